@@ -1,0 +1,204 @@
+"""fp64 CPU oracle of the decode hot path (ctypes front end of qkv_oracle.c).
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. The CUDA library and
+its Python binding never import it, and the two share no code: the only
+common inputs are the arrays drawn by ``workloads``.
+
+Every function takes and returns numpy arrays. bf16 and fp16 values travel as
+``uint16`` bit patterns; results are float64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "qkv_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Compile qkv_oracle.c with gcc (no fast-math, no FP contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+                               "-D_DEFAULT_SOURCE", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class YarnParams(ctypes.Structure):
+    _fields_ = [("rope_base", ctypes.c_double), ("rot_dim", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("factor", ctypes.c_double), ("orig_max_pos", ctypes.c_int64),
+                ("beta_fast", ctypes.c_double), ("beta_slow", ctypes.c_double),
+                ("ext_factor", ctypes.c_double), ("attn_factor", ctypes.c_double)]
+
+
+def _params(spec: Dict) -> YarnParams:
+    return YarnParams(float(spec["rope_base"]), int(spec["rot_dim"]), 0, float(spec.get("factor", 1.0)),
+                      int(spec.get("orig_max_pos", 262144)), float(spec.get("beta_fast", 32.0)),
+                      float(spec.get("beta_slow", 1.0)), float(spec.get("ext_factor", -1.0)),
+                      float(spec.get("attn_factor", 0.0)))
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        d, i32, i64, vp = ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
+        P = ctypes.POINTER(YarnParams)
+        sig = {
+            "oracle_yarn_theta": (d, [P, vp, vp, vp]),
+            "oracle_yarn_table": (None, [P, i64, i64, vp, vp]),
+            "oracle_rope_apply_f64": (None, [vp, vp, vp, i32, i32, i32, P]),
+            "oracle_rope_apply_bf16": (None, [vp, vp, vp, i32, i32, i32, P]),
+            "oracle_quantize_cell": (None, [vp, vp, vp]),
+            "oracle_kv_write_f4": (i32, [vp, vp, vp, i64, vp, vp, vp, vp, i32, i32, i32, i64]),
+            "oracle_paged_attention": (None, [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32,
+                                              d, vp, vp, i32]),
+            "oracle_lse_merge": (None, [vp, vp, i32, i32, i32, vp, vp]),
+            "oracle_max_threads": (i32, []),
+            "oracle_f64_to_f16_array": (None, [vp, vp, i64]),
+            "oracle_f16_to_f64_array": (None, [vp, vp, i64]),
+            "oracle_f64_to_bf16_array": (None, [vp, vp, i64]),
+            "oracle_bf16_to_f64_array": (None, [vp, vp, i64]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(_lib, name)
+            fn.restype, fn.argtypes = res, args
+    return _lib
+
+
+def _p(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def _c(a, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ---------------------------------------------------------------------------
+# formats
+
+def f64_to_f16(x) -> np.ndarray:
+    x = _c(x, np.float64); y = np.empty(x.shape, np.uint16)
+    lib().oracle_f64_to_f16_array(_p(x), _p(y), x.size); return y
+
+
+def f16_to_f64(x) -> np.ndarray:
+    x = _c(x, np.uint16); y = np.empty(x.shape, np.float64)
+    lib().oracle_f16_to_f64_array(_p(x), _p(y), x.size); return y
+
+
+def f64_to_bf16(x) -> np.ndarray:
+    x = _c(x, np.float64); y = np.empty(x.shape, np.uint16)
+    lib().oracle_f64_to_bf16_array(_p(x), _p(y), x.size); return y
+
+
+def bf16_to_f64(x) -> np.ndarray:
+    x = _c(x, np.uint16); y = np.empty(x.shape, np.float64)
+    lib().oracle_bf16_to_f64_array(_p(x), _p(y), x.size); return y
+
+
+# ---------------------------------------------------------------------------
+# rotary
+
+def yarn_theta(spec: Dict) -> Tuple[np.ndarray, float, float, float]:
+    """(theta [rot_dim/2], mscale, low, high)."""
+    p = _params(spec)
+    th = np.empty(p.rot_dim // 2, np.float64)
+    lo, hi = ctypes.c_double(), ctypes.c_double()
+    ms = lib().oracle_yarn_theta(ctypes.byref(p), _p(th), ctypes.addressof(lo), ctypes.addressof(hi))
+    return th, ms, lo.value, hi.value
+
+
+def yarn_table(spec: Dict, pos0: int, n_pos: int) -> Tuple[np.ndarray, np.ndarray]:
+    p = _params(spec)
+    c = np.empty((n_pos, p.rot_dim // 2)); s = np.empty_like(c)
+    lib().oracle_yarn_table(ctypes.byref(p), pos0, n_pos, _p(c), _p(s))
+    return c, s
+
+
+def rope_apply_f64(x, positions, spec: Dict) -> np.ndarray:
+    """x float64 [n_tok][n_heads][head_dim] -> rotated copy (float64)."""
+    x = _c(x, np.float64); pos = _c(positions, np.int64); y = np.empty_like(x)
+    p = _params(spec)
+    lib().oracle_rope_apply_f64(_p(x), _p(y), _p(pos), x.shape[0], x.shape[1], x.shape[2], ctypes.byref(p))
+    return y
+
+
+def rope_apply_bf16(x, positions, spec: Dict) -> np.ndarray:
+    """x bf16 bits [n_tok][n_heads][head_dim] -> rotated bf16 bits."""
+    x = _c(x, np.uint16); pos = _c(positions, np.int64); y = np.empty_like(x)
+    p = _params(spec)
+    lib().oracle_rope_apply_bf16(_p(x), _p(y), _p(pos), x.shape[0], x.shape[1], x.shape[2], ctypes.byref(p))
+    return y
+
+
+# ---------------------------------------------------------------------------
+# F4 cache
+
+def quantize_cell(x32) -> Tuple[np.ndarray, int]:
+    x = _c(x32, np.uint16); assert x.size == 32
+    b = np.empty(16, np.uint8); s = np.empty(1, np.uint16)
+    lib().oracle_quantize_cell(_p(x), _p(b), _p(s))
+    return b, int(s[0])
+
+
+def empty_cache(num_pages: int, kv_heads: int, block_size: int, head_dim: int):
+    """Zeroed (k_data, k_scale, v_data, v_scale) in the paged layout."""
+    data = lambda: np.zeros((num_pages, kv_heads, block_size, head_dim // 2), np.uint8)
+    scale = lambda: np.zeros((num_pages, kv_heads, block_size, head_dim // 32), np.uint16)
+    return data(), scale(), data(), scale()
+
+
+def kv_write_f4(k, v, slots, cache, kv_heads: int, head_dim: int, block_size: int) -> int:
+    """Quantise rows of k, v (bf16 bits [n_tok][kv_heads][head_dim]) into
+    ``cache`` (in place) at ``slots``; returns the number of bad slots."""
+    k = _c(k, np.uint16); v = _c(v, np.uint16); sl = _c(slots, np.int64)
+    kd, ks, vd, vs = cache
+    for a in cache:
+        assert a.flags.c_contiguous
+    return lib().oracle_kv_write_f4(_p(k), _p(v), _p(sl), sl.size, _p(kd), _p(ks), _p(vd), _p(vs),
+                                    kv_heads, head_dim, block_size, kd.shape[0])
+
+
+# ---------------------------------------------------------------------------
+# attention
+
+def paged_attention(q, cache, page_table, tok_begin, tok_end, q_heads: int, kv_heads: int,
+                    head_dim: int, block_size: int, softmax_scale: Optional[float] = None,
+                    n_threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """Exact softmax attention per (sequence, query head) over the token range
+    [tok_begin[s], tok_end[s]). Returns (out [n_seq][Hq][D], lse2 [n_seq][Hq])."""
+    q = _c(q, np.uint16); pt = _c(page_table, np.int32)
+    tb = _c(tok_begin, np.int32); te = _c(tok_end, np.int32)
+    n_seq = pt.shape[0]
+    kd, ks, vd, vs = (np.ascontiguousarray(a) for a in cache)
+    out = np.empty((n_seq, q_heads, head_dim)); lse2 = np.empty((n_seq, q_heads))
+    sc = float(softmax_scale) if softmax_scale else 1.0 / np.sqrt(head_dim)
+    lib().oracle_paged_attention(_p(q), _p(kd), _p(ks), _p(vd), _p(vs), _p(pt), pt.shape[1], _p(tb), _p(te),
+                                 n_seq, q_heads, kv_heads, head_dim, block_size, sc, _p(out), _p(lse2),
+                                 n_threads)
+    return out, lse2
+
+
+def lse_merge(o_parts, lse2_parts) -> Tuple[np.ndarray, np.ndarray]:
+    """o_parts [n_parts][rows][D], lse2_parts [n_parts][rows] -> (out, lse2)."""
+    o = _c(o_parts, np.float64); l = _c(lse2_parts, np.float64)
+    n, rows, d = o.shape
+    out = np.empty((rows, d)); lse2 = np.empty(rows)
+    lib().oracle_lse_merge(_p(o), _p(l), n, rows, d, _p(out), _p(lse2))
+    return out, lse2
+
+
+def max_threads() -> int:
+    return lib().oracle_max_threads()

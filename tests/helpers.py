@@ -1,0 +1,38 @@
+"""Shared test helpers: building oracle-side caches from the seeded workloads.
+(Test infrastructure; uses the oracle and the generator only.)"""
+import numpy as np
+
+import oracle
+import workloads
+
+
+def oracle_layer(w, layer=0, inputs=None, with_step=True):
+    """Quantise a workload layer into an oracle cache. Returns (inputs, cache).
+    With ``with_step`` the decode step's (unroped) k_new/v_new are written too,
+    at the step slots; rotary is the caller's business."""
+    x = inputs if inputs is not None else workloads.host_layer(w, layer)
+    cache = oracle.empty_cache(w.num_pages, w.kv_heads, w.block_size, w.head_dim)
+    bad = oracle.kv_write_f4(x["k_cache"], x["v_cache"], x["cache_slots"], cache, w.kv_heads, w.head_dim,
+                             w.block_size)
+    assert bad == 0
+    if with_step:
+        bad = oracle.kv_write_f4(x["k_new"], x["v_new"], x["step_slots"], cache, w.kv_heads, w.head_dim,
+                                 w.block_size)
+        assert bad == 0
+    return x, cache
+
+
+def dense_dequant(cache, page_table, seq, n_tok, block_size):
+    """[n_tok][Hkv][D] float64 K and V of one sequence, by an explicit gather
+    (independent of the oracle's paged walk)."""
+    kd, ks, vd, vs = cache
+    t = np.arange(n_tok)
+    pages = page_table[seq, t // block_size]
+    off = t % block_size
+
+    def deq(d, s):
+        b = d[pages, :, off, :]                        # [n_tok][Hkv][D/2] u8
+        codes = np.stack([b & 15, b >> 4], -1).reshape(b.shape[0], b.shape[1], -1).astype(np.float64)
+        sc = s[pages, :, off, :].view(np.float16).astype(np.float64)   # [n_tok][Hkv][D/32]
+        return (codes - 8) * np.repeat(sc, 32, axis=-1)
+    return deq(kd, ks), deq(vd, vs)
