@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the paged F4 attention hot path on B200.
+
+One step = one decode token for every sequence of the workload through all
+its full-attention layers: the YaRN table row(s) of the step positions, the
+partial rotary of q and of the new key, the F4 write of the new K/V, the
+split-KV paged attention and the log2-sum-exp merge -- 1 + 5 x layers kernel
+launches, replayed from a CUDA graph.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). ``value`` is the whole-job rate of algorithmic
+K/V bytes (packed data + fp16 scales + page-table entries + q in + out) in
+GB/s, device-timed with CUDA events, max over ranks. Each rank runs its own
+copy of the workload (independent sequences): weak scaling, no collective on
+the data path. ``--impl reference`` times the fp64 CPU oracle on the host
+cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "paged F4 decode-attn K/V GB/s (% of B200 HBM peak); tokens/s per layer at 262k"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=workloads.YARN_262K.name, choices=sorted(workloads.BY_NAME))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="host-time budget of the CPU baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- peaks / profiles
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("decode_split.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "quantized_paged_kv_yarn_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per split-kernel launch from the committed ncu summary, if
+    it was taken from the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"paged_decode_split_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_traffic = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_hash or not m_traffic or m_hash.group(1) != kernel_source_hash():
+        return None
+    return int(m_traffic.group(1))
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device, period_s: float = 0.005):
+        self.period = period_s
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- CPU oracle sample
+
+def oracle_step_sample(w: workloads.Workload, n_tok: int, seed: int = 1):
+    """Build a host sample of the workload (same recipe, first ``n_tok``
+    context tokens of the first sequence) and return a callable that runs one
+    oracle decode step on it, plus the algorithmic bytes that step covers."""
+    import oracle
+    s = workloads.Workload(name=w.name + "_sample", n_layers=1, seq_lens=(n_tok,),
+                           num_pages=-(-n_tok // w.block_size), block_size=w.block_size, q_heads=w.q_heads,
+                           kv_heads=w.kv_heads, head_dim=w.head_dim, rot_dim=w.rot_dim, rope_base=w.rope_base,
+                           yarn_factor=w.yarn_factor, orig_max_pos=w.orig_max_pos, beta_fast=w.beta_fast,
+                           beta_slow=w.beta_slow, first_position=w.first_position + w.seq_lens[0] - n_tok,
+                           head_scale=w.head_scale, k_outlier_frac=w.k_outlier_frac, seed=seed)
+    x = workloads.host_layer(s)
+    cache = oracle.empty_cache(s.num_pages, s.kv_heads, s.block_size, s.head_dim)
+    oracle.kv_write_f4(x["k_cache"], x["v_cache"], x["cache_slots"], cache, s.kv_heads, s.head_dim, s.block_size)
+    spec = workloads.yarn_spec(s)
+
+    def step():
+        q = oracle.rope_apply_bf16(x["q"], x["positions"], spec)
+        k = oracle.rope_apply_bf16(x["k_new"], x["positions"], spec)
+        oracle.kv_write_f4(k, x["v_new"], x["step_slots"], cache, s.kv_heads, s.head_dim, s.block_size)
+        return oracle.paged_attention(q, cache, x["page_table"], [0], x["seq_lens"], s.q_heads, s.kv_heads,
+                                      s.head_dim, s.block_size)
+
+    return step, s.algorithmic_bytes_per_layer(), oracle.max_threads()
+
+
+def calibrate_sample(w, seconds: float):
+    """Token count whose oracle step takes about ``seconds`` on this host."""
+    probe = min(2048, w.seq_lens[0])
+    step, _, _ = oracle_step_sample(w, probe)
+    t0 = time.perf_counter()
+    step()
+    dt = max(time.perf_counter() - t0, 1e-4)
+    n = int(probe * seconds / dt) // w.block_size * w.block_size
+    return max(w.block_size, min(w.seq_lens[0], n))
+
+
+def cpu_baseline(w, seconds: float):
+    n_tok = calibrate_sample(w, seconds)
+    step, nbytes, cores = oracle_step_sample(w, n_tok)
+    t0 = time.perf_counter()
+    step()
+    dt = time.perf_counter() - t0
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"one layer, first sequence, {n_tok} of {w.seq_lens[0]} context tokens "
+                      f"(rotary + F4 write of the new token + exact attention, fp64), {dt:.1f} s"}
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return
+    w = workloads.BY_NAME[args.workload]
+    per_step = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    n_tok = calibrate_sample(w, per_step)
+    step, nbytes, cores = oracle_step_sample(w, n_tok)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    value = nbytes / dt / 1e9
+    sample = (f"each step: one layer, first sequence, {n_tok} of {w.seq_lens[0]} context tokens "
+              f"(rotary + F4 write + exact attention, fp64 oracle)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, args),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def config_of(w, args):
+    return {"workload": w.name, "layers": w.n_layers, "seq_lens": list(w.seq_lens), "q_heads": w.q_heads,
+            "kv_heads": w.kv_heads, "head_dim": w.head_dim, "rot_dim": w.rot_dim, "block_size": w.block_size,
+            "yarn_factor": w.yarn_factor, "step_positions": w.step_positions, "parallelism": f"replicas{args.gpus}",
+            "l2": "inputs larger than L2: each layer's cache exceeds 126 MB and the step walks all layers"}
+
+
+# --------------------------------------------------------------------------- our arm
+
+class Bench:
+    def __init__(self, w: workloads.Workload, device, seed_offset: int):
+        import torch
+
+        import quantized_paged_kv_yarn_b200 as qkv
+        self.torch, self.qkv, self.w, self.dev = torch, qkv, w, device
+        w = dataclass_replace(w, seed=w.seed + seed_offset)
+        self.w = w
+        self.L = w.n_layers
+        self.caches, self.q_raw, self.kn_raw, self.vn = [], [], [], []
+        for layer in range(self.L):
+            x = workloads.device_layer(w, layer, device)
+            c = qkv.PagedF4Cache.allocate(w.num_pages, w.kv_heads, w.block_size, w.head_dim, device=device)
+            c.write(x["k_cache"], x["v_cache"], x["cache_slots"])
+            self.caches.append(c)
+            self.q_raw.append(x["q"])
+            self.kn_raw.append(x["k_new"])
+            self.vn.append(x["v_new"])
+            if layer == 0:
+                self.page_table, self.seq_lens = x["page_table"], x["seq_lens"]
+                self.positions, self.step_slots = x["positions"], x["step_slots"]
+            del x
+        torch.cuda.synchronize()
+        self.q_rot = [torch.empty_like(t) for t in self.q_raw]
+        self.k_rot = [torch.empty_like(t) for t in self.kn_raw]
+        self.out = [torch.empty_like(t) for t in self.q_raw]
+        pos = w.step_positions
+        self.pos0, self.n_rows = min(pos), max(pos) - min(pos) + 1
+        self.cos = torch.empty((self.n_rows, w.rot_dim // 2), dtype=torch.float32, device=device)
+        self.sin = torch.empty_like(self.cos)
+        self.params = qkv.YarnParams.make(**workloads.yarn_spec(w))
+        self.att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.launches_per_step = 1 + 5 * self.L
+        # host side of the end-to-end measurement (pinned)
+        self.h_q = [t.cpu().pin_memory() for t in self.q_raw]
+        self.h_kn = [t.cpu().pin_memory() for t in self.kn_raw]
+        self.h_vn = [t.cpu().pin_memory() for t in self.vn]
+        self.h_pos = self.positions.cpu().pin_memory()
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.out]
+
+    def step(self):
+        q, w = self.qkv, self.w
+        q.qkv_yarn_rope_table(self.params, self.pos0, self.n_rows, self.cos, self.sin)
+        for l in range(self.L):
+            q.qkv_rope_apply(self.q_raw[l], self.q_rot[l], self.positions, self.cos, self.sin, self.pos0, w.rot_dim,
+                             device_status=self.status)
+            q.qkv_rope_apply(self.kn_raw[l], self.k_rot[l], self.positions, self.cos, self.sin, self.pos0,
+                             w.rot_dim, device_status=self.status)
+            self.caches[l].write(self.k_rot[l], self.vn[l], self.step_slots, device_status=self.status)
+            self.att(self.out[l], self.q_rot[l], self.caches[l], self.page_table, self.seq_lens,
+                     num_splits=w.num_splits, device_status=self.status)
+
+    def e2e_step(self):
+        """Host buffers in, the step, the result back to the host."""
+        for l in range(self.L):
+            self.q_raw[l].copy_(self.h_q[l], non_blocking=True)
+            self.kn_raw[l].copy_(self.h_kn[l], non_blocking=True)
+            self.vn[l].copy_(self.h_vn[l], non_blocking=True)
+        self.positions.copy_(self.h_pos, non_blocking=True)
+        self.step()
+        for l in range(self.L):
+            self.h_out[l].copy_(self.out[l], non_blocking=True)
+
+    def io_bytes(self):
+        nb = lambda ts: sum(t.numel() * t.element_size() for t in ts)
+        return nb(self.h_q) + nb(self.h_kn) + nb(self.h_vn) + nb([self.h_pos]), nb(self.h_out)
+
+    def capture(self, fn):
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    def split_kernel_ms(self, reps: int):
+        """Average duration of the split-pass kernel alone, CUDA events on its
+        stream around each launch, each layer's cache in turn (cold in L2)."""
+        torch, qkv, w = self.torch, self.qkv, self.w
+        rows = w.n_seq * w.q_heads
+        ms = self.att.max_splits
+        o_parts = torch.empty((ms, rows, w.head_dim), dtype=torch.float32, device=self.dev)
+        l_parts = torch.empty((ms, rows), dtype=torch.float32, device=self.dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps * self.L)]
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=self.dev)
+        for i in range(reps * self.L):
+            l = i % self.L
+            c = self.caches[l]
+            if self.L == 1:
+                flush.zero_()
+            ev[i][0].record()
+            qkv.qkv_paged_decode_split_f4(o_parts, l_parts, self.q_rot[l], c.k_data, c.k_scale, c.v_data,
+                                          c.v_scale, self.page_table, self.seq_lens, w.kv_heads,
+                                          num_splits=w.num_splits)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        t = [a.elapsed_time(b) for a, b in ev]
+        return float(np.mean(t)), float(np.median(t))
+
+
+def dataclass_replace(w, **kw):
+    import dataclasses
+    return dataclasses.replace(w, **kw)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    w = workloads.BY_NAME[args.workload]
+    b = Bench(w, dev, seed_offset=rank)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm the library (tensor maps, occupancy) before any capture
+    b.step()
+    torch.cuda.synchronize()
+    if args.no_graph:
+        run_step, run_e2e = b.step, b.e2e_step
+    else:
+        g_step = b.capture(b.step)
+        g_e2e = b.capture(b.e2e_step)
+        run_step, run_e2e = g_step.replay, g_e2e.replay
+
+    # ---- device-timed steps
+    for _ in range(args.warmup):
+        run_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            run_step()
+        e1.record()
+        torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    status = int(b.status.item())
+
+    # ---- end to end through host buffers
+    for _ in range(max(1, args.warmup // 2)):
+        run_e2e()
+    barrier()
+    e0.record()
+    for _ in range(args.steps):
+        run_e2e()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    # ---- the dominant kernel alone, for the roofline
+    split_ms_mean, split_ms_median = b.split_kernel_ms(reps=max(1, min(args.steps, 50) // 5))
+    split_ms_mean = max_over_ranks(split_ms_mean)
+
+    if rank != 0:
+        return
+    per_layer = w.algorithmic_bytes_per_layer()
+    step_bytes = per_layer * w.n_layers
+    value = world * step_bytes / (ms * 1e-3) / 1e9
+    e2e_value = world * step_bytes / (ms_e2e * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+    out_bytes = 2 * w.n_seq * w.q_heads * w.head_dim
+    split_bytes = per_layer - out_bytes  # the merge writes out
+    achieved = split_bytes / (split_ms_mean * 1e-3) / 1e9
+    traffic = profiled_traffic(w.name)
+    bi, bo = b.io_bytes()
+    clocks = clk.summary()
+    result = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 mma, f32 accumulate (u4 cache)", "data": "synthetic",
+        "config": config_of(w, args),
+        "pct_of_hbm_peak": 100.0 * value / world / peak,
+        "decode_tokens_per_s_per_layer": world * w.n_seq * w.n_layers / (ms * 1e-3),
+        "context_tokens_per_s": world * sum(w.seq_lens) * w.n_layers / (ms * 1e-3),
+        "device_status": status,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "paged_decode_split_kernel", "peak_kind": f"{peak_kind} (copy bandwidth)",
+                     "kernel_ms": split_ms_mean, "kernel_ms_median": split_ms_median,
+                     "algorithmic_bytes_per_launch": split_bytes},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+                "ms_per_step": ms_e2e},
+        "gpu_launches": b.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    print(json.dumps(result), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device(f"cuda:{local_rank}"))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,229 @@
+/*
+ * qkv.h -- C ABI of the B200 (sm_100a) decode hot path for long-context
+ * serving over a paged, 4-bit ("F4") K/V cache with YaRN partial rotary.
+ *
+ * The operations follow these sources (page title, section):
+ *   [YARN]  mistral.rs PR "YaRN rope scaling, 4-bit F4 packed KV cache, and
+ *           hybrid paged attention for Qwen3.5-Next long-context serving",
+ *           section 1: YaRN for a partial rotary, llama.cpp-style corr_dims
+ *           ramp from beta_fast/beta_slow, table scale 1 + 0.1 ln(factor).
+ *   [AUTO]  ignis docs "context-and-speculation", --model-rope-scaling: auto
+ *           factor max_context / 262,144; the attention factor applies to
+ *           queries and keys alike.
+ *   [F4]    same PR, section 2: packed 4-bit cache written by a
+ *           reshape-and-cache kernel through a slot mapping, values
+ *           (nibble - 8) * scale, 32 values per 16-byte cell.
+ *   [PAGED] same PR section 2 (v1/v2 paged attention dequantising cells
+ *           inline) and ignis "context-and-speculation" (the KV pool in
+ *           64-token pages, lanes sharing one pool).
+ *   [FOLD]  FreeToken issue #568 "Serving ...'s 1M-token window on one 24 GB
+ *           card", proposed solution item 2: partial results folded by
+ *           log2-sum-exp.
+ *
+ * Conventions for every call:
+ *   - Array arguments are DEVICE pointers owned by the caller, except where a
+ *     comment says "host". The library allocates no memory.
+ *   - bf16 and fp16 values travel as uint16_t bit patterns.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream);
+ *     the library never synchronises the host.
+ *   - Return value: QKV_OK, or an error code below when an argument is
+ *     invalid (nothing is launched) or a launch fails.
+ *   - Data-dependent problems found on the device (a page id outside the
+ *     pool, a slot outside the pool, a position outside the table, a length
+ *     past the page table) never trap: the kernel skips the offending item
+ *     and ORs a QKV_DEV_* flag into `*device_status` when that pointer is not
+ *     NULL. The caller zeroes the word and reads it when convenient.
+ *   - Kernels contain no waits on other blocks. The waits on their own copy
+ *     barriers are bounded; one that runs out sets QKV_DEV_TIMEOUT and the
+ *     block returns.
+ */
+#ifndef QKV_H_
+#define QKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QKV_API __attribute__((visibility("default")))
+#else
+#define QKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* qkv_stream_t;
+
+/* Return codes. */
+#define QKV_OK 0
+#define QKV_EINVAL 1       /* invalid argument (null pointer, bad size or alignment) */
+#define QKV_EUNSUPPORTED 2 /* valid, but outside the compiled shapes */
+#define QKV_ECUDA 3        /* a CUDA launch or driver call failed */
+
+/* Device status flags (ORed into *device_status). */
+#define QKV_DEV_BAD_POSITION 0x1 /* rope position outside the table: token left unrotated */
+#define QKV_DEV_BAD_SLOT 0x2     /* write slot >= num_pages * block_size: token skipped */
+#define QKV_DEV_BAD_PAGE 0x4     /* page id < 0 or >= num_pages: page skipped */
+#define QKV_DEV_BAD_SEQLEN 0x8   /* seq_len < 0 or > max_pages_per_seq * block_size: clamped */
+#define QKV_DEV_TIMEOUT 0x10     /* a bounded wait on a copy barrier ran out */
+
+/* Rotary configuration [YARN], [AUTO].
+ *   rope_base    frequency base (1e7 for the workloads here).
+ *   rot_dim      rotated dims per head (the first rot_dim of head_dim);
+ *                even, 2..512.
+ *   factor       YaRN scale s >= 1; 1 = no scaling (textbook RoPE table).
+ *   orig_max_pos trained context length the ramp is measured against.
+ *   beta_fast, beta_slow  ramp bounds in turns over orig_max_pos (32, 1).
+ *   ext_factor   ramp weight; < 0 selects 1 when factor > 1, else 0.
+ *   attn_factor  table scale; <= 0 selects 1 + 0.1 ln(factor) when
+ *                factor > 1, else 1.
+ * Pair j < rot_dim/2 has omega_j = rope_base^(-2j/rot_dim) and angle step
+ *   theta_j = (omega_j / s) (1 - r_j e) + omega_j r_j e,
+ * r_j = 1 - clamp((j - low) / max(0.001, high - low), 0, 1), where low =
+ * max(0, floor(c(beta_fast))), high = min(rot_dim - 1, ceil(c(beta_slow))),
+ * c(b) = rot_dim ln(orig_max_pos / (2 pi b)) / (2 ln rope_base). */
+typedef struct {
+  double rope_base;
+  int32_t rot_dim;
+  int32_t reserved; /* set to 0 */
+  double factor;
+  int64_t orig_max_pos;
+  double beta_fast;
+  double beta_slow;
+  double ext_factor;
+  double attn_factor;
+} qkv_yarn_params;
+
+/* [AUTO] Host-only helper: the YaRN factor the auto rule picks for a
+ * maximum context. Returns 0 when no scaling is needed (max_context <=
+ * orig_max_pos), -1 when the context is refused (factor above 64 or a
+ * non-positive argument), else max_context / orig_max_pos. */
+QKV_API double qkv_yarn_auto_factor(int64_t max_context, int64_t orig_max_pos);
+
+/* a1 [YARN] YaRN rotary table.
+ *   params   HOST pointer.
+ *   cos_out, sin_out  float [n_pos][rot_dim/2]; row i is position
+ *            pos_start + i; each value is mscale * cos|sin(p * theta_j) with
+ *            the angle formed and evaluated in double, stored as float.
+ * EINVAL: null pointer, n_pos < 0, pos_start < 0, rot_dim odd or out of
+ * range, factor < 1, rope_base <= 1, orig_max_pos <= 0. */
+QKV_API int qkv_yarn_rope_table(const qkv_yarn_params* params, int64_t pos_start, int64_t n_pos,
+                        float* cos_out, float* sin_out, qkv_stream_t stream);
+
+/* a2 [YARN], [AUTO] Partial NEOX rotary on q or k rows.
+ *   x_in, x_out  bf16 [n_tok][n_heads][head_dim]; x_out may equal x_in
+ *                (in place); otherwise the ranges must not overlap.
+ *   positions    int64 [n_tok], position of each token.
+ *   cos_tab, sin_tab  a table from qkv_yarn_rope_table covering positions
+ *                table_pos_start .. table_pos_start + table_len - 1.
+ * For j < rot_dim/2: (x_j, x_{j+rot/2}) -> (x_j c - x_{j+rot/2} s,
+ * x_{j+rot/2} c + x_j s) in float, rounded to bf16 (nearest even); dims >=
+ * rot_dim are copied. A position outside the table copies the token
+ * unrotated and sets QKV_DEV_BAD_POSITION.
+ * n_tok == 0 or n_heads == 0 returns QKV_OK without touching any pointer.
+ * EINVAL: null pointer, n_tok/n_heads < 0, rot_dim odd or > head_dim,
+ * head_dim odd, table_len < 0, distinct x_in/x_out that overlap. */
+QKV_API int qkv_rope_apply(const uint16_t* x_in, uint16_t* x_out, const int64_t* positions, int32_t n_tok,
+                   int32_t n_heads, int32_t head_dim, int32_t rot_dim, const float* cos_tab,
+                   const float* sin_tab, int64_t table_pos_start, int64_t table_len,
+                   int32_t* device_status, qkv_stream_t stream);
+
+/* a3 [F4] Quantise and write new K/V rows into the paged F4 cache.
+ *   k, v          bf16 [n_tok][kv_heads][head_dim].
+ *   slot_mapping  int64 [n_tok]: page * block_size + offset; < 0 skips the
+ *                 token; >= num_pages * block_size skips it and sets
+ *                 QKV_DEV_BAD_SLOT.
+ *   k_data, v_data    u8  [num_pages][kv_heads][block_size][head_dim/2]
+ *   k_scale, v_scale  fp16 [num_pages][kv_heads][block_size][head_dim/32]
+ * Per 32-value cell: scale = fp16(amax / 7), round to nearest even,
+ * saturating at 65504; code = clamp(rint(x / scale), -8, 7) + 8 (all 8 when
+ * scale is 0); byte b holds element 2b in bits 0-3 and 2b+1 in bits 4-7.
+ * The result is bit-identical to evaluating both divisions exactly.
+ * n_tok == 0 returns QKV_OK without touching any pointer.
+ * EINVAL: null pointer, n_tok < 0, head_dim not a multiple of 32 or > 256,
+ * kv_heads < 1, block_size < 1, num_pages < 1, k/v not 16-byte aligned. */
+QKV_API int qkv_kv_write_f4(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping,
+                    int32_t n_tok, uint8_t* k_data, uint16_t* k_scale, uint8_t* v_data,
+                    uint16_t* v_scale, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                    int64_t num_pages, int32_t* device_status, qkv_stream_t stream);
+
+/* Number of splits per sequence the automatic plan aims for on the current
+ * device (resident split blocks / kv_heads); a workspace sized with this as
+ * max_splits never limits the automatic plan. Host-only; returns 0 when no
+ * CUDA device is present. */
+QKV_API int32_t qkv_paged_decode_auto_splits(int32_t kv_heads, int32_t block_size);
+
+/* Bytes of workspace qkv_paged_decode_attn_f4 needs: max_splits *
+ * n_seq * q_heads * (head_dim + 1) floats, rounded up to 256 bytes. */
+QKV_API size_t qkv_paged_decode_workspace_bytes(int32_t n_seq, int32_t q_heads, int32_t head_dim,
+                                        int32_t max_splits);
+
+/* a4 [PAGED], [FOLD] Split pass of paged GQA decode attention.
+ *   q         bf16 [n_seq][q_heads][head_dim] (already rotated).
+ *   k_data, k_scale, v_data, v_scale  the F4 cache (layout as in
+ *             qkv_kv_write_f4).
+ *   page_table  int32 [n_seq][max_pages_per_seq]; token i of sequence s is
+ *             in page page_table[s][i / block_size] at offset i % block_size.
+ *   seq_lens  int32 [n_seq], context tokens of each sequence.
+ *   softmax_scale  0 selects 1/sqrt(head_dim).
+ *   num_splits  > 0: every sequence is cut into min(num_splits, max_splits)
+ *             splits; 0: the plan balances pages over the device (splits of
+ *             about sum(pages) / auto_splits pages each, at most max_splits
+ *             per sequence). Split i of a sequence with n pages covers pages
+ *             [i*n/S, (i+1)*n/S).
+ *   o_parts   float [max_splits][n_seq * q_heads][head_dim]: partial output
+ *             of split i for row (s, h) at [i][s * q_heads + h], normalised
+ *             by its own softmax sum.
+ *   lse2_parts float [max_splits][n_seq * q_heads]: log2 of the split's
+ *             softmax normaliser, log2 sum_t 2^(score_t log2 e); -inf for an
+ *             empty or unused split (its o_parts row is then unspecified).
+ * Shapes compiled: head_dim 256, q_heads / kv_heads in {1, 2, 4, 8},
+ * block_size in {16, 32, 64}; others return QKV_EUNSUPPORTED. Cache and q
+ * pointers must be 16-byte aligned (EINVAL otherwise). */
+QKV_API int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int32_t max_splits,
+                              const uint16_t* q, const uint8_t* k_data, const uint16_t* k_scale,
+                              const uint8_t* v_data, const uint16_t* v_scale,
+                              const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
+                              int32_t q_heads, int32_t kv_heads, int32_t head_dim,
+                              int32_t block_size, int32_t max_pages_per_seq, int64_t num_pages,
+                              float softmax_scale, int32_t num_splits, int32_t* device_status,
+                              qkv_stream_t stream);
+
+/* a5 [FOLD] log2-sum-exp merge of partial attention results.
+ *   o_parts   float [n_parts][rows][head_dim], lse2_parts float [n_parts][rows].
+ *   out       bf16 [rows][head_dim] (nearest even); lse2_out float [rows] or NULL.
+ * Per row: M = max_i lse2_i; w_i = 2^(lse2_i - M); out = sum_i w_i o_i /
+ * sum_i w_i; lse2 = M + log2 sum_i w_i. Parts with lse2 = -inf carry no
+ * weight and their o rows are not read; a row without any gives out = 0 and
+ * lse2 = -inf.
+ * EINVAL: null pointer, n_parts < 1, rows < 0, head_dim not a multiple of 4
+ * or > 1024. */
+QKV_API int qkv_lse_merge(const float* o_parts, const float* lse2_parts, int32_t n_parts, int32_t rows,
+                  int32_t head_dim, uint16_t* out, float* lse2_out, qkv_stream_t stream);
+
+/* a4 + a5: the decode attention of one layer. Runs the split pass into
+ * `workspace` (see qkv_paged_decode_workspace_bytes) and merges it into
+ * `out` (bf16 [n_seq][q_heads][head_dim]) and `lse2_out` (float
+ * [n_seq][q_heads] or NULL). Arguments and errors as in the two calls;
+ * EINVAL also when workspace_bytes is too small or workspace is not
+ * 256-byte aligned. */
+QKV_API int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q,
+                             const uint8_t* k_data, const uint16_t* k_scale,
+                             const uint8_t* v_data, const uint16_t* v_scale,
+                             const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
+                             int32_t q_heads, int32_t kv_heads, int32_t head_dim,
+                             int32_t block_size, int32_t max_pages_per_seq, int64_t num_pages,
+                             float softmax_scale, int32_t num_splits, int32_t max_splits,
+                             void* workspace, size_t workspace_bytes, int32_t* device_status,
+                             qkv_stream_t stream);
+
+/* Static text for a return code. */
+QKV_API const char* qkv_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKV_H_ */

@@ -1,0 +1,195 @@
+"""ctypes declarations of include/qkv.h and argument marshalling."""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqkv.so")
+
+QKV_OK, QKV_EINVAL, QKV_EUNSUPPORTED, QKV_ECUDA = 0, 1, 2, 3
+DEV_BAD_POSITION, DEV_BAD_SLOT, DEV_BAD_PAGE, DEV_BAD_SEQLEN, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
+
+
+class QkvError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {qkv_status_string(code)} (status {code})")
+        self.code = code
+
+
+class YarnParams(ctypes.Structure):
+    """Mirror of qkv_yarn_params."""
+    _fields_ = [("rope_base", ctypes.c_double), ("rot_dim", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("factor", ctypes.c_double), ("orig_max_pos", ctypes.c_int64),
+                ("beta_fast", ctypes.c_double), ("beta_slow", ctypes.c_double),
+                ("ext_factor", ctypes.c_double), ("attn_factor", ctypes.c_double)]
+
+    @classmethod
+    def make(cls, rope_base=1e7, rot_dim=64, factor=1.0, orig_max_pos=262144, beta_fast=32.0, beta_slow=1.0,
+             ext_factor=-1.0, attn_factor=0.0):
+        return cls(float(rope_base), int(rot_dim), 0, float(factor), int(orig_max_pos), float(beta_fast),
+                   float(beta_slow), float(ext_factor), float(attn_factor))
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m quantized_paged_kv_yarn_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i32, _i64, _f32, _f64, _sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                    ctypes.c_double, ctypes.c_size_t)
+_SIGS = {
+    "qkv_yarn_auto_factor": (_f64, [_i64, _i64]),
+    "qkv_yarn_rope_table": (ctypes.c_int, [ctypes.POINTER(YarnParams), _i64, _i64, _vp, _vp, _vp]),
+    "qkv_rope_apply": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i64, _i64, _vp, _vp]),
+    "qkv_kv_write_f4": (ctypes.c_int, [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i64, _vp,
+                                       _vp]),
+    "qkv_paged_decode_auto_splits": (_i32, [_i32, _i32]),
+    "qkv_paged_decode_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
+    "qkv_paged_decode_split_f4": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+                                                 _i32, _i32, _i32, _i32, _i64, _f32, _i32, _vp, _vp]),
+    "qkv_lse_merge": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "qkv_paged_decode_attn_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                                                _i32, _i32, _i32, _i64, _f32, _i32, _i32, _vp, _sz, _vp, _vp]),
+    "qkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype, _fn.argtypes = _res, _args
+
+
+def exported_symbols():
+    return sorted(_SIGS)
+
+
+def qkv_status_string(code: int) -> str:
+    return lib.qkv_status_string(int(code)).decode()
+
+
+def _check(fn: str, rc: int):
+    if rc != QKV_OK:
+        raise QkvError(fn, rc)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+_U16 = (torch.bfloat16, torch.float16, torch.int16, torch.uint16)
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, dtypes=None, numel=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name}: has {t.numel()} elements, needs {numel}")
+    return t.data_ptr()
+
+
+def qkv_yarn_auto_factor(max_context: int, orig_max_pos: int = 262144) -> float:
+    return lib.qkv_yarn_auto_factor(int(max_context), int(orig_max_pos))
+
+
+def qkv_yarn_rope_table(params: YarnParams, pos_start: int, n_pos: int, cos_out: torch.Tensor,
+                        sin_out: torch.Tensor, stream=None):
+    n = n_pos * (params.rot_dim // 2)
+    _check("qkv_yarn_rope_table", lib.qkv_yarn_rope_table(
+        ctypes.byref(params), int(pos_start), int(n_pos), _ptr(cos_out, "cos_out", (torch.float32,), n),
+        _ptr(sin_out, "sin_out", (torch.float32,), n), _stream(stream)))
+
+
+def qkv_rope_apply(x_in, x_out, positions, cos_tab, sin_tab, table_pos_start: int, rot_dim: int,
+                   device_status=None, stream=None):
+    """x_in/x_out bf16 [n_tok][n_heads][head_dim] (x_out may be x_in)."""
+    n_tok, n_heads, head_dim = x_in.shape
+    if tuple(x_out.shape) != (n_tok, n_heads, head_dim):
+        raise ValueError("x_out shape")
+    half = rot_dim // 2
+    _check("qkv_rope_apply", lib.qkv_rope_apply(
+        _ptr(x_in, "x_in", _U16), _ptr(x_out, "x_out", _U16), _ptr(positions, "positions", (torch.int64,), n_tok),
+        n_tok, n_heads, head_dim, rot_dim, _ptr(cos_tab, "cos_tab", (torch.float32,)),
+        _ptr(sin_tab, "sin_tab", (torch.float32,)), int(table_pos_start), cos_tab.numel() // half,
+        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+
+
+def qkv_kv_write_f4(k, v, slot_mapping, k_data, k_scale, v_data, v_scale, device_status=None, stream=None):
+    """k/v bf16 [n_tok][kv_heads][head_dim]; cache tensors shaped
+    [num_pages][kv_heads][block_size][head_dim/2 | head_dim/32]."""
+    n_tok, kv_heads, head_dim = k.shape
+    num_pages, kvh2, block_size, half_bytes = k_data.shape
+    if kvh2 != kv_heads or half_bytes != head_dim // 2 or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("cache/input shapes disagree")
+    _check("qkv_kv_write_f4", lib.qkv_kv_write_f4(
+        _ptr(k, "k", _U16), _ptr(v, "v", _U16), _ptr(slot_mapping, "slot_mapping", (torch.int64,), n_tok), n_tok,
+        _ptr(k_data, "k_data", (torch.uint8,)), _ptr(k_scale, "k_scale", _U16), _ptr(v_data, "v_data", (torch.uint8,)),
+        _ptr(v_scale, "v_scale", _U16), kv_heads, head_dim, block_size, num_pages,
+        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+
+
+def qkv_paged_decode_auto_splits(kv_heads: int, block_size: int) -> int:
+    return lib.qkv_paged_decode_auto_splits(int(kv_heads), int(block_size))
+
+
+def qkv_paged_decode_workspace_bytes(n_seq: int, q_heads: int, head_dim: int, max_splits: int) -> int:
+    return lib.qkv_paged_decode_workspace_bytes(int(n_seq), int(q_heads), int(head_dim), int(max_splits))
+
+
+def _cache_args(k_data, k_scale, v_data, v_scale):
+    return (_ptr(k_data, "k_data", (torch.uint8,)), _ptr(k_scale, "k_scale", _U16),
+            _ptr(v_data, "v_data", (torch.uint8,)), _ptr(v_scale, "v_scale", _U16))
+
+
+def qkv_paged_decode_split_f4(o_parts, lse2_parts, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens,
+                              kv_heads: int, softmax_scale: float = 0.0, num_splits: int = 0,
+                              device_status=None, stream=None):
+    """o_parts float [max_splits][n_seq*q_heads][head_dim], lse2_parts float
+    [max_splits][n_seq*q_heads]."""
+    n_seq, q_heads, head_dim = q.shape
+    max_splits = o_parts.shape[0]
+    num_pages, _, block_size, _ = k_data.shape
+    _check("qkv_paged_decode_split_f4", lib.qkv_paged_decode_split_f4(
+        _ptr(o_parts, "o_parts", (torch.float32,), max_splits * n_seq * q_heads * head_dim),
+        _ptr(lse2_parts, "lse2_parts", (torch.float32,), max_splits * n_seq * q_heads), max_splits,
+        _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),
+        _ptr(page_table, "page_table", (torch.int32,)), _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq), n_seq,
+        q_heads, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, float(softmax_scale),
+        int(num_splits), _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+
+
+def qkv_lse_merge(o_parts, lse2_parts, out, lse2_out=None, stream=None):
+    """o_parts float [n_parts][rows][head_dim] -> out bf16 [rows][head_dim]."""
+    n_parts, rows, head_dim = o_parts.shape
+    _check("qkv_lse_merge", lib.qkv_lse_merge(
+        _ptr(o_parts, "o_parts", (torch.float32,)), _ptr(lse2_parts, "lse2_parts", (torch.float32,), n_parts * rows),
+        n_parts, rows, head_dim, _ptr(out, "out", _U16, rows * head_dim),
+        _ptr(lse2_out, "lse2_out", (torch.float32,), rows), _stream(stream)))
+
+
+def qkv_paged_decode_attn_f4(out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, kv_heads: int,
+                             workspace, max_splits: int, lse2_out=None, softmax_scale: float = 0.0,
+                             num_splits: int = 0, device_status=None, stream=None):
+    """out bf16 [n_seq][q_heads][head_dim]; workspace a uint8 CUDA tensor of
+    at least qkv_paged_decode_workspace_bytes(...) bytes."""
+    n_seq, q_heads, head_dim = q.shape
+    num_pages, _, block_size, _ = k_data.shape
+    _check("qkv_paged_decode_attn_f4", lib.qkv_paged_decode_attn_f4(
+        _ptr(out, "out", _U16, n_seq * q_heads * head_dim), _ptr(lse2_out, "lse2_out", (torch.float32,)),
+        _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),
+        _ptr(page_table, "page_table", (torch.int32,)), _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq), n_seq,
+        q_heads, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, float(softmax_scale),
+        int(num_splits), int(max_splits), _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))

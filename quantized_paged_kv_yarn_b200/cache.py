@@ -1,0 +1,69 @@
+"""Device memory plumbing around the C ABI: the paged F4 cache of one layer
+and a decode-attention helper that owns its workspace. PyTorch supplies the
+memory and streams; every computation is a library call."""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+from . import _abi
+
+
+@dataclasses.dataclass
+class PagedF4Cache:
+    """One layer's F4 cache: data u8 [num_pages][kv_heads][block][head_dim/2]
+    and fp16 scales [num_pages][kv_heads][block][head_dim/32], for K and V."""
+
+    k_data: torch.Tensor
+    k_scale: torch.Tensor
+    v_data: torch.Tensor
+    v_scale: torch.Tensor
+
+    @classmethod
+    def allocate(cls, num_pages: int, kv_heads: int, block_size: int, head_dim: int, device="cuda"):
+        d = lambda: torch.zeros((num_pages, kv_heads, block_size, head_dim // 2), dtype=torch.uint8, device=device)
+        s = lambda: torch.zeros((num_pages, kv_heads, block_size, head_dim // 32), dtype=torch.float16,
+                                device=device)
+        return cls(d(), s(), d(), s())
+
+    @property
+    def num_pages(self) -> int:
+        return self.k_data.shape[0]
+
+    @property
+    def kv_heads(self) -> int:
+        return self.k_data.shape[1]
+
+    @property
+    def block_size(self) -> int:
+        return self.k_data.shape[2]
+
+    @property
+    def head_dim(self) -> int:
+        return self.k_data.shape[3] * 2
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.k_data, self.k_scale, self.v_data, self.v_scale))
+
+    def write(self, k, v, slot_mapping, device_status=None, stream=None):
+        _abi.qkv_kv_write_f4(k, v, slot_mapping, self.k_data, self.k_scale, self.v_data, self.v_scale,
+                             device_status=device_status, stream=stream)
+
+
+class DecodeAttention:
+    """Split pass + log2-sum-exp merge with a workspace sized once."""
+
+    def __init__(self, n_seq: int, q_heads: int, kv_heads: int, head_dim: int, block_size: int,
+                 max_splits: int = 0, device="cuda"):
+        self.kv_heads = kv_heads
+        self.max_splits = max_splits or max(1, _abi.qkv_paged_decode_auto_splits(kv_heads, block_size))
+        nbytes = _abi.qkv_paged_decode_workspace_bytes(n_seq, q_heads, head_dim, self.max_splits)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+    def __call__(self, out, q, cache: PagedF4Cache, page_table, seq_lens, lse2_out=None, softmax_scale=0.0,
+                 num_splits=0, device_status=None, stream=None):
+        _abi.qkv_paged_decode_attn_f4(out, q, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale,
+                                      page_table, seq_lens, self.kv_heads, self.workspace, self.max_splits,
+                                      lse2_out=lse2_out, softmax_scale=softmax_scale, num_splits=num_splits,
+                                      device_status=device_status, stream=stream)

@@ -36,3 +36,41 @@ def dense_dequant(cache, page_table, seq, n_tok, block_size):
         sc = s[pages, :, off, :].view(np.float16).astype(np.float64)   # [n_tok][Hkv][D/32]
         return (codes - 8) * np.repeat(sc, 32, axis=-1)
     return deq(kd, ks), deq(vd, vs)
+
+
+# ---------------------------------------------------------------------------
+# device-side helpers for the GPU parity tests
+
+def to_dev(a, device="cuda"):
+    """numpy -> torch CUDA tensor; uint16 (bf16/fp16 bits) travel as int16."""
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).to(device)
+
+
+def to_host(t, dtype=None):
+    a = t.detach().cpu().numpy()
+    if dtype is not None:
+        a = a.view(dtype)
+    return a
+
+
+def bf16_ulp(x):
+    """Spacing of bf16 numbers at |x| (float64 in, float64 out)."""
+    ax = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(ax, 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+# The attention tolerance: 2e-3 on top of the bf16 rounding of the output
+# (half a bf16 ulp of the exact value).
+ATOL_ATTN = 2e-3
+
+
+def attn_within(gpu_bf16_bits, ref_f64, atol=ATOL_ATTN):
+    g = workloads.bf16_bits_to_f32(gpu_bf16_bits).astype(np.float64)
+    err = np.abs(g - ref_f64)
+    bound = atol + 0.5 * bf16_ulp(ref_f64)
+    return err, bound

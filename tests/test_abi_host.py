@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/qkv.h declares, and rejects invalid arguments before
+launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT, read_golden
+
+HEADER = os.path.join(ROOT, "include", "qkv.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^QKV_API\s+[\w\s\*]+?\b(qkv_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def qkv():
+    from quantized_paged_kv_yarn_b200 import build as b
+    b.build()
+    import quantized_paged_kv_yarn_b200 as q
+    return q
+
+
+def test_exports_every_declared_symbol(qkv):
+    declared = _declared()
+    assert len(declared) >= 10
+    lib = ctypes.CDLL(qkv.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(qkv.exported_symbols()) == declared
+
+
+def test_auto_factor_rule_printed_examples(qkv):
+    _, rows = read_golden("yarn_auto_factor.txt")
+    for ctx, want in rows:
+        got = qkv.qkv_yarn_auto_factor(int(ctx), 262144)
+        assert got == float(want), (ctx, got, want)
+
+
+def test_status_strings(qkv):
+    assert qkv.qkv_status_string(0) == "ok"
+    assert "invalid" in qkv.qkv_status_string(1)
+    assert "unsupported" in qkv.qkv_status_string(2)
+    assert qkv.qkv_status_string(99) == "unknown status"
+
+
+def test_workspace_bytes(qkv):
+    n = qkv.qkv_paged_decode_workspace_bytes(3, 16, 256, 74)
+    rows = 3 * 16 * 74
+    assert n == ((rows * 256 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    assert qkv.qkv_paged_decode_workspace_bytes(-1, 16, 256, 4) == 0
+
+
+FAKE = ctypes.c_void_p(4096)  # never dereferenced: validation fails first
+NUL = None
+
+
+def test_invalid_arguments_rejected_before_launch(qkv):
+    L = qkv.lib
+    # rope table: odd rot_dim, factor < 1, null outputs
+    p = qkv.YarnParams.make(rot_dim=63)
+    assert L.qkv_yarn_rope_table(ctypes.byref(p), 0, 4, FAKE, FAKE, NUL) == 1
+    p = qkv.YarnParams.make(factor=0.5)
+    assert L.qkv_yarn_rope_table(ctypes.byref(p), 0, 4, FAKE, FAKE, NUL) == 1
+    p = qkv.YarnParams.make()
+    assert L.qkv_yarn_rope_table(ctypes.byref(p), 0, 4, NUL, FAKE, NUL) == 1
+    assert L.qkv_yarn_rope_table(ctypes.byref(p), 0, 0, FAKE, FAKE, NUL) == 0   # nothing to do
+    # rope apply: rot > head_dim, overlapping distinct buffers, empty
+    assert L.qkv_rope_apply(FAKE, FAKE, FAKE, 1, 1, 64, 128, FAKE, FAKE, 0, 10, NUL, NUL) == 1
+    assert L.qkv_rope_apply(ctypes.c_void_p(4096), ctypes.c_void_p(4098), FAKE, 1, 1, 64, 64, FAKE, FAKE, 0, 10,
+                            NUL, NUL) == 1
+    assert L.qkv_rope_apply(FAKE, FAKE, FAKE, 0, 16, 256, 64, FAKE, FAKE, 0, 10, NUL, NUL) == 0
+    # kv write: head_dim not a multiple of 32, misaligned input, null cache
+    assert L.qkv_kv_write_f4(FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, 4, 48, 64, 8, NUL, NUL) == 1
+    assert L.qkv_kv_write_f4(ctypes.c_void_p(4098), FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, 4, 256, 64, 8, NUL,
+                             NUL) == 1
+    assert L.qkv_kv_write_f4(FAKE, FAKE, FAKE, 1, NUL, FAKE, FAKE, FAKE, 4, 256, 64, 8, NUL, NUL) == 1
+    assert L.qkv_kv_write_f4(FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, 4, 256, 64, 8, NUL, NUL) == 0
+    # split pass: unsupported head_dim / group / block, bad group divisibility, null
+    args = lambda hq, hkv, d, blk, ms=4: (FAKE, FAKE, ms, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, hq, hkv, d,
+                                          blk, 16, 64, ctypes.c_float(0.0), 0, NUL, NUL)
+    assert L.qkv_paged_decode_split_f4(*args(16, 4, 128, 64)) == 2
+    assert L.qkv_paged_decode_split_f4(*args(12, 4, 256, 64)) == 2     # group of 3
+    assert L.qkv_paged_decode_split_f4(*args(16, 4, 256, 128)) == 2    # block 128
+    assert L.qkv_paged_decode_split_f4(*args(16, 3, 256, 64)) == 1     # 16 % 3
+    assert L.qkv_paged_decode_split_f4(*args(16, 4, 256, 64, 0)) == 1  # max_splits 0
+    a = list(args(16, 4, 256, 64)); a[3] = NUL
+    assert L.qkv_paged_decode_split_f4(*a) == 1
+    a = list(args(16, 4, 256, 64)); a[4] = ctypes.c_void_p(4100)       # cache not 16-byte aligned
+    assert L.qkv_paged_decode_split_f4(*a) == 1
+    # merge: bad head_dim, no parts, empty rows
+    assert L.qkv_lse_merge(FAKE, FAKE, 4, 8, 30, FAKE, NUL, NUL) == 1
+    assert L.qkv_lse_merge(FAKE, FAKE, 0, 8, 256, FAKE, NUL, NUL) == 1
+    assert L.qkv_lse_merge(FAKE, FAKE, 4, 0, 256, FAKE, NUL, NUL) == 0
+    # one-call attention: workspace too small or misaligned
+    wa = lambda ws, nb: (FAKE, NUL, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 16, 4, 256, 64, 16, 64,
+                         ctypes.c_float(0.0), 0, 4, ws, nb, NUL, NUL)
+    need = qkv.qkv_paged_decode_workspace_bytes(1, 16, 256, 4)
+    assert L.qkv_paged_decode_attn_f4(*wa(FAKE, need - 1)) == 1
+    assert L.qkv_paged_decode_attn_f4(*wa(ctypes.c_void_p(4096 + 16), need)) == 1
