@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="host-time budget of the CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="run fewer layers than the workload has (a smaller case for profiler captures)")
     return ap.parse_args()
 
 
@@ -342,6 +344,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device(f"cuda:{local_rank}")
     torch.cuda.set_device(dev)
     w = workloads.BY_NAME[args.workload]
+    if args.layers:
+        w = dataclass_replace(w, n_layers=args.layers)
     b = Bench(w, dev, seed_offset=rank)
 
     def barrier():

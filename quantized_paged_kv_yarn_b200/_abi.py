@@ -36,7 +36,7 @@ class YarnParams(ctypes.Structure):
 
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built; run `python -m quantized_paged_kv_yarn_b200.build`")
+    raise ImportError(f"{LIB_PATH} is not built; run `python quantized_paged_kv_yarn_b200/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -193,3 +193,4 @@ def qkv_paged_decode_attn_f4(out, q, k_data, k_scale, v_data, v_scale, page_tabl
         q_heads, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, float(softmax_scale),
         int(num_splits), int(max_splits), _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+

@@ -1,6 +1,6 @@
 """Build the C-ABI CUDA library libqkv.so in-tree for sm_100a.
 
-    python -m quantized_paged_kv_yarn_b200.build [--force]
+    python quantized_paged_kv_yarn_b200/build.py [--force]
 
 Each .cu under csrc/ compiles to an object in _build/ (parallel), then nvcc
 links them into quantized_paged_kv_yarn_b200/libqkv.so with the static CUDA

@@ -19,8 +19,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def qkv():
-    from quantized_paged_kv_yarn_b200 import build as b
-    b.build()
+    import __graft_entry__
+    __graft_entry__._build_module().build()
     import quantized_paged_kv_yarn_b200 as q
     return q
 
