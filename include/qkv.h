@@ -219,6 +219,39 @@ QKV_API int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint1
                              void* workspace, size_t workspace_bytes, int32_t* device_status,
                              qkv_stream_t stream);
 
+/* Size of the partials array compiled into the library for
+ * qkv_paged_decode_attn_f4_static (8 MiB per GPU that loads the library). */
+#define QKV_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* Decode attention (a4 + a5) without caller-provided scratch. The paper has
+ * no counterpart to this call; it exists for callers that cannot call
+ * cudaMalloc: plugins inside a host engine that owns all device memory, and
+ * runtimes that forbid allocation after start-up (cudaMalloc can
+ * synchronise the device and fragments a pre-planned budget).
+ * Same arguments and results as qkv_paged_decode_attn_f4, minus the
+ * workspace: the partials live in a QKV_STATIC_SCRATCH_BYTES array compiled
+ * into the library. The call allocates nothing. Splits per sequence: num_splits
+ * when > 0, else qkv_paged_decode_auto_splits(kv_heads, block_size).
+ *   - EINVAL when qkv_paged_decode_workspace_bytes(n_seq, q_heads, head_dim,
+ *     splits) exceeds QKV_STATIC_SCRATCH_BYTES (for 16 query heads of
+ *     dimension 256 and 74 splits: up to 6 sequences).
+ *   - The first call on a device resolves the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents (nothing in it needs to start at zero). Calls whose
+ *     kernels overlap on the GPU -- on different streams, or from different
+ *     host threads -- race on it: order them on one stream. */
+QKV_API int qkv_paged_decode_attn_f4_static(uint16_t* out, float* lse2_out, const uint16_t* q,
+                                            const uint8_t* k_data, const uint16_t* k_scale,
+                                            const uint8_t* v_data, const uint16_t* v_scale,
+                                            const int32_t* page_table, const int32_t* seq_lens,
+                                            int32_t n_seq, int32_t q_heads, int32_t kv_heads,
+                                            int32_t head_dim, int32_t block_size,
+                                            int32_t max_pages_per_seq, int64_t num_pages,
+                                            float softmax_scale, int32_t num_splits,
+                                            int32_t* device_status, qkv_stream_t stream);
+
 /* Static text for a return code. */
 QKV_API const char* qkv_status_string(int status);
 

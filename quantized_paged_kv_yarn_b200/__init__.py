@@ -22,6 +22,8 @@ from ._abi import (  # noqa: F401
     qkv_kv_write_f4,
     qkv_lse_merge,
     qkv_paged_decode_attn_f4,
+    qkv_paged_decode_attn_f4_static,
+    STATIC_SCRATCH_BYTES,
     qkv_paged_decode_auto_splits,
     qkv_paged_decode_split_f4,
     qkv_paged_decode_workspace_bytes,

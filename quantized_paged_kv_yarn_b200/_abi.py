@@ -55,6 +55,8 @@ _SIGS = {
     "qkv_lse_merge": (ctypes.c_int, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "qkv_paged_decode_attn_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                                                 _i32, _i32, _i32, _i64, _f32, _i32, _i32, _vp, _sz, _vp, _vp]),
+    "qkv_paged_decode_attn_f4_static": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+                                                       _i32, _i32, _i32, _i32, _i64, _f32, _i32, _vp, _vp]),
     "qkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -194,3 +196,22 @@ def qkv_paged_decode_attn_f4(out, q, k_data, k_scale, v_data, v_scale, page_tabl
         int(num_splits), int(max_splits), _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
 
+
+STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def qkv_paged_decode_attn_f4_static(out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, kv_heads: int,
+                                    lse2_out=None, softmax_scale: float = 0.0, num_splits: int = 0,
+                                    device_status=None, stream=None):
+    """Decode attention with the partials in the library's own device array
+    (no workspace argument, no allocation). For callers that cannot allocate
+    device memory; see include/qkv.h for the size limit and the rule that
+    overlapping calls race on the shared array."""
+    n_seq, q_heads, head_dim = q.shape
+    num_pages, _, block_size, _ = k_data.shape
+    _check("qkv_paged_decode_attn_f4_static", lib.qkv_paged_decode_attn_f4_static(
+        _ptr(out, "out", _U16, n_seq * q_heads * head_dim), _ptr(lse2_out, "lse2_out", (torch.float32,)),
+        _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),
+        _ptr(page_table, "page_table", (torch.int32,)), _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq), n_seq,
+        q_heads, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, float(softmax_scale),
+        int(num_splits), _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
