@@ -9,25 +9,27 @@
 // folded by log2-sum-exp); ignis docs "context-and-speculation" (64-token KV
 // pages; lanes sharing one pool).
 //
-// Design (B200, sm_100a). The step is HBM-bound: 288 bytes of packed K/V and
+// Design (B200, sm_100a). The step streams bytes: 288 bytes of packed K/V and
 // scales per token and KV head feed 2 x 4 x 256 multiply-adds. One CTA owns
 // (split, sequence, KV head) so the G query heads of the group share every
-// dequantised page.
-//  * Thread 0 streams 64-token stages (one 64-token page, or 2/4
-//    pages of 32/16 tokens) into a 4-deep shared-memory ring: the packed
-//    K and V rows by 2-D TMA with the 128-byte swizzle, their fp16 scales by
-//    1-D bulk copies, all completing on one mbarrier per stage.
-//  * Four consumer warps take 16 tokens of each stage. ldmatrix delivers the
-//    packed nibbles already in mma-fragment order (plain for K, transposed
-//    for V); a LOP3 + fp16 FMA pair turns 2 nibbles into 2 exact fp16 values
+// dequantised page; 4 warps, 2 CTAs per SM.
+//  * 64-token stages (one 64-token page, or 2/4 pages of 32/16 tokens) fill a
+//    4-slot shared-memory ring: the packed K and V rows by 2-D TMA with the
+//    128-byte swizzle, their fp16 scales by 1-D bulk copies, all completing
+//    on one mbarrier per slot. Warp w issues the stages R = w (mod 4), so the
+//    issue work is spread evenly and no warp paces the others; a slot is
+//    refilled by its warp once all four warps have released it.
+//  * Each warp takes 16 tokens of a stage. ldmatrix delivers the packed
+//    nibbles already in mma-fragment order (plain for K, transposed for V);
+//    a LOP3 + fp16 add/FMA pair turns 2 nibbles into 2 exact fp16 values
 //    (n - 8) in registers. Q K^T and P V run on the tensor cores as
-//    m16n8k16 fp16 MMAs with fp32 accumulation; the per-cell K scale is
-//    applied to each cell's fp32 partial sum and the per-cell V scale is
-//    folded into the probabilities (the B operand) of that cell.
+//    m16n8k16 fp16 MMAs with fp32 accumulation; each 32-dim cell of K is its
+//    own MMA chain scaled by that token's cell scale in fp32, and the per-cell
+//    V scale is folded into the probabilities (the B operand) of that cell.
 //  * The running max / sum live in registers (base-2 exponent); the four
 //    warps are combined through shared memory and the CTA writes one fp32
 //    partial and its lse2 per query head. The merge kernel folds splits.
-// Dequantised tiles never touch shared memory: staging bf16 tiles for
+// Dequantised tiles never touch shared memory: staging fp16 tiles for
 // tcgen05 would need ~4x the shared-memory bandwidth of the packed bytes.
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -85,6 +87,13 @@ using namespace split;
 
 __device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 
+// 2^x for the softmax weights (hardware approximation, subnormal results flushed to 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float half_at(const uint4& v, int i) {
   const uint32_t w = (i < 2) ? v.x : (i < 4) ? v.y : (i < 6) ? v.z : v.w;
   const unsigned short b = (i & 1) ? (unsigned short)(w >> 16) : (unsigned short)(w & 0xffff);
@@ -103,18 +112,37 @@ __device__ __forceinline__ int seq_len_of(const Params& p, int s, int block, boo
 }
 
 // Split plan. Fixed: min(num_splits, max_splits) splits per sequence.
-// Automatic: pages are cut into pieces of P = ceil(total pages / target),
-// so the grid holds about `target` busy CTAs per KV head whatever the mix of
+// Automatic: pages are cut into pieces of about total pages / target, so the
+// grid holds at most `target` busy CTAs per KV head whatever the mix of
 // lengths. Split i of a sequence with n pages covers [i*n/S, (i+1)*n/S).
+__device__ long long splits_for(const Params& p, int block, long long P) {
+  long long total = 0;
+  for (int s = 0; s < p.n_seq; ++s) total += ((seq_len_of(p, s, block, false) + block - 1) / block + P - 1) / P;
+  return total;
+}
+
 __device__ void plan(const Params& p, int seq, int split, int block, int& S, int& pg0, int& pg1, int& L) {
   L = seq_len_of(p, seq, block, split == 0 && blockIdx.z == 0);
   const int n = (L + block - 1) / block;
   if (p.num_splits > 0) {
     S = min(p.num_splits, p.max_splits);
   } else {
-    long long T = 0;
-    for (int s = 0; s < p.n_seq; ++s) T += (seq_len_of(p, s, block, false) + block - 1) / block;
-    const long long P = max(1LL, (T + p.target - 1) / p.target);
+    // Pieces of P pages with sum_s ceil(n_s / P) <= target, so the busy CTAs
+    // fit the resident slots in one wave.
+    long long T = 0, nmax = 1;
+    for (int s = 0; s < p.n_seq; ++s) {
+      const long long ns = (seq_len_of(p, s, block, false) + block - 1) / block;
+      T += ns;
+      nmax = max(nmax, ns);
+    }
+    long long P;
+    if (p.target <= p.n_seq) {
+      P = nmax;  // one split per sequence
+    } else {
+      P = max(1LL, (T + p.target - 1) / p.target);
+      for (int k = 0; k < 4 && splits_for(p, block, P) > p.target; ++k) ++P;
+      if (splits_for(p, block, P) > p.target) P = max(P, (T + p.target - p.n_seq - 1) / (p.target - p.n_seq));
+    }
     S = (int)min((long long)p.max_splits, max(1LL, (n + P - 1) / P));
   }
   pg0 = (int)((long long)split * n / S);
@@ -160,30 +188,58 @@ __global__ void __launch_bounds__(THREADS, 2)
   __syncthreads();
 
   // ------------------------------------------------------------ copy issue
-  // Thread 0 fills the ring: stage `it` holds tokens t_begin + 64 it ...
-  // +63, i.e. 64 / BLOCK pages, each as four copies (K rows, V rows by TMA
-  // with the 128-byte swizzle; K and V scales by bulk copy). It refills a
-  // slot once all warps have released it, NS stages ahead of the compute.
+  // Stage `it` holds tokens t_begin + 64 it ... +63, i.e. 64 / BLOCK pages,
+  // each as four copies (K rows, V rows by TMA with the 128-byte swizzle; K
+  // and V scales by bulk copy). Warp w issues the stages R = w (mod 4), so
+  // the issue work is spread evenly over the warps; lane j of warp w keeps
+  // the page ids of the j-th next of those stages (32 per refresh, the next
+  // 32 prefetched), so no copy waits on a page-table load.
+  static_assert(NS == CWARPS, "one ring slot per issuing warp");
   const uint64_t pol = policy_evict_first();
-  const int32_t* pt = p.page_table + (size_t)seq * p.max_pages;
+  const int32_t* pt = p.page_table + (size_t)seq * p.max_pages + pg0;
+  const int npg = pg1 - pg0;
   volatile int* abort_flag = &sm.abort_flag;
-  auto issue = [&](int it) {
-    const int st = it % NS;
-    const int tok0 = t_begin + it * STAGE_TOK;
+  int id_cur[PPS], id_nxt[PPS];
+  int id_base = 0;  // index (R / CWARPS) of the stage held by lane 0
+  auto load_ids = [&](int base, int (&dst)[PPS]) {
+    const int R = (base + lane) * CWARPS + warp;
+#pragma unroll
+    for (int k = 0; k < PPS; ++k) {
+      const int pi = R * PPS + k;
+      dst[k] = pi < npg ? pt[pi] : -1;
+    }
+  };
+  load_ids(0, id_cur);
+  load_ids(32, id_nxt);
+  // called by all lanes of warp R % CWARPS, with R increasing
+  auto issue = [&](int R) {
+    const int st = R % NS;
+    const int j = R / CWARPS;
+    if (j >= id_base + 32) {
+      id_base += 32;
+#pragma unroll
+      for (int k = 0; k < PPS; ++k) id_cur[k] = id_nxt[k];
+      load_ids(id_base + 32, id_nxt);
+    }
     int phys[PPS];
+#pragma unroll
+    for (int k = 0; k < PPS; ++k) phys[k] = __shfl_sync(FULL_MASK, id_cur[k], (j - id_base) & 31);
+    if (lane != 0) return;
+    const int tok0 = t_begin + R * STAGE_TOK;
     unsigned long long mask = 0;
     uint32_t bytes = 0;
 #pragma unroll
     for (int k = 0; k < PPS; ++k) {
-      phys[k] = -1;
       const int tk = tok0 + k * BLOCK;
-      if (tk >= t_end) continue;
-      const int pid = pt[tk / BLOCK];
-      if (pid < 0 || (int64_t)pid >= p.num_pages) {
-        flag(p.status, QKV_DEV_BAD_PAGE);
+      if (tk >= t_end) {
+        phys[k] = -1;
         continue;
       }
-      phys[k] = pid;
+      if (phys[k] < 0 || (int64_t)phys[k] >= p.num_pages) {
+        flag(p.status, QKV_DEV_BAD_PAGE);
+        phys[k] = -1;
+        continue;
+      }
       const int nv = min(BLOCK, t_end - tk);
       const unsigned long long bits = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
       mask |= bits << (k * BLOCK);
@@ -202,10 +258,9 @@ __global__ void __launch_bounds__(THREADS, 2)
       bulk_load(&sm.vs[st][k * BLOCK * SROW_BYTES], p.v_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
                 &sm.full[st], pol);
     }
-    sm.issued = it + 1;
+    atomicMax(&sm.issued, R + 1);
   };
-  if (threadIdx.x == 0)
-    for (int it = 0; it < min(NS, n_it); ++it) issue(it);
+  if (warp < n_it) issue(warp);  // stages 0 .. NS-1, one per warp
 
   // ------------------------------------------------------------ consumers
   const int g = lane >> 2, t = lane & 3;
@@ -265,21 +320,14 @@ __global__ void __launch_bounds__(THREADS, 2)
   const uint32_t ld_row = (uint32_t)((((lane >> 3) & 1) * 8 + (lane & 7)) * ROW_BYTES);
   const int sw = lane & 7;  // 128B swizzle: chunk index ^= row index mod 8
   const int co = lane >> 4;
+  uint32_t ld_off[CELLS / 2];  // this lane's ldmatrix address offset for cell pair cp
+#pragma unroll
+  for (int cp = 0; cp < CELLS / 2; ++cp) ld_off[cp] = ld_row + ((uint32_t)((2 * cp + co) ^ sw) << 4);
   float(*tr)[TR_STRIDE] = sm.tr[warp];
   bool aborted = false;
 
   for (int it = 0; it < n_it; ++it) {
     const int st = it % NS;
-    // refill the slot released by the previous iteration
-    if (threadIdx.x == 0 && it >= 1 && it - 1 + NS < n_it && !*abort_flag) {
-      const int pv = it - 1;
-      if (mbar_wait_bounded(&sm.empty[pv % NS], (pv / NS) & 1)) {
-        issue(pv + NS);
-      } else {
-        flag(p.status, QKV_DEV_TIMEOUT);
-        *abort_flag = 1;
-      }
-    }
     if (!aborted && !mbar_wait_bounded(&sm.full[st], (it / NS) & 1)) {
       flag(p.status, QKV_DEV_TIMEOUT);
       *abort_flag = 1;
@@ -294,33 +342,60 @@ __global__ void __launch_bounds__(THREADS, 2)
       const uint8_t* vsb = &sm.vs[st][warp * 16 * SROW_BYTES];
       const bool partial = tmask != 0xffffu;
 
-      // ---- scores: S[token][head] for tokens g, g+8 and heads 2t, 2t+1
+      // All shared-memory reads of the tile up front: packed K and V in
+      // fragment order, the K scales of tokens g and g+8, the V scales of
+      // tokens 2t, 2t+1, 2t+8, 2t+9.
+      uint32_t kw[CELLS / 2][4], vw[CELLS / 2][4];
+#pragma unroll
+      for (int cp = 0; cp < CELLS / 2; ++cp) ldsm_x4(kbase + ld_off[cp], kw[cp]);
       const uint4 skA = lds128(ksb + g * SROW_BYTES);
       const uint4 skB = lds128(ksb + (g + 8) * SROW_BYTES);
+#pragma unroll
+      for (int cp = 0; cp < CELLS / 2; ++cp) ldsm_x4_trans(vbase + ld_off[cp], vw[cp]);
+      uint4 sv0 = lds128(vsb + (2 * t) * SROW_BYTES);
+      uint4 sv1 = lds128(vsb + (2 * t + 1) * SROW_BYTES);
+      uint4 sv2 = lds128(vsb + (2 * t + 8) * SROW_BYTES);
+      uint4 sv3 = lds128(vsb + (2 * t + 9) * SROW_BYTES);
+
+      // ---- scores S[token][head] for tokens g, g+8 and heads 2t, 2t+1:
+      //      eight independent per-cell MMA chains, then the cell scales
+      float d[CELLS][4];
+#pragma unroll
+      for (int c = 0; c < CELLS; ++c) {
+        const uint32_t wa = kw[c >> 1][2 * (c & 1)], wb = kw[c >> 1][2 * (c & 1) + 1];
+        d[c][0] = d[c][1] = d[c][2] = d[c][3] = 0.f;
+        mma_f16(d[c], nib_lo(wa), nib_lo(wb), nib_hi(wa), nib_hi(wb), qb[c][0][0], qb[c][0][1]);
+      }
+#pragma unroll
+      for (int c = 0; c < CELLS; ++c) {
+        const uint32_t wa = kw[c >> 1][2 * (c & 1)] >> 8, wb = kw[c >> 1][2 * (c & 1) + 1] >> 8;
+        mma_f16(d[c], nib_lo(wa), nib_lo(wb), nib_hi(wa), nib_hi(wb), qb[c][1][0], qb[c][1][1]);
+      }
       float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+      const uint32_t ka[4] = {skA.x, skA.y, skA.z, skA.w}, kb[4] = {skB.x, skB.y, skB.z, skB.w};
 #pragma unroll
-      for (int cp = 0; cp < CELLS / 2; ++cp) {
-        uint32_t r[4];
-        ldsm_x4(kbase + ld_row + ((uint32_t)((2 * cp + co) ^ sw) << 4), r);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int c = 2 * cp + hh;
-          const uint32_t wa = r[2 * hh], wb = r[2 * hh + 1];
-          float d[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_f16(d, nib_lo(wa), nib_lo(wb), nib_hi(wa), nib_hi(wb), qb[c][0][0], qb[c][0][1]);
-          mma_f16(d, nib_lo(wa >> 8), nib_lo(wb >> 8), nib_hi(wa >> 8), nib_hi(wb >> 8), qb[c][1][0],
-                  qb[c][1][1]);
-          const float sa = half_at(skA, c), sb = half_at(skB, c);
-          s0 = fmaf(sa, d[0], s0);
-          s1 = fmaf(sa, d[1], s1);
-          s2 = fmaf(sb, d[2], s2);
-          s3 = fmaf(sb, d[3], s3);
-        }
+      for (int c2 = 0; c2 < CELLS / 2; ++c2) {
+        const float2 fa = __half22float2(u32_as_h2(ka[c2])), fb = __half22float2(u32_as_h2(kb[c2]));
+        s0 = fmaf(fa.x, d[2 * c2][0], s0);
+        s1 = fmaf(fa.x, d[2 * c2][1], s1);
+        s2 = fmaf(fb.x, d[2 * c2][2], s2);
+        s3 = fmaf(fb.x, d[2 * c2][3], s3);
+        s0 = fmaf(fa.y, d[2 * c2 + 1][0], s0);
+        s1 = fmaf(fa.y, d[2 * c2 + 1][1], s1);
+        s2 = fmaf(fb.y, d[2 * c2 + 1][2], s2);
+        s3 = fmaf(fb.y, d[2 * c2 + 1][3], s3);
       }
       s0 *= score_scale; s1 *= score_scale; s2 *= score_scale; s3 *= score_scale;
       if (partial) {
         if (!((tmask >> g) & 1u)) s0 = s1 = -INFINITY;
         if (!((tmask >> (g + 8)) & 1u)) s2 = s3 = -INFINITY;
+        // the weights of absent tokens are exactly 0; make their scales 0 too
+        // (a stale slot may hold any bit pattern)
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        if (!((tmask >> (2 * t)) & 1u)) sv0 = z4;
+        if (!((tmask >> (2 * t + 1)) & 1u)) sv1 = z4;
+        if (!((tmask >> (2 * t + 8)) & 1u)) sv2 = z4;
+        if (!((tmask >> (2 * t + 9)) & 1u)) sv3 = z4;
       }
 
       // ---- transpose to the PV B-operand layout: head g, tokens 2t, 2t+1, 2t+8, 2t+9
@@ -349,10 +424,10 @@ __global__ void __launch_bounds__(THREADS, 2)
       mt = fmaxf(mt, __shfl_xor_sync(FULL_MASK, mt, 2));
       const float m_new = fmaxf(m_run, mt);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = (g < G) ? exp2f(m_run - m_use) : 1.f;
+      const float alpha = (g < G) ? ex2(m_run - m_use) : 1.f;
       float pr[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) pr[i] = exp2f(sc[i] - m_use);
+      for (int i = 0; i < 4; ++i) pr[i] = ex2(sc[i] - m_use);
       l_run = l_run * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
       m_run = m_new;
       const float al0 = __shfl_sync(FULL_MASK, alpha, (8 * t) & 31);
@@ -367,40 +442,38 @@ __global__ void __launch_bounds__(THREADS, 2)
           }
       }
 
-      // ---- P V with the V scale folded into P per cell
-      const uint4 sv0 = lds128(vsb + (2 * t) * SROW_BYTES);
-      const uint4 sv1 = lds128(vsb + (2 * t + 1) * SROW_BYTES);
-      const uint4 sv2 = lds128(vsb + (2 * t + 8) * SROW_BYTES);
-      const uint4 sv3 = lds128(vsb + (2 * t + 9) * SROW_BYTES);
-      bool vok[4] = {true, true, true, true};
-      if (partial) {
-        vok[0] = (tmask >> (2 * t)) & 1u;
-        vok[1] = (tmask >> (2 * t + 1)) & 1u;
-        vok[2] = (tmask >> (2 * t + 8)) & 1u;
-        vok[3] = (tmask >> (2 * t + 9)) & 1u;
-      }
+      // ---- P V with the V scale folded into P per cell (packed fp16)
+      const __half2 p01 = __floats2half2_rn(pr[0], pr[1]), p23 = __floats2half2_rn(pr[2], pr[3]);
+      const uint32_t s0w[4] = {sv0.x, sv0.y, sv0.z, sv0.w}, s1w[4] = {sv1.x, sv1.y, sv1.z, sv1.w};
+      const uint32_t s2w[4] = {sv2.x, sv2.y, sv2.z, sv2.w}, s3w[4] = {sv3.x, sv3.y, sv3.z, sv3.w};
 #pragma unroll
-      for (int cp = 0; cp < CELLS / 2; ++cp) {
-        uint32_t z[4];
-        ldsm_x4_trans(vbase + ld_row + ((uint32_t)((2 * cp + co) ^ sw) << 4), z);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int c = 2 * cp + hh;
-          float b0 = pr[0] * half_at(sv0, c), b1 = pr[1] * half_at(sv1, c);
-          float b2 = pr[2] * half_at(sv2, c), b3 = pr[3] * half_at(sv3, c);
-          if (partial) {
-            b0 = vok[0] ? b0 : 0.f; b1 = vok[1] ? b1 : 0.f;
-            b2 = vok[2] ? b2 : 0.f; b3 = vok[3] ? b3 : 0.f;
-          }
-          const uint32_t b01 = pack_f16x2(b0, b1), b23 = pack_f16x2(b2, b3);
-          const uint32_t za = z[2 * hh], zb = z[2 * hh + 1];
-          mma_f16(acc[c][0], nib_lo(za), nib_hi(za), nib_lo(zb), nib_hi(zb), b01, b23);
-          mma_f16(acc[c][1], nib_lo(za >> 8), nib_hi(za >> 8), nib_lo(zb >> 8), nib_hi(zb >> 8), b01, b23);
-        }
+      for (int c = 0; c < CELLS; ++c) {
+        const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;
+        const uint32_t b01 = h2_as_u32(__hmul2(p01, u32_as_h2(__byte_perm(s0w[c >> 1], s1w[c >> 1], sel))));
+        const uint32_t b23 = h2_as_u32(__hmul2(p23, u32_as_h2(__byte_perm(s2w[c >> 1], s3w[c >> 1], sel))));
+        const uint32_t za = vw[c >> 1][2 * (c & 1)], zb = vw[c >> 1][2 * (c & 1) + 1];
+        mma_f16(acc[c][0], nib_lo(za), nib_hi(za), nib_lo(zb), nib_hi(zb), b01, b23);
+        mma_f16(acc[c][1], nib_lo(za >> 8), nib_hi(za >> 8), nib_lo(zb >> 8), nib_hi(zb >> 8), b01, b23);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[st]);
+    // The slot of the previous iteration (all warps have normally left it by
+    // now) is refilled NS - 1 iterations ahead of its use, by its own warp.
+    if (it >= 1 && it - 1 + NS < n_it && ((it - 1) % CWARPS) == warp) {
+      const int pv = it - 1;
+      int go = 1;
+      if (lane == 0) {
+        if (*abort_flag) {
+          go = 0;
+        } else if (!mbar_wait_bounded(&sm.empty[pv % NS], (pv / NS) & 1)) {
+          flag(p.status, QKV_DEV_TIMEOUT);
+          *abort_flag = 1;
+          go = 0;
+        }
+      }
+      if (__shfl_sync(FULL_MASK, go, 0)) issue(pv + NS);
+    }
   }
 
   // ------------------------------------------------------------ combine the 4 warps
