@@ -12,20 +12,24 @@
 // Design (B200, sm_100a). The step streams bytes: 288 bytes of packed K/V and
 // scales per token and KV head feed 2 x 4 x 256 multiply-adds. One CTA owns
 // (split, sequence, KV head) so the G query heads of the group share every
-// dequantised page; 4 warps, 2 CTAs per SM.
+// dequantised page; 4 warps, 3 CTAs per SM (168 registers per thread).
 //  * 64-token stages (one 64-token page, or 2/4 pages of 32/16 tokens) fill a
-//    4-slot shared-memory ring: the packed K and V rows by 2-D TMA with the
+//    3-slot shared-memory ring: the packed K and V rows by 2-D TMA with the
 //    128-byte swizzle, their fp16 scales by 1-D bulk copies, all completing
 //    on one mbarrier per slot. Warp w issues the stages R = w (mod 4), so the
 //    issue work is spread evenly and no warp paces the others; a slot is
-//    refilled by its warp once all four warps have released it.
+//    refilled once all four warps have released it.
 //  * Each warp takes 16 tokens of a stage. ldmatrix delivers the packed
-//    nibbles already in mma-fragment order (plain for K, transposed for V);
-//    a LOP3 + fp16 add/FMA pair turns 2 nibbles into 2 exact fp16 values
-//    (n - 8) in registers. Q K^T and P V run on the tensor cores as
-//    m16n8k16 fp16 MMAs with fp32 accumulation; each 32-dim cell of K is its
-//    own MMA chain scaled by that token's cell scale in fp32, and the per-cell
-//    V scale is folded into the probabilities (the B operand) of that cell.
+//    nibbles already in mma-fragment order (plain for K, transposed for V).
+//    Q K^T and P V run on the tensor cores as m16n8k16 fp16 MMAs with fp32
+//    accumulation. K nibbles enter the MMA raw, as fp16 subnormals
+//    (n * 2^-24 in bits 0-3, n * 2^-20 in bits 4-7, both exact): q carries
+//    16 q on the low-nibble positions and each 32-dim cell's MMA chain starts
+//    from -8 * 2^-20 * sum(q over the cell), so the chain yields
+//    2^-20 * sum((n - 8) q) with one AND per fp16 pair. V nibbles become
+//    exact fp16 (n - 8) with a LOP3 + one fp16 add/FMA per pair. Each cell
+//    chain of K is scaled by that token's cell scale in fp32; the per-cell V
+//    scale is folded into the probabilities (the B operand) of that cell.
 //  * The running max / sum live in registers (base-2 exponent); the four
 //    warps are combined through shared memory and the CTA writes one fp32
 //    partial and its lse2 per query head. The merge kernel folds splits.
@@ -47,7 +51,7 @@ constexpr int CELLS = D / 32;        // 8 cells of 32 values per row
 constexpr int ROW_BYTES = D / 2;     // 128 packed bytes per token
 constexpr int SROW_BYTES = CELLS * 2;  // 16 bytes of fp16 scales per token
 constexpr int STAGE_TOK = 64;
-constexpr int NS = 4;                // ring depth
+constexpr int NS = 3;                // ring depth
 constexpr int CWARPS = 4;            // warps; each takes 16 tokens of a stage
 constexpr int THREADS = CWARPS * 32;
 constexpr int TR_STRIDE = 20;        // padded row of the score transpose buffer
@@ -58,6 +62,8 @@ struct __align__(1024) Smem {
   uint8_t ks[NS][STAGE_TOK * SROW_BYTES];
   uint8_t vs[NS][STAGE_TOK * SROW_BYTES];
   float tr[CWARPS][8][TR_STRIDE];
+  uint4 qfrag[CELLS][32];  // per cell and lane: the 4 fp16x2 B registers of both k-steps
+  float qbias[CELLS][8];   // per cell and head: -8 * 2^-20 * sum of the cell's q (accumulator start)
   float wm[CWARPS][8];
   float wl[CWARPS][8];
   unsigned long long mask[NS];
@@ -86,6 +92,16 @@ struct Params {
 using namespace split;
 
 __device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+
+// D = A * B + C with C given separately (no copy of C into D first).
+__device__ __forceinline__ void mma_f16_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1, float c0, float c1, float c2, float c3) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %11, %12, %13};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2), "f"(c3));
+}
 
 // 2^x for the softmax weights (hardware approximation, subnormal results flushed to 0)
 __device__ __forceinline__ float ex2(float x) {
@@ -150,7 +166,7 @@ __device__ void plan(const Params& p, int seq, int split, int block, int& S, int
 }
 
 template <int BLOCK, int G>
-__global__ void __launch_bounds__(THREADS, 2)
+__global__ void __launch_bounds__(THREADS, 3)
     paged_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                               const Params p) {
   static_assert(STAGE_TOK % BLOCK == 0, "pages must tile a stage");
@@ -194,7 +210,6 @@ __global__ void __launch_bounds__(THREADS, 2)
   // the issue work is spread evenly over the warps; lane j of warp w keeps
   // the page ids of the j-th next of those stages (32 per refresh, the next
   // 32 prefetched), so no copy waits on a page-table load.
-  static_assert(NS == CWARPS, "one ring slot per issuing warp");
   const uint64_t pol = policy_evict_first();
   const int32_t* pt = p.page_table + (size_t)seq * p.max_pages + pg0;
   const int npg = pg1 - pg0;
@@ -260,7 +275,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
     atomicMax(&sm.issued, R + 1);
   };
-  if (warp < n_it) issue(warp);  // stages 0 .. NS-1, one per warp
+  if (warp < min(NS, n_it)) issue(warp);  // stages 0 .. NS-1
 
   // ------------------------------------------------------------ consumers
   const int g = lane >> 2, t = lane & 3;
@@ -269,7 +284,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   // 32-dim cell the k index is permuted to match the nibble order the
   // unpack produces: k-step ks, fragment register r, half i <-> dim
   // 8t + 2ks + r + 4i.
-  uint32_t qb[CELLS][2][2];
+  uint32_t qb[CELLS][2][2];  // built here, kept in shared memory
   float score_scale = p.score_scale;
   {
     float qf[CELLS][8];
@@ -293,18 +308,34 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(FULL_MASK, qmax, o));
-    // Keep q inside the fp16 range with an exact power-of-two prescale.
+    // q enters the MMA as fp16 with an exact power-of-two prescale: the
+    // low-nibble positions take 16 q (their K values are n * 2^-24), the
+    // high-nibble positions q (K values n * 2^-20), so every product is
+    // 2^-20 * n * q; 16 * max|q| stays below 2^15.
     const int qexp = (int)((__float_as_uint(qmax) >> 23) & 0xff) - 127;
-    const int shift = qexp >= 15 ? qexp - 14 : 0;
-    score_scale = ldexpf(score_scale, shift);
+    const int shift = qexp >= 11 ? qexp - 10 : 0;
+    score_scale = ldexpf(score_scale, shift + 20);
 #pragma unroll
-    for (int c = 0; c < CELLS; ++c)
+    for (int c = 0; c < CELLS; ++c) {
+      float qs = 0.f;  // sum of this lane's 8 dims of the cell, as the MMA sees them
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
-        qb[c][ks][0] = pack_f16x2(ldexpf(qf[c][2 * ks], -shift), ldexpf(qf[c][2 * ks + 4], -shift));
-        qb[c][ks][1] = pack_f16x2(ldexpf(qf[c][2 * ks + 1], -shift), ldexpf(qf[c][2 * ks + 5], -shift));
+        const __half2 lo = __floats2half2_rn(ldexpf(qf[c][2 * ks], -shift), ldexpf(qf[c][2 * ks + 4], -shift));
+        const __half2 hi = __floats2half2_rn(ldexpf(qf[c][2 * ks + 1], -shift), ldexpf(qf[c][2 * ks + 5], -shift));
+        const float2 lf = __half22float2(lo), hf = __half22float2(hi);
+        qs += (lf.x + lf.y) + (hf.x + hf.y);
+        qb[c][ks][0] = h2_as_u32(__hmul2(lo, u32_as_h2(0x4C004C00u)));  // x16, exact
+        qb[c][ks][1] = h2_as_u32(hi);
       }
+      qs += __shfl_xor_sync(FULL_MASK, qs, 1);
+      qs += __shfl_xor_sync(FULL_MASK, qs, 2);
+      if (warp == 0 && t == 0) sm.qbias[c][g] = (g < G) ? -8.0f * ldexpf(qs, -20) : 0.f;
+    }
+    if (warp == 0)
+#pragma unroll
+      for (int c = 0; c < CELLS; ++c) sm.qfrag[c][lane] = make_uint4(qb[c][0][0], qb[c][0][1], qb[c][1][0], qb[c][1][1]);
   }
+  __syncthreads();
 
   float acc[CELLS][2][4];
 #pragma unroll
@@ -342,49 +373,45 @@ __global__ void __launch_bounds__(THREADS, 2)
       const uint8_t* vsb = &sm.vs[st][warp * 16 * SROW_BYTES];
       const bool partial = tmask != 0xffffu;
 
-      // All shared-memory reads of the tile up front: packed K and V in
-      // fragment order, the K scales of tokens g and g+8, the V scales of
-      // tokens 2t, 2t+1, 2t+8, 2t+9.
-      uint32_t kw[CELLS / 2][4], vw[CELLS / 2][4];
-#pragma unroll
-      for (int cp = 0; cp < CELLS / 2; ++cp) ldsm_x4(kbase + ld_off[cp], kw[cp]);
       const uint4 skA = lds128(ksb + g * SROW_BYTES);
       const uint4 skB = lds128(ksb + (g + 8) * SROW_BYTES);
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+      const uint32_t ka[4] = {skA.x, skA.y, skA.z, skA.w}, kb[4] = {skB.x, skB.y, skB.z, skB.w};
 #pragma unroll
-      for (int cp = 0; cp < CELLS / 2; ++cp) ldsm_x4_trans(vbase + ld_off[cp], vw[cp]);
+      for (int grp = 0; grp < 2; ++grp) {
+        uint32_t kw[2][4];
+        ldsm_x4(kbase + ld_off[2 * grp], kw[0]);
+        ldsm_x4(kbase + ld_off[2 * grp + 1], kw[1]);
+        float d[4][4];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = 4 * grp + cc;
+          const uint4 qv = sm.qfrag[c][lane];
+          const float2 bias = *reinterpret_cast<const float2*>(&sm.qbias[c][2 * t]);
+          const uint32_t wa = kw[cc >> 1][2 * (cc & 1)], wb = kw[cc >> 1][2 * (cc & 1) + 1];
+          const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
+          // raw nibbles as fp16 subnormals: n * 2^-24 (bits 0-3), n * 2^-20 (bits 4-7)
+          mma_f16_c(d[cc], wa & 0x000F000Fu, wb & 0x000F000Fu, wa & 0x00F000F0u, wb & 0x00F000F0u, qv.x, qv.y,
+                    bias.x, bias.y, bias.x, bias.y);
+          mma_f16(d[cc], wa8 & 0x000F000Fu, wb8 & 0x000F000Fu, wa8 & 0x00F000F0u, wb8 & 0x00F000F0u, qv.z, qv.w);
+        }
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const float2 fa = __half22float2(u32_as_h2(ka[2 * grp + c2])), fb = __half22float2(u32_as_h2(kb[2 * grp + c2]));
+          s0 = fmaf(fa.x, d[2 * c2][0], s0);
+          s1 = fmaf(fa.x, d[2 * c2][1], s1);
+          s2 = fmaf(fb.x, d[2 * c2][2], s2);
+          s3 = fmaf(fb.x, d[2 * c2][3], s3);
+          s0 = fmaf(fa.y, d[2 * c2 + 1][0], s0);
+          s1 = fmaf(fa.y, d[2 * c2 + 1][1], s1);
+          s2 = fmaf(fb.y, d[2 * c2 + 1][2], s2);
+          s3 = fmaf(fb.y, d[2 * c2 + 1][3], s3);
+        }
+      }
       uint4 sv0 = lds128(vsb + (2 * t) * SROW_BYTES);
       uint4 sv1 = lds128(vsb + (2 * t + 1) * SROW_BYTES);
       uint4 sv2 = lds128(vsb + (2 * t + 8) * SROW_BYTES);
       uint4 sv3 = lds128(vsb + (2 * t + 9) * SROW_BYTES);
-
-      // ---- scores S[token][head] for tokens g, g+8 and heads 2t, 2t+1:
-      //      eight independent per-cell MMA chains, then the cell scales
-      float d[CELLS][4];
-#pragma unroll
-      for (int c = 0; c < CELLS; ++c) {
-        const uint32_t wa = kw[c >> 1][2 * (c & 1)], wb = kw[c >> 1][2 * (c & 1) + 1];
-        d[c][0] = d[c][1] = d[c][2] = d[c][3] = 0.f;
-        mma_f16(d[c], nib_lo(wa), nib_lo(wb), nib_hi(wa), nib_hi(wb), qb[c][0][0], qb[c][0][1]);
-      }
-#pragma unroll
-      for (int c = 0; c < CELLS; ++c) {
-        const uint32_t wa = kw[c >> 1][2 * (c & 1)] >> 8, wb = kw[c >> 1][2 * (c & 1) + 1] >> 8;
-        mma_f16(d[c], nib_lo(wa), nib_lo(wb), nib_hi(wa), nib_hi(wb), qb[c][1][0], qb[c][1][1]);
-      }
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-      const uint32_t ka[4] = {skA.x, skA.y, skA.z, skA.w}, kb[4] = {skB.x, skB.y, skB.z, skB.w};
-#pragma unroll
-      for (int c2 = 0; c2 < CELLS / 2; ++c2) {
-        const float2 fa = __half22float2(u32_as_h2(ka[c2])), fb = __half22float2(u32_as_h2(kb[c2]));
-        s0 = fmaf(fa.x, d[2 * c2][0], s0);
-        s1 = fmaf(fa.x, d[2 * c2][1], s1);
-        s2 = fmaf(fb.x, d[2 * c2][2], s2);
-        s3 = fmaf(fb.x, d[2 * c2][3], s3);
-        s0 = fmaf(fa.y, d[2 * c2 + 1][0], s0);
-        s1 = fmaf(fa.y, d[2 * c2 + 1][1], s1);
-        s2 = fmaf(fb.y, d[2 * c2 + 1][2], s2);
-        s3 = fmaf(fb.y, d[2 * c2 + 1][3], s3);
-      }
       s0 *= score_scale; s1 *= score_scale; s2 *= score_scale; s3 *= score_scale;
       if (partial) {
         if (!((tmask >> g) & 1u)) s0 = s1 = -INFINITY;
@@ -446,12 +473,14 @@ __global__ void __launch_bounds__(THREADS, 2)
       const __half2 p01 = __floats2half2_rn(pr[0], pr[1]), p23 = __floats2half2_rn(pr[2], pr[3]);
       const uint32_t s0w[4] = {sv0.x, sv0.y, sv0.z, sv0.w}, s1w[4] = {sv1.x, sv1.y, sv1.z, sv1.w};
       const uint32_t s2w[4] = {sv2.x, sv2.y, sv2.z, sv2.w}, s3w[4] = {sv3.x, sv3.y, sv3.z, sv3.w};
+      uint32_t vw[2][4];
 #pragma unroll
       for (int c = 0; c < CELLS; ++c) {
+        if ((c & 1) == 0) ldsm_x4_trans(vbase + ld_off[c >> 1], vw[(c >> 1) & 1]);
         const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;
         const uint32_t b01 = h2_as_u32(__hmul2(p01, u32_as_h2(__byte_perm(s0w[c >> 1], s1w[c >> 1], sel))));
         const uint32_t b23 = h2_as_u32(__hmul2(p23, u32_as_h2(__byte_perm(s2w[c >> 1], s3w[c >> 1], sel))));
-        const uint32_t za = vw[c >> 1][2 * (c & 1)], zb = vw[c >> 1][2 * (c & 1) + 1];
+        const uint32_t za = vw[(c >> 1) & 1][2 * (c & 1)], zb = vw[(c >> 1) & 1][2 * (c & 1) + 1];
         mma_f16(acc[c][0], nib_lo(za), nib_hi(za), nib_lo(zb), nib_hi(zb), b01, b23);
         mma_f16(acc[c][1], nib_lo(za >> 8), nib_hi(za >> 8), nib_lo(zb >> 8), nib_hi(zb >> 8), b01, b23);
       }
@@ -460,7 +489,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     if (lane == 0) mbar_arrive(&sm.empty[st]);
     // The slot of the previous iteration (all warps have normally left it by
     // now) is refilled NS - 1 iterations ahead of its use, by its own warp.
-    if (it >= 1 && it - 1 + NS < n_it && ((it - 1) % CWARPS) == warp) {
+    if (it >= 1 && it - 1 + NS < n_it && ((it - 1 + NS) % CWARPS) == warp) {
       const int pv = it - 1;
       int go = 1;
       if (lane == 0) {
