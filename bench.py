@@ -3,9 +3,9 @@
 
 One step = one decode token for every sequence of the workload through all
 its full-attention layers: the YaRN table row(s) of the step positions, the
-partial rotary of q and of the new key, the F4 write of the new K/V, the
-split-KV paged attention and the log2-sum-exp merge -- 1 + 5 x layers kernel
-launches, replayed from a CUDA graph.
+partial rotary of q and of the new key with the F4 write of the new K/V (one
+launch), the split-KV paged attention and the log2-sum-exp merge -- 1 + 3 x
+layers kernel launches, replayed from a CUDA graph.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -264,7 +264,7 @@ class Bench:
         self.params = qkv.YarnParams.make(**workloads.yarn_spec(w))
         self.att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
-        self.launches_per_step = 1 + 5 * self.L
+        self.launches_per_step = 1 + 3 * self.L
         # host side of the end-to-end measurement (pinned)
         self.h_q = [t.cpu().pin_memory() for t in self.q_raw]
         self.h_kn = [t.cpu().pin_memory() for t in self.kn_raw]
@@ -276,13 +276,14 @@ class Bench:
         q, w = self.qkv, self.w
         q.qkv_yarn_rope_table(self.params, self.pos0, self.n_rows, self.cos, self.sin)
         for l in range(self.L):
-            q.qkv_rope_apply(self.q_raw[l], self.q_rot[l], self.positions, self.cos, self.sin, self.pos0, w.rot_dim,
-                             device_status=self.status)
-            q.qkv_rope_apply(self.kn_raw[l], self.k_rot[l], self.positions, self.cos, self.sin, self.pos0,
-                             w.rot_dim, device_status=self.status)
-            self.caches[l].write(self.k_rot[l], self.vn[l], self.step_slots, device_status=self.status)
-            self.att(self.out[l], self.q_rot[l], self.caches[l], self.page_table, self.seq_lens,
-                     num_splits=w.num_splits, device_status=self.status)
+            c = self.caches[l]
+            # a2 + a3 in one launch: rotary of q and of the new k, F4 write of k and v
+            q.qkv_rope_kv_write_f4(self.q_raw[l], self.q_rot[l], self.kn_raw[l], self.vn[l], self.positions,
+                                   self.step_slots, self.cos, self.sin, self.pos0, w.rot_dim, c.k_data, c.k_scale,
+                                   c.v_data, c.v_scale, device_status=self.status)
+            # a4 + a5
+            self.att(self.out[l], self.q_rot[l], c, self.page_table, self.seq_lens, num_splits=w.num_splits,
+                     device_status=self.status)
 
     def e2e_step(self):
         """Host buffers in, the step, the result back to the host."""

@@ -149,6 +149,25 @@ QKV_API int qkv_kv_write_f4(const uint16_t* k, const uint16_t* v, const int64_t*
                     uint16_t* v_scale, int32_t kv_heads, int32_t head_dim, int32_t block_size,
                     int64_t num_pages, int32_t* device_status, qkv_stream_t stream);
 
+/* a2 + a3 in one launch: the partial rotary of q and of the new k, and the
+ * F4 write of the rotated k and of v through the slot mapping.
+ *   q_in, q_out  bf16 [n_tok][q_heads][head_dim] (q_out may equal q_in).
+ *   k_in, v_in   bf16 [n_tok][kv_heads][head_dim], not modified.
+ *   k_out        bf16 [n_tok][kv_heads][head_dim] receives the rotated k, or
+ *                NULL.
+ * Other arguments as in qkv_rope_apply and qkv_kv_write_f4; the results are
+ * bit-identical to qkv_rope_apply on q and on k followed by
+ * qkv_kv_write_f4 of the rotated k and v. rot_dim must be a multiple of 16.
+ * n_tok == 0 returns QKV_OK without touching any pointer. */
+QKV_API int qkv_rope_kv_write_f4(const uint16_t* q_in, uint16_t* q_out, const uint16_t* k_in,
+                                 const uint16_t* v_in, uint16_t* k_out, const int64_t* positions,
+                                 const int64_t* slot_mapping, int32_t n_tok, int32_t q_heads,
+                                 int32_t kv_heads, int32_t head_dim, int32_t rot_dim,
+                                 const float* cos_tab, const float* sin_tab, int64_t table_pos_start,
+                                 int64_t table_len, uint8_t* k_data, uint16_t* k_scale,
+                                 uint8_t* v_data, uint16_t* v_scale, int32_t block_size,
+                                 int64_t num_pages, int32_t* device_status, qkv_stream_t stream);
+
 /* Number of splits per sequence the automatic plan aims for on the current
  * device (resident split blocks / kv_heads); a workspace sized with this as
  * max_splits never limits the automatic plan. Host-only; returns 0 when no

@@ -28,6 +28,7 @@ from ._abi import (  # noqa: F401
     qkv_paged_decode_split_f4,
     qkv_paged_decode_workspace_bytes,
     qkv_rope_apply,
+    qkv_rope_kv_write_f4,
     qkv_status_string,
     qkv_yarn_auto_factor,
     qkv_yarn_rope_table,

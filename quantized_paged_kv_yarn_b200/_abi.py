@@ -48,6 +48,8 @@ _SIGS = {
     "qkv_rope_apply": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i64, _i64, _vp, _vp]),
     "qkv_kv_write_f4": (ctypes.c_int, [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i64, _vp,
                                        _vp]),
+    "qkv_rope_kv_write_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp,
+                                            _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i64, _vp, _vp]),
     "qkv_paged_decode_auto_splits": (_i32, [_i32, _i32]),
     "qkv_paged_decode_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "qkv_paged_decode_split_f4": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
@@ -139,6 +141,23 @@ def qkv_kv_write_f4(k, v, slot_mapping, k_data, k_scale, v_data, v_scale, device
         _ptr(k, "k", _U16), _ptr(v, "v", _U16), _ptr(slot_mapping, "slot_mapping", (torch.int64,), n_tok), n_tok,
         _ptr(k_data, "k_data", (torch.uint8,)), _ptr(k_scale, "k_scale", _U16), _ptr(v_data, "v_data", (torch.uint8,)),
         _ptr(v_scale, "v_scale", _U16), kv_heads, head_dim, block_size, num_pages,
+        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+
+
+def qkv_rope_kv_write_f4(q_in, q_out, k_in, v_in, positions, slot_mapping, cos_tab, sin_tab, table_pos_start: int,
+                         rot_dim: int, k_data, k_scale, v_data, v_scale, k_out=None, device_status=None, stream=None):
+    """Rotary of q (q_in -> q_out) and of k, and the F4 write of the rotated k
+    and of v, in one launch."""
+    n_tok, q_heads, head_dim = q_in.shape
+    _, kv_heads, _ = k_in.shape
+    num_pages, _, block_size, _ = k_data.shape
+    half = rot_dim // 2
+    _check("qkv_rope_kv_write_f4", lib.qkv_rope_kv_write_f4(
+        _ptr(q_in, "q_in", _U16), _ptr(q_out, "q_out", _U16), _ptr(k_in, "k_in", _U16), _ptr(v_in, "v_in", _U16),
+        _ptr(k_out, "k_out", _U16), _ptr(positions, "positions", (torch.int64,), n_tok),
+        _ptr(slot_mapping, "slot_mapping", (torch.int64,), n_tok), n_tok, q_heads, kv_heads, head_dim, rot_dim,
+        _ptr(cos_tab, "cos_tab", (torch.float32,)), _ptr(sin_tab, "sin_tab", (torch.float32,)), int(table_pos_start),
+        cos_tab.numel() // half, *_cache_args(k_data, k_scale, v_data, v_scale), block_size, num_pages,
         _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
 
 

@@ -26,8 +26,42 @@ constexpr unsigned FULL_MASK = 0xffffffffu;
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;
 
+// Programmatic dependent launch. Every kernel of the library is launched
+// with programmatic stream serialization allowed, so it may be scheduled
+// while its predecessor in the stream is still running. It calls
+// pdl_wait() before touching any global memory -- the wait returns once the
+// predecessor grid has completed and its writes are visible -- and then
+// pdl_release() so its own successor may be scheduled early in turn.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch with programmatic stream serialization allowed (see pdl_wait).
+inline cudaError_t launch_pdl(const void* kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              void** args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, kernel, args);
+}
+
 __device__ __forceinline__ void flag(int32_t* status, int32_t bits) {
   if (status) atomicOr(status, bits);
+}
+
+// NEOX rotation of the pair (x0, x1) = (x_j, x_{j+rot/2}) by (c, s), float,
+// with a fixed rounding order so every kernel produces the same bits.
+__device__ __forceinline__ float rot_first(float x0, float x1, float c, float s) {
+  return __fmaf_rn(x0, c, -__fmul_rn(x1, s));
+}
+__device__ __forceinline__ float rot_second(float x0, float x1, float c, float s) {
+  return __fmaf_rn(x1, c, __fmul_rn(x0, s));
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

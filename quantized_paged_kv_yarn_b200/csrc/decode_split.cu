@@ -176,6 +176,8 @@ __global__ void __launch_bounds__(THREADS, 3)
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
+  pdl_wait();
+  pdl_release();
   const int split = blockIdx.x, seq = blockIdx.y, kvh = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows = p.n_seq * p.q_heads;
@@ -742,7 +744,7 @@ extern "C" int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int3
   // covers every slot the merge reads.
   dim3 grid((unsigned)max_splits, (unsigned)n_seq, (unsigned)kv_heads);
   void* args[] = {(void*)&tm_k, (void*)&tm_v, (void*)&p};
-  if (cudaLaunchKernel(fn, grid, dim3(THREADS), args, SMEM_BYTES, stream) != cudaSuccess) {
+  if (launch_pdl(fn, grid, dim3(THREADS), SMEM_BYTES, stream, args) != cudaSuccess) {
     (void)cudaGetLastError();
     return QKV_ECUDA;
   }

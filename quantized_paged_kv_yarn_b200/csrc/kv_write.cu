@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(256) kv_write_f4_kernel(
     const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, const int64_t* __restrict__ slots,
     int n_tok, uint8_t* __restrict__ k_data, __half* __restrict__ k_scale, uint8_t* __restrict__ v_data,
     __half* __restrict__ v_scale, int kv_heads, int head_dim, int block, int64_t num_pages, int32_t* status) {
+  pdl_wait();
+  pdl_release();
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (item >= (int64_t)n_tok * kv_heads * 2) return;
@@ -95,9 +97,13 @@ extern "C" int qkv_kv_write_f4(const uint16_t* k, const uint16_t* v, const int64
   if (warps == 0) return QKV_OK;
   const int64_t blocks = (warps + 7) / 8;
   if (blocks > 0x7fffffff) return QKV_EINVAL;
-  kv_write_f4_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
-      k, v, slot_mapping, n_tok, k_data, reinterpret_cast<__half*>(k_scale), v_data,
-      reinterpret_cast<__half*>(v_scale), kv_heads, head_dim, block_size, num_pages, device_status);
-  QKV_LAUNCH_CHECK();
+  __half* ks = reinterpret_cast<__half*>(k_scale);
+  __half* vs = reinterpret_cast<__half*>(v_scale);
+  int nt = n_tok, kvh = kv_heads, hd = head_dim, bs = block_size;
+  void* args[] = {&k, &v, &slot_mapping, &nt, &k_data, &ks, &v_data, &vs, &kvh, &hd, &bs, &num_pages, &device_status};
+  if (launch_pdl((const void*)kv_write_f4_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, args) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QKV_ECUDA;
+  }
   return QKV_OK;
 }

@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* _
                                                                   int n_parts, int rows, int head_dim,
                                                                   __nv_bfloat16* __restrict__ out,
                                                                   float* __restrict__ lse2_out) {
+  pdl_wait();
+  pdl_release();
   __shared__ float red[MERGE_THREADS / 32];
   __shared__ float4 part[MERGE_GROUPS][16];
   const int row = blockIdx.x;
@@ -100,9 +102,13 @@ extern "C" int qkv_lse_merge(const float* o_parts, const float* lse2_parts, int3
     return QKV_EINVAL;
   if (rows == 0) return QKV_OK;
   dim3 grid((unsigned)rows, (unsigned)((head_dim + MERGE_DIMS - 1) / MERGE_DIMS));
-  lse_merge_kernel<<<grid, MERGE_THREADS, 0, stream>>>(o_parts, lse2_parts, n_parts, rows, head_dim,
-                                                       reinterpret_cast<__nv_bfloat16*>(out), lse2_out);
-  QKV_LAUNCH_CHECK();
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+  int np = n_parts, nr = rows, hd = head_dim;
+  void* args[] = {&o_parts, &lse2_parts, &np, &nr, &hd, &o, &lse2_out};
+  if (launch_pdl((const void*)lse_merge_kernel, grid, dim3(MERGE_THREADS), 0, stream, args) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QKV_ECUDA;
+  }
   return QKV_OK;
 }
 

@@ -42,6 +42,8 @@ __device__ double yarn_theta(const YarnDev& p, int j, double* mscale) {
 __global__ void __launch_bounds__(256) yarn_table_kernel(YarnDev p, int64_t pos_start, int64_t n_pos,
                                                          float* __restrict__ cos_out,
                                                          float* __restrict__ sin_out) {
+  pdl_wait();
+  pdl_release();
   __shared__ double s_theta[MAX_ROT_HALF];
   __shared__ double s_ms;
   const int half = p.rot / 2;
@@ -73,6 +75,8 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const __nv_bfloat16* x_
                                                          const float* __restrict__ sin_tab,
                                                          int64_t tab_start, int64_t tab_len,
                                                          int32_t* status) {
+  pdl_wait();
+  pdl_release();
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (item >= (int64_t)n_tok * n_heads) return;
@@ -87,8 +91,8 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const __nv_bfloat16* x_
     const float x0 = __bfloat162float(xi[j]), x1 = __bfloat162float(xi[j + half]);
     if (ok) {
       const float c = cos_tab[row * half + j], s = sin_tab[row * half + j];
-      xo[j] = __float2bfloat16_rn(x0 * c - x1 * s);
-      xo[j + half] = __float2bfloat16_rn(x1 * c + x0 * s);
+      xo[j] = __float2bfloat16_rn(rot_first(x0, x1, c, s));
+      xo[j + half] = __float2bfloat16_rn(rot_second(x0, x1, c, s));
     } else {
       xo[j] = xi[j];
       xo[j + half] = xi[j + half];
@@ -122,8 +126,11 @@ extern "C" int qkv_yarn_rope_table(const qkv_yarn_params* params, int64_t pos_st
   const int64_t total = n_pos * (q.rot_dim / 2);
   const int64_t blocks = (total + 255) / 256;
   if (blocks > 0x7fffffff) return QKV_EINVAL;
-  yarn_table_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p, pos_start, n_pos, cos_out, sin_out);
-  QKV_LAUNCH_CHECK();
+  void* args[] = {&p, &pos_start, &n_pos, &cos_out, &sin_out};
+  if (launch_pdl((const void*)yarn_table_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, args) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QKV_ECUDA;
+  }
   return QKV_OK;
 }
 
@@ -144,9 +151,14 @@ extern "C" int qkv_rope_apply(const uint16_t* x_in, uint16_t* x_out, const int64
   const int64_t items = (int64_t)n_tok * n_heads;
   if (items == 0) return QKV_OK;
   const int64_t blocks = (items + 7) / 8;
-  rope_apply_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
-      reinterpret_cast<const __nv_bfloat16*>(x_in), reinterpret_cast<__nv_bfloat16*>(x_out), positions,
-      n_tok, n_heads, head_dim, rot_dim, cos_tab, sin_tab, table_pos_start, table_len, device_status);
-  QKV_LAUNCH_CHECK();
+  const __nv_bfloat16* xi = reinterpret_cast<const __nv_bfloat16*>(x_in);
+  __nv_bfloat16* xo = reinterpret_cast<__nv_bfloat16*>(x_out);
+  int nt = n_tok, nh = n_heads, hd = head_dim, rd = rot_dim;
+  void* args[] = {&xi, &xo, &positions, &nt, &nh, &hd, &rd, &cos_tab, &sin_tab, &table_pos_start, &table_len,
+                  &device_status};
+  if (launch_pdl((const void*)rope_apply_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, args) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QKV_ECUDA;
+  }
   return QKV_OK;
 }

@@ -147,3 +147,54 @@ def test_kv_write_exhaustive_bf16(qkv, amax_bits):
     assert st == 0
     for a, b in zip(got, ref):
         assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("inplace", [False, True])
+@pytest.mark.parametrize("rot", [64, 128, 256])
+def test_rope_kv_write_fused_matches_two_calls(qkv, rot, inplace):
+    """The one-launch rotary + F4 write gives the same bits as qkv_rope_apply
+    on q and k followed by qkv_kv_write_f4 (and so the oracle parity of those
+    two calls carries over)."""
+    spec = dict(YARN4, rot_dim=rot)
+    rng = np.random.default_rng(13)
+    n_tok, hq, hkv, d, B, P = 9, 16, 4, 256, 16, 12
+    q = workloads.f32_to_bf16_bits((rng.standard_normal((n_tok, hq, d)) * 2).astype(np.float32))
+    k = workloads.f32_to_bf16_bits((rng.standard_normal((n_tok, hkv, d)) * 3).astype(np.float32))
+    v = workloads.f32_to_bf16_bits(rng.standard_normal((n_tok, hkv, d)).astype(np.float32))
+    pos = np.sort(rng.integers(262144, 1048576, n_tok)).astype(np.int64)
+    slots = rng.permutation(P * B)[:n_tok].astype(np.int64)
+    slots[2] = -1
+    p0 = int(pos.min())
+    c, s = _table(qkv, spec, p0, int(pos.max()) - p0 + 1)
+    # two calls
+    q2 = torch.empty_like(to_dev(q))
+    k2 = torch.empty_like(to_dev(k))
+    qkv.qkv_rope_apply(to_dev(q), q2, to_dev(pos), c, s, p0, rot)
+    qkv.qkv_rope_apply(to_dev(k), k2, to_dev(pos), c, s, p0, rot)
+    ref = qkv.PagedF4Cache.allocate(P, hkv, B, d)
+    ref.write(k2, to_dev(v), to_dev(slots))
+    # one launch
+    qi = to_dev(q)
+    qo = qi if inplace else torch.empty_like(qi)
+    ko = torch.empty_like(to_dev(k))
+    got = qkv.PagedF4Cache.allocate(P, hkv, B, d)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    qkv.qkv_rope_kv_write_f4(qi, qo, to_dev(k), to_dev(v), to_dev(pos), to_dev(slots), c, s, p0, rot, got.k_data,
+                             got.k_scale, got.v_data, got.v_scale, k_out=ko, device_status=st)
+    assert int(st.item()) == 0
+    assert torch.equal(qo, q2) and torch.equal(ko, k2)
+    for a, b in zip((got.k_data, got.k_scale, got.v_data, got.v_scale), (ref.k_data, ref.k_scale, ref.v_data,
+                                                                          ref.v_scale)):
+        assert torch.equal(a, b)
+
+
+def test_rope_kv_write_fused_flags(qkv):
+    k = to_dev(np.full((2, 1, 256), 0x3F80, np.uint16))
+    q = to_dev(np.full((2, 2, 256), 0x3F80, np.uint16))
+    c, s = _table(qkv, YARN4, 100, 10)
+    cache = qkv.PagedF4Cache.allocate(2, 1, 16, 256)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    qkv.qkv_rope_kv_write_f4(q, q, k, k, to_dev(np.array([105, 200], np.int64)), to_dev(np.array([3, 32], np.int64)),
+                             c, s, 100, 64, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale,
+                             device_status=st)
+    assert int(st.item()) == qkv.DEV_BAD_POSITION | qkv.DEV_BAD_SLOT
