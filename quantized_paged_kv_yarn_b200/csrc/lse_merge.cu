@@ -6,17 +6,20 @@
 // F4 packed KV cache, ...", section 2.
 //
 // Per row: M = max_i lse2_i, w_i = 2^(lse2_i - M), out = sum_i w_i o_i /
-// sum_i w_i, lse2 = M + log2 sum_i w_i. One CTA per (row, 64-dim chunk):
-// 8 groups of 16 lanes split the parts, each lane carries 4 dims.
+// sum_i w_i, lse2 = M + log2 sum_i w_i.
 #include <math.h>
 
 #include "common.cuh"
 
 namespace qkv {
 
-constexpr int MERGE_THREADS = 128;
-constexpr int MERGE_GROUPS = MERGE_THREADS / 16;
-constexpr int MERGE_DIMS = 64;
+// One CTA per (row, 128-dim chunk). 16 warps split the parts (warp w takes
+// parts w, w + 16, ...); each lane carries 4 dims, so a warp covers the
+// chunk. A thread issues the loads of all its parts before using them.
+constexpr int MERGE_WARPS = 16;
+constexpr int MERGE_THREADS = MERGE_WARPS * 32;
+constexpr int MERGE_DIMS = 128;
+constexpr int MERGE_UNROLL = 8;  // parts per warp in flight
 
 __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* __restrict__ o_parts,
                                                                   const float* __restrict__ lse2_parts,
@@ -25,8 +28,8 @@ __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* _
                                                                   float* __restrict__ lse2_out) {
   pdl_wait();
   pdl_release();
-  __shared__ float red[MERGE_THREADS / 32];
-  __shared__ float4 part[MERGE_GROUPS][16];
+  __shared__ float red[MERGE_WARPS];
+  __shared__ float4 part[MERGE_WARPS][32];
   const int row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -39,7 +42,7 @@ __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* _
   __syncthreads();
   float M = red[0];
 #pragma unroll
-  for (int w = 1; w < MERGE_THREADS / 32; ++w) M = fmaxf(M, red[w]);
+  for (int w = 1; w < MERGE_WARPS; ++w) M = fmaxf(M, red[w]);
   __syncthreads();
   float ws = 0.f;
   if (M != -INFINITY)
@@ -53,38 +56,49 @@ __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* _
   __syncthreads();
   float W = 0.f;
 #pragma unroll
-  for (int w = 0; w < MERGE_THREADS / 32; ++w) W += red[w];
+  for (int w = 0; w < MERGE_WARPS; ++w) W += red[w];
 
-  // weighted sum of this CTA's 64 dims
-  const int grp = tid >> 4, l16 = tid & 15;
-  const int d = blockIdx.y * MERGE_DIMS + 4 * l16;
+  // weighted sum of this CTA's dims, MERGE_UNROLL parts per warp at a time
+  const int d = blockIdx.y * MERGE_DIMS + 4 * lane;
+  const bool dim_ok = d < head_dim;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (M != -INFINITY && d < head_dim)
-    for (int i = grp; i < n_parts; i += MERGE_GROUPS) {
-      const float l = lse2_parts[(size_t)i * rows + row];
-      if (l == -INFINITY) continue;
-      const float w = exp2f(l - M);
-      const float4 x = *reinterpret_cast<const float4*>(o_parts + ((size_t)i * rows + row) * head_dim + d);
-      acc.x = fmaf(w, x.x, acc.x);
-      acc.y = fmaf(w, x.y, acc.y);
-      acc.z = fmaf(w, x.z, acc.z);
-      acc.w = fmaf(w, x.w, acc.w);
-    }
-  part[grp][l16] = acc;
-  __syncthreads();
-  if (grp == 0 && d < head_dim) {
-    float4 s = part[0][l16];
+  if (M != -INFINITY && dim_ok)
+    for (int base = warp; base < n_parts; base += MERGE_WARPS * MERGE_UNROLL) {
+      float lw[MERGE_UNROLL];
+      float4 x[MERGE_UNROLL];
 #pragma unroll
-    for (int g = 1; g < MERGE_GROUPS; ++g) {
-      const float4 x = part[g][l16];
+      for (int u = 0; u < MERGE_UNROLL; ++u) {
+        const int i = base + u * MERGE_WARPS;
+        lw[u] = i < n_parts ? lse2_parts[(size_t)i * rows + row] : -INFINITY;
+      }
+#pragma unroll
+      for (int u = 0; u < MERGE_UNROLL; ++u) {
+        const int i = base + u * MERGE_WARPS;
+        x[u] = (lw[u] != -INFINITY) ? *reinterpret_cast<const float4*>(o_parts + ((size_t)i * rows + row) * head_dim + d)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < MERGE_UNROLL; ++u) {
+        const float w = (lw[u] != -INFINITY) ? exp2f(lw[u] - M) : 0.f;
+        acc.x = fmaf(w, x[u].x, acc.x);
+        acc.y = fmaf(w, x[u].y, acc.y);
+        acc.z = fmaf(w, x[u].z, acc.z);
+        acc.w = fmaf(w, x[u].w, acc.w);
+      }
+    }
+  part[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0 && dim_ok) {
+    float4 s = part[0][lane];
+#pragma unroll
+    for (int w = 1; w < MERGE_WARPS; ++w) {
+      const float4 x = part[w][lane];
       s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
     }
     const float inv = W > 0.f ? 1.f / W : 0.f;
-    __nv_bfloat162 lo = __floats2bfloat162_rn(s.x * inv, s.y * inv);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(s.z * inv, s.w * inv);
     __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + (size_t)row * head_dim + d);
-    dst[0] = lo;
-    dst[1] = hi;
+    dst[0] = __floats2bfloat162_rn(s.x * inv, s.y * inv);
+    dst[1] = __floats2bfloat162_rn(s.z * inv, s.w * inv);
   }
   if (tid == 0 && blockIdx.y == 0 && lse2_out) lse2_out[row] = W > 0.f ? M + log2f(W) : -INFINITY;
 }
