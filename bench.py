@@ -55,6 +55,25 @@ def parse_args():
     return ap.parse_args()
 
 
+# --------------------------------------------------------------------------- ranks
+
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Max of a per-rank value over all ranks (identity when alone)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbps(bytes_per_rank_step: int, ms_per_step_max: float, world: int) -> float:
+    """Weak scaling: every rank moves its own bytes; the job takes the
+    slowest rank's time."""
+    return world * bytes_per_rank_step / (ms_per_step_max * 1e-3) / 1e9
+
+
 # --------------------------------------------------------------------------- peaks / profiles
 
 def hbm_peak():
@@ -355,11 +374,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     # warm the library (tensor maps, occupancy) before any capture
     b.step()
@@ -406,8 +421,8 @@ def run_ours(args, rank, world, local_rank):
         return
     per_layer = w.algorithmic_bytes_per_layer()
     step_bytes = per_layer * w.n_layers
-    value = world * step_bytes / (ms * 1e-3) / 1e9
-    e2e_value = world * step_bytes / (ms_e2e * 1e-3) / 1e9
+    value = whole_job_gbps(step_bytes, ms, world)
+    e2e_value = whole_job_gbps(step_bytes, ms_e2e, world)
     peak, peak_kind = hbm_peak()
     out_bytes = 2 * w.n_seq * w.q_heads * w.head_dim
     split_bytes = per_layer - out_bytes  # the merge writes out
