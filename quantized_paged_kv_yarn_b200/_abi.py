@@ -137,6 +137,8 @@ def qkv_kv_write_f4(k, v, slot_mapping, k_data, k_scale, v_data, v_scale, device
     num_pages, kvh2, block_size, half_bytes = k_data.shape
     if kvh2 != kv_heads or half_bytes != head_dim // 2 or tuple(v.shape) != tuple(k.shape):
         raise ValueError("cache/input shapes disagree")
+    if slot_mapping.numel() != n_tok:
+        raise ValueError(f"slot_mapping has {slot_mapping.numel()} entries for {n_tok} tokens")
     _check("qkv_kv_write_f4", lib.qkv_kv_write_f4(
         _ptr(k, "k", _U16), _ptr(v, "v", _U16), _ptr(slot_mapping, "slot_mapping", (torch.int64,), n_tok), n_tok,
         _ptr(k_data, "k_data", (torch.uint8,)), _ptr(k_scale, "k_scale", _U16), _ptr(v_data, "v_data", (torch.uint8,)),
@@ -152,6 +154,11 @@ def qkv_rope_kv_write_f4(q_in, q_out, k_in, v_in, positions, slot_mapping, cos_t
     _, kv_heads, _ = k_in.shape
     num_pages, _, block_size, _ = k_data.shape
     half = rot_dim // 2
+    if (tuple(q_out.shape) != tuple(q_in.shape) or tuple(k_in.shape) != (n_tok, kv_heads, head_dim)
+            or tuple(v_in.shape) != tuple(k_in.shape) or (k_out is not None and tuple(k_out.shape) != tuple(k_in.shape))):
+        raise ValueError("q/k/v shapes disagree")
+    if slot_mapping.numel() != n_tok or positions.numel() != n_tok:
+        raise ValueError("positions and slot_mapping need one entry per token")
     _check("qkv_rope_kv_write_f4", lib.qkv_rope_kv_write_f4(
         _ptr(q_in, "q_in", _U16), _ptr(q_out, "q_out", _U16), _ptr(k_in, "k_in", _U16), _ptr(v_in, "v_in", _U16),
         _ptr(k_out, "k_out", _U16), _ptr(positions, "positions", (torch.int64,), n_tok),

@@ -1,6 +1,6 @@
 // common.cuh -- device helpers shared by the kernels of the decode hot path
 // (sm_100a): shared-memory addressing, mbarriers with bounded waits, TMA and
-// bulk copies, ldmatrix, warp-level MMA and the nibble -> fp16 unpack.
+// bulk copies, ldmatrix and warp-level MMA.
 #pragma once
 
 #include <cuda.h>
@@ -161,6 +161,10 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
                : "r"(addr));
 }
 
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
 // D += A * B, m16n8k16, fp16 inputs, fp32 accumulate.
 __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                         uint32_t b0, uint32_t b1) {
@@ -171,37 +175,7 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1,
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// ---------------------------------------------------------------- nibble unpack
-//
-// A 32-bit word w holds nibbles n0..n7 (n0 in bits 0-3). With the fp16
-// exponent field of 1024 ORed in, the nibbles at bits 0-3 / 16-19 read as
-// the fp16 pair (1024 + n0, 1024 + n4), and the nibbles at bits 4-7 / 20-23
-// as (1024 + 16 n1, 1024 + 16 n5). One fp16 add or fma then yields the signed
-// values n - 8 exactly.
-
-__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(orv));
-  return r;
-}
-
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
-
-// (n0, n4) - 8 as fp16x2
-__device__ __forceinline__ uint32_t nib_lo(uint32_t w) {
-  const __half2 x = u32_as_h2(lop_and_or(w, 0x000F000Fu, 0x64006400u));
-  return h2_as_u32(__hsub2(x, u32_as_h2(0x64086408u)));  // 1032
-}
-// (n1, n5) - 8 as fp16x2
-__device__ __forceinline__ uint32_t nib_hi(uint32_t w) {
-  const __half2 x = u32_as_h2(lop_and_or(w, 0x00F000F0u, 0x64006400u));
-  // (1024 + 16 n) / 16 - 72 = n - 8
-  return h2_as_u32(__hfma2(x, u32_as_h2(0x2C002C00u), u32_as_h2(0xD480D480u)));
-}
-
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  return h2_as_u32(__floats2half2_rn(lo, hi));
-}
 
 }  // namespace qkv

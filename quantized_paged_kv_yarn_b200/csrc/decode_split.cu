@@ -26,10 +26,12 @@
 //    (n * 2^-24 in bits 0-3, n * 2^-20 in bits 4-7, both exact): q carries
 //    16 q on the low-nibble positions and each 32-dim cell's MMA chain starts
 //    from -8 * 2^-20 * sum(q over the cell), so the chain yields
-//    2^-20 * sum((n - 8) q) with one AND per fp16 pair. V nibbles become
-//    exact fp16 (n - 8) with a LOP3 + one fp16 add/FMA per pair. Each cell
-//    chain of K is scaled by that token's cell scale in fp32; the per-cell V
-//    scale is folded into the probabilities (the B operand) of that cell.
+//    2^-20 * sum((n - 8) q) with one AND per fp16 pair. V nibbles enter the
+//    same way; there the -8 offset is one extra MMA per tile, the sum over
+//    tokens of p * v_scale per (cell, head), subtracted in the epilogue.
+//    Each cell chain of K is scaled by that token's cell scale in fp32; the
+//    per-cell V scale is folded into the probabilities (the B operand) of
+//    that cell.
 //  * The running max / sum live in registers (base-2 exponent); the four
 //    warps are combined through shared memory and the CTA writes one fp32
 //    partial and its lse2 per query head. The merge kernel folds splits.
@@ -347,6 +349,8 @@ __global__ void __launch_bounds__(THREADS, 3)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[c][k][i] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;
+  // vsum[j] = running sum over tokens of p(token, head 2t+j) * v_scale(token, cell g)
+  float vsum[2] = {0.f, 0.f};
 
   // ldmatrix row owned by this lane: matrix mi = lane / 8 covers tokens
   // 8 * (mi & 1) .. +7 of the warp's 16 and cell 2 * cp + (mi >> 1).
@@ -469,12 +473,30 @@ __global__ void __launch_bounds__(THREADS, 3)
             acc[c][k][0] *= al0; acc[c][k][1] *= al1;
             acc[c][k][2] *= al0; acc[c][k][3] *= al1;
           }
+        vsum[0] *= al0;
+        vsum[1] *= al1;
       }
 
-      // ---- P V with the V scale folded into P per cell (packed fp16)
+      // ---- P V with the V scale folded into P per cell (packed fp16). The V
+      // nibbles enter raw, as fp16 subnormals (n * 2^-24 on MMA rows 0-7,
+      // n * 2^-20 on rows 8-15); the -8 offset is accounted for once per
+      // tile by vsum += S_v^T P (cell x head), applied in the epilogue.
       const __half2 p01 = __floats2half2_rn(pr[0], pr[1]), p23 = __floats2half2_rn(pr[2], pr[3]);
       const uint32_t s0w[4] = {sv0.x, sv0.y, sv0.z, sv0.w}, s1w[4] = {sv1.x, sv1.y, sv1.z, sv1.w};
       const uint32_t s2w[4] = {sv2.x, sv2.y, sv2.z, sv2.w}, s3w[4] = {sv3.x, sv3.y, sv3.z, sv3.w};
+      {
+        // A = the tile's V scales transposed: row = cell g, k = tokens 2t, 2t+1 (+8)
+        uint32_t st0, st1;
+        ldsm_x2_trans(smem_u32(vsb) + (uint32_t)((lane & 15) * SROW_BYTES), st0, st1);
+        if (partial) {  // absent tokens: a stale slot may hold any bit pattern
+          st0 &= (((tmask >> (2 * t)) & 1u) ? 0x0000ffffu : 0u) | (((tmask >> (2 * t + 1)) & 1u) ? 0xffff0000u : 0u);
+          st1 &= (((tmask >> (2 * t + 8)) & 1u) ? 0x0000ffffu : 0u) | (((tmask >> (2 * t + 9)) & 1u) ? 0xffff0000u : 0u);
+        }
+        float dd[4];
+        mma_f16_c(dd, st0, 0u, st1, 0u, h2_as_u32(p01), h2_as_u32(p23), vsum[0], vsum[1], 0.f, 0.f);
+        vsum[0] = dd[0];
+        vsum[1] = dd[1];
+      }
       uint32_t vw[2][4];
 #pragma unroll
       for (int c = 0; c < CELLS; ++c) {
@@ -483,8 +505,9 @@ __global__ void __launch_bounds__(THREADS, 3)
         const uint32_t b01 = h2_as_u32(__hmul2(p01, u32_as_h2(__byte_perm(s0w[c >> 1], s1w[c >> 1], sel))));
         const uint32_t b23 = h2_as_u32(__hmul2(p23, u32_as_h2(__byte_perm(s2w[c >> 1], s3w[c >> 1], sel))));
         const uint32_t za = vw[(c >> 1) & 1][2 * (c & 1)], zb = vw[(c >> 1) & 1][2 * (c & 1) + 1];
-        mma_f16(acc[c][0], nib_lo(za), nib_hi(za), nib_lo(zb), nib_hi(zb), b01, b23);
-        mma_f16(acc[c][1], nib_lo(za >> 8), nib_hi(za >> 8), nib_lo(zb >> 8), nib_hi(zb >> 8), b01, b23);
+        const uint32_t za8 = za >> 8, zb8 = zb >> 8;
+        mma_f16(acc[c][0], za & 0x000F000Fu, za & 0x00F000F0u, zb & 0x000F000Fu, zb & 0x00F000F0u, b01, b23);
+        mma_f16(acc[c][1], za8 & 0x000F000Fu, za8 & 0x00F000F0u, zb8 & 0x000F000Fu, zb8 & 0x00F000F0u, b01, b23);
       }
     }
     __syncwarp();
@@ -537,6 +560,20 @@ __global__ void __launch_bounds__(THREADS, 3)
 #pragma unroll
       for (int w = 0; w < CWARPS; ++w) M = fmaxf(M, sm.wm[w][h]);
       fw[j] = (M == -INFINITY) ? 0.f : exp2f(sm.wm[warp][h] - M);
+    }
+  }
+  // Undo the subnormal encoding of V: rows 0-7 carry 2^-24 * sum(n p s),
+  // rows 8-15 2^-20 * sum(n p s); the -8 offset is 8 * sum(p s) per cell.
+#pragma unroll
+  for (int c = 0; c < CELLS; ++c) {
+    const float b0 = 8.f * __shfl_sync(FULL_MASK, vsum[0], 4 * c + t);
+    const float b1 = 8.f * __shfl_sync(FULL_MASK, vsum[1], 4 * c + t);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      acc[c][k][0] = fmaf(acc[c][k][0], 16777216.f, -b0);
+      acc[c][k][1] = fmaf(acc[c][k][1], 16777216.f, -b1);
+      acc[c][k][2] = fmaf(acc[c][k][2], 1048576.f, -b0);
+      acc[c][k][3] = fmaf(acc[c][k][3], 1048576.f, -b1);
     }
   }
 #pragma unroll

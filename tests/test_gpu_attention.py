@@ -65,6 +65,7 @@ CASES = [
     ((2500,), 16, 4, 4, 300, 7),
     ((700, 1), 32, 16, 16, 30, 100),     # more splits than pages: empty splits
     ((5000, 3000, 10), 64, 16, 4, 140, 0),
+    ((1000, 31, 4097, 0, 1), 32, 32, 4, 200, 0),  # an empty context and a single token among others
 ]
 
 

@@ -43,7 +43,9 @@ class Workload:
     ``seq_lens`` counts every context token of a sequence, including the one
     the decode step writes: the cache is pre-filled with ``L - 1`` tokens at
     positions ``first_position ... first_position + L - 2`` and the step runs
-    at position ``first_position + L - 1``.
+    at position ``first_position + L - 1``. ``L = 0`` is an empty context:
+    nothing is pre-filled, the step writes no token (its slot is -1) and its
+    query is rotated at ``first_position``.
     """
 
     name: str
@@ -78,7 +80,7 @@ class Workload:
 
     @property
     def step_positions(self) -> List[int]:
-        return [self.first_position + L - 1 for L in self.seq_lens]
+        return [self.first_position + max(L - 1, 0) for L in self.seq_lens]
 
     def algorithmic_bytes_per_layer(self) -> int:
         """K/V data + fp16 scales of every context token, page-table entries,
@@ -173,14 +175,14 @@ def cache_slots(w: Workload, pt: np.ndarray) -> np.ndarray:
     the order of the generated K/V rows: sequence by sequence, token by token."""
     out = []
     for s, L in enumerate(w.seq_lens):
-        t = np.arange(L - 1, dtype=np.int64)
+        t = np.arange(max(L - 1, 0), dtype=np.int64)
         out.append(pt[s, t // w.block_size].astype(np.int64) * w.block_size + t % w.block_size)
     return np.concatenate(out) if out else np.zeros(0, np.int64)
 
 
 def step_slots(w: Workload, pt: np.ndarray) -> np.ndarray:
     """int64 slot of the token each sequence's decode step writes."""
-    return np.array([int(pt[s, (L - 1) // w.block_size]) * w.block_size + (L - 1) % w.block_size
+    return np.array([int(pt[s, (L - 1) // w.block_size]) * w.block_size + (L - 1) % w.block_size if L > 0 else -1
                      for s, L in enumerate(w.seq_lens)], dtype=np.int64)
 
 
@@ -205,13 +207,13 @@ def host_layer(w: Workload, layer: int = 0) -> Dict[str, np.ndarray]:
     """All inputs of one layer's decode step, as host arrays.
 
     Keys: ``q`` [n_seq][Hq][D], ``k_cache``/``v_cache`` [T][Hkv][D] (T = sum
-    of L - 1, rows ordered as ``cache_slots``), ``k_new``/``v_new``
+    of max(L - 1, 0), rows ordered as ``cache_slots``), ``k_new``/``v_new``
     [n_seq][Hkv][D] (bf16 bits, uint16); ``page_table``, ``cache_slots``,
     ``step_slots``, ``seq_lens`` (int32), ``positions`` (int64, step position
     of each sequence).
     """
     f = _head_factors(w, layer)
-    T = sum(L - 1 for L in w.seq_lens)
+    T = sum(max(L - 1, 0) for L in w.seq_lens)
     d = w.head_dim
 
     def normal(stream, shape, head_f, head_axis):
@@ -248,7 +250,7 @@ def device_layer(w: Workload, layer: int, device) -> Dict[str, "object"]:
     import torch
 
     f = _head_factors(w, layer)
-    T = sum(L - 1 for L in w.seq_lens)
+    T = sum(max(L - 1, 0) for L in w.seq_lens)
     d = w.head_dim
 
     def gen(stream):
