@@ -223,7 +223,7 @@ def qkv_paged_decode_attn_f4(out, q, k_data, k_scale, v_data, v_scale, page_tabl
         _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
 
 
-STATIC_SCRATCH_BYTES = 8 << 20
+STATIC_SCRATCH_BYTES = 16 << 20
 
 
 def qkv_paged_decode_attn_f4_static(out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, kv_heads: int,

@@ -10,31 +10,38 @@
 // pages; lanes sharing one pool).
 //
 // Design (B200, sm_100a). The step streams bytes: 288 bytes of packed K/V and
-// scales per token and KV head feed 2 x 4 x 256 multiply-adds. One CTA owns
+// scales per token and KV head feed 2 x G x 256 multiply-adds. One CTA owns
 // (split, sequence, KV head) so the G query heads of the group share every
-// dequantised page; 4 warps, 3 CTAs per SM (168 registers per thread).
-//  * 64-token stages (one 64-token page, or 2/4 pages of 32/16 tokens) fill a
-//    3-slot shared-memory ring: the packed K and V rows by 2-D TMA with the
-//    128-byte swizzle, their fp16 scales by 1-D bulk copies, all completing
-//    on one mbarrier per slot. Warp w issues the stages R = w (mod 4), so the
-//    issue work is spread evenly and no warp paces the others; a slot is
-//    refilled once all four warps have released it.
-//  * Each warp takes 16 tokens of a stage. ldmatrix delivers the packed
-//    nibbles already in mma-fragment order (plain for K, transposed for V).
-//    Q K^T and P V run on the tensor cores as m16n8k16 fp16 MMAs with fp32
-//    accumulation. K nibbles enter the MMA raw, as fp16 subnormals
-//    (n * 2^-24 in bits 0-3, n * 2^-20 in bits 4-7, both exact): q carries
-//    16 q on the low-nibble positions and each 32-dim cell's MMA chain starts
-//    from -8 * 2^-20 * sum(q over the cell), so the chain yields
-//    2^-20 * sum((n - 8) q) with one AND per fp16 pair. V nibbles enter the
-//    same way; there the -8 offset is one extra MMA per tile, the sum over
-//    tokens of p * v_scale per (cell, head), subtracted in the epilogue.
-//    Each cell chain of K is scaled by that token's cell scale in fp32; the
-//    per-cell V scale is folded into the probabilities (the B operand) of
-//    that cell.
-//  * The running max / sum live in registers (base-2 exponent); the four
-//    warps are combined through shared memory and the CTA writes one fp32
-//    partial and its lse2 per query head. The merge kernel folds splits.
+// page it reads; 4 warps, 4 CTAs per SM.
+//  * 64-token stages (one 64-token page, or 2/4 pages of 32/16 tokens). The
+//    packed K rows and their fp16 scales fill a 2-slot K ring, the V rows and
+//    scales a 3-slot V ring (V of a stage is read last): rows by 2-D TMA with
+//    the 128-byte swizzle, scales by 1-D bulk copies, each half of a stage
+//    completing on its own mbarrier. Both halves of stage i + 2 are issued
+//    at the CTA barrier of stage i, which shows their slots free, by the warp
+//    that owns the stage (stage R belongs to warp R mod 4).
+//  * Q K^T: warp w scores tokens 16w .. 16w + 15 of the stage. ldmatrix
+//    delivers the packed nibbles in mma-fragment order and they enter an
+//    m16n8k16 fp16 MMA (fp32 accumulate) raw, as fp16 subnormals (n * 2^-24
+//    in bits 0-3, n * 2^-20 in bits 4-7): q carries 16 q on the low-nibble
+//    positions and the -8 code offset is the chain's start value, -8 * 2^-20
+//    * sum(q over the cell). One MMA covers two cells: its 8 columns are
+//    (query head, cell parity), so each lane ends with both cells of one
+//    head and scales them by their own per-token cell scales in fp32.
+//  * Softmax: base-2 scores against one running max m per head shared by the
+//    whole CTA, probabilities 2^(x - m - SLACK). A stage whose scores all
+//    stay below m + SLACK (after the first stages, nearly all) needs one CTA
+//    barrier: the warps write their probabilities (fp16) to shared memory and
+//    the barrier, which also ORs a "new max" flag, publishes them. Otherwise
+//    the warps exchange tile maxima, rescale and rewrite.
+//  * P V: warp w owns dims 64w .. 64w + 63 (cells 2w, 2w+1) over all 64
+//    tokens of the stage: V^T (ldmatrix.trans, nibbles as fp16 subnormals) is
+//    the A operand, P times the token's V cell scale (one packed fp16
+//    multiply) the B operand. The -8 offset is sum_t p * v_scale per (cell,
+//    head), one extra MMA per 16 tokens, subtracted at the end. Each lane
+//    keeps 16 fp32 accumulators.
+//  * The CTA writes one fp32 partial per query head (each warp its own dims)
+//    and its lse2; the merge kernel folds the splits.
 // Dequantised tiles never touch shared memory: staging fp16 tiles for
 // tcgen05 would need ~4x the shared-memory bandwidth of the packed bytes.
 #include <cudaTypedefs.h>
@@ -42,39 +49,60 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 
 namespace qkv {
 
 namespace split {
-constexpr int D = 256;               // head_dim
-constexpr int CELLS = D / 32;        // 8 cells of 32 values per row
-constexpr int ROW_BYTES = D / 2;     // 128 packed bytes per token
+constexpr int D = 256;                 // head_dim
+constexpr int CELLS = D / 32;          // 8 cells of 32 values per row
+constexpr int PAIRS = CELLS / 2;       // cell pairs, one MMA chain each
+constexpr int ROW_BYTES = D / 2;       // 128 packed bytes per token
 constexpr int SROW_BYTES = CELLS * 2;  // 16 bytes of fp16 scales per token
 constexpr int STAGE_TOK = 64;
-constexpr int NS = 3;                // ring depth
-constexpr int CWARPS = 4;            // warps; each takes 16 tokens of a stage
+constexpr int NSK = 2;                 // K ring depth
+constexpr int NSV = 3;                 // V ring depth (V of a stage is read last)
+constexpr int CWARPS = 4;              // warps
 constexpr int THREADS = CWARPS * 32;
-constexpr int TR_STRIDE = 20;        // padded row of the score transpose buffer
+constexpr int PROW = STAGE_TOK + 8;    // padded probability row (fp16): conflict-free B loads
+constexpr uint32_t LO4 = 0x000F000Fu;  // nibble of bits 0-3 of each 16-bit half
+constexpr uint32_t HI4 = 0x00F000F0u;  // nibble of bits 4-7 of each 16-bit half
+// The running max of a head moves only when a score exceeds it by more than
+// SLACK (base-2 units); probabilities are taken against m + SLACK, so they
+// stay <= 1 and the fp16 product p * v_scale cannot overflow.
+constexpr float SLACK = 2.0f;
 
-struct __align__(1024) Smem {
-  uint8_t k[NS][STAGE_TOK * ROW_BYTES];  // 8 KiB each, 1024-aligned (128B swizzle atom)
-  uint8_t v[NS][STAGE_TOK * ROW_BYTES];
-  uint8_t ks[NS][STAGE_TOK * SROW_BYTES];
-  uint8_t vs[NS][STAGE_TOK * SROW_BYTES];
-  float tr[CWARPS][8][TR_STRIDE];
-  uint4 qfrag[CELLS][32];  // per cell and lane: the 4 fp16x2 B registers of both k-steps
-  float qbias[CELLS][8];   // per cell and head: -8 * 2^-20 * sum of the cell's q (accumulator start)
-  float wm[CWARPS][8];
-  float wl[CWARPS][8];
-  unsigned long long mask[NS];
-  uint64_t full[NS];
-  uint64_t empty[NS];
-  int abort_flag;
-  int issued;
+// Query-head quads: G <= 4 heads fit one MMA tile of (head, cell parity)
+// columns; G = 8 takes two.
+template <int G>
+struct Cfg {
+  static constexpr int HQ = (G + 3) / 4;
+  static constexpr int MIN_BLOCKS = 4;  // up to 128 registers: no operand shuffling
 };
-constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;  // + alignment slack
+
+template <int HQ>
+struct __align__(1024) Smem {
+  uint8_t k[NSK][STAGE_TOK * ROW_BYTES];  // 8 KiB each, 1024-aligned (128B swizzle atom)
+  uint8_t v[NSV][STAGE_TOK * ROW_BYTES];
+  uint8_t ks[NSK][STAGE_TOK * SROW_BYTES];
+  uint8_t vs[NSV][STAGE_TOK * SROW_BYTES];
+  uint4 qfrag[HQ][PAIRS][2][32];  // per lane: the B registers of the 4 MMAs of a cell pair
+  uint16_t prob[2][8][PROW];      // fp16 probabilities [stage parity][query head][token]
+  float4 qbias[HQ][PAIRS][4];     // per lane t: chain start of columns 2t, 2t+1 (twice, rows g and g+8)
+  float tmax[CWARPS][8];
+  float wl[CWARPS][8];
+  unsigned long long mask[NSK];  // tokens present in the stage of each K slot
+  uint64_t kfull[NSK];
+  uint64_t vfull[NSV];
+  int abort_flag;
+  int issued;  // stages issued so far (both halves)
+};
+template <int HQ>
+constexpr size_t smem_bytes() {
+  return sizeof(Smem<HQ>) + 1024;  // + alignment slack
+}
 
 struct Params {
   float* o_parts;
@@ -94,6 +122,7 @@ struct Params {
 using namespace split;
 
 __device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ uint32_t lds32(const void* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
 // D = A * B + C with C given separately (no copy of C into D first).
 __device__ __forceinline__ void mma_f16_c(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -112,10 +141,37 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ float half_at(const uint4& v, int i) {
-  const uint32_t w = (i < 2) ? v.x : (i < 4) ? v.y : (i < 6) ? v.z : v.w;
-  const unsigned short b = (i & 1) ? (unsigned short)(w >> 16) : (unsigned short)(w & 0xffff);
-  return __half2float(__ushort_as_half(b));
+// CTA barrier 1 over all THREADS threads that also returns the OR of `pred`.
+__device__ __forceinline__ bool bar_red_or(bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, 1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)pred), "n"(THREADS)
+      : "memory");
+  return out != 0;
+}
+
+__device__ __forceinline__ void bar_cta() { asm volatile("bar.sync 1, %0;" ::"n"(THREADS) : "memory"); }
+
+// Wait for phase `parity` of a copy barrier. False when the CTA is aborting
+// (another warp set the flag) or the wait limit ran out (then this sets it).
+__device__ __forceinline__ bool wait_copies(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                            int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (*abort_flag) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+      flag(status, QKV_DEV_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+  }
 }
 
 // Context length of a sequence, clamped to what its page-table row holds.
@@ -129,59 +185,73 @@ __device__ __forceinline__ int seq_len_of(const Params& p, int s, int block, boo
   return L;
 }
 
+// ceil(a / b) for a >= 0, b > 0 (32-bit division: a few instructions)
+__device__ __forceinline__ uint32_t cdiv(uint32_t a, uint32_t b) { return (a + b - 1) / b; }
+
+// floor(a * b / c) for a, b >= 0, c > 0, in 32-bit arithmetic when a * b fits
+__device__ __forceinline__ int muldiv(uint32_t a, uint32_t b, uint32_t c) {
+  const unsigned long long ab = (unsigned long long)a * b;
+  return (ab >> 32) == 0 ? (int)((uint32_t)ab / c) : (int)(ab / c);
+}
+
 // Split plan. Fixed: min(num_splits, max_splits) splits per sequence.
 // Automatic: pages are cut into pieces of about total pages / target, so the
 // grid holds at most `target` busy CTAs per KV head whatever the mix of
 // lengths. Split i of a sequence with n pages covers [i*n/S, (i+1)*n/S).
-__device__ long long splits_for(const Params& p, int block, long long P) {
+__device__ long long splits_for(const Params& p, int block, uint32_t P) {
   long long total = 0;
-  for (int s = 0; s < p.n_seq; ++s) total += ((seq_len_of(p, s, block, false) + block - 1) / block + P - 1) / P;
+  for (int s = 0; s < p.n_seq; ++s) total += cdiv(cdiv((uint32_t)seq_len_of(p, s, block, false), block), P);
   return total;
 }
 
 __device__ void plan(const Params& p, int seq, int split, int block, int& S, int& pg0, int& pg1, int& L) {
   L = seq_len_of(p, seq, block, split == 0 && blockIdx.z == 0);
-  const int n = (L + block - 1) / block;
+  const uint32_t n = cdiv((uint32_t)L, (uint32_t)block);
   if (p.num_splits > 0) {
     S = min(p.num_splits, p.max_splits);
   } else {
     // Pieces of P pages with sum_s ceil(n_s / P) <= target, so the busy CTAs
     // fit the resident slots in one wave.
-    long long T = 0, nmax = 1;
+    long long T = 0;
+    uint32_t nmax = 1;
     for (int s = 0; s < p.n_seq; ++s) {
-      const long long ns = (seq_len_of(p, s, block, false) + block - 1) / block;
+      const uint32_t ns = cdiv((uint32_t)seq_len_of(p, s, block, false), (uint32_t)block);
       T += ns;
       nmax = max(nmax, ns);
     }
-    long long P;
+    uint32_t P;
     if (p.target <= p.n_seq) {
       P = nmax;  // one split per sequence
     } else {
-      P = max(1LL, (T + p.target - 1) / p.target);
+      P = (uint32_t)max(1LL, (T + p.target - 1) / p.target);
       for (int k = 0; k < 4 && splits_for(p, block, P) > p.target; ++k) ++P;
-      if (splits_for(p, block, P) > p.target) P = max(P, (T + p.target - p.n_seq - 1) / (p.target - p.n_seq));
+      if (splits_for(p, block, P) > p.target)
+        P = max(P, (uint32_t)((T + p.target - p.n_seq - 1) / (p.target - p.n_seq)));
     }
-    S = (int)min((long long)p.max_splits, max(1LL, (n + P - 1) / P));
+    S = (int)min((uint32_t)p.max_splits, max(1u, cdiv(n, P)));
   }
-  pg0 = (int)((long long)split * n / S);
-  pg1 = (int)((long long)(split + 1) * n / S);
+  pg0 = muldiv((uint32_t)split, n, (uint32_t)S);
+  pg1 = muldiv((uint32_t)split + 1, n, (uint32_t)S);
 }
 
 template <int BLOCK, int G>
-__global__ void __launch_bounds__(THREADS, 3)
+__global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
     paged_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                               const Params p) {
   static_assert(STAGE_TOK % BLOCK == 0, "pages must tile a stage");
-  static_assert(G >= 1 && G <= 8, "one n8 MMA tile holds the query group");
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8, "query heads per KV head");
+  constexpr int HQ = Cfg<G>::HQ;
   constexpr int PPS = STAGE_TOK / BLOCK;  // pages per stage
+  using SmemT = Smem<HQ>;
 
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SmemT& sm = *reinterpret_cast<SmemT*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   pdl_wait();
   pdl_release();
   const int split = blockIdx.x, seq = blockIdx.y, kvh = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
   const int rows = p.n_seq * p.q_heads;
   const int row0 = seq * p.q_heads + kvh * G;  // first query-head row of this group
   float* lse_out = p.lse2_parts + (size_t)split * rows + row0;
@@ -197,119 +267,124 @@ __global__ void __launch_bounds__(THREADS, 3)
   const int n_it = t_end > t_begin ? (t_end - t_begin + STAGE_TOK - 1) / STAGE_TOK : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], CWARPS);
-    }
+    for (int s = 0; s < NSK; ++s) mbar_init(&sm.kfull[s], 1);
+    for (int s = 0; s < NSV; ++s) mbar_init(&sm.vfull[s], 1);
     sm.abort_flag = 0;
     sm.issued = 0;
     fence_barrier_init();
   }
+  // probability rows of absent query heads (G < 8) are read as zeros
+  for (int i = threadIdx.x; i < (int)(sizeof(sm.prob) / 4); i += THREADS)
+    reinterpret_cast<uint32_t*>(&sm.prob[0][0][0])[i] = 0u;
   __syncthreads();
 
   // ------------------------------------------------------------ copy issue
-  // Stage `it` holds tokens t_begin + 64 it ... +63, i.e. 64 / BLOCK pages,
-  // each as four copies (K rows, V rows by TMA with the 128-byte swizzle; K
-  // and V scales by bulk copy). Warp w issues the stages R = w (mod 4), so
-  // the issue work is spread evenly over the warps; lane j of warp w keeps
-  // the page ids of the j-th next of those stages (32 per refresh, the next
-  // 32 prefetched), so no copy waits on a page-table load.
+  // Stage R holds tokens t_begin + 64 R ... + 63, i.e. 64 / BLOCK pages. Its
+  // K half (rows by TMA, scales by bulk copy) completes on kfull[R % NSK],
+  // its V half on vfull[R % NSV]. Stage R belongs to warp R % 4, which issues
+  // both halves at once; each warp holds the page ids of its next stage,
+  // loaded one of its stages ahead, so no copy waits on the page table.
   const uint64_t pol = policy_evict_first();
   const int32_t* pt = p.page_table + (size_t)seq * p.max_pages + pg0;
   const int npg = pg1 - pg0;
+  const int full_stages = (t_end - t_begin) / STAGE_TOK;  // stages with all 64 tokens
   volatile int* abort_flag = &sm.abort_flag;
-  int id_cur[PPS], id_nxt[PPS];
-  int id_base = 0;  // index (R / CWARPS) of the stage held by lane 0
-  auto load_ids = [&](int base, int (&dst)[PPS]) {
-    const int R = (base + lane) * CWARPS + warp;
+  // the host keeps num_pages * kv_heads * block below 2^31
+  const uint32_t num_pages32 = (uint32_t)p.num_pages;
+  int ids[PPS];
+  auto load_ids = [&](int R) {
 #pragma unroll
     for (int k = 0; k < PPS; ++k) {
       const int pi = R * PPS + k;
-      dst[k] = pi < npg ? pt[pi] : -1;
+      ids[k] = pi < npg ? pt[pi] : -1;
     }
   };
-  load_ids(0, id_cur);
-  load_ids(32, id_nxt);
-  // called by all lanes of warp R % CWARPS, with R increasing
+  load_ids(warp);
+  // Called by all lanes of warp R % 4, with R increasing by 4 each time.
   auto issue = [&](int R) {
-    const int st = R % NS;
-    const int j = R / CWARPS;
-    if (j >= id_base + 32) {
-      id_base += 32;
-#pragma unroll
-      for (int k = 0; k < PPS; ++k) id_cur[k] = id_nxt[k];
-      load_ids(id_base + 32, id_nxt);
-    }
     int phys[PPS];
 #pragma unroll
-    for (int k = 0; k < PPS; ++k) phys[k] = __shfl_sync(FULL_MASK, id_cur[k], (j - id_base) & 31);
+    for (int k = 0; k < PPS; ++k) phys[k] = ids[k];
+    load_ids(R + CWARPS);
     if (lane != 0) return;
-    const int tok0 = t_begin + R * STAGE_TOK;
-    unsigned long long mask = 0;
-    uint32_t bytes = 0;
+    const int ks = R % NSK, vs = R % NSV;
+    bool all_ok = R < full_stages;
 #pragma unroll
-    for (int k = 0; k < PPS; ++k) {
-      const int tk = tok0 + k * BLOCK;
-      if (tk >= t_end) {
-        phys[k] = -1;
-        continue;
+    for (int k = 0; k < PPS; ++k) all_ok = all_ok && (uint32_t)phys[k] < num_pages32;
+    unsigned long long mask = ~0ull;
+    uint32_t npages = PPS;
+    if (!all_ok) {  // the last, partial stage or an invalid page id
+      const int tok0 = t_begin + R * STAGE_TOK;
+      mask = 0;
+      npages = 0;
+#pragma unroll
+      for (int k = 0; k < PPS; ++k) {
+        const int tk = tok0 + k * BLOCK;
+        if (tk >= t_end) {
+          phys[k] = -1;
+        } else if ((uint32_t)phys[k] >= num_pages32) {  // negative ids wrap to large
+          flag(p.status, QKV_DEV_BAD_PAGE);
+          phys[k] = -1;
+        } else {
+          const int nv = min(BLOCK, t_end - tk);
+          const unsigned long long bits = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
+          mask |= bits << (k * BLOCK);
+          ++npages;
+        }
       }
-      if (phys[k] < 0 || (int64_t)phys[k] >= p.num_pages) {
-        flag(p.status, QKV_DEV_BAD_PAGE);
-        phys[k] = -1;
-        continue;
-      }
-      const int nv = min(BLOCK, t_end - tk);
-      const unsigned long long bits = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
-      mask |= bits << (k * BLOCK);
-      bytes += 2u * BLOCK * (ROW_BYTES + SROW_BYTES);
     }
-    sm.mask[st] = mask;
-    mbar_arrive_expect_tx(&sm.full[st], bytes);
+    sm.mask[ks] = mask;
+    const uint32_t bytes = npages * BLOCK * (ROW_BYTES + SROW_BYTES);
+    mbar_arrive_expect_tx(&sm.kfull[ks], bytes);
+    mbar_arrive_expect_tx(&sm.vfull[vs], bytes);
 #pragma unroll
     for (int k = 0; k < PPS; ++k) {
       if (phys[k] < 0) continue;
       const int row = (phys[k] * p.kv_heads + kvh) * BLOCK;
-      tma_load_2d(&sm.k[st][k * BLOCK * ROW_BYTES], &tm_k, &sm.full[st], 0, row, pol);
-      tma_load_2d(&sm.v[st][k * BLOCK * ROW_BYTES], &tm_v, &sm.full[st], 0, row, pol);
-      bulk_load(&sm.ks[st][k * BLOCK * SROW_BYTES], p.k_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
-                &sm.full[st], pol);
-      bulk_load(&sm.vs[st][k * BLOCK * SROW_BYTES], p.v_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
-                &sm.full[st], pol);
+      tma_load_2d(&sm.k[ks][k * BLOCK * ROW_BYTES], &tm_k, &sm.kfull[ks], 0, row, pol);
+      bulk_load(&sm.ks[ks][k * BLOCK * SROW_BYTES], p.k_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
+                &sm.kfull[ks], pol);
+      tma_load_2d(&sm.v[vs][k * BLOCK * ROW_BYTES], &tm_v, &sm.vfull[vs], 0, row, pol);
+      bulk_load(&sm.vs[vs][k * BLOCK * SROW_BYTES], p.v_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
+                &sm.vfull[vs], pol);
     }
     atomicMax(&sm.issued, R + 1);
   };
-  if (warp < min(NS, n_it)) issue(warp);  // stages 0 .. NS-1
+  // stages 0 and 1; stage R + 2 follows at the CTA barrier of stage R
+  if (warp < 2 && warp < n_it) issue(warp);
 
-  // ------------------------------------------------------------ consumers
-  const int g = lane >> 2, t = lane & 3;
-
-  // q as the B operand (k = head_dim slice, n = query head). Within each
-  // 32-dim cell the k index is permuted to match the nibble order the
-  // unpack produces: k-step ks, fragment register r, half i <-> dim
-  // 8t + 2ks + r + 4i.
-  uint32_t qb[CELLS][2][2];  // built here, kept in shared memory
+  // ------------------------------------------------------------ q as the B operand
+  // Column n of the Q K^T tile is (query head n >> 1 of the quad, cell
+  // parity n & 1). Lane (g, t) builds column g: head 4 hq + (g >> 1), cell
+  // 2 pp + (g & 1), dims 8t .. 8t + 7 of that cell. The 4 MMAs of a pair
+  // take the nibble variants v = 0..3 (dims 8t + v and 8t + 4 + v); rows 0-7
+  // of the k index come from the even cell, rows 8-15 from the odd one.
   float score_scale = p.score_scale;
   {
-    float qf[CELLS][8];
+    const int hl = g >> 1, par = g & 1;
+    const bool col_ok = G >= 4 || hl < G;
+    float qf[HQ][PAIRS][8];
     float qmax = 0.f;
 #pragma unroll
-    for (int c = 0; c < CELLS; ++c) {
-      if (g < G) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(p.q + (size_t)(row0 + g) * D + 32 * c + 8 * t);
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    for (int hq = 0; hq < HQ; ++hq)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          qf[c][2 * i] = __uint_as_float(w[i] << 16);
-          qf[c][2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+      for (int pp = 0; pp < PAIRS; ++pp) {
+        if (col_ok) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(p.q + (size_t)(row0 + 4 * hq + hl) * D +
+                                                            32 * (2 * pp + par) + 8 * t);
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            qf[hq][pp][2 * i] = __uint_as_float(w[i] << 16);
+            qf[hq][pp][2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) qf[hq][pp][i] = 0.f;
         }
-      } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) qf[c][i] = 0.f;
+        for (int i = 0; i < 8; ++i) qmax = fmaxf(qmax, fabsf(qf[hq][pp][i]));
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) qmax = fmaxf(qmax, fabsf(qf[c][i]));
-    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(FULL_MASK, qmax, o));
     // q enters the MMA as fp16 with an exact power-of-two prescale: the
@@ -318,256 +393,330 @@ __global__ void __launch_bounds__(THREADS, 3)
     // 2^-20 * n * q; 16 * max|q| stays below 2^15.
     const int qexp = (int)((__float_as_uint(qmax) >> 23) & 0xff) - 127;
     const int shift = qexp >= 11 ? qexp - 10 : 0;
-    score_scale = ldexpf(score_scale, shift + 20);
+    // exact powers of two (shift <= 117): 2^-shift scales q, 2^(shift + 20) the scores
+    const float down = __int_as_float((127 - shift) << 23);
+    score_scale = score_scale * 1048576.f * __int_as_float((127 + shift) << 23);
 #pragma unroll
-    for (int c = 0; c < CELLS; ++c) {
-      float qs = 0.f;  // sum of this lane's 8 dims of the cell, as the MMA sees them
+    for (int hq = 0; hq < HQ; ++hq)
 #pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        const __half2 lo = __floats2half2_rn(ldexpf(qf[c][2 * ks], -shift), ldexpf(qf[c][2 * ks + 4], -shift));
-        const __half2 hi = __floats2half2_rn(ldexpf(qf[c][2 * ks + 1], -shift), ldexpf(qf[c][2 * ks + 5], -shift));
-        const float2 lf = __half22float2(lo), hf = __half22float2(hi);
-        qs += (lf.x + lf.y) + (hf.x + hf.y);
-        qb[c][ks][0] = h2_as_u32(__hmul2(lo, u32_as_h2(0x4C004C00u)));  // x16, exact
-        qb[c][ks][1] = h2_as_u32(hi);
+      for (int pp = 0; pp < PAIRS; ++pp) {
+        uint32_t bv[4];
+        float qs = 0.f;  // sum of this lane's 8 dims, as the MMA sees them
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const __half2 h = __floats2half2_rn(qf[hq][pp][v] * down, qf[hq][pp][v + 4] * down);
+          const float2 f = __half22float2(h);
+          qs += f.x + f.y;
+          bv[v] = (v & 1) ? h2_as_u32(h) : h2_as_u32(__hmul2(h, u32_as_h2(0x4C004C00u)));  // x16, exact
+        }
+        uint32_t b0[4], b1[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          b0[v] = par ? 0u : bv[v];
+          b1[v] = par ? bv[v] : 0u;
+        }
+        if (warp == 0) {
+          sm.qfrag[hq][pp][0][lane] = make_uint4(b0[0], b1[0], b0[1], b1[1]);
+          sm.qfrag[hq][pp][1][lane] = make_uint4(b0[2], b1[2], b0[3], b1[3]);
+        }
+        qs += __shfl_xor_sync(FULL_MASK, qs, 1);
+        qs += __shfl_xor_sync(FULL_MASK, qs, 2);
+        // column g starts its chain at -8 * 2^-20 * sum of the cell's q
+        if (warp == 0 && t == 0) {
+          float* b4 = reinterpret_cast<float*>(&sm.qbias[hq][pp][g >> 1]);
+          b4[g & 1] = b4[(g & 1) + 2] = col_ok ? qs * -7.62939453125e-06f : 0.f;  // -8 * 2^-20
+        }
       }
-      qs += __shfl_xor_sync(FULL_MASK, qs, 1);
-      qs += __shfl_xor_sync(FULL_MASK, qs, 2);
-      if (warp == 0 && t == 0) sm.qbias[c][g] = (g < G) ? -8.0f * ldexpf(qs, -20) : 0.f;
-    }
-    if (warp == 0)
-#pragma unroll
-      for (int c = 0; c < CELLS; ++c) sm.qfrag[c][lane] = make_uint4(qb[c][0][0], qb[c][0][1], qb[c][1][0], qb[c][1][1]);
   }
   __syncthreads();
 
-  float acc[CELLS][2][4];
+  // ------------------------------------------------------------ main loop
+  // QK side: lane (g, t) holds head 4 hq + t of tokens g and g + 8 of the
+  // warp's 16. PV side: columns 2t, 2t+1 are query heads 2t, 2t+1; rows are
+  // dims of the warp's two cells.
+  bool head_ok[HQ];
 #pragma unroll
-  for (int c = 0; c < CELLS; ++c)
+  for (int hq = 0; hq < HQ; ++hq) head_ok[hq] = G >= 4 || t < G;
+  float m_run[HQ], m_ref[HQ], thr[HQ], l_run[HQ];
+#pragma unroll
+  for (int hq = 0; hq < HQ; ++hq) {
+    m_run[hq] = -INFINITY;  // running max of the scaled scores (base 2)
+    m_ref[hq] = 0.f;        // exponent reference: m_run + SLACK, or 0 while m_run = -inf
+    thr[hq] = -INFINITY;    // 0, or -inf while m_run = -inf: the fast path needs x - m_ref <= thr
+    l_run[hq] = 0.f;
+  }
+  float acc[2][2][4];
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
 #pragma unroll
     for (int k = 0; k < 2; ++k)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[c][k][i] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
-  // vsum[j] = running sum over tokens of p(token, head 2t+j) * v_scale(token, cell g)
+  // vsum[j] = running sum, over this warp's k-step of every stage, of
+  // p(token, head 2t + j) * v_scale(token, cell g)
   float vsum[2] = {0.f, 0.f};
 
-  // ldmatrix row owned by this lane: matrix mi = lane / 8 covers tokens
-  // 8 * (mi & 1) .. +7 of the warp's 16 and cell 2 * cp + (mi >> 1).
-  const uint32_t ld_row = (uint32_t)((((lane >> 3) & 1) * 8 + (lane & 7)) * ROW_BYTES);
-  const int sw = lane & 7;  // 128B swizzle: chunk index ^= row index mod 8
-  const int co = lane >> 4;
-  uint32_t ld_off[CELLS / 2];  // this lane's ldmatrix address offset for cell pair cp
+  // K ldmatrix (plain): matrix mi = lane / 8 covers tokens 16w + 8 (mi & 1)
+  // .. +7 and cell 2 pp + (mi >> 1); 128B swizzle: chunk ^= row mod 8.
+  const int sw = lane & 7;
+  uint32_t koff[PAIRS];
 #pragma unroll
-  for (int cp = 0; cp < CELLS / 2; ++cp) ld_off[cp] = ld_row + ((uint32_t)((2 * cp + co) ^ sw) << 4);
-  float(*tr)[TR_STRIDE] = sm.tr[warp];
+  for (int pp = 0; pp < PAIRS; ++pp)
+    koff[pp] = (uint32_t)((16 * warp + 8 * ((lane >> 3) & 1) + sw) * ROW_BYTES) +
+               ((uint32_t)((2 * pp + (lane >> 4)) ^ sw) << 4);
+  // V ldmatrix (transposed) of k-step kk: tokens 16 kk + 8 (mi & 1) .. +7,
+  // cell 2w + (mi >> 1).
+  const uint32_t voff = (uint32_t)((8 * ((lane >> 3) & 1) + sw) * ROW_BYTES) +
+                        ((uint32_t)((2 * warp + (lane >> 4)) ^ sw) << 4);
   bool aborted = false;
+  int st = 0, vst = 0;           // K and V slots of stage it
+  uint32_t ph = 0, vph = 0;      // their phase parities
 
   for (int it = 0; it < n_it; ++it) {
-    const int st = it % NS;
-    if (!aborted && !mbar_wait_bounded(&sm.full[st], (it / NS) & 1)) {
-      flag(p.status, QKV_DEV_TIMEOUT);
-      *abort_flag = 1;
-    }
-    // warp-uniform, so the .aligned ldmatrix / mma below see a converged warp
-    aborted = __any_sync(FULL_MASK, aborted || (*abort_flag != 0));
-    const uint32_t tmask = aborted ? 0u : (uint32_t)((sm.mask[st] >> (16 * warp)) & 0xffffu);
-    if (tmask != 0u) {
-      const uint32_t kbase = smem_u32(&sm.k[st][warp * 16 * ROW_BYTES]);
-      const uint32_t vbase = smem_u32(&sm.v[st][warp * 16 * ROW_BYTES]);
-      const uint8_t* ksb = &sm.ks[st][warp * 16 * SROW_BYTES];
-      const uint8_t* vsb = &sm.vs[st][warp * 16 * SROW_BYTES];
-      const bool partial = tmask != 0xffffu;
-
+    // ---------------- scores of the warp's 16 tokens
+    // (aborted is warp-uniform, so the .aligned ldmatrix / mma below see a
+    // converged warp)
+    aborted = __any_sync(FULL_MASK, aborted || !wait_copies(&sm.kfull[st], ph, abort_flag, p.status));
+    const unsigned long long smask = aborted ? 0ull : sm.mask[st];
+    const uint32_t wmask = (uint32_t)(smask >> (16 * warp)) & 0xffffu;
+    float sg[HQ], sg8[HQ];
+#pragma unroll
+    for (int hq = 0; hq < HQ; ++hq) sg[hq] = sg8[hq] = 0.f;
+    if (wmask != 0u) {
+      const uint32_t kbase = smem_u32(&sm.k[st][0]);
+      const uint8_t* ksb = &sm.ks[st][16 * warp * SROW_BYTES];
       const uint4 skA = lds128(ksb + g * SROW_BYTES);
       const uint4 skB = lds128(ksb + (g + 8) * SROW_BYTES);
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-      const uint32_t ka[4] = {skA.x, skA.y, skA.z, skA.w}, kb[4] = {skB.x, skB.y, skB.z, skB.w};
+      const uint32_t sa[4] = {skA.x, skA.y, skA.z, skA.w}, sb[4] = {skB.x, skB.y, skB.z, skB.w};
 #pragma unroll
-      for (int grp = 0; grp < 2; ++grp) {
-        uint32_t kw[2][4];
-        ldsm_x4(kbase + ld_off[2 * grp], kw[0]);
-        ldsm_x4(kbase + ld_off[2 * grp + 1], kw[1]);
-        float d[4][4];
+      for (int pp = 0; pp < PAIRS; ++pp) {
+        uint32_t kw[4];
+        ldsm_x4(kbase + koff[pp], kw);  // tok g / g+8 of cell 2pp, then of cell 2pp+1
+        uint32_t kh[4];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int c = 4 * grp + cc;
-          const uint4 qv = sm.qfrag[c][lane];
-          const float2 bias = *reinterpret_cast<const float2*>(&sm.qbias[c][2 * t]);
-          const uint32_t wa = kw[cc >> 1][2 * (cc & 1)], wb = kw[cc >> 1][2 * (cc & 1) + 1];
-          const uint32_t wa8 = wa >> 8, wb8 = wb >> 8;
-          // raw nibbles as fp16 subnormals: n * 2^-24 (bits 0-3), n * 2^-20 (bits 4-7)
-          mma_f16_c(d[cc], wa & 0x000F000Fu, wb & 0x000F000Fu, wa & 0x00F000F0u, wb & 0x00F000F0u, qv.x, qv.y,
-                    bias.x, bias.y, bias.x, bias.y);
-          mma_f16(d[cc], wa8 & 0x000F000Fu, wb8 & 0x000F000Fu, wa8 & 0x00F000F0u, wb8 & 0x00F000F0u, qv.z, qv.w);
-        }
+        for (int i = 0; i < 4; ++i) kh[i] = kw[i] >> 8;
+        const float2 fa = __half22float2(u32_as_h2(sa[pp])), fb = __half22float2(u32_as_h2(sb[pp]));
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          const float2 fa = __half22float2(u32_as_h2(ka[2 * grp + c2])), fb = __half22float2(u32_as_h2(kb[2 * grp + c2]));
-          s0 = fmaf(fa.x, d[2 * c2][0], s0);
-          s1 = fmaf(fa.x, d[2 * c2][1], s1);
-          s2 = fmaf(fb.x, d[2 * c2][2], s2);
-          s3 = fmaf(fb.x, d[2 * c2][3], s3);
-          s0 = fmaf(fa.y, d[2 * c2 + 1][0], s0);
-          s1 = fmaf(fa.y, d[2 * c2 + 1][1], s1);
-          s2 = fmaf(fb.y, d[2 * c2 + 1][2], s2);
-          s3 = fmaf(fb.y, d[2 * c2 + 1][3], s3);
+        for (int hq = 0; hq < HQ; ++hq) {
+          const uint4 qa = sm.qfrag[hq][pp][0][lane], qb = sm.qfrag[hq][pp][1][lane];
+          const float4 bias = sm.qbias[hq][pp][t];
+          float d[4];
+          mma_f16_c(d, kw[0] & LO4, kw[1] & LO4, kw[2] & LO4, kw[3] & LO4, qa.x, qa.y, bias.x, bias.y, bias.z,
+                    bias.w);
+          mma_f16(d, kw[0] & HI4, kw[1] & HI4, kw[2] & HI4, kw[3] & HI4, qa.z, qa.w);
+          mma_f16(d, kh[0] & LO4, kh[1] & LO4, kh[2] & LO4, kh[3] & LO4, qb.x, qb.y);
+          mma_f16(d, kh[0] & HI4, kh[1] & HI4, kh[2] & HI4, kh[3] & HI4, qb.z, qb.w);
+          // columns 2t (even cell) and 2t+1 (odd cell) of head t
+          sg[hq] = fmaf(fa.x, d[0], sg[hq]);
+          sg[hq] = fmaf(fa.y, d[1], sg[hq]);
+          sg8[hq] = fmaf(fb.x, d[2], sg8[hq]);
+          sg8[hq] = fmaf(fb.y, d[3], sg8[hq]);
         }
       }
-      uint4 sv0 = lds128(vsb + (2 * t) * SROW_BYTES);
-      uint4 sv1 = lds128(vsb + (2 * t + 1) * SROW_BYTES);
-      uint4 sv2 = lds128(vsb + (2 * t + 8) * SROW_BYTES);
-      uint4 sv3 = lds128(vsb + (2 * t + 9) * SROW_BYTES);
-      s0 *= score_scale; s1 *= score_scale; s2 *= score_scale; s3 *= score_scale;
-      if (partial) {
-        if (!((tmask >> g) & 1u)) s0 = s1 = -INFINITY;
-        if (!((tmask >> (g + 8)) & 1u)) s2 = s3 = -INFINITY;
-        // the weights of absent tokens are exactly 0; make their scales 0 too
-        // (a stale slot may hold any bit pattern)
-        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-        if (!((tmask >> (2 * t)) & 1u)) sv0 = z4;
-        if (!((tmask >> (2 * t + 1)) & 1u)) sv1 = z4;
-        if (!((tmask >> (2 * t + 8)) & 1u)) sv2 = z4;
-        if (!((tmask >> (2 * t + 9)) & 1u)) sv3 = z4;
-      }
+    }
+    const bool okA = (wmask >> g) & 1u, okB = (wmask >> (g + 8)) & 1u;
 
-      // ---- transpose to the PV B-operand layout: head g, tokens 2t, 2t+1, 2t+8, 2t+9
-      __syncwarp();
-      if (2 * t < G) {
-        tr[2 * t][g] = s0;
-        tr[2 * t][g + 8] = s2;
-        if (2 * t + 1 < G) {
-          tr[2 * t + 1][g] = s1;
-          tr[2 * t + 1][g + 8] = s3;
+    // ---------------- probabilities against the CTA's running max
+    const int pb = it & 1;
+    float xA[HQ], xB[HQ], psum[HQ];
+    bool need = false;
+#pragma unroll
+    for (int hq = 0; hq < HQ; ++hq) {
+      xA[hq] = (okA && head_ok[hq]) ? sg[hq] * score_scale : -INFINITY;
+      xB[hq] = (okB && head_ok[hq]) ? sg8[hq] * score_scale : -INFINITY;
+      const float yA = xA[hq] - m_ref[hq], yB = xB[hq] - m_ref[hq];
+      need |= (yA > thr[hq]) || (yB > thr[hq]);
+      const float pA = ex2(yA), pB = ex2(yB);
+      psum[hq] = pA + pB;
+      uint16_t* pr = &sm.prob[pb][4 * hq + t][16 * warp + g];
+      pr[0] = __half_as_ushort(__float2half_rn(pA));
+      pr[8] = __half_as_ushort(__float2half_rn(pB));
+    }
+    // All warps are done with K of this stage and with V of the previous
+    // one; the probabilities of this stage are published.
+    const bool any_new_max = bar_red_or(need);
+    if (any_new_max) {
+      // Some head's running max moves: exchange the tile maxima, rescale.
+#pragma unroll
+      for (int hq = 0; hq < HQ; ++hq) {
+        float tm = fmaxf(xA[hq], xB[hq]);
+        tm = fmaxf(tm, __shfl_xor_sync(FULL_MASK, tm, 4));
+        tm = fmaxf(tm, __shfl_xor_sync(FULL_MASK, tm, 8));
+        tm = fmaxf(tm, __shfl_xor_sync(FULL_MASK, tm, 16));
+        if (g == 0) sm.tmax[warp][4 * hq + t] = tm;
+      }
+      bar_cta();
+      float alpha[HQ];
+#pragma unroll
+      for (int hq = 0; hq < HQ; ++hq) {
+        float mn = m_run[hq];
+#pragma unroll
+        for (int w = 0; w < CWARPS; ++w) mn = fmaxf(mn, sm.tmax[w][4 * hq + t]);
+        const float mu = (mn == -INFINITY) ? 0.f : mn + SLACK;
+        alpha[hq] = (m_run[hq] == -INFINITY) ? 0.f : ex2(m_ref[hq] - mu);  // nothing accumulated yet: 0
+        m_run[hq] = mn;
+        m_ref[hq] = mu;
+        thr[hq] = (mn == -INFINITY) ? -INFINITY : 0.f;
+        const float pA = ex2(xA[hq] - mu), pB = ex2(xB[hq] - mu);
+        l_run[hq] = l_run[hq] * alpha[hq] + (pA + pB);
+        uint16_t* pr = &sm.prob[pb][4 * hq + t][16 * warp + g];
+        pr[0] = __half_as_ushort(__float2half_rn(pA));
+        pr[8] = __half_as_ushort(__float2half_rn(pB));
+      }
+      // PV columns 2t, 2t+1 are heads 2t, 2t+1: their alphas sit on the lanes
+      // t' = 2t mod 4 and 2t+1 mod 4 of quad (2t) / 4.
+      const int src0 = (lane & ~3) | ((2 * t) & 3), src1 = src0 | 1;
+      float al0 = __shfl_sync(FULL_MASK, alpha[0], src0), al1 = __shfl_sync(FULL_MASK, alpha[0], src1);
+      if (HQ > 1) {
+        const float b0 = __shfl_sync(FULL_MASK, alpha[HQ - 1], src0), b1 = __shfl_sync(FULL_MASK, alpha[HQ - 1], src1);
+        if (t >= 2) {
+          al0 = b0;
+          al1 = b1;
         }
       }
-      __syncwarp();
-      float sc[4];
-      if (g < G) {
-        const float2 a = *reinterpret_cast<const float2*>(&tr[g][2 * t]);
-        const float2 b = *reinterpret_cast<const float2*>(&tr[g][2 * t + 8]);
-        sc[0] = a.x; sc[1] = a.y; sc[2] = b.x; sc[3] = b.y;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          acc[c][k][0] *= al0;
+          acc[c][k][1] *= al1;
+          acc[c][k][2] *= al0;
+          acc[c][k][3] *= al1;
+        }
+      vsum[0] *= al0;
+      vsum[1] *= al1;
+      bar_cta();
+    } else {
+#pragma unroll
+      for (int hq = 0; hq < HQ; ++hq) l_run[hq] += psum[hq];
+    }
+
+    // ---------------- refill: K of stage it + 2 (slot of stage it), V of stage it + 1
+    // K of stage it + 2 goes to the K slot of stage it, V to the slot of
+    // stage it - 1: all warps are past both.
+    if (!aborted && it + 2 < n_it && ((it + 2) % CWARPS) == warp) issue(it + 2);
+
+    // ---------------- P V over the stage's 64 tokens, dims of cells 2w, 2w+1
+    if (!aborted) aborted = __any_sync(FULL_MASK, !wait_copies(&sm.vfull[vst], vph, abort_flag, p.status));
+    if (!aborted && smask != 0ull) {
+      const uint32_t vbase = smem_u32(&sm.v[vst][0]) + voff;
+      const uint8_t* vsb = &sm.vs[vst][0];
+      const uint16_t* prow = &sm.prob[pb][g][0];
+      // k-step kk: tokens 16 kk .. 16 kk + 15; `partial` masks absent tokens
+      auto pv_step = [&](int kk, uint32_t km, auto partial) {
+        const uint32_t b01 = lds32(prow + 16 * kk + 2 * t);
+        const uint32_t b23 = lds32(prow + 16 * kk + 2 * t + 8);
+        const uint8_t* sr = vsb + (16 * kk + 2 * t) * SROW_BYTES + 4 * warp;  // cells 2w, 2w+1
+        uint32_t s0 = lds32(sr), s1 = lds32(sr + SROW_BYTES), s2 = lds32(sr + 8 * SROW_BYTES),
+                 s3 = lds32(sr + 9 * SROW_BYTES);
+        if constexpr (decltype(partial)::value) {  // a stale slot may hold any bit pattern
+          s0 = ((km >> (2 * t)) & 1u) ? s0 : 0u;
+          s1 = ((km >> (2 * t + 1)) & 1u) ? s1 : 0u;
+          s2 = ((km >> (2 * t + 8)) & 1u) ? s2 : 0u;
+          s3 = ((km >> (2 * t + 9)) & 1u) ? s3 : 0u;
+        }
+        uint32_t vw[4];
+        ldsm_x4_trans(vbase + (uint32_t)(16 * kk * ROW_BYTES), vw);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t sel = c ? 0x7632u : 0x5410u;
+          const uint32_t b01c = h2_as_u32(__hmul2(u32_as_h2(b01), u32_as_h2(__byte_perm(s0, s1, sel))));
+          const uint32_t b23c = h2_as_u32(__hmul2(u32_as_h2(b23), u32_as_h2(__byte_perm(s2, s3, sel))));
+          const uint32_t za = vw[2 * c], zb = vw[2 * c + 1];
+          const uint32_t za8 = za >> 8, zb8 = zb >> 8;
+          mma_f16(acc[c][0], za & LO4, za & HI4, zb & LO4, zb & HI4, b01c, b23c);
+          mma_f16(acc[c][1], za8 & LO4, za8 & HI4, zb8 & LO4, zb8 & HI4, b01c, b23c);
+        }
+      };
+      if (smask == ~0ull) {
+#pragma unroll
+        for (int kk = 0; kk < STAGE_TOK / 16; ++kk) pv_step(kk, 0xffffu, std::false_type{});
       } else {
-        sc[0] = sc[1] = sc[2] = sc[3] = -INFINITY;
+#pragma unroll
+        for (int kk = 0; kk < STAGE_TOK / 16; ++kk) {
+          const uint32_t km = (uint32_t)(smask >> (16 * kk)) & 0xffffu;
+          if (km != 0u) pv_step(kk, km, std::true_type{});
+        }
       }
-
-      // ---- online softmax in base 2 (per head g; lanes of one g agree)
-      float mt = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-      mt = fmaxf(mt, __shfl_xor_sync(FULL_MASK, mt, 1));
-      mt = fmaxf(mt, __shfl_xor_sync(FULL_MASK, mt, 2));
-      const float m_new = fmaxf(m_run, mt);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = (g < G) ? ex2(m_run - m_use) : 1.f;
-      float pr[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) pr[i] = ex2(sc[i] - m_use);
-      l_run = l_run * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-      m_run = m_new;
-      const float al0 = __shfl_sync(FULL_MASK, alpha, (8 * t) & 31);
-      const float al1 = __shfl_sync(FULL_MASK, alpha, (8 * t + 4) & 31);
-      if (__any_sync(FULL_MASK, alpha != 1.f)) {
-#pragma unroll
-        for (int c = 0; c < CELLS; ++c)
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            acc[c][k][0] *= al0; acc[c][k][1] *= al1;
-            acc[c][k][2] *= al0; acc[c][k][3] *= al1;
-          }
-        vsum[0] *= al0;
-        vsum[1] *= al1;
-      }
-
-      // ---- P V with the V scale folded into P per cell (packed fp16). The V
-      // nibbles enter raw, as fp16 subnormals (n * 2^-24 on MMA rows 0-7,
-      // n * 2^-20 on rows 8-15); the -8 offset is accounted for once per
-      // tile by vsum += S_v^T P (cell x head), applied in the epilogue.
-      const __half2 p01 = __floats2half2_rn(pr[0], pr[1]), p23 = __floats2half2_rn(pr[2], pr[3]);
-      const uint32_t s0w[4] = {sv0.x, sv0.y, sv0.z, sv0.w}, s1w[4] = {sv1.x, sv1.y, sv1.z, sv1.w};
-      const uint32_t s2w[4] = {sv2.x, sv2.y, sv2.z, sv2.w}, s3w[4] = {sv3.x, sv3.y, sv3.z, sv3.w};
-      {
-        // A = the tile's V scales transposed: row = cell g, k = tokens 2t, 2t+1 (+8)
+      // The -8 offset: this warp sums p * v_scale over its own k-step (tokens
+      // 16w .. 16w + 15) for every cell; the warps' sums add up at the end.
+      if (wmask != 0u) {
+        const uint32_t b01 = lds32(prow + 16 * warp + 2 * t);
+        const uint32_t b23 = lds32(prow + 16 * warp + 2 * t + 8);
+        // A: the V scales transposed, row = cell g, k = tokens
         uint32_t st0, st1;
-        ldsm_x2_trans(smem_u32(vsb) + (uint32_t)((lane & 15) * SROW_BYTES), st0, st1);
-        if (partial) {  // absent tokens: a stale slot may hold any bit pattern
-          st0 &= (((tmask >> (2 * t)) & 1u) ? 0x0000ffffu : 0u) | (((tmask >> (2 * t + 1)) & 1u) ? 0xffff0000u : 0u);
-          st1 &= (((tmask >> (2 * t + 8)) & 1u) ? 0x0000ffffu : 0u) | (((tmask >> (2 * t + 9)) & 1u) ? 0xffff0000u : 0u);
+        ldsm_x2_trans(smem_u32(vsb) + (uint32_t)((16 * warp + (lane & 15)) * SROW_BYTES), st0, st1);
+        if (wmask != 0xffffu) {
+          st0 &= (((wmask >> (2 * t)) & 1u) ? 0x0000ffffu : 0u) | (((wmask >> (2 * t + 1)) & 1u) ? 0xffff0000u : 0u);
+          st1 &= (((wmask >> (2 * t + 8)) & 1u) ? 0x0000ffffu : 0u) |
+                 (((wmask >> (2 * t + 9)) & 1u) ? 0xffff0000u : 0u);
         }
         float dd[4];
-        mma_f16_c(dd, st0, 0u, st1, 0u, h2_as_u32(p01), h2_as_u32(p23), vsum[0], vsum[1], 0.f, 0.f);
+        mma_f16_c(dd, st0, 0u, st1, 0u, b01, b23, vsum[0], vsum[1], 0.f, 0.f);
         vsum[0] = dd[0];
         vsum[1] = dd[1];
       }
-      uint32_t vw[2][4];
-#pragma unroll
-      for (int c = 0; c < CELLS; ++c) {
-        if ((c & 1) == 0) ldsm_x4_trans(vbase + ld_off[c >> 1], vw[(c >> 1) & 1]);
-        const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;
-        const uint32_t b01 = h2_as_u32(__hmul2(p01, u32_as_h2(__byte_perm(s0w[c >> 1], s1w[c >> 1], sel))));
-        const uint32_t b23 = h2_as_u32(__hmul2(p23, u32_as_h2(__byte_perm(s2w[c >> 1], s3w[c >> 1], sel))));
-        const uint32_t za = vw[(c >> 1) & 1][2 * (c & 1)], zb = vw[(c >> 1) & 1][2 * (c & 1) + 1];
-        const uint32_t za8 = za >> 8, zb8 = zb >> 8;
-        mma_f16(acc[c][0], za & 0x000F000Fu, za & 0x00F000F0u, zb & 0x000F000Fu, zb & 0x00F000F0u, b01, b23);
-        mma_f16(acc[c][1], za8 & 0x000F000Fu, za8 & 0x00F000F0u, zb8 & 0x000F000Fu, zb8 & 0x00F000F0u, b01, b23);
-      }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.empty[st]);
-    // The slot of the previous iteration (all warps have normally left it by
-    // now) is refilled NS - 1 iterations ahead of its use, by its own warp.
-    if (it >= 1 && it - 1 + NS < n_it && ((it - 1 + NS) % CWARPS) == warp) {
-      const int pv = it - 1;
-      int go = 1;
-      if (lane == 0) {
-        if (*abort_flag) {
-          go = 0;
-        } else if (!mbar_wait_bounded(&sm.empty[pv % NS], (pv / NS) & 1)) {
-          flag(p.status, QKV_DEV_TIMEOUT);
-          *abort_flag = 1;
-          go = 0;
-        }
-      }
-      if (__shfl_sync(FULL_MASK, go, 0)) issue(pv + NS);
+    if (++st == NSK) {
+      st = 0;
+      ph ^= 1u;
+    }
+    if (++vst == NSV) {
+      vst = 0;
+      vph ^= 1u;
     }
   }
 
-  // ------------------------------------------------------------ combine the 4 warps
-  l_run += __shfl_xor_sync(FULL_MASK, l_run, 1);
-  l_run += __shfl_xor_sync(FULL_MASK, l_run, 2);
-  if (t == 0 && g < G) {
-    sm.wm[warp][g] = m_run;
-    sm.wl[warp][g] = l_run;
+  // ------------------------------------------------------------ epilogue
+#pragma unroll
+  for (int hq = 0; hq < HQ; ++hq) {
+    float l = l_run[hq];
+    l += __shfl_xor_sync(FULL_MASK, l, 4);
+    l += __shfl_xor_sync(FULL_MASK, l, 8);
+    l += __shfl_xor_sync(FULL_MASK, l, 16);
+    if (g == 0) sm.wl[warp][4 * hq + t] = l;
   }
   __syncthreads();
   if (*abort_flag) {
     // Leave only after every copy issued here has landed.
     if (threadIdx.x == 0) {
       const int issued = sm.issued;
-      for (int it = max(0, issued - NS); it < issued; ++it)
-        if (!mbar_wait_bounded(&sm.full[it % NS], (it / NS) & 1)) flag(p.status, QKV_DEV_TIMEOUT);
+      for (int r = max(0, issued - NSK); r < issued; ++r)
+        if (!mbar_wait_bounded(&sm.kfull[r % NSK], (r / NSK) & 1)) flag(p.status, QKV_DEV_TIMEOUT);
+      for (int r = max(0, issued - NSV); r < issued; ++r)
+        if (!mbar_wait_bounded(&sm.vfull[r % NSV], (r / NSV) & 1)) flag(p.status, QKV_DEV_TIMEOUT);
     }
     if (threadIdx.x < G) lse_out[threadIdx.x] = -INFINITY;
     return;
   }
-  // Each warp scales its accumulator to the CTA-wide max and parks it in
-  // the (now idle) K ring: slab[warp][head][dim].
-  float* slab = reinterpret_cast<float*>(&sm.k[0][0]);
-  float fw[2] = {0.f, 0.f};
+  // the warps' offset sums, parked in the (now idle) K ring: [warp][lane][2]
+  float2* vsp = reinterpret_cast<float2*>(&sm.k[0][0]);
+  vsp[warp * 32 + lane] = make_float2(vsum[0], vsum[1]);
+  __syncthreads();
+  float inv[2];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
     const int h = 2 * t + j;
-    if (h < G) {
-      float M = -INFINITY;
+    float Ls = 0.f;
+    if (h < G)
 #pragma unroll
-      for (int w = 0; w < CWARPS; ++w) M = fmaxf(M, sm.wm[w][h]);
-      fw[j] = (M == -INFINITY) ? 0.f : exp2f(sm.wm[warp][h] - M);
-    }
+      for (int w = 0; w < CWARPS; ++w) Ls += sm.wl[w][h];
+    inv[j] = Ls > 0.f ? 1.f / Ls : 0.f;
   }
   // Undo the subnormal encoding of V: rows 0-7 carry 2^-24 * sum(n p s),
   // rows 8-15 2^-20 * sum(n p s); the -8 offset is 8 * sum(p s) per cell.
 #pragma unroll
-  for (int c = 0; c < CELLS; ++c) {
-    const float b0 = 8.f * __shfl_sync(FULL_MASK, vsum[0], 4 * c + t);
-    const float b1 = 8.f * __shfl_sync(FULL_MASK, vsum[1], 4 * c + t);
+  for (int c = 0; c < 2; ++c) {
+    const int cell = 2 * warp + c;
+    float b0 = 0.f, b1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < CWARPS; ++w) {
+      const float2 v = vsp[w * 32 + 4 * cell + t];
+      b0 += v.x;
+      b1 += v.y;
+    }
+    b0 *= 8.f;
+    b1 *= 8.f;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       acc[c][k][0] = fmaf(acc[c][k][0], 16777216.f, -b0);
@@ -580,36 +729,26 @@ __global__ void __launch_bounds__(THREADS, 3)
   for (int j = 0; j < 2; ++j) {
     const int h = 2 * t + j;
     if (h < G) {
-      float* dst = slab + ((size_t)warp * 8 + h) * D;
+      float* dst = p.o_parts + ((size_t)split * rows + row0 + h) * D + 4 * g;
 #pragma unroll
-      for (int c = 0; c < CELLS; ++c) {
-        const float4 o = make_float4(fw[j] * acc[c][0][j], fw[j] * acc[c][0][j + 2], fw[j] * acc[c][1][j],
-                                     fw[j] * acc[c][1][j + 2]);
-        *reinterpret_cast<float4*>(dst + 32 * c + 4 * g) = o;
+      for (int c = 0; c < 2; ++c) {
+        const float4 o = make_float4(inv[j] * acc[c][0][j], inv[j] * acc[c][0][j + 2], inv[j] * acc[c][1][j],
+                                     inv[j] * acc[c][1][j + 2]);
+        *reinterpret_cast<float4*>(dst + 32 * (2 * warp + c)) = o;
       }
     }
   }
-  __syncthreads();
-  // Sum the warps, normalise, write the partial of this split.
-  const int tid = threadIdx.x;  // 0 .. 127
-  for (int e = tid; e < G * (D / 4); e += CWARPS * 32) {
-    const int h = e / (D / 4), d4 = e % (D / 4);
-    float M = -INFINITY;
+  if (warp == 0 && g == 0) {
 #pragma unroll
-    for (int w = 0; w < CWARPS; ++w) M = fmaxf(M, sm.wm[w][h]);
-    float Lsum = 0.f;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int hq = 0; hq < HQ; ++hq) {
+      const int h = 4 * hq + t;
+      if (h < G) {
+        float Ls = 0.f;
 #pragma unroll
-    for (int w = 0; w < CWARPS; ++w) {
-      const float f = (M == -INFINITY) ? 0.f : exp2f(sm.wm[w][h] - M);
-      Lsum += f * sm.wl[w][h];
-      const float4 x = *reinterpret_cast<const float4*>(slab + ((size_t)w * 8 + h) * D + 4 * d4);
-      o.x += x.x; o.y += x.y; o.z += x.z; o.w += x.w;
+        for (int w = 0; w < CWARPS; ++w) Ls += sm.wl[w][h];
+        lse_out[h] = Ls > 0.f ? m_ref[hq] + log2f(Ls) : -INFINITY;
+      }
     }
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    o.x *= inv; o.y *= inv; o.z *= inv; o.w *= inv;
-    *reinterpret_cast<float4*>(p.o_parts + ((size_t)split * rows + row0 + h) * D + 4 * d4) = o;
-    if (d4 == 0) lse_out[h] = Lsum > 0.f ? M + log2f(Lsum) : -INFINITY;
   }
 }
 
@@ -655,6 +794,8 @@ const void* kernel_ptr() {
   return reinterpret_cast<const void*>(&paged_decode_split_kernel<BLOCK, G>);
 }
 
+size_t kernel_smem(int G) { return G > 4 ? smem_bytes<2>() : smem_bytes<1>(); }
+
 const void* pick_kernel(int block, int G) {
 #define QKV_PICK(B)                         \
   if (block == B) {                         \
@@ -683,10 +824,11 @@ int prepare(const void* fn, int block, int G) {
   const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
   std::lock_guard<std::mutex> lock(mu);
   if (occ[dev][bi][gi] == 0) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) != cudaSuccess)
+    const size_t smem = kernel_smem(G);
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return 0;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, THREADS, SMEM_BYTES) != cudaSuccess || n < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, THREADS, smem) != cudaSuccess || n < 1)
       return 0;
     occ[dev][bi][gi] = n;
   }
@@ -781,7 +923,7 @@ extern "C" int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int3
   // covers every slot the merge reads.
   dim3 grid((unsigned)max_splits, (unsigned)n_seq, (unsigned)kv_heads);
   void* args[] = {(void*)&tm_k, (void*)&tm_v, (void*)&p};
-  if (launch_pdl(fn, grid, dim3(THREADS), SMEM_BYTES, stream, args) != cudaSuccess) {
+  if (launch_pdl(fn, grid, dim3(THREADS), kernel_smem(G), stream, args) != cudaSuccess) {
     (void)cudaGetLastError();
     return QKV_ECUDA;
   }

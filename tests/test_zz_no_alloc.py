@@ -74,10 +74,10 @@ def test_static_scratch_refuses_oversize(qkv):
     w = workloads.small("noalloc_big", seq_lens=(64,) * 4, num_pages=8, block_size=64)
     x, cache = _inputs(qkv, w)
     out, lse = _outputs(w)
-    need = qkv.qkv_paged_decode_workspace_bytes(w.n_seq, w.q_heads, w.head_dim, 200)
+    need = qkv.qkv_paged_decode_workspace_bytes(w.n_seq, w.q_heads, w.head_dim, 400)
     assert need > qkv.STATIC_SCRATCH_BYTES
     with pytest.raises(qkv.QkvError) as e:
         qkv.qkv_paged_decode_attn_f4_static(out, to_dev(x["q"]), cache.k_data, cache.k_scale, cache.v_data,
                                             cache.v_scale, to_dev(x["page_table"]), to_dev(x["seq_lens"]),
-                                            w.kv_heads, num_splits=200)
+                                            w.kv_heads, num_splits=400)
     assert e.value.code == 1
