@@ -469,55 +469,110 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
   const uint32_t voff = (uint32_t)((8 * ((lane >> 3) & 1) + sw) * ROW_BYTES) +
                         ((uint32_t)((2 * warp + (lane >> 4)) ^ sw) << 4);
   bool aborted = false;
-  int st = 0, vst = 0;           // K and V slots of stage it
-  uint32_t ph = 0, vph = 0;      // their phase parities
+  float sg[HQ], sg8[HQ];  // raw scores of tokens g, g + 8 of the warp's 16 (head 4 hq + t)
 
-  for (int it = 0; it < n_it; ++it) {
-    // ---------------- scores of the warp's 16 tokens
-    // (aborted is warp-uniform, so the .aligned ldmatrix / mma below see a
-    // converged warp)
-    aborted = __any_sync(FULL_MASK, aborted || !wait_copies(&sm.kfull[st], ph, abort_flag, p.status));
-    const unsigned long long smask = aborted ? 0ull : sm.mask[st];
-    const uint32_t wmask = (uint32_t)(smask >> (16 * warp)) & 0xffffu;
-    float sg[HQ], sg8[HQ];
+  // Q K^T of the warp's 16 tokens of the stage in K slot `ks`.
+  auto qk_math = [&](int ks) {
+    const uint32_t kbase = smem_u32(&sm.k[ks][0]);
+    const uint8_t* ksb = &sm.ks[ks][16 * warp * SROW_BYTES];
+    const uint4 skA = lds128(ksb + g * SROW_BYTES);
+    const uint4 skB = lds128(ksb + (g + 8) * SROW_BYTES);
+    const uint32_t sa[4] = {skA.x, skA.y, skA.z, skA.w}, sb[4] = {skB.x, skB.y, skB.z, skB.w};
 #pragma unroll
-    for (int hq = 0; hq < HQ; ++hq) sg[hq] = sg8[hq] = 0.f;
-    if (wmask != 0u) {
-      const uint32_t kbase = smem_u32(&sm.k[st][0]);
-      const uint8_t* ksb = &sm.ks[st][16 * warp * SROW_BYTES];
-      const uint4 skA = lds128(ksb + g * SROW_BYTES);
-      const uint4 skB = lds128(ksb + (g + 8) * SROW_BYTES);
-      const uint32_t sa[4] = {skA.x, skA.y, skA.z, skA.w}, sb[4] = {skB.x, skB.y, skB.z, skB.w};
+    for (int pp = 0; pp < PAIRS; ++pp) {
+      uint32_t kw[4];
+      ldsm_x4(kbase + koff[pp], kw);  // tok g / g+8 of cell 2pp, then of cell 2pp+1
+      uint32_t kh[4];
 #pragma unroll
-      for (int pp = 0; pp < PAIRS; ++pp) {
-        uint32_t kw[4];
-        ldsm_x4(kbase + koff[pp], kw);  // tok g / g+8 of cell 2pp, then of cell 2pp+1
-        uint32_t kh[4];
+      for (int i = 0; i < 4; ++i) kh[i] = kw[i] >> 8;
+      const float2 fa = __half22float2(u32_as_h2(sa[pp])), fb = __half22float2(u32_as_h2(sb[pp]));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) kh[i] = kw[i] >> 8;
-        const float2 fa = __half22float2(u32_as_h2(sa[pp])), fb = __half22float2(u32_as_h2(sb[pp]));
-#pragma unroll
-        for (int hq = 0; hq < HQ; ++hq) {
-          const uint4 qa = sm.qfrag[hq][pp][0][lane], qb = sm.qfrag[hq][pp][1][lane];
-          const float4 bias = sm.qbias[hq][pp][t];
-          float d[4];
-          mma_f16_c(d, kw[0] & LO4, kw[1] & LO4, kw[2] & LO4, kw[3] & LO4, qa.x, qa.y, bias.x, bias.y, bias.z,
-                    bias.w);
-          mma_f16(d, kw[0] & HI4, kw[1] & HI4, kw[2] & HI4, kw[3] & HI4, qa.z, qa.w);
-          mma_f16(d, kh[0] & LO4, kh[1] & LO4, kh[2] & LO4, kh[3] & LO4, qb.x, qb.y);
-          mma_f16(d, kh[0] & HI4, kh[1] & HI4, kh[2] & HI4, kh[3] & HI4, qb.z, qb.w);
-          // columns 2t (even cell) and 2t+1 (odd cell) of head t
-          sg[hq] = fmaf(fa.x, d[0], sg[hq]);
-          sg[hq] = fmaf(fa.y, d[1], sg[hq]);
-          sg8[hq] = fmaf(fb.x, d[2], sg8[hq]);
-          sg8[hq] = fmaf(fb.y, d[3], sg8[hq]);
-        }
+      for (int hq = 0; hq < HQ; ++hq) {
+        const uint4 qa = sm.qfrag[hq][pp][0][lane], qb = sm.qfrag[hq][pp][1][lane];
+        const float4 bias = sm.qbias[hq][pp][t];
+        float d[4];
+        mma_f16_c(d, kw[0] & LO4, kw[1] & LO4, kw[2] & LO4, kw[3] & LO4, qa.x, qa.y, bias.x, bias.y, bias.z,
+                  bias.w);
+        mma_f16(d, kw[0] & HI4, kw[1] & HI4, kw[2] & HI4, kw[3] & HI4, qa.z, qa.w);
+        mma_f16(d, kh[0] & LO4, kh[1] & LO4, kh[2] & LO4, kh[3] & LO4, qb.x, qb.y);
+        mma_f16(d, kh[0] & HI4, kh[1] & HI4, kh[2] & HI4, kh[3] & HI4, qb.z, qb.w);
+        // columns 2t (even cell) and 2t+1 (odd cell) of head t
+        sg[hq] = fmaf(fa.x, d[0], sg[hq]);
+        sg[hq] = fmaf(fa.y, d[1], sg[hq]);
+        sg8[hq] = fmaf(fb.x, d[2], sg8[hq]);
+        sg8[hq] = fmaf(fb.y, d[3], sg8[hq]);
       }
     }
-    const bool okA = (wmask >> g) & 1u, okB = (wmask >> (g + 8)) & 1u;
+  };
 
-    // ---------------- probabilities against the CTA's running max
-    const int pb = it & 1;
+  // P V of the 64 tokens of the stage in V slot `vs` (probabilities in
+  // buffer `pb`) into the dims of cells 2w, 2w+1; `partial` masks absent
+  // tokens of `smask` (a stale slot may hold any bit pattern).
+  auto pv_math = [&](int vs, int pb, unsigned long long smask, auto partial) {
+    const uint32_t vbase = smem_u32(&sm.v[vs][0]) + voff;
+    const uint8_t* vsb = &sm.vs[vs][0];
+    const uint16_t* prow = &sm.prob[pb][g][0];
+    auto pv_step = [&](int kk, uint32_t km) {
+      const uint32_t b01 = lds32(prow + 16 * kk + 2 * t);
+      const uint32_t b23 = lds32(prow + 16 * kk + 2 * t + 8);
+      const uint8_t* sr = vsb + (16 * kk + 2 * t) * SROW_BYTES + 4 * warp;  // cells 2w, 2w+1
+      uint32_t s0 = lds32(sr), s1 = lds32(sr + SROW_BYTES), s2 = lds32(sr + 8 * SROW_BYTES),
+               s3 = lds32(sr + 9 * SROW_BYTES);
+      if constexpr (decltype(partial)::value) {
+        s0 = ((km >> (2 * t)) & 1u) ? s0 : 0u;
+        s1 = ((km >> (2 * t + 1)) & 1u) ? s1 : 0u;
+        s2 = ((km >> (2 * t + 8)) & 1u) ? s2 : 0u;
+        s3 = ((km >> (2 * t + 9)) & 1u) ? s3 : 0u;
+      }
+      uint32_t vw[4];
+      ldsm_x4_trans(vbase + (uint32_t)(16 * kk * ROW_BYTES), vw);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const uint32_t sel = c ? 0x7632u : 0x5410u;
+        const uint32_t b01c = h2_as_u32(__hmul2(u32_as_h2(b01), u32_as_h2(__byte_perm(s0, s1, sel))));
+        const uint32_t b23c = h2_as_u32(__hmul2(u32_as_h2(b23), u32_as_h2(__byte_perm(s2, s3, sel))));
+        const uint32_t za = vw[2 * c], zb = vw[2 * c + 1];
+        const uint32_t za8 = za >> 8, zb8 = zb >> 8;
+        mma_f16(acc[c][0], za & LO4, za & HI4, zb & LO4, zb & HI4, b01c, b23c);
+        mma_f16(acc[c][1], za8 & LO4, za8 & HI4, zb8 & LO4, zb8 & HI4, b01c, b23c);
+      }
+    };
+    if constexpr (decltype(partial)::value) {
+#pragma unroll
+      for (int kk = 0; kk < STAGE_TOK / 16; ++kk) {
+        const uint32_t km = (uint32_t)(smask >> (16 * kk)) & 0xffffu;
+        if (km != 0u) pv_step(kk, km);
+      }
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < STAGE_TOK / 16; ++kk) pv_step(kk, 0xffffu);
+    }
+    // The -8 offset: this warp sums p * v_scale over its own k-step (tokens
+    // 16w .. 16w + 15) for every cell; the warps' sums add up at the end.
+    const uint32_t wm = (uint32_t)(smask >> (16 * warp)) & 0xffffu;
+    if (!decltype(partial)::value || wm != 0u) {
+      const uint32_t b01 = lds32(prow + 16 * warp + 2 * t);
+      const uint32_t b23 = lds32(prow + 16 * warp + 2 * t + 8);
+      // A: the V scales transposed, row = cell g, k = tokens
+      uint32_t st0, st1;
+      ldsm_x2_trans(smem_u32(vsb) + (uint32_t)((16 * warp + (lane & 15)) * SROW_BYTES), st0, st1);
+      if constexpr (decltype(partial)::value) {
+        st0 &= (((wm >> (2 * t)) & 1u) ? 0x0000ffffu : 0u) | (((wm >> (2 * t + 1)) & 1u) ? 0xffff0000u : 0u);
+        st1 &= (((wm >> (2 * t + 8)) & 1u) ? 0x0000ffffu : 0u) | (((wm >> (2 * t + 9)) & 1u) ? 0xffff0000u : 0u);
+      }
+      float dd[4];
+      mma_f16_c(dd, st0, 0u, st1, 0u, b01, b23, vsum[0], vsum[1], 0.f, 0.f);
+      vsum[0] = dd[0];
+      vsum[1] = dd[1];
+    }
+  };
+
+  // Probabilities of the scored stage (its tokens in wm) against the CTA's
+  // running max, written to buffer pb; then the CTA barrier that publishes
+  // them. All warps are then past Q K^T of that stage and P V of the one
+  // before it.
+  auto publish = [&](int pb, uint32_t wm) {
+    const bool okA = (wm >> g) & 1u, okB = (wm >> (g + 8)) & 1u;
     float xA[HQ], xB[HQ], psum[HQ];
     bool need = false;
 #pragma unroll
@@ -532,10 +587,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
       pr[0] = __half_as_ushort(__float2half_rn(pA));
       pr[8] = __half_as_ushort(__float2half_rn(pB));
     }
-    // All warps are done with K of this stage and with V of the previous
-    // one; the probabilities of this stage are published.
-    const bool any_new_max = bar_red_or(need);
-    if (any_new_max) {
+    if (bar_red_or(need)) {
       // Some head's running max moves: exchange the tile maxima, rescale.
 #pragma unroll
       for (int hq = 0; hq < HQ; ++hq) {
@@ -590,76 +642,61 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
 #pragma unroll
       for (int hq = 0; hq < HQ; ++hq) l_run[hq] += psum[hq];
     }
+  };
 
-    // ---------------- refill: K of stage it + 2 (slot of stage it), V of stage it + 1
-    // K of stage it + 2 goes to the K slot of stage it, V to the slot of
-    // stage it - 1: all warps are past both.
-    if (!aborted && it + 2 < n_it && ((it + 2) % CWARPS) == warp) issue(it + 2);
-
-    // ---------------- P V over the stage's 64 tokens, dims of cells 2w, 2w+1
-    if (!aborted) aborted = __any_sync(FULL_MASK, !wait_copies(&sm.vfull[vst], vph, abort_flag, p.status));
-    if (!aborted && smask != 0ull) {
-      const uint32_t vbase = smem_u32(&sm.v[vst][0]) + voff;
-      const uint8_t* vsb = &sm.vs[vst][0];
-      const uint16_t* prow = &sm.prob[pb][g][0];
-      // k-step kk: tokens 16 kk .. 16 kk + 15; `partial` masks absent tokens
-      auto pv_step = [&](int kk, uint32_t km, auto partial) {
-        const uint32_t b01 = lds32(prow + 16 * kk + 2 * t);
-        const uint32_t b23 = lds32(prow + 16 * kk + 2 * t + 8);
-        const uint8_t* sr = vsb + (16 * kk + 2 * t) * SROW_BYTES + 4 * warp;  // cells 2w, 2w+1
-        uint32_t s0 = lds32(sr), s1 = lds32(sr + SROW_BYTES), s2 = lds32(sr + 8 * SROW_BYTES),
-                 s3 = lds32(sr + 9 * SROW_BYTES);
-        if constexpr (decltype(partial)::value) {  // a stale slot may hold any bit pattern
-          s0 = ((km >> (2 * t)) & 1u) ? s0 : 0u;
-          s1 = ((km >> (2 * t + 1)) & 1u) ? s1 : 0u;
-          s2 = ((km >> (2 * t + 8)) & 1u) ? s2 : 0u;
-          s3 = ((km >> (2 * t + 9)) & 1u) ? s3 : 0u;
-        }
-        uint32_t vw[4];
-        ldsm_x4_trans(vbase + (uint32_t)(16 * kk * ROW_BYTES), vw);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint32_t sel = c ? 0x7632u : 0x5410u;
-          const uint32_t b01c = h2_as_u32(__hmul2(u32_as_h2(b01), u32_as_h2(__byte_perm(s0, s1, sel))));
-          const uint32_t b23c = h2_as_u32(__hmul2(u32_as_h2(b23), u32_as_h2(__byte_perm(s2, s3, sel))));
-          const uint32_t za = vw[2 * c], zb = vw[2 * c + 1];
-          const uint32_t za8 = za >> 8, zb8 = zb >> 8;
-          mma_f16(acc[c][0], za & LO4, za & HI4, zb & LO4, zb & HI4, b01c, b23c);
-          mma_f16(acc[c][1], za8 & LO4, za8 & HI4, zb8 & LO4, zb8 & HI4, b01c, b23c);
-        }
-      };
-      if (smask == ~0ull) {
-#pragma unroll
-        for (int kk = 0; kk < STAGE_TOK / 16; ++kk) pv_step(kk, 0xffffu, std::false_type{});
-      } else {
-#pragma unroll
-        for (int kk = 0; kk < STAGE_TOK / 16; ++kk) {
-          const uint32_t km = (uint32_t)(smask >> (16 * kk)) & 0xffffu;
-          if (km != 0u) pv_step(kk, km, std::true_type{});
-        }
-      }
-      // The -8 offset: this warp sums p * v_scale over its own k-step (tokens
-      // 16w .. 16w + 15) for every cell; the warps' sums add up at the end.
-      if (wmask != 0u) {
-        const uint32_t b01 = lds32(prow + 16 * warp + 2 * t);
-        const uint32_t b23 = lds32(prow + 16 * warp + 2 * t + 8);
-        // A: the V scales transposed, row = cell g, k = tokens
-        uint32_t st0, st1;
-        ldsm_x2_trans(smem_u32(vsb) + (uint32_t)((16 * warp + (lane & 15)) * SROW_BYTES), st0, st1);
-        if (wmask != 0xffffu) {
-          st0 &= (((wmask >> (2 * t)) & 1u) ? 0x0000ffffu : 0u) | (((wmask >> (2 * t + 1)) & 1u) ? 0xffff0000u : 0u);
-          st1 &= (((wmask >> (2 * t + 8)) & 1u) ? 0x0000ffffu : 0u) |
-                 (((wmask >> (2 * t + 9)) & 1u) ? 0xffff0000u : 0u);
-        }
-        float dd[4];
-        mma_f16_c(dd, st0, 0u, st1, 0u, b01, b23, vsum[0], vsum[1], 0.f, 0.f);
-        vsum[0] = dd[0];
-        vsum[1] = dd[1];
-      }
+  // Software pipeline: iteration `it` multiplies stage it into the
+  // accumulators and scores stage it + 1, so the two run as one straight
+  // block on full stages; the CTA barrier sits between the scoring and the
+  // P V of each stage. Stage s + 2 is issued at the barrier of stage s.
+  int kst = 0, vst = 0;       // K slot of the next stage to score, V slot of stage it
+  uint32_t kph = 0, vph = 0;  // their phase parities
+  unsigned long long smask_n = 0;  // token mask of the next stage to score
+  auto next_k = [&]() {
+    if (++kst == NSK) {
+      kst = 0;
+      kph ^= 1u;
     }
-    if (++st == NSK) {
-      st = 0;
-      ph ^= 1u;
+  };
+  if (n_it > 0) {
+    // (aborted is warp-uniform, so the .aligned ldmatrix / mma see a converged warp)
+    aborted = __any_sync(FULL_MASK, !wait_copies(&sm.kfull[0], 0, abort_flag, p.status));
+    smask_n = aborted ? 0ull : sm.mask[0];
+    const uint32_t wm = (uint32_t)(smask_n >> (16 * warp)) & 0xffffu;
+#pragma unroll
+    for (int hq = 0; hq < HQ; ++hq) sg[hq] = sg8[hq] = 0.f;
+    if (wm != 0u) qk_math(0);
+    publish(0, wm);
+    if (!aborted && 2 < n_it && warp == 2) issue(2);
+    next_k();
+  }
+  for (int it = 0; it < n_it; ++it) {
+    const unsigned long long smask = smask_n;  // stage it
+    const bool nxt = it + 1 < n_it;
+    if (!aborted) {
+      bool ok = wait_copies(&sm.vfull[vst], vph, abort_flag, p.status);
+      if (nxt) ok = ok && wait_copies(&sm.kfull[kst], kph, abort_flag, p.status);
+      aborted = __any_sync(FULL_MASK, !ok);
+    }
+    smask_n = (nxt && !aborted) ? sm.mask[kst] : 0ull;
+    const uint32_t wm_n = (uint32_t)(smask_n >> (16 * warp)) & 0xffffu;
+    const int pb = it & 1;
+#pragma unroll
+    for (int hq = 0; hq < HQ; ++hq) sg[hq] = sg8[hq] = 0.f;
+    if (!aborted && smask == ~0ull && (smask_n == ~0ull || !nxt)) {
+      // full stages: one straight block
+      pv_math(vst, pb, smask, std::false_type{});
+      if (nxt) qk_math(kst);
+    } else {
+      if (!aborted && smask != 0ull) pv_math(vst, pb, smask, std::true_type{});
+      if (wm_n != 0u) qk_math(kst);
+    }
+    if (nxt) {
+      publish(pb ^ 1, wm_n);
+      // K of stage it + 3 replaces stage it + 1 (scored), V replaces stage it
+      // (multiplied); warp-uniform, since the issue shuffles nothing but
+      // loads on every lane.
+      if (!aborted && it + 3 < n_it && ((it + 3) % CWARPS) == warp) issue(it + 3);
+      next_k();
     }
     if (++vst == NSV) {
       vst = 0;
