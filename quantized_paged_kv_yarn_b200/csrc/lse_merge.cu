@@ -13,13 +13,16 @@
 
 namespace qkv {
 
-// One CTA per (row, 128-dim chunk). 16 warps split the parts (warp w takes
-// parts w, w + 16, ...); each lane carries 4 dims, so a warp covers the
-// chunk. A thread issues the loads of all its parts before using them.
+// One CTA per (row, 64-dim chunk); 16 warps split the parts (warp w takes
+// parts w, w + 16, ...). A warp first loads the lse2 of up to 32 of its
+// parts with one load per lane, takes their max and weights, then issues the
+// loads of all those parts' 64-dim rows (2 dims per lane) before using them,
+// so a row costs two dependent global-latency rounds per 32 x 16 parts. The
+// warps' (max, weight sum, weighted sum) are combined in shared memory.
 constexpr int MERGE_WARPS = 16;
 constexpr int MERGE_THREADS = MERGE_WARPS * 32;
-constexpr int MERGE_DIMS = 128;
-constexpr int MERGE_UNROLL = 8;  // parts per warp in flight
+constexpr int MERGE_DIMS = 64;
+constexpr int MERGE_BATCH = 8;  // part rows a lane has in flight at once
 
 __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* __restrict__ o_parts,
                                                                   const float* __restrict__ lse2_parts,
@@ -28,79 +31,83 @@ __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* _
                                                                   float* __restrict__ lse2_out) {
   pdl_wait();
   pdl_release();
-  __shared__ float red[MERGE_WARPS];
-  __shared__ float4 part[MERGE_WARPS][32];
+  __shared__ float wm[MERGE_WARPS], wsum[MERGE_WARPS];
+  __shared__ float2 wacc[MERGE_WARPS][32];
   const int row = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-  // M and the weight sum over all parts
-  float m = -INFINITY;
-  for (int i = tid; i < n_parts; i += MERGE_THREADS) m = fmaxf(m, lse2_parts[(size_t)i * rows + row]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, o));
-  if (lane == 0) red[warp] = m;
-  __syncthreads();
-  float M = red[0];
-#pragma unroll
-  for (int w = 1; w < MERGE_WARPS; ++w) M = fmaxf(M, red[w]);
-  __syncthreads();
-  float ws = 0.f;
-  if (M != -INFINITY)
-    for (int i = tid; i < n_parts; i += MERGE_THREADS) {
-      const float l = lse2_parts[(size_t)i * rows + row];
-      if (l != -INFINITY) ws += exp2f(l - M);
-    }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(FULL_MASK, ws, o);
-  if (lane == 0) red[warp] = ws;
-  __syncthreads();
-  float W = 0.f;
-#pragma unroll
-  for (int w = 0; w < MERGE_WARPS; ++w) W += red[w];
-
-  // weighted sum of this CTA's dims, MERGE_UNROLL parts per warp at a time
-  const int d = blockIdx.y * MERGE_DIMS + 4 * lane;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int d = blockIdx.y * MERGE_DIMS + 2 * lane;
   const bool dim_ok = d < head_dim;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (M != -INFINITY && dim_ok)
-    for (int base = warp; base < n_parts; base += MERGE_WARPS * MERGE_UNROLL) {
-      float lw[MERGE_UNROLL];
-      float4 x[MERGE_UNROLL];
+
+  // running (max, weight sum, weighted sum) of this warp's parts
+  float m = -INFINITY, ws = 0.f;
+  float2 acc = make_float2(0.f, 0.f);
+  for (int base = warp; base < n_parts; base += MERGE_WARPS * 32) {
+    // lane j holds part base + 16 j of this round
+    const int my = base + MERGE_WARPS * lane;
+    const float l = my < n_parts ? lse2_parts[(size_t)my * rows + row] : -INFINITY;
+    float mr = l;
 #pragma unroll
-      for (int u = 0; u < MERGE_UNROLL; ++u) {
-        const int i = base + u * MERGE_WARPS;
-        lw[u] = i < n_parts ? lse2_parts[(size_t)i * rows + row] : -INFINITY;
+    for (int o = 16; o > 0; o >>= 1) mr = fmaxf(mr, __shfl_xor_sync(FULL_MASK, mr, o));
+    if (mr == -INFINITY) continue;  // nothing in this round
+    const float mn = fmaxf(m, mr);
+    const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+    acc.x *= alpha;
+    acc.y *= alpha;
+    ws *= alpha;
+    m = mn;
+    const float wt = (l == -INFINITY) ? 0.f : exp2f(l - m);
+    float wsr = wt;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsr += __shfl_xor_sync(FULL_MASK, wsr, o);
+    ws += wsr;
+    const int cnt = min(32, (n_parts - base + MERGE_WARPS - 1) / MERGE_WARPS);
+    for (int j0 = 0; j0 < cnt; j0 += MERGE_BATCH) {
+      float2 x[MERGE_BATCH];
+      float w[MERGE_BATCH];
+#pragma unroll
+      for (int u = 0; u < MERGE_BATCH; ++u) {
+        const int j = j0 + u;
+        w[u] = __shfl_sync(FULL_MASK, wt, j & 31);
+        x[u] = make_float2(0.f, 0.f);
+        if (j < cnt && w[u] != 0.f && dim_ok)
+          x[u] = *reinterpret_cast<const float2*>(o_parts + ((size_t)(base + MERGE_WARPS * j) * rows + row) * head_dim + d);
       }
 #pragma unroll
-      for (int u = 0; u < MERGE_UNROLL; ++u) {
-        const int i = base + u * MERGE_WARPS;
-        x[u] = (lw[u] != -INFINITY) ? *reinterpret_cast<const float4*>(o_parts + ((size_t)i * rows + row) * head_dim + d)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < MERGE_UNROLL; ++u) {
-        const float w = (lw[u] != -INFINITY) ? exp2f(lw[u] - M) : 0.f;
-        acc.x = fmaf(w, x[u].x, acc.x);
-        acc.y = fmaf(w, x[u].y, acc.y);
-        acc.z = fmaf(w, x[u].z, acc.z);
-        acc.w = fmaf(w, x[u].w, acc.w);
+      for (int u = 0; u < MERGE_BATCH; ++u) {
+        if (j0 + u < cnt) {
+          acc.x = fmaf(w[u], x[u].x, acc.x);
+          acc.y = fmaf(w[u], x[u].y, acc.y);
+        }
       }
     }
-  part[warp][lane] = acc;
+  }
+  if (lane == 0) {
+    wm[warp] = m;
+    wsum[warp] = ws;
+  }
+  wacc[warp][lane] = acc;
   __syncthreads();
-  if (warp == 0 && dim_ok) {
-    float4 s = part[0][lane];
+  if (warp == 0) {
+    float M = -INFINITY;
 #pragma unroll
-    for (int w = 1; w < MERGE_WARPS; ++w) {
-      const float4 x = part[w][lane];
-      s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
+    for (int w = 0; w < MERGE_WARPS; ++w) M = fmaxf(M, wm[w]);
+    float W = 0.f;
+    float2 o = make_float2(0.f, 0.f);
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < MERGE_WARPS; ++w) {
+        const float f = (wm[w] == -INFINITY) ? 0.f : exp2f(wm[w] - M);
+        W = fmaf(f, wsum[w], W);
+        const float2 a = wacc[w][lane];
+        o.x = fmaf(f, a.x, o.x);
+        o.y = fmaf(f, a.y, o.y);
+      }
     }
     const float inv = W > 0.f ? 1.f / W : 0.f;
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + (size_t)row * head_dim + d);
-    dst[0] = __floats2bfloat162_rn(s.x * inv, s.y * inv);
-    dst[1] = __floats2bfloat162_rn(s.z * inv, s.w * inv);
+    if (dim_ok)
+      *reinterpret_cast<__nv_bfloat162*>(out + (size_t)row * head_dim + d) = __floats2bfloat162_rn(o.x * inv, o.y * inv);
+    if (lane == 0 && blockIdx.y == 0 && lse2_out) lse2_out[row] = W > 0.f ? M + log2f(W) : -INFINITY;
   }
-  if (tid == 0 && blockIdx.y == 0 && lse2_out) lse2_out[row] = W > 0.f ? M + log2f(W) : -INFINITY;
 }
 
 }  // namespace qkv
@@ -111,7 +118,7 @@ extern "C" int qkv_lse_merge(const float* o_parts, const float* lse2_parts, int3
                              int32_t head_dim, uint16_t* out, float* lse2_out, qkv_stream_t stream) {
   if (!o_parts || !lse2_parts || !out) return QKV_EINVAL;
   if (n_parts < 1 || rows < 0 || head_dim < 4 || head_dim % 4 || head_dim > 1024) return QKV_EINVAL;
-  if (((uintptr_t)o_parts & 15) || ((uintptr_t)lse2_parts & 3) || ((uintptr_t)out & 7) ||
+  if (((uintptr_t)o_parts & 15) || ((uintptr_t)lse2_parts & 3) || ((uintptr_t)out & 3) ||
       ((uintptr_t)lse2_out & 3))
     return QKV_EINVAL;
   if (rows == 0) return QKV_OK;
