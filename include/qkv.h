@@ -253,7 +253,7 @@ QKV_API int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint1
  * when > 0, else qkv_paged_decode_auto_splits(kv_heads, block_size).
  *   - EINVAL when qkv_paged_decode_workspace_bytes(n_seq, q_heads, head_dim,
  *     splits) exceeds QKV_STATIC_SCRATCH_BYTES (16 query heads of dimension
- *     256 at a B200's automatic 148 splits: up to 6 sequences).
+ *     256 at a B200's automatic 37 splits: up to 27 sequences).
  *   - The first call on a device resolves the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.

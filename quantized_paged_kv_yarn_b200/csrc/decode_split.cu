@@ -64,8 +64,11 @@ constexpr int SROW_BYTES = CELLS * 2;  // 16 bytes of fp16 scales per token
 constexpr int STAGE_TOK = 64;
 constexpr int NSK = 2;                 // K ring depth
 constexpr int NSV = 3;                 // V ring depth (V of a stage is read last)
-constexpr int CWARPS = 4;              // warps
-constexpr int THREADS = CWARPS * 32;
+constexpr int GWARPS = 4;              // warps of a group; a group processes whole stages
+constexpr int GROUPS = 4;              // groups per CTA, sharing the split's stages
+constexpr int GTHREADS = GWARPS * 32;
+constexpr int THREADS = GROUPS * GTHREADS;
+constexpr int INIT = 6;                // a group's first local stages, assigned without claims
 constexpr int PROW = STAGE_TOK + 8;    // padded probability row (fp16): conflict-free B loads
 constexpr uint32_t LO4 = 0x000F000Fu;  // nibble of bits 0-3 of each 16-bit half
 constexpr uint32_t HI4 = 0x00F000F0u;  // nibble of bits 4-7 of each 16-bit half
@@ -79,25 +82,33 @@ constexpr float SLACK = 2.0f;
 template <int G>
 struct Cfg {
   static constexpr int HQ = (G + 3) / 4;
-  static constexpr int MIN_BLOCKS = 4;  // up to 128 registers: no operand shuffling
 };
 
-template <int HQ>
-struct __align__(1024) Smem {
+// One group's rings, probabilities and bookkeeping.
+struct __align__(1024) GroupSmem {
   uint8_t k[NSK][STAGE_TOK * ROW_BYTES];  // 8 KiB each, 1024-aligned (128B swizzle atom)
   uint8_t v[NSV][STAGE_TOK * ROW_BYTES];
   uint8_t ks[NSK][STAGE_TOK * SROW_BYTES];
   uint8_t vs[NSV][STAGE_TOK * SROW_BYTES];
-  uint4 qfrag[HQ][PAIRS][2][32];  // per lane: the B registers of the 4 MMAs of a cell pair
-  uint16_t prob[2][8][PROW];      // fp16 probabilities [stage parity][query head][token]
-  float4 qbias[HQ][PAIRS][4];     // per lane t: chain start of columns 2t, 2t+1 (twice, rows g and g+8)
-  float tmax[CWARPS][8];
-  float wl[CWARPS][8];
+  uint16_t prob[2][8][PROW];  // fp16 probabilities [stage parity][query head][token]
+  float tmax[GWARPS][8];
+  float wl[GWARPS][8];
   unsigned long long mask[NSK];  // tokens present in the stage of each K slot
   uint64_t kfull[NSK];
   uint64_t vfull[NSV];
+  int n_local;  // the group's stage count, once a claim ran past the split
+  int issued;   // local stages issued so far
+};
+
+template <int HQ>
+struct __align__(1024) Smem {
+  GroupSmem grp[GROUPS];
+  uint4 qfrag[HQ][PAIRS][2][32];  // per lane: the B registers of the 4 MMAs of a cell pair
+  float4 qbias[HQ][PAIRS][4];     // per lane t: chain start of columns 2t, 2t+1 (twice, rows g and g+8)
+  float gm[GROUPS][8];            // per group and head: exponent reference of its sums
+  float gl[GROUPS][8];            // per group and head: softmax sum
+  int next;                       // next stage of the split to claim
   int abort_flag;
-  int issued;  // stages issued so far (both halves)
 };
 template <int HQ>
 constexpr size_t smem_bytes() {
@@ -141,21 +152,22 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// CTA barrier 1 over all THREADS threads that also returns the OR of `pred`.
-__device__ __forceinline__ bool bar_red_or(bool pred) {
+// Named barrier `id` over one group's GTHREADS threads that also returns the
+// OR of `pred` over them.
+__device__ __forceinline__ bool bar_red_or(uint32_t id, bool pred) {
   uint32_t out;
   asm volatile(
       "{\n\t.reg .pred pi, po;\n\t"
       "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.or.pred po, 1, %2, pi;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\t"
       "selp.u32 %0, 1, 0, po;\n\t}"
       : "=r"(out)
-      : "r"((uint32_t)pred), "n"(THREADS)
+      : "r"((uint32_t)pred), "r"(id), "n"(GTHREADS)
       : "memory");
   return out != 0;
 }
 
-__device__ __forceinline__ void bar_cta() { asm volatile("bar.sync 1, %0;" ::"n"(THREADS) : "memory"); }
+__device__ __forceinline__ void bar_sync(uint32_t id) { asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(GTHREADS) : "memory"); }
 
 // Wait for phase `parity` of a copy barrier. False when the CTA is aborting
 // (another warp set the flag) or the wait limit ran out (then this sets it).
@@ -235,7 +247,7 @@ __device__ void plan(const Params& p, int seq, int split, int block, int& S, int
 }
 
 template <int BLOCK, int G>
-__global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
+__global__ void __launch_bounds__(THREADS, 1)
     paged_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                               const Params p) {
   static_assert(STAGE_TOK % BLOCK == 0, "pages must tile a stage");
@@ -251,10 +263,12 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
   pdl_release();
   const int split = blockIdx.x, seq = blockIdx.y, kvh = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp / GWARPS, gw = warp % GWARPS;  // group, warp within the group
   const int g = lane >> 2, t = lane & 3;
   const int rows = p.n_seq * p.q_heads;
-  const int row0 = seq * p.q_heads + kvh * G;  // first query-head row of this group
+  const int row0 = seq * p.q_heads + kvh * G;  // first query-head row of this CTA
   float* lse_out = p.lse2_parts + (size_t)split * rows + row0;
+  GroupSmem& gs = sm.grp[grp];
 
   int S, pg0, pg1, L;
   plan(p, seq, split, BLOCK, S, pg0, pg1, L);
@@ -267,47 +281,74 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
   const int n_it = t_end > t_begin ? (t_end - t_begin + STAGE_TOK - 1) / STAGE_TOK : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NSK; ++s) mbar_init(&sm.kfull[s], 1);
-    for (int s = 0; s < NSV; ++s) mbar_init(&sm.vfull[s], 1);
+    for (int q = 0; q < GROUPS; ++q) {
+      for (int s = 0; s < NSK; ++s) mbar_init(&sm.grp[q].kfull[s], 1);
+      for (int s = 0; s < NSV; ++s) mbar_init(&sm.grp[q].vfull[s], 1);
+      // local stages j < INIT of group q are stages q + GROUPS j of the split
+      const int valid = min(INIT, max(0, (n_it - q + GROUPS - 1) / GROUPS));
+      sm.grp[q].n_local = valid < INIT ? valid : 0x7fffffff;
+      sm.grp[q].issued = 0;
+    }
+    sm.next = GROUPS * INIT;
     sm.abort_flag = 0;
-    sm.issued = 0;
     fence_barrier_init();
   }
   // probability rows of absent query heads (G < 8) are read as zeros
-  for (int i = threadIdx.x; i < (int)(sizeof(sm.prob) / 4); i += THREADS)
-    reinterpret_cast<uint32_t*>(&sm.prob[0][0][0])[i] = 0u;
+  for (int i = threadIdx.x % GTHREADS; i < (int)(sizeof(gs.prob) / 4); i += GTHREADS)
+    reinterpret_cast<uint32_t*>(&gs.prob[0][0][0])[i] = 0u;
   __syncthreads();
 
   // ------------------------------------------------------------ copy issue
-  // Stage R holds tokens t_begin + 64 R ... + 63, i.e. 64 / BLOCK pages. Its
-  // K half (rows by TMA, scales by bulk copy) completes on kfull[R % NSK],
-  // its V half on vfull[R % NSV]. Stage R belongs to warp R % 4, which issues
-  // both halves at once; each warp holds the page ids of its next stage,
-  // loaded one of its stages ahead, so no copy waits on the page table.
+  // Stage R of the split holds tokens t_begin + 64 R ... + 63, i.e. 64 /
+  // BLOCK pages. The four groups share the split's stages dynamically: a
+  // group's local stage j is stage grp + 4 j for j < INIT, then whatever the
+  // next claim on the CTA's counter returns, claimed in order, so a group
+  // that runs faster takes more stages and all groups finish together. Local
+  // stage j belongs to warp j % 4 of the group, which claims it four of its
+  // stages ahead (with its page ids) and issues both halves of it (K rows and
+  // scales on kfull[j % NSK], V on vfull[j % NSV]) at the group barrier of
+  // local stage j - 2. The first claim past the split sets n_local, the
+  // group's stage count.
   const uint64_t pol = policy_evict_first();
   const int32_t* pt = p.page_table + (size_t)seq * p.max_pages + pg0;
   const int npg = pg1 - pg0;
   const int full_stages = (t_end - t_begin) / STAGE_TOK;  // stages with all 64 tokens
   volatile int* abort_flag = &sm.abort_flag;
+  volatile int* n_local = &gs.n_local;
   // the host keeps num_pages * kv_heads * block below 2^31
   const uint32_t num_pages32 = (uint32_t)p.num_pages;
+  int held = n_it;  // stage of the split held for this warp's next local stage (>= n_it: none)
   int ids[PPS];
-  auto load_ids = [&](int R) {
+  // claim local stage j (all lanes of warp j % 4, j increasing by 4)
+  auto claim = [&](int j) {
+    int R;
+    if (j < INIT) {
+      R = grp + GROUPS * j;
+    } else {
+      R = 0;
+      if (lane == 0) R = atomicAdd(&sm.next, 1);
+      R = __shfl_sync(FULL_MASK, R, 0);
+    }
+    held = R;
+    if (R >= n_it) {
+      if (lane == 0 && j >= INIT) atomicMin(&gs.n_local, j);
+      return;
+    }
 #pragma unroll
     for (int k = 0; k < PPS; ++k) {
       const int pi = R * PPS + k;
       ids[k] = pi < npg ? pt[pi] : -1;
     }
   };
-  load_ids(warp);
-  // Called by all lanes of warp R % 4, with R increasing by 4 each time.
-  auto issue = [&](int R) {
+  // issue local stage j and claim j + 4 (all lanes of warp j % 4)
+  auto issue = [&](int j, bool copy) {
+    const int R = held;
     int phys[PPS];
 #pragma unroll
     for (int k = 0; k < PPS; ++k) phys[k] = ids[k];
-    load_ids(R + CWARPS);
-    if (lane != 0) return;
-    const int ks = R % NSK, vs = R % NSV;
+    claim(j + GWARPS);
+    if (R >= n_it || !copy || lane != 0) return;
+    const int ks = j % NSK, vs = j % NSV;
     bool all_ok = R < full_stages;
 #pragma unroll
     for (int k = 0; k < PPS; ++k) all_ok = all_ok && (uint32_t)phys[k] < num_pages32;
@@ -333,25 +374,28 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
         }
       }
     }
-    sm.mask[ks] = mask;
+    gs.mask[ks] = mask;
     const uint32_t bytes = npages * BLOCK * (ROW_BYTES + SROW_BYTES);
-    mbar_arrive_expect_tx(&sm.kfull[ks], bytes);
-    mbar_arrive_expect_tx(&sm.vfull[vs], bytes);
+    mbar_arrive_expect_tx(&gs.kfull[ks], bytes);
+    mbar_arrive_expect_tx(&gs.vfull[vs], bytes);
 #pragma unroll
     for (int k = 0; k < PPS; ++k) {
       if (phys[k] < 0) continue;
       const int row = (phys[k] * p.kv_heads + kvh) * BLOCK;
-      tma_load_2d(&sm.k[ks][k * BLOCK * ROW_BYTES], &tm_k, &sm.kfull[ks], 0, row, pol);
-      bulk_load(&sm.ks[ks][k * BLOCK * SROW_BYTES], p.k_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
-                &sm.kfull[ks], pol);
-      tma_load_2d(&sm.v[vs][k * BLOCK * ROW_BYTES], &tm_v, &sm.vfull[vs], 0, row, pol);
-      bulk_load(&sm.vs[vs][k * BLOCK * SROW_BYTES], p.v_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
-                &sm.vfull[vs], pol);
+      tma_load_2d(&gs.k[ks][k * BLOCK * ROW_BYTES], &tm_k, &gs.kfull[ks], 0, row, pol);
+      bulk_load(&gs.ks[ks][k * BLOCK * SROW_BYTES], p.k_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
+                &gs.kfull[ks], pol);
+      tma_load_2d(&gs.v[vs][k * BLOCK * ROW_BYTES], &tm_v, &gs.vfull[vs], 0, row, pol);
+      bulk_load(&gs.vs[vs][k * BLOCK * SROW_BYTES], p.v_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
+                &gs.vfull[vs], pol);
     }
-    atomicMax(&sm.issued, R + 1);
+    atomicMax(&gs.issued, j + 1);
   };
-  // stages 0 and 1; stage R + 2 follows at the CTA barrier of stage R
-  if (warp < 2 && warp < n_it) issue(warp);
+  // local stage 0 now, 1 after the q set-up (so that every group's first
+  // stage is queued at the memory ahead of the second ones); stage j + 2
+  // follows at the group barrier of stage j
+  claim(gw);
+  if (gw == 0) issue(0, true);
 
   // ------------------------------------------------------------ q as the B operand
   // Column n of the Q K^T tile is (query head n >> 1 of the quad, cell
@@ -428,6 +472,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
         }
       }
   }
+  if (gw == 1) issue(1, true);
   __syncthreads();
 
   // ------------------------------------------------------------ main loop
@@ -440,7 +485,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
   float m_run[HQ], m_ref[HQ], thr[HQ], l_run[HQ];
 #pragma unroll
   for (int hq = 0; hq < HQ; ++hq) {
-    m_run[hq] = -INFINITY;  // running max of the scaled scores (base 2)
+    m_run[hq] = -INFINITY;  // the group's running max of the scaled scores (base 2)
     m_ref[hq] = 0.f;        // exponent reference: m_run + SLACK, or 0 while m_run = -inf
     thr[hq] = -INFINITY;    // 0, or -inf while m_run = -inf: the fast path needs x - m_ref <= thr
     l_run[hq] = 0.f;
@@ -462,19 +507,20 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
   uint32_t koff[PAIRS];
 #pragma unroll
   for (int pp = 0; pp < PAIRS; ++pp)
-    koff[pp] = (uint32_t)((16 * warp + 8 * ((lane >> 3) & 1) + sw) * ROW_BYTES) +
+    koff[pp] = (uint32_t)((16 * gw + 8 * ((lane >> 3) & 1) + sw) * ROW_BYTES) +
                ((uint32_t)((2 * pp + (lane >> 4)) ^ sw) << 4);
   // V ldmatrix (transposed) of k-step kk: tokens 16 kk + 8 (mi & 1) .. +7,
   // cell 2w + (mi >> 1).
   const uint32_t voff = (uint32_t)((8 * ((lane >> 3) & 1) + sw) * ROW_BYTES) +
-                        ((uint32_t)((2 * warp + (lane >> 4)) ^ sw) << 4);
+                        ((uint32_t)((2 * gw + (lane >> 4)) ^ sw) << 4);
+  const uint32_t bar_id = 1 + grp;  // the group's named barrier (0 is __syncthreads)
   bool aborted = false;
   float sg[HQ], sg8[HQ];  // raw scores of tokens g, g + 8 of the warp's 16 (head 4 hq + t)
 
   // Q K^T of the warp's 16 tokens of the stage in K slot `ks`.
   auto qk_math = [&](int ks) {
-    const uint32_t kbase = smem_u32(&sm.k[ks][0]);
-    const uint8_t* ksb = &sm.ks[ks][16 * warp * SROW_BYTES];
+    const uint32_t kbase = smem_u32(&gs.k[ks][0]);
+    const uint8_t* ksb = &gs.ks[ks][16 * gw * SROW_BYTES];
     const uint4 skA = lds128(ksb + g * SROW_BYTES);
     const uint4 skB = lds128(ksb + (g + 8) * SROW_BYTES);
     const uint32_t sa[4] = {skA.x, skA.y, skA.z, skA.w}, sb[4] = {skB.x, skB.y, skB.z, skB.w};
@@ -509,13 +555,13 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
   // buffer `pb`) into the dims of cells 2w, 2w+1; `partial` masks absent
   // tokens of `smask` (a stale slot may hold any bit pattern).
   auto pv_math = [&](int vs, int pb, unsigned long long smask, auto partial) {
-    const uint32_t vbase = smem_u32(&sm.v[vs][0]) + voff;
-    const uint8_t* vsb = &sm.vs[vs][0];
-    const uint16_t* prow = &sm.prob[pb][g][0];
+    const uint32_t vbase = smem_u32(&gs.v[vs][0]) + voff;
+    const uint8_t* vsb = &gs.vs[vs][0];
+    const uint16_t* prow = &gs.prob[pb][g][0];
     auto pv_step = [&](int kk, uint32_t km) {
       const uint32_t b01 = lds32(prow + 16 * kk + 2 * t);
       const uint32_t b23 = lds32(prow + 16 * kk + 2 * t + 8);
-      const uint8_t* sr = vsb + (16 * kk + 2 * t) * SROW_BYTES + 4 * warp;  // cells 2w, 2w+1
+      const uint8_t* sr = vsb + (16 * kk + 2 * t) * SROW_BYTES + 4 * gw;  // cells 2w, 2w+1
       uint32_t s0 = lds32(sr), s1 = lds32(sr + SROW_BYTES), s2 = lds32(sr + 8 * SROW_BYTES),
                s3 = lds32(sr + 9 * SROW_BYTES);
       if constexpr (decltype(partial)::value) {
@@ -548,14 +594,14 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
       for (int kk = 0; kk < STAGE_TOK / 16; ++kk) pv_step(kk, 0xffffu);
     }
     // The -8 offset: this warp sums p * v_scale over its own k-step (tokens
-    // 16w .. 16w + 15) for every cell; the warps' sums add up at the end.
-    const uint32_t wm = (uint32_t)(smask >> (16 * warp)) & 0xffffu;
+    // 16w .. 16w + 15) for every cell; the group's warps add up at the end.
+    const uint32_t wm = (uint32_t)(smask >> (16 * gw)) & 0xffffu;
     if (!decltype(partial)::value || wm != 0u) {
-      const uint32_t b01 = lds32(prow + 16 * warp + 2 * t);
-      const uint32_t b23 = lds32(prow + 16 * warp + 2 * t + 8);
+      const uint32_t b01 = lds32(prow + 16 * gw + 2 * t);
+      const uint32_t b23 = lds32(prow + 16 * gw + 2 * t + 8);
       // A: the V scales transposed, row = cell g, k = tokens
       uint32_t st0, st1;
-      ldsm_x2_trans(smem_u32(vsb) + (uint32_t)((16 * warp + (lane & 15)) * SROW_BYTES), st0, st1);
+      ldsm_x2_trans(smem_u32(vsb) + (uint32_t)((16 * gw + (lane & 15)) * SROW_BYTES), st0, st1);
       if constexpr (decltype(partial)::value) {
         st0 &= (((wm >> (2 * t)) & 1u) ? 0x0000ffffu : 0u) | (((wm >> (2 * t + 1)) & 1u) ? 0xffff0000u : 0u);
         st1 &= (((wm >> (2 * t + 8)) & 1u) ? 0x0000ffffu : 0u) | (((wm >> (2 * t + 9)) & 1u) ? 0xffff0000u : 0u);
@@ -567,10 +613,10 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
     }
   };
 
-  // Probabilities of the scored stage (its tokens in wm) against the CTA's
-  // running max, written to buffer pb; then the CTA barrier that publishes
-  // them. All warps are then past Q K^T of that stage and P V of the one
-  // before it.
+  // Probabilities of the scored stage (its tokens in wm) against the group's
+  // running max, written to buffer pb; then the group barrier that publishes
+  // them. The group's warps are then past Q K^T of that stage and P V of the
+  // one before it.
   auto publish = [&](int pb, uint32_t wm) {
     const bool okA = (wm >> g) & 1u, okB = (wm >> (g + 8)) & 1u;
     float xA[HQ], xB[HQ], psum[HQ];
@@ -583,11 +629,11 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
       need |= (yA > thr[hq]) || (yB > thr[hq]);
       const float pA = ex2(yA), pB = ex2(yB);
       psum[hq] = pA + pB;
-      uint16_t* pr = &sm.prob[pb][4 * hq + t][16 * warp + g];
+      uint16_t* pr = &gs.prob[pb][4 * hq + t][16 * gw + g];
       pr[0] = __half_as_ushort(__float2half_rn(pA));
       pr[8] = __half_as_ushort(__float2half_rn(pB));
     }
-    if (bar_red_or(need)) {
+    if (bar_red_or(bar_id, need)) {
       // Some head's running max moves: exchange the tile maxima, rescale.
 #pragma unroll
       for (int hq = 0; hq < HQ; ++hq) {
@@ -595,15 +641,15 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
         tm = fmaxf(tm, __shfl_xor_sync(FULL_MASK, tm, 4));
         tm = fmaxf(tm, __shfl_xor_sync(FULL_MASK, tm, 8));
         tm = fmaxf(tm, __shfl_xor_sync(FULL_MASK, tm, 16));
-        if (g == 0) sm.tmax[warp][4 * hq + t] = tm;
+        if (g == 0) gs.tmax[gw][4 * hq + t] = tm;
       }
-      bar_cta();
+      bar_sync(bar_id);
       float alpha[HQ];
 #pragma unroll
       for (int hq = 0; hq < HQ; ++hq) {
         float mn = m_run[hq];
 #pragma unroll
-        for (int w = 0; w < CWARPS; ++w) mn = fmaxf(mn, sm.tmax[w][4 * hq + t]);
+        for (int w = 0; w < GWARPS; ++w) mn = fmaxf(mn, gs.tmax[w][4 * hq + t]);
         const float mu = (mn == -INFINITY) ? 0.f : mn + SLACK;
         alpha[hq] = (m_run[hq] == -INFINITY) ? 0.f : ex2(m_ref[hq] - mu);  // nothing accumulated yet: 0
         m_run[hq] = mn;
@@ -611,7 +657,7 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
         thr[hq] = (mn == -INFINITY) ? -INFINITY : 0.f;
         const float pA = ex2(xA[hq] - mu), pB = ex2(xB[hq] - mu);
         l_run[hq] = l_run[hq] * alpha[hq] + (pA + pB);
-        uint16_t* pr = &sm.prob[pb][4 * hq + t][16 * warp + g];
+        uint16_t* pr = &gs.prob[pb][4 * hq + t][16 * gw + g];
         pr[0] = __half_as_ushort(__float2half_rn(pA));
         pr[8] = __half_as_ushort(__float2half_rn(pB));
       }
@@ -637,18 +683,21 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
         }
       vsum[0] *= al0;
       vsum[1] *= al1;
-      bar_cta();
+      bar_sync(bar_id);
     } else {
 #pragma unroll
       for (int hq = 0; hq < HQ; ++hq) l_run[hq] += psum[hq];
     }
   };
 
-  // Software pipeline: iteration `it` multiplies stage it into the
-  // accumulators and scores stage it + 1, so the two run as one straight
-  // block on full stages; the CTA barrier sits between the scoring and the
-  // P V of each stage. Stage s + 2 is issued at the barrier of stage s.
-  int kst = 0, vst = 0;       // K slot of the next stage to score, V slot of stage it
+  // Software pipeline: iteration `it` multiplies local stage it into the
+  // accumulators and scores local stage it + 1, so the two run as one
+  // straight block on full stages; the group barrier sits between the
+  // scoring and the P V of each stage. Local stage j + 2 is issued at the
+  // barrier of local stage j. The stage count n_local is read only for stages
+  // whose claim was made at least four barriers earlier, so every warp of the
+  // group sees the same count.
+  int kst = 0, vst = 0;       // K slot of the next local stage to score, V slot of local stage it
   uint32_t kph = 0, vph = 0;  // their phase parities
   unsigned long long smask_n = 0;  // token mask of the next stage to score
   auto next_k = [&]() {
@@ -657,97 +706,100 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
       kph ^= 1u;
     }
   };
-  if (n_it > 0) {
+  if (*n_local > 0) {
     // (aborted is warp-uniform, so the .aligned ldmatrix / mma see a converged warp)
-    aborted = __any_sync(FULL_MASK, !wait_copies(&sm.kfull[0], 0, abort_flag, p.status));
-    smask_n = aborted ? 0ull : sm.mask[0];
-    const uint32_t wm = (uint32_t)(smask_n >> (16 * warp)) & 0xffffu;
+    aborted = __any_sync(FULL_MASK, !wait_copies(&gs.kfull[0], 0, abort_flag, p.status));
+    smask_n = aborted ? 0ull : gs.mask[0];
+    const uint32_t wm = (uint32_t)(smask_n >> (16 * gw)) & 0xffffu;
 #pragma unroll
     for (int hq = 0; hq < HQ; ++hq) sg[hq] = sg8[hq] = 0.f;
     if (wm != 0u) qk_math(0);
     publish(0, wm);
-    if (!aborted && 2 < n_it && warp == 2) issue(2);
+    if (gw == 2) issue(2, !aborted);
     next_k();
-  }
-  for (int it = 0; it < n_it; ++it) {
-    const unsigned long long smask = smask_n;  // stage it
-    const bool nxt = it + 1 < n_it;
-    if (!aborted) {
-      bool ok = wait_copies(&sm.vfull[vst], vph, abort_flag, p.status);
-      if (nxt) ok = ok && wait_copies(&sm.kfull[kst], kph, abort_flag, p.status);
-      aborted = __any_sync(FULL_MASK, !ok);
-    }
-    smask_n = (nxt && !aborted) ? sm.mask[kst] : 0ull;
-    const uint32_t wm_n = (uint32_t)(smask_n >> (16 * warp)) & 0xffffu;
-    const int pb = it & 1;
+    for (int it = 0;; ++it) {
+      const unsigned long long smask = smask_n;  // local stage it
+      const bool nxt = it + 1 < *n_local;
+      if (!aborted) {
+        bool ok = wait_copies(&gs.vfull[vst], vph, abort_flag, p.status);
+        if (nxt) ok = ok && wait_copies(&gs.kfull[kst], kph, abort_flag, p.status);
+        aborted = __any_sync(FULL_MASK, !ok);
+      }
+      smask_n = (nxt && !aborted) ? gs.mask[kst] : 0ull;
+      const uint32_t wm_n = (uint32_t)(smask_n >> (16 * gw)) & 0xffffu;
+      const int pb = it & 1;
 #pragma unroll
-    for (int hq = 0; hq < HQ; ++hq) sg[hq] = sg8[hq] = 0.f;
-    if (!aborted && smask == ~0ull && (smask_n == ~0ull || !nxt)) {
-      // full stages: one straight block
-      pv_math(vst, pb, smask, std::false_type{});
-      if (nxt) qk_math(kst);
-    } else {
-      if (!aborted && smask != 0ull) pv_math(vst, pb, smask, std::true_type{});
-      if (wm_n != 0u) qk_math(kst);
-    }
-    if (nxt) {
+      for (int hq = 0; hq < HQ; ++hq) sg[hq] = sg8[hq] = 0.f;
+      if (!aborted && smask == ~0ull && (smask_n == ~0ull || !nxt)) {
+        // full stages: one straight block
+        pv_math(vst, pb, smask, std::false_type{});
+        if (nxt) qk_math(kst);
+      } else {
+        if (!aborted && smask != 0ull) pv_math(vst, pb, smask, std::true_type{});
+        if (wm_n != 0u) qk_math(kst);
+      }
+      if (!nxt) break;
       publish(pb ^ 1, wm_n);
-      // K of stage it + 3 replaces stage it + 1 (scored), V replaces stage it
-      // (multiplied); warp-uniform, since the issue shuffles nothing but
-      // loads on every lane.
-      if (!aborted && it + 3 < n_it && ((it + 3) % CWARPS) == warp) issue(it + 3);
+      // local stage it + 3 takes the K slot of stage it + 1 (scored) and the
+      // V slot of stage it (multiplied); its claim is kept going even when
+      // aborting, so that the stage count gets set.
+      if (((it + 3) % GWARPS) == gw) issue(it + 3, !aborted);
       next_k();
-    }
-    if (++vst == NSV) {
-      vst = 0;
-      vph ^= 1u;
+      if (++vst == NSV) {
+        vst = 0;
+        vph ^= 1u;
+      }
     }
   }
 
   // ------------------------------------------------------------ epilogue
+  // Per group: softmax sums of the warps, offset sums of the warps (in the
+  // group's idle V scale slots), and the decoded accumulators.
 #pragma unroll
   for (int hq = 0; hq < HQ; ++hq) {
     float l = l_run[hq];
     l += __shfl_xor_sync(FULL_MASK, l, 4);
     l += __shfl_xor_sync(FULL_MASK, l, 8);
     l += __shfl_xor_sync(FULL_MASK, l, 16);
-    if (g == 0) sm.wl[warp][4 * hq + t] = l;
+    if (g == 0) gs.wl[gw][4 * hq + t] = l;
   }
   __syncthreads();
   if (*abort_flag) {
     // Leave only after every copy issued here has landed.
-    if (threadIdx.x == 0) {
-      const int issued = sm.issued;
+    if (threadIdx.x < GROUPS) {
+      GroupSmem& q = sm.grp[threadIdx.x];
+      const int issued = q.issued;
       for (int r = max(0, issued - NSK); r < issued; ++r)
-        if (!mbar_wait_bounded(&sm.kfull[r % NSK], (r / NSK) & 1)) flag(p.status, QKV_DEV_TIMEOUT);
+        if (!mbar_wait_bounded(&q.kfull[r % NSK], (r / NSK) & 1)) flag(p.status, QKV_DEV_TIMEOUT);
       for (int r = max(0, issued - NSV); r < issued; ++r)
-        if (!mbar_wait_bounded(&sm.vfull[r % NSV], (r / NSV) & 1)) flag(p.status, QKV_DEV_TIMEOUT);
+        if (!mbar_wait_bounded(&q.vfull[r % NSV], (r / NSV) & 1)) flag(p.status, QKV_DEV_TIMEOUT);
     }
     if (threadIdx.x < G) lse_out[threadIdx.x] = -INFINITY;
     return;
   }
-  // the warps' offset sums, parked in the (now idle) K ring: [warp][lane][2]
-  float2* vsp = reinterpret_cast<float2*>(&sm.k[0][0]);
-  vsp[warp * 32 + lane] = make_float2(vsum[0], vsum[1]);
-  __syncthreads();
-  float inv[2];
+  float2* vsp = reinterpret_cast<float2*>(&gs.vs[0][0]);
+  vsp[gw * 32 + lane] = make_float2(vsum[0], vsum[1]);
+  bar_sync(bar_id);
+  // the group's softmax sum and exponent reference per head
+  if (gw == 0 && g == 0) {
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int h = 2 * t + j;
-    float Ls = 0.f;
-    if (h < G)
+    for (int hq = 0; hq < HQ; ++hq) {
+      const int h = 4 * hq + t;
+      float Ls = 0.f;
 #pragma unroll
-      for (int w = 0; w < CWARPS; ++w) Ls += sm.wl[w][h];
-    inv[j] = Ls > 0.f ? 1.f / Ls : 0.f;
+      for (int w = 0; w < GWARPS; ++w) Ls += gs.wl[w][h];
+      sm.gl[grp][h] = Ls;
+      sm.gm[grp][h] = m_ref[hq];
+    }
   }
   // Undo the subnormal encoding of V: rows 0-7 carry 2^-24 * sum(n p s),
   // rows 8-15 2^-20 * sum(n p s); the -8 offset is 8 * sum(p s) per cell.
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
-    const int cell = 2 * warp + c;
+    const int cell = 2 * gw + c;
     float b0 = 0.f, b1 = 0.f;
 #pragma unroll
-    for (int w = 0; w < CWARPS; ++w) {
+    for (int w = 0; w < GWARPS; ++w) {
       const float2 v = vsp[w * 32 + 4 * cell + t];
       b0 += v.x;
       b1 += v.y;
@@ -762,30 +814,53 @@ __global__ void __launch_bounds__(THREADS, Cfg<G>::MIN_BLOCKS)
       acc[c][k][3] = fmaf(acc[c][k][3], 1048576.f, -b1);
     }
   }
+  __syncthreads();
+  // Fold the groups: weights 2^(m_ref of the group - M) per head.
+  float* slab = reinterpret_cast<float*>(&sm.grp[0].k[0][0]);  // [group][head][dim], in idle rings
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
     const int h = 2 * t + j;
     if (h < G) {
-      float* dst = p.o_parts + ((size_t)split * rows + row0 + h) * D + 4 * g;
+      float M = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < GROUPS; ++q)
+        if (sm.gl[q][h] > 0.f) M = fmaxf(M, sm.gm[q][h]);
+      const float f = (sm.gl[grp][h] > 0.f) ? exp2f(sm.gm[grp][h] - M) : 0.f;
+      float* dst = slab + ((size_t)grp * G + h) * D + 4 * g;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        const float4 o = make_float4(inv[j] * acc[c][0][j], inv[j] * acc[c][0][j + 2], inv[j] * acc[c][1][j],
-                                     inv[j] * acc[c][1][j + 2]);
-        *reinterpret_cast<float4*>(dst + 32 * (2 * warp + c)) = o;
+        const float4 o = make_float4(f * acc[c][0][j], f * acc[c][0][j + 2], f * acc[c][1][j], f * acc[c][1][j + 2]);
+        *reinterpret_cast<float4*>(dst + 32 * (2 * gw + c)) = o;
       }
     }
   }
-  if (warp == 0 && g == 0) {
+  __syncthreads();
+  // Sum the groups, normalise, write the partial of this split.
+  for (int e = threadIdx.x; e < G * (D / 4); e += THREADS) {
+    const int h = e / (D / 4), d4 = e % (D / 4);
+    float M = -INFINITY;
 #pragma unroll
-    for (int hq = 0; hq < HQ; ++hq) {
-      const int h = 4 * hq + t;
-      if (h < G) {
-        float Ls = 0.f;
+    for (int q = 0; q < GROUPS; ++q)
+      if (sm.gl[q][h] > 0.f) M = fmaxf(M, sm.gm[q][h]);
+    float Ls = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w = 0; w < CWARPS; ++w) Ls += sm.wl[w][h];
-        lse_out[h] = Ls > 0.f ? m_ref[hq] + log2f(Ls) : -INFINITY;
-      }
+    for (int q = 0; q < GROUPS; ++q) {
+      const float f = (sm.gl[q][h] > 0.f) ? exp2f(sm.gm[q][h] - M) : 0.f;
+      Ls = fmaf(f, sm.gl[q][h], Ls);
+      const float4 x = *reinterpret_cast<const float4*>(slab + ((size_t)q * G + h) * D + 4 * d4);
+      o.x += x.x;
+      o.y += x.y;
+      o.z += x.z;
+      o.w += x.w;
     }
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+    o.x *= inv;
+    o.y *= inv;
+    o.z *= inv;
+    o.w *= inv;
+    *reinterpret_cast<float4*>(p.o_parts + ((size_t)split * rows + row0 + h) * D + 4 * d4) = o;
+    if (d4 == 0) lse_out[h] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
   }
 }
 
