@@ -195,3 +195,28 @@ def test_unsupported_shapes_raise(qkv):
     with pytest.raises(qkv.QkvError) as e:
         _run_attn(qkv, w, x, cache)
     assert e.value.code == 2
+
+
+def test_workspace_reuse_across_calls(qkv):
+    """One workspace serves calls with different inputs, split counts and
+    sequence counts in a row; each matches the oracle."""
+    att = qkv.DecodeAttention(3, 16, 4, 256, 64, max_splits=16)
+    calls = [
+        (workloads.small("reuse_a", seq_lens=(3000, 70, 1), num_pages=60, block_size=64, head_scale=True,
+                         page_alloc="interleaved"), 0),
+        (workloads.small("reuse_b", seq_lens=(1200, 4000), num_pages=90, block_size=64, seed=5,
+                         page_alloc="interleaved"), 7),
+        (workloads.small("reuse_c", seq_lens=(64,), num_pages=2, block_size=64, seed=9), 16),
+    ]
+    for w, splits in calls:
+        x, ref = oracle_layer(w)
+        cache = _dev_cache(qkv, w, x)
+        out = torch.empty((w.n_seq, w.q_heads, w.head_dim), dtype=torch.int16, device="cuda")
+        lse = torch.empty((w.n_seq, w.q_heads), dtype=torch.float32, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        att(out, to_dev(x["q"]), cache, to_dev(x["page_table"]), to_dev(x["seq_lens"]), lse2_out=lse,
+            num_splits=splits, device_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        ref_out, ref_lse = _oracle_attn(w, x, ref)
+        _assert_close(to_host(out, np.uint16), to_host(lse), ref_out, ref_lse)
