@@ -202,3 +202,34 @@ def lse_merge(o_parts, lse2_parts) -> Tuple[np.ndarray, np.ndarray]:
 
 def max_threads() -> int:
     return lib().oracle_max_threads()
+
+
+def dense_attention(q, k, v, softmax_scale: Optional[float] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Exact softmax attention of one sequence over unquantised K/V: the plain
+    definition out = softmax(q k^T * scale) v, in float64 (the bf16 "oracle
+    format" the ignis docs "context-and-speculation" run every correctness
+    check against, KV pool section, --model-kv-format).
+
+    q bf16 bits [Hq][D]; k, v bf16 bits [T][Hkv][D] (or float arrays); query
+    head h reads KV head h // (Hq / Hkv). Returns (out [Hq][D], lse2 [Hq]),
+    lse2 = log2 sum_t exp(score_t)."""
+    def f64(a):
+        a = np.asarray(a)
+        return bf16_to_f64(a) if a.dtype == np.uint16 else a.astype(np.float64)
+    qf, kf, vf = f64(q), f64(k), f64(v)
+    hq, d = qf.shape
+    hkv = kf.shape[1]
+    g = hq // hkv
+    sc = float(softmax_scale) if softmax_scale else 1.0 / np.sqrt(d)
+    out = np.zeros((hq, d))
+    lse2 = np.full(hq, -np.inf)
+    if kf.shape[0] == 0:
+        return out, lse2
+    for h in range(hq):
+        s = kf[:, h // g, :] @ qf[h] * sc                    # [T]
+        m = s.max()
+        e = np.exp(s - m)
+        z = e.sum()
+        out[h] = (e @ vf[:, h // g, :]) / z
+        lse2[h] = (m + np.log(z)) / np.log(2.0)
+    return out, lse2
