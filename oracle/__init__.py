@@ -61,9 +61,10 @@ def lib() -> ctypes.CDLL:
             "oracle_rope_apply_f64": (None, [vp, vp, vp, i32, i32, i32, P]),
             "oracle_rope_apply_bf16": (None, [vp, vp, vp, i32, i32, i32, P]),
             "oracle_quantize_cell": (None, [vp, vp, vp]),
-            "oracle_kv_write_f4": (i32, [vp, vp, vp, i64, vp, vp, vp, vp, i32, i32, i32, i64]),
+            "oracle_quantize_group": (None, [vp, i32, vp, vp]),
+            "oracle_kv_write_f4": (i32, [vp, vp, vp, i64, vp, vp, vp, vp, i32, i32, i32, i64, i32]),
             "oracle_paged_attention": (None, [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32,
-                                              d, vp, vp, i32]),
+                                              d, vp, vp, i32, i32]),
             "oracle_lse_merge": (None, [vp, vp, i32, i32, i32, vp, vp]),
             "oracle_max_threads": (i32, []),
             "oracle_f64_to_f16_array": (None, [vp, vp, i64]),
@@ -153,11 +154,26 @@ def quantize_cell(x32) -> Tuple[np.ndarray, int]:
     return b, int(s[0])
 
 
-def empty_cache(num_pages: int, kv_heads: int, block_size: int, head_dim: int):
-    """Zeroed (k_data, k_scale, v_data, v_scale) in the paged layout."""
+def quantize_group(x) -> Tuple[np.ndarray, int]:
+    """One group of n values (n even) sharing a scale: (bytes [n/2], scale bits)."""
+    x = _c(x, np.uint16); n = x.size; assert n % 2 == 0 and n <= 1024
+    b = np.empty(n // 2, np.uint8); s = np.empty(1, np.uint16)
+    lib().oracle_quantize_group(_p(x), n, _p(b), _p(s))
+    return b, int(s[0])
+
+
+def empty_cache(num_pages: int, kv_heads: int, block_size: int, head_dim: int, v_group: int = 32):
+    """Zeroed (k_data, k_scale, v_data, v_scale) in the paged layout. K has
+    one scale per 32-value cell; V one per v_group values (32, or head_dim for
+    one scale per token, the PR's own V layout)."""
     data = lambda: np.zeros((num_pages, kv_heads, block_size, head_dim // 2), np.uint8)
-    scale = lambda: np.zeros((num_pages, kv_heads, block_size, head_dim // 32), np.uint16)
-    return data(), scale(), data(), scale()
+    scale = lambda g: np.zeros((num_pages, kv_heads, block_size, head_dim // g), np.uint16)
+    return data(), scale(32), data(), scale(v_group)
+
+
+def v_group_of(cache, head_dim: int) -> int:
+    """Values per V scale of a cache from empty_cache."""
+    return head_dim // cache[3].shape[-1]
 
 
 def kv_write_f4(k, v, slots, cache, kv_heads: int, head_dim: int, block_size: int) -> int:
@@ -168,7 +184,7 @@ def kv_write_f4(k, v, slots, cache, kv_heads: int, head_dim: int, block_size: in
     for a in cache:
         assert a.flags.c_contiguous
     return lib().oracle_kv_write_f4(_p(k), _p(v), _p(sl), sl.size, _p(kd), _p(ks), _p(vd), _p(vs),
-                                    kv_heads, head_dim, block_size, kd.shape[0])
+                                    kv_heads, head_dim, block_size, kd.shape[0], v_group_of(cache, head_dim))
 
 
 # ---------------------------------------------------------------------------
@@ -187,7 +203,7 @@ def paged_attention(q, cache, page_table, tok_begin, tok_end, q_heads: int, kv_h
     sc = float(softmax_scale) if softmax_scale else 1.0 / np.sqrt(head_dim)
     lib().oracle_paged_attention(_p(q), _p(kd), _p(ks), _p(vd), _p(vs), _p(pt), pt.shape[1], _p(tb), _p(te),
                                  n_seq, q_heads, kv_heads, head_dim, block_size, sc, _p(out), _p(lse2),
-                                 n_threads)
+                                 n_threads, v_group_of(cache, head_dim))
     return out, lse2
 
 

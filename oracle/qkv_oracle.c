@@ -197,38 +197,47 @@ void oracle_rope_apply_bf16(const uint16_t* x, uint16_t* out, const int64_t* pos
 /* ------------------------------------------------------------------------- */
 /* F4 quantisation [F4].                                                     */
 
-/* One 32-value cell: scale = fp16(amax / 7) (saturating at 65504), code_i =
- * clamp(rint(x_i / scale), -8, 7) + 8, all codes 8 when scale is 0; byte b
- * holds element 2b in bits 0-3 and element 2b+1 in bits 4-7. */
-void oracle_quantize_cell(const uint16_t* x, uint8_t* bytes, uint16_t* scale_out) {
+/* A group of n values (n even, <= 1024) sharing one scale: scale =
+ * fp16(amax / 7) (saturating at 65504), code_i = clamp(rint(x_i / scale),
+ * -8, 7) + 8, all codes 8 when scale is 0; byte b holds element 2b in bits
+ * 0-3 and element 2b+1 in bits 4-7. The PR's K cells are groups of 32; its V
+ * scale is "one scale per token per V head", a group of head_dim. */
+void oracle_quantize_group(const uint16_t* x, int n, uint8_t* bytes, uint16_t* scale_out) {
   double amax = 0;
-  for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(oracle_bf16_to_f64(x[i])));
+  for (int i = 0; i < n; ++i) amax = fmax(amax, fabs(oracle_bf16_to_f64(x[i])));
   uint16_t sc = oracle_f64_to_f16(amax / 7.0);
   if ((sc & 0x7FFF) == 0x7C00) sc = 0x7BFF; /* saturate to 65504 */
   const double s = oracle_f16_to_f64(sc);
-  int code[32];
-  for (int i = 0; i < 32; ++i) {
+  int code[1024];
+  for (int i = 0; i < n; ++i) {
     if (s == 0) { code[i] = 8; continue; }
     double r = nearbyint(oracle_bf16_to_f64(x[i]) / s); /* ties to even */
     if (r < -8) r = -8;
     if (r > 7) r = 7;
     code[i] = (int)r + 8;
   }
-  for (int b = 0; b < 16; ++b) bytes[b] = (uint8_t)(code[2 * b] | (code[2 * b + 1] << 4));
+  for (int b = 0; b < n / 2; ++b) bytes[b] = (uint8_t)(code[2 * b] | (code[2 * b + 1] << 4));
   *scale_out = sc;
+}
+
+/* One 32-value cell. */
+void oracle_quantize_cell(const uint16_t* x, uint8_t* bytes, uint16_t* scale_out) {
+  oracle_quantize_group(x, 32, bytes, scale_out);
 }
 
 /* Paged cache, per layer and for each of K and V:
  *   data  u8  [num_pages][kv_heads][block_size][head_dim/2]
- *   scale f16 [num_pages][kv_heads][block_size][head_dim/32]
+ *   scale f16 [num_pages][kv_heads][block_size][head_dim/32] for K, and
+ *             [num_pages][kv_heads][block_size][head_dim/v_group] for V
+ *             (v_group 32: per cell; head_dim: one scale per token)
  * Token i of a sequence lives in page page_table[i / B] at offset i % B; a
  * write goes to slot = page * B + offset. Slots < 0 are skipped; slots past
  * the pool are skipped and counted. Returns the count of skipped bad slots. */
 int oracle_kv_write_f4(const uint16_t* k, const uint16_t* v, const int64_t* slots, int64_t n_tok,
                        uint8_t* k_data, uint16_t* k_scale, uint8_t* v_data, uint16_t* v_scale,
-                       int kv_heads, int head_dim, int block_size, int64_t num_pages) {
+                       int kv_heads, int head_dim, int block_size, int64_t num_pages, int v_group) {
   int bad = 0;
-  const int cells = head_dim / 32;
+  const int cells = head_dim / 32, vgroups = head_dim / v_group;
   for (int64_t t = 0; t < n_tok; ++t) {
     const int64_t slot = slots[t];
     if (slot < 0) continue;
@@ -239,18 +248,23 @@ int oracle_kv_write_f4(const uint16_t* k, const uint16_t* v, const int64_t* slot
       for (int c = 0; c < cells; ++c) {
         const size_t src = ((size_t)t * kv_heads + h) * head_dim + 32 * c;
         oracle_quantize_cell(k + src, k_data + row * (head_dim / 2) + 16 * c, k_scale + row * cells + c);
-        oracle_quantize_cell(v + src, v_data + row * (head_dim / 2) + 16 * c, v_scale + row * cells + c);
+      }
+      for (int c = 0; c < vgroups; ++c) {
+        const size_t src = ((size_t)t * kv_heads + h) * head_dim + (size_t)v_group * c;
+        oracle_quantize_group(v + src, v_group, v_data + row * (head_dim / 2) + (v_group / 2) * c,
+                              v_scale + row * vgroups + c);
       }
     }
   }
   return bad;
 }
 
-/* Dequantised element d of the cache row: (code - 8) * scale, exact in double. */
-static double deq(const uint8_t* data, const uint16_t* scale, size_t row, int head_dim, int d) {
+/* Dequantised element d of the cache row: (code - 8) * scale, exact in
+ * double; `group` values share a scale. */
+static double deq(const uint8_t* data, const uint16_t* scale, size_t row, int head_dim, int group, int d) {
   const uint8_t byte = data[row * (head_dim / 2) + d / 2];
   const int code = (d & 1) ? (byte >> 4) : (byte & 15);
-  return (code - 8) * oracle_f16_to_f64(scale[row * (head_dim / 32) + d / 32]);
+  return (code - 8) * oracle_f16_to_f64(scale[row * (head_dim / group) + d / group]);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -268,7 +282,7 @@ void oracle_paged_attention(const uint16_t* q, const uint8_t* k_data, const uint
                             const int32_t* page_table, int max_pages_per_seq,
                             const int32_t* tok_begin, const int32_t* tok_end, int n_seq,
                             int q_heads, int kv_heads, int head_dim, int block_size,
-                            double softmax_scale, double* out, double* lse2, int n_threads) {
+                            double softmax_scale, double* out, double* lse2, int n_threads, int v_group) {
   const int group = q_heads / kv_heads;
   const long rows = (long)n_seq * q_heads;
 #ifdef _OPENMP
@@ -288,7 +302,7 @@ void oracle_paged_attention(const uint16_t* q, const uint8_t* k_data, const uint
     for (int t = t0; t < t1; ++t) {
       const size_t row = ((size_t)page_table[(size_t)s * max_pages_per_seq + t / block_size] * kv_heads + kvh) * block_size + t % block_size;
       double dot = 0;
-      for (int d = 0; d < head_dim; ++d) dot += qd[d] * deq(k_data, k_scale, row, head_dim, d);
+      for (int d = 0; d < head_dim; ++d) dot += qd[d] * deq(k_data, k_scale, row, head_dim, 32, d);
       const double sc = softmax_scale * dot;
       if (sc > m) m = sc;
     }
@@ -297,10 +311,10 @@ void oracle_paged_attention(const uint16_t* q, const uint8_t* k_data, const uint
     for (int t = t0; t < t1; ++t) {
       const size_t row = ((size_t)page_table[(size_t)s * max_pages_per_seq + t / block_size] * kv_heads + kvh) * block_size + t % block_size;
       double dot = 0;
-      for (int d = 0; d < head_dim; ++d) dot += qd[d] * deq(k_data, k_scale, row, head_dim, d);
+      for (int d = 0; d < head_dim; ++d) dot += qd[d] * deq(k_data, k_scale, row, head_dim, 32, d);
       const double w = exp(softmax_scale * dot - m);
       z += w;
-      for (int d = 0; d < head_dim; ++d) o[d] += w * deq(v_data, v_scale, row, head_dim, d);
+      for (int d = 0; d < head_dim; ++d) o[d] += w * deq(v_data, v_scale, row, head_dim, v_group, d);
     }
     for (int d = 0; d < head_dim; ++d) o[d] /= z;
     lse2[r] = (m + log(z)) / log(2.0);

@@ -92,3 +92,24 @@ def test_deviation_report_runs_small():
     r = f4_deviation.deviation(f4_deviation.sample(workloads.TINY_4K, 1024))
     assert r["tokens"] == 1024
     assert 0 < r["rel_out"] < 0.5 and np.isfinite(r["max_abs_lse2"])
+
+
+def test_dense_equals_paged_per_token_v_scale():
+    """Per-token V scales: on V rows that one power-of-two scale per row
+    stores exactly, paged attention over the F4 cache equals the dense bf16
+    attention (K stored exactly per cell as before)."""
+    rng = np.random.default_rng(12)
+    hq, hkv, d, block, T = 8, 2, 256, 16, 90
+    k, _ = _exact_rows(rng, T, hkv, d)
+    vcodes = rng.integers(1, 16, size=(T, hkv, d))
+    vcodes[..., 5] = 15
+    vexp = rng.integers(0, 6, size=(T, hkv, 1))
+    v = workloads.f32_to_bf16_bits(((vcodes - 8) * np.ldexp(1.0, -vexp)).astype(np.float32))
+    q = workloads.f32_to_bf16_bits(rng.standard_normal((1, hq, d)).astype(np.float32))
+    pages = -(-T // block)
+    cache = oracle.empty_cache(pages, hkv, block, d, v_group=d)
+    pt = np.arange(pages, dtype=np.int32)[None, :]
+    assert oracle.kv_write_f4(k, v, np.arange(T, dtype=np.int64), cache, hkv, d, block) == 0
+    o4, l4 = oracle.paged_attention(q, cache, pt, [0], [T], hq, hkv, d, block)
+    ob, lb = oracle.dense_attention(q[0], k, v)
+    assert np.max(np.abs(o4[0] - ob)) <= 1e-12 and np.max(np.abs(l4[0] - lb)) <= 1e-12

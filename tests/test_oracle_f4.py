@@ -151,3 +151,76 @@ def test_kv_write_layout_and_skips():
     written[1, :, 3] = written[0, :, 0] = True
     assert np.all(kd[~written] == 0) and np.all(ks[~written] == 0)
     assert np.all(vd[~written] == 0) and np.all(vs[~written] == 0)
+
+
+# --------------------------------------------------------------------------
+# One V scale per token (the PR's own V layout: "one scale per token per V
+# head"): the same quantiser over a group of head_dim values.
+
+def _group_codes(b):
+    b = np.asarray(b, dtype=np.uint8)
+    return np.stack([b & 15, b >> 4], axis=-1).reshape(-1).astype(np.int64)
+
+
+@pytest.mark.parametrize("n", [64, 128, 256])
+def test_group_nearest_code_and_bound(n):
+    """Per-token groups: every code is the nearest grid point (ties to even,
+    clamped), |x - x_hat| <= scale / 2, and the largest element lands on code
+    1 or 15 -- found by exhaustive search over the 16 codes."""
+    rng = np.random.default_rng(n)
+    for trial in range(200):
+        x = workloads.f32_to_bf16_bits((rng.standard_normal(n) * 10.0 ** rng.uniform(-3, 3)).astype(np.float32))
+        b, s = oracle.quantize_group(x)
+        sc = oracle.f16_to_f64(np.array([s]))[0]
+        xv = oracle.bf16_to_f64(x)
+        assert s == int(oracle.f64_to_f16(np.array([np.abs(xv).max() / 7.0]))[0])
+        grid = (np.arange(16) - 8) * sc
+        dist = np.abs(xv[:, None] - grid[None, :])
+        best = dist.min(axis=1, keepdims=True)
+        cand = dist == best
+        want = np.where(cand.sum(1) > 1, np.argmax(cand & (np.arange(16) % 2 == 0), axis=1), np.argmax(cand, axis=1))
+        codes = _group_codes(b)
+        assert np.array_equal(codes, want)
+        assert np.all(np.abs(xv - (codes - 8) * sc) <= sc / 2 * (1 + 1e-12))
+        assert codes[np.argmax(np.abs(xv))] in (1, 15)
+
+
+def test_group_of_32_is_the_cell():
+    for x in _random_cells(200, 4):
+        assert oracle.quantize_group(x)[1] == oracle.quantize_cell(x)[1]
+        assert np.array_equal(oracle.quantize_group(x)[0], oracle.quantize_cell(x)[0])
+
+
+def test_group_zero_and_roundtrip():
+    b, s = oracle.quantize_group(np.zeros(256, np.uint16))
+    assert s == 0 and np.all(b == 0x88)
+    rng = np.random.default_rng(8)
+    codes = rng.integers(1, 16, 256)
+    codes[17] = 15
+    x = workloads.f32_to_bf16_bits(((codes - 8) * 0.125).astype(np.float32))
+    b, s = oracle.quantize_group(x)
+    assert oracle.f16_to_f64(np.array([s]))[0] == 0.125
+    assert np.array_equal(_group_codes(b), codes)
+
+
+def test_kv_write_per_token_v_scale():
+    """kv_write_f4 into a cache with one V scale per token stores, for every
+    (token, head), the group quantisation of the V row and the cell
+    quantisation of the K row."""
+    rng = np.random.default_rng(3)
+    n, hkv, d, block = 20, 2, 256, 16
+    k = workloads.f32_to_bf16_bits(rng.standard_normal((n, hkv, d)).astype(np.float32))
+    v = workloads.f32_to_bf16_bits((rng.standard_normal((n, hkv, d)) * 3).astype(np.float32))
+    cache = oracle.empty_cache(2, hkv, block, d, v_group=d)
+    assert cache[3].shape == (2, hkv, block, 1)
+    slots = rng.permutation(2 * block)[:n].astype(np.int64)
+    assert oracle.kv_write_f4(k, v, slots, cache, hkv, d, block) == 0
+    for t in range(n):
+        page, off = divmod(int(slots[t]), block)
+        for h in range(hkv):
+            vb, vs = oracle.quantize_group(v[t, h])
+            assert np.array_equal(cache[2][page, h, off], vb) and cache[3][page, h, off, 0] == vs
+            for c in range(d // 32):
+                kb, ks = oracle.quantize_cell(k[t, h, 32 * c:32 * c + 32])
+                assert np.array_equal(cache[0][page, h, off, 16 * c:16 * c + 16], kb)
+                assert cache[1][page, h, off, c] == ks
