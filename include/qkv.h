@@ -149,6 +149,21 @@ QKV_API int qkv_kv_write_f4(const uint16_t* k, const uint16_t* v, const int64_t*
                     uint16_t* v_scale, int32_t kv_heads, int32_t head_dim, int32_t block_size,
                     int64_t num_pages, int32_t* device_status, qkv_stream_t stream);
 
+/* a3 with the V scale layout as a parameter. The mistral.rs PR's own F4
+ * cache keeps "one scale per 32-value K cell and one scale per token per V
+ * head"; qkv_kv_write_f4 gives V the K layout.
+ *   v_group   values of a V row sharing one scale: 32 (v_scale as in
+ *             qkv_kv_write_f4) or head_dim (v_scale fp16
+ *             [num_pages][kv_heads][block_size][1], one scale per token and
+ *             head: fp16(amax of the row / 7), same rounding and codes).
+ * K is always quantised per 32-value cell. Other arguments, results and
+ * errors as in qkv_kv_write_f4; EINVAL also for any other v_group. */
+QKV_API int qkv_kv_write_f4_v(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping,
+                              int32_t n_tok, uint8_t* k_data, uint16_t* k_scale, uint8_t* v_data,
+                              uint16_t* v_scale, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                              int64_t num_pages, int32_t v_group, int32_t* device_status,
+                              qkv_stream_t stream);
+
 /* a2 + a3 in one launch: the partial rotary of q and of the new k, and the
  * F4 write of the rotated k and of v through the slot mapping.
  *   q_in, q_out  bf16 [n_tok][q_heads][head_dim] (q_out may equal q_in).
@@ -167,6 +182,17 @@ QKV_API int qkv_rope_kv_write_f4(const uint16_t* q_in, uint16_t* q_out, const ui
                                  int64_t table_len, uint8_t* k_data, uint16_t* k_scale,
                                  uint8_t* v_data, uint16_t* v_scale, int32_t block_size,
                                  int64_t num_pages, int32_t* device_status, qkv_stream_t stream);
+
+/* qkv_rope_kv_write_f4 with the V scale layout of qkv_kv_write_f4_v. */
+QKV_API int qkv_rope_kv_write_f4_v(const uint16_t* q_in, uint16_t* q_out, const uint16_t* k_in,
+                                   const uint16_t* v_in, uint16_t* k_out, const int64_t* positions,
+                                   const int64_t* slot_mapping, int32_t n_tok, int32_t q_heads,
+                                   int32_t kv_heads, int32_t head_dim, int32_t rot_dim,
+                                   const float* cos_tab, const float* sin_tab, int64_t table_pos_start,
+                                   int64_t table_len, uint8_t* k_data, uint16_t* k_scale,
+                                   uint8_t* v_data, uint16_t* v_scale, int32_t block_size,
+                                   int64_t num_pages, int32_t v_group, int32_t* device_status,
+                                   qkv_stream_t stream);
 
 /* Number of splits per sequence the automatic plan aims for on the current
  * device (resident split blocks / kv_heads); a workspace sized with this as
@@ -210,6 +236,20 @@ QKV_API int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int32_t
                               float softmax_scale, int32_t num_splits, int32_t* device_status,
                               qkv_stream_t stream);
 
+/* qkv_paged_decode_split_f4 over a cache written with qkv_kv_write_f4_v:
+ * v_group 32 (V scale per cell) or head_dim (one V scale per token; the P V
+ * product then takes one scale per token for all of the row). EINVAL for
+ * any other v_group; other arguments as in qkv_paged_decode_split_f4. */
+QKV_API int qkv_paged_decode_split_f4_v(float* o_parts, float* lse2_parts, int32_t max_splits,
+                                        const uint16_t* q, const uint8_t* k_data,
+                                        const uint16_t* k_scale, const uint8_t* v_data,
+                                        const uint16_t* v_scale, const int32_t* page_table,
+                                        const int32_t* seq_lens, int32_t n_seq, int32_t q_heads,
+                                        int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                        int32_t max_pages_per_seq, int64_t num_pages,
+                                        float softmax_scale, int32_t num_splits, int32_t v_group,
+                                        int32_t* device_status, qkv_stream_t stream);
+
 /* a5 [FOLD] log2-sum-exp merge of partial attention results.
  *   o_parts   float [n_parts][rows][head_dim], lse2_parts float [n_parts][rows].
  *   out       bf16 [rows][head_dim] (nearest even); lse2_out float [rows] or NULL.
@@ -237,6 +277,19 @@ QKV_API int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint1
                              float softmax_scale, int32_t num_splits, int32_t max_splits,
                              void* workspace, size_t workspace_bytes, int32_t* device_status,
                              qkv_stream_t stream);
+
+/* qkv_paged_decode_attn_f4 over a cache written with qkv_kv_write_f4_v
+ * (v_group 32 or head_dim). */
+QKV_API int qkv_paged_decode_attn_f4_v(uint16_t* out, float* lse2_out, const uint16_t* q,
+                                       const uint8_t* k_data, const uint16_t* k_scale,
+                                       const uint8_t* v_data, const uint16_t* v_scale,
+                                       const int32_t* page_table, const int32_t* seq_lens,
+                                       int32_t n_seq, int32_t q_heads, int32_t kv_heads,
+                                       int32_t head_dim, int32_t block_size,
+                                       int32_t max_pages_per_seq, int64_t num_pages,
+                                       float softmax_scale, int32_t num_splits, int32_t max_splits,
+                                       int32_t v_group, void* workspace, size_t workspace_bytes,
+                                       int32_t* device_status, qkv_stream_t stream);
 
 /* Size of the partials array compiled into the library for
  * qkv_paged_decode_attn_f4_static (16 MiB per GPU that loads the library). */

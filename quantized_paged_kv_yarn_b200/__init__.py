@@ -32,5 +32,6 @@ from ._abi import (  # noqa: F401
     qkv_status_string,
     qkv_yarn_auto_factor,
     qkv_yarn_rope_table,
+    v_group_of,
 )
 from .cache import DecodeAttention, PagedF4Cache  # noqa: F401

@@ -60,6 +60,15 @@ _SIGS = {
     "qkv_paged_decode_attn_f4_static": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
                                                        _i32, _i32, _i32, _i32, _i64, _f32, _i32, _vp, _vp]),
     "qkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "qkv_kv_write_f4_v": (ctypes.c_int, [_vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i64, _i32, _vp,
+                                         _vp]),
+    "qkv_rope_kv_write_f4_v": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp,
+                                              _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _vp, _vp]),
+    "qkv_paged_decode_split_f4_v": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+                                                   _i32, _i32, _i32, _i32, _i64, _f32, _i32, _i32, _vp, _vp]),
+    "qkv_paged_decode_attn_f4_v": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                                                  _i32, _i32, _i32, _i64, _f32, _i32, _i32, _i32, _vp, _sz, _vp,
+                                                  _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -130,20 +139,31 @@ def qkv_rope_apply(x_in, x_out, positions, cos_tab, sin_tab, table_pos_start: in
         _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
 
 
+def v_group_of(v_scale, head_dim: int) -> int:
+    """Values per V scale of a cache: 32 (per cell) or head_dim (per token)."""
+    return head_dim // v_scale.shape[-1]
+
+
 def qkv_kv_write_f4(k, v, slot_mapping, k_data, k_scale, v_data, v_scale, device_status=None, stream=None):
     """k/v bf16 [n_tok][kv_heads][head_dim]; cache tensors shaped
-    [num_pages][kv_heads][block_size][head_dim/2 | head_dim/32]."""
+    [num_pages][kv_heads][block_size][head_dim/2 | head_dim/32]; v_scale's
+    last dim 1 selects one V scale per token (qkv_kv_write_f4_v)."""
     n_tok, kv_heads, head_dim = k.shape
     num_pages, kvh2, block_size, half_bytes = k_data.shape
     if kvh2 != kv_heads or half_bytes != head_dim // 2 or tuple(v.shape) != tuple(k.shape):
         raise ValueError("cache/input shapes disagree")
     if slot_mapping.numel() != n_tok:
         raise ValueError(f"slot_mapping has {slot_mapping.numel()} entries for {n_tok} tokens")
-    _check("qkv_kv_write_f4", lib.qkv_kv_write_f4(
-        _ptr(k, "k", _U16), _ptr(v, "v", _U16), _ptr(slot_mapping, "slot_mapping", (torch.int64,), n_tok), n_tok,
-        _ptr(k_data, "k_data", (torch.uint8,)), _ptr(k_scale, "k_scale", _U16), _ptr(v_data, "v_data", (torch.uint8,)),
-        _ptr(v_scale, "v_scale", _U16), kv_heads, head_dim, block_size, num_pages,
-        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+    args = (_ptr(k, "k", _U16), _ptr(v, "v", _U16), _ptr(slot_mapping, "slot_mapping", (torch.int64,), n_tok), n_tok,
+            _ptr(k_data, "k_data", (torch.uint8,)), _ptr(k_scale, "k_scale", _U16),
+            _ptr(v_data, "v_data", (torch.uint8,)), _ptr(v_scale, "v_scale", _U16), kv_heads, head_dim, block_size,
+            num_pages)
+    tail = (_ptr(device_status, "device_status", (torch.int32,)), _stream(stream))
+    vg = v_group_of(v_scale, head_dim)
+    if vg == 32:
+        _check("qkv_kv_write_f4", lib.qkv_kv_write_f4(*args, *tail))
+    else:
+        _check("qkv_kv_write_f4_v", lib.qkv_kv_write_f4_v(*args, vg, *tail))
 
 
 def qkv_rope_kv_write_f4(q_in, q_out, k_in, v_in, positions, slot_mapping, cos_tab, sin_tab, table_pos_start: int,
@@ -159,13 +179,18 @@ def qkv_rope_kv_write_f4(q_in, q_out, k_in, v_in, positions, slot_mapping, cos_t
         raise ValueError("q/k/v shapes disagree")
     if slot_mapping.numel() != n_tok or positions.numel() != n_tok:
         raise ValueError("positions and slot_mapping need one entry per token")
-    _check("qkv_rope_kv_write_f4", lib.qkv_rope_kv_write_f4(
-        _ptr(q_in, "q_in", _U16), _ptr(q_out, "q_out", _U16), _ptr(k_in, "k_in", _U16), _ptr(v_in, "v_in", _U16),
-        _ptr(k_out, "k_out", _U16), _ptr(positions, "positions", (torch.int64,), n_tok),
-        _ptr(slot_mapping, "slot_mapping", (torch.int64,), n_tok), n_tok, q_heads, kv_heads, head_dim, rot_dim,
-        _ptr(cos_tab, "cos_tab", (torch.float32,)), _ptr(sin_tab, "sin_tab", (torch.float32,)), int(table_pos_start),
-        cos_tab.numel() // half, *_cache_args(k_data, k_scale, v_data, v_scale), block_size, num_pages,
-        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+    args = (_ptr(q_in, "q_in", _U16), _ptr(q_out, "q_out", _U16), _ptr(k_in, "k_in", _U16), _ptr(v_in, "v_in", _U16),
+            _ptr(k_out, "k_out", _U16), _ptr(positions, "positions", (torch.int64,), n_tok),
+            _ptr(slot_mapping, "slot_mapping", (torch.int64,), n_tok), n_tok, q_heads, kv_heads, head_dim, rot_dim,
+            _ptr(cos_tab, "cos_tab", (torch.float32,)), _ptr(sin_tab, "sin_tab", (torch.float32,)),
+            int(table_pos_start), cos_tab.numel() // half, *_cache_args(k_data, k_scale, v_data, v_scale), block_size,
+            num_pages)
+    tail = (_ptr(device_status, "device_status", (torch.int32,)), _stream(stream))
+    vg = v_group_of(v_scale, head_dim)
+    if vg == 32:
+        _check("qkv_rope_kv_write_f4", lib.qkv_rope_kv_write_f4(*args, *tail))
+    else:
+        _check("qkv_rope_kv_write_f4_v", lib.qkv_rope_kv_write_f4_v(*args, vg, *tail))
 
 
 def qkv_paged_decode_auto_splits(kv_heads: int, block_size: int) -> int:
@@ -189,13 +214,18 @@ def qkv_paged_decode_split_f4(o_parts, lse2_parts, q, k_data, k_scale, v_data, v
     n_seq, q_heads, head_dim = q.shape
     max_splits = o_parts.shape[0]
     num_pages, _, block_size, _ = k_data.shape
-    _check("qkv_paged_decode_split_f4", lib.qkv_paged_decode_split_f4(
-        _ptr(o_parts, "o_parts", (torch.float32,), max_splits * n_seq * q_heads * head_dim),
-        _ptr(lse2_parts, "lse2_parts", (torch.float32,), max_splits * n_seq * q_heads), max_splits,
-        _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),
-        _ptr(page_table, "page_table", (torch.int32,)), _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq), n_seq,
-        q_heads, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, float(softmax_scale),
-        int(num_splits), _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+    args = (_ptr(o_parts, "o_parts", (torch.float32,), max_splits * n_seq * q_heads * head_dim),
+            _ptr(lse2_parts, "lse2_parts", (torch.float32,), max_splits * n_seq * q_heads), max_splits,
+            _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),
+            _ptr(page_table, "page_table", (torch.int32,)), _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq),
+            n_seq, q_heads, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, float(softmax_scale),
+            int(num_splits))
+    tail = (_ptr(device_status, "device_status", (torch.int32,)), _stream(stream))
+    vg = v_group_of(v_scale, head_dim)
+    if vg == 32:
+        _check("qkv_paged_decode_split_f4", lib.qkv_paged_decode_split_f4(*args, *tail))
+    else:
+        _check("qkv_paged_decode_split_f4_v", lib.qkv_paged_decode_split_f4_v(*args, vg, *tail))
 
 
 def qkv_lse_merge(o_parts, lse2_parts, out, lse2_out=None, stream=None):
@@ -214,13 +244,18 @@ def qkv_paged_decode_attn_f4(out, q, k_data, k_scale, v_data, v_scale, page_tabl
     at least qkv_paged_decode_workspace_bytes(...) bytes."""
     n_seq, q_heads, head_dim = q.shape
     num_pages, _, block_size, _ = k_data.shape
-    _check("qkv_paged_decode_attn_f4", lib.qkv_paged_decode_attn_f4(
-        _ptr(out, "out", _U16, n_seq * q_heads * head_dim), _ptr(lse2_out, "lse2_out", (torch.float32,)),
-        _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),
-        _ptr(page_table, "page_table", (torch.int32,)), _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq), n_seq,
-        q_heads, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, float(softmax_scale),
-        int(num_splits), int(max_splits), _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+    args = (_ptr(out, "out", _U16, n_seq * q_heads * head_dim), _ptr(lse2_out, "lse2_out", (torch.float32,)),
+            _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),
+            _ptr(page_table, "page_table", (torch.int32,)), _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq),
+            n_seq, q_heads, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, float(softmax_scale),
+            int(num_splits), int(max_splits))
+    ws = (_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size())
+    tail = (_ptr(device_status, "device_status", (torch.int32,)), _stream(stream))
+    vg = v_group_of(v_scale, head_dim)
+    if vg == 32:
+        _check("qkv_paged_decode_attn_f4", lib.qkv_paged_decode_attn_f4(*args, *ws, *tail))
+    else:
+        _check("qkv_paged_decode_attn_f4_v", lib.qkv_paged_decode_attn_f4_v(*args, vg, *ws, *tail))
 
 
 STATIC_SCRATCH_BYTES = 16 << 20
@@ -235,6 +270,8 @@ def qkv_paged_decode_attn_f4_static(out, q, k_data, k_scale, v_data, v_scale, pa
     overlapping calls race on the shared array."""
     n_seq, q_heads, head_dim = q.shape
     num_pages, _, block_size, _ = k_data.shape
+    if v_group_of(v_scale, head_dim) != 32:
+        raise ValueError("qkv_paged_decode_attn_f4_static takes caches with one V scale per 32-value cell")
     _check("qkv_paged_decode_attn_f4_static", lib.qkv_paged_decode_attn_f4_static(
         _ptr(out, "out", _U16, n_seq * q_heads * head_dim), _ptr(lse2_out, "lse2_out", (torch.float32,)),
         _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),

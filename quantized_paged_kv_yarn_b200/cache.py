@@ -13,7 +13,10 @@ from . import _abi
 @dataclasses.dataclass
 class PagedF4Cache:
     """One layer's F4 cache: data u8 [num_pages][kv_heads][block][head_dim/2]
-    and fp16 scales [num_pages][kv_heads][block][head_dim/32], for K and V."""
+    and fp16 scales [num_pages][kv_heads][block][head_dim/32], for K and V;
+    with v_group=head_dim the V scales are [num_pages][kv_heads][block][1]
+    (one per token and head). The library calls read the V layout from the
+    last dimension of v_scale."""
 
     k_data: torch.Tensor
     k_scale: torch.Tensor
@@ -21,11 +24,14 @@ class PagedF4Cache:
     v_scale: torch.Tensor
 
     @classmethod
-    def allocate(cls, num_pages: int, kv_heads: int, block_size: int, head_dim: int, device="cuda"):
+    def allocate(cls, num_pages: int, kv_heads: int, block_size: int, head_dim: int, device="cuda",
+                 v_group: int = 32):
+        if v_group not in (32, head_dim):
+            raise ValueError(f"v_group must be 32 or head_dim ({head_dim}), got {v_group}")
         d = lambda: torch.zeros((num_pages, kv_heads, block_size, head_dim // 2), dtype=torch.uint8, device=device)
-        s = lambda: torch.zeros((num_pages, kv_heads, block_size, head_dim // 32), dtype=torch.float16,
-                                device=device)
-        return cls(d(), s(), d(), s())
+        s = lambda g: torch.zeros((num_pages, kv_heads, block_size, head_dim // g), dtype=torch.float16,
+                                  device=device)
+        return cls(d(), s(32), d(), s(v_group))
 
     @property
     def num_pages(self) -> int:
@@ -42,6 +48,10 @@ class PagedF4Cache:
     @property
     def head_dim(self) -> int:
         return self.k_data.shape[3] * 2
+
+    @property
+    def v_group(self) -> int:
+        return _abi.v_group_of(self.v_scale, self.head_dim)
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in (self.k_data, self.k_scale, self.v_data, self.v_scale))

@@ -246,7 +246,7 @@ __device__ void plan(const Params& p, int seq, int split, int block, int& S, int
   pg1 = muldiv((uint32_t)split + 1, n, (uint32_t)S);
 }
 
-template <int BLOCK, int G>
+template <int BLOCK, int G, bool VTOK>
 __global__ void __launch_bounds__(THREADS, 1)
     paged_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                               const Params p) {
@@ -254,6 +254,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "query heads per KV head");
   constexpr int HQ = Cfg<G>::HQ;
   constexpr int PPS = STAGE_TOK / BLOCK;  // pages per stage
+  // V scales: one per 32-value cell (16 bytes per token), or one per token
+  constexpr int VSROW = VTOK ? 2 : SROW_BYTES;
+  constexpr int VCELLS = VTOK ? 1 : CELLS;
   using SmemT = Smem<HQ>;
 
   extern __shared__ uint8_t smem_raw[];
@@ -375,9 +378,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
     gs.mask[ks] = mask;
-    const uint32_t bytes = npages * BLOCK * (ROW_BYTES + SROW_BYTES);
-    mbar_arrive_expect_tx(&gs.kfull[ks], bytes);
-    mbar_arrive_expect_tx(&gs.vfull[vs], bytes);
+    mbar_arrive_expect_tx(&gs.kfull[ks], npages * BLOCK * (ROW_BYTES + SROW_BYTES));
+    mbar_arrive_expect_tx(&gs.vfull[vs], npages * BLOCK * (ROW_BYTES + VSROW));
 #pragma unroll
     for (int k = 0; k < PPS; ++k) {
       if (phys[k] < 0) continue;
@@ -386,8 +388,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       bulk_load(&gs.ks[ks][k * BLOCK * SROW_BYTES], p.k_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
                 &gs.kfull[ks], pol);
       tma_load_2d(&gs.v[vs][k * BLOCK * ROW_BYTES], &tm_v, &gs.vfull[vs], 0, row, pol);
-      bulk_load(&gs.vs[vs][k * BLOCK * SROW_BYTES], p.v_scale + (size_t)row * CELLS, BLOCK * SROW_BYTES,
-                &gs.vfull[vs], pol);
+      bulk_load(&gs.vs[vs][k * BLOCK * VSROW], p.v_scale + (size_t)row * VCELLS, BLOCK * VSROW, &gs.vfull[vs],
+                pol);
     }
     atomicMax(&gs.issued, j + 1);
   };
@@ -561,6 +563,35 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto pv_step = [&](int kk, uint32_t km) {
       const uint32_t b01 = lds32(prow + 16 * kk + 2 * t);
       const uint32_t b23 = lds32(prow + 16 * kk + 2 * t + 8);
+      if constexpr (VTOK) {
+        // one scale per token: the pair of tokens 2t, 2t+1 (and +8) is one
+        // word, and one B operand serves both cells
+        const uint16_t* sv = reinterpret_cast<const uint16_t*>(vsb) + 16 * kk + 2 * t;
+        uint32_t s01 = lds32(sv), s89 = lds32(sv + 8);
+        if constexpr (decltype(partial)::value) {
+          s01 &= (((km >> (2 * t)) & 1u) ? 0x0000ffffu : 0u) | (((km >> (2 * t + 1)) & 1u) ? 0xffff0000u : 0u);
+          s89 &= (((km >> (2 * t + 8)) & 1u) ? 0x0000ffffu : 0u) | (((km >> (2 * t + 9)) & 1u) ? 0xffff0000u : 0u);
+        }
+        const uint32_t b01c = h2_as_u32(__hmul2(u32_as_h2(b01), u32_as_h2(s01)));
+        const uint32_t b23c = h2_as_u32(__hmul2(u32_as_h2(b23), u32_as_h2(s89)));
+        uint32_t vw[4];
+        ldsm_x4_trans(vbase + (uint32_t)(16 * kk * ROW_BYTES), vw);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint32_t za = vw[2 * c], zb = vw[2 * c + 1];
+          const uint32_t za8 = za >> 8, zb8 = zb >> 8;
+          mma_f16(acc[c][0], za & LO4, za & HI4, zb & LO4, zb & HI4, b01c, b23c);
+          mma_f16(acc[c][1], za8 & LO4, za8 & HI4, zb8 & LO4, zb8 & HI4, b01c, b23c);
+        }
+        // the -8 offset, sum over tokens of p * v_scale per head: an MMA
+        // with an all-ones A sums the B columns
+        constexpr uint32_t ONES = 0x3C003C00u;  // fp16 pair (1, 1)
+        float dd[4];
+        mma_f16_c(dd, ONES, ONES, ONES, ONES, b01c, b23c, vsum[0], vsum[1], 0.f, 0.f);
+        vsum[0] = dd[0];
+        vsum[1] = dd[1];
+        return;
+      }
       const uint8_t* sr = vsb + (16 * kk + 2 * t) * SROW_BYTES + 4 * gw;  // cells 2w, 2w+1
       uint32_t s0 = lds32(sr), s1 = lds32(sr + SROW_BYTES), s2 = lds32(sr + 8 * SROW_BYTES),
                s3 = lds32(sr + 9 * SROW_BYTES);
@@ -596,7 +627,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // The -8 offset: this warp sums p * v_scale over its own k-step (tokens
     // 16w .. 16w + 15) for every cell; the group's warps add up at the end.
     const uint32_t wm = (uint32_t)(smask >> (16 * gw)) & 0xffffu;
-    if (!decltype(partial)::value || wm != 0u) {
+    if (!VTOK && (!decltype(partial)::value || wm != 0u)) {
       const uint32_t b01 = lds32(prow + 16 * gw + 2 * t);
       const uint32_t b23 = lds32(prow + 16 * gw + 2 * t + 8);
       // A: the V scales transposed, row = cell g, k = tokens
@@ -798,11 +829,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   for (int c = 0; c < 2; ++c) {
     const int cell = 2 * gw + c;
     float b0 = 0.f, b1 = 0.f;
+    if constexpr (VTOK) {  // the warp's own sum covers every token and cell
+      b0 = vsum[0];
+      b1 = vsum[1];
+    } else {
 #pragma unroll
-    for (int w = 0; w < GWARPS; ++w) {
-      const float2 v = vsp[w * 32 + 4 * cell + t];
-      b0 += v.x;
-      b1 += v.y;
+      for (int w = 0; w < GWARPS; ++w) {
+        const float2 v = vsp[w * 32 + 4 * cell + t];
+        b0 += v.x;
+        b1 += v.y;
+      }
     }
     b0 *= 8.f;
     b1 *= 8.f;
@@ -902,19 +938,20 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, int block) {
 }
 
 template <int BLOCK, int G>
-const void* kernel_ptr() {
-  return reinterpret_cast<const void*>(&paged_decode_split_kernel<BLOCK, G>);
+const void* kernel_ptr(bool vtok) {
+  return vtok ? reinterpret_cast<const void*>(&paged_decode_split_kernel<BLOCK, G, true>)
+              : reinterpret_cast<const void*>(&paged_decode_split_kernel<BLOCK, G, false>);
 }
 
 size_t kernel_smem(int G) { return G > 4 ? smem_bytes<2>() : smem_bytes<1>(); }
 
-const void* pick_kernel(int block, int G) {
+const void* pick_kernel(int block, int G, bool vtok = false) {
 #define QKV_PICK(B)                         \
   if (block == B) {                         \
-    if (G == 1) return kernel_ptr<B, 1>();  \
-    if (G == 2) return kernel_ptr<B, 2>();  \
-    if (G == 4) return kernel_ptr<B, 4>();  \
-    if (G == 8) return kernel_ptr<B, 8>();  \
+    if (G == 1) return kernel_ptr<B, 1>(vtok);  \
+    if (G == 2) return kernel_ptr<B, 2>(vtok);  \
+    if (G == 4) return kernel_ptr<B, 4>(vtok);  \
+    if (G == 8) return kernel_ptr<B, 8>(vtok);  \
   }
   QKV_PICK(16)
   QKV_PICK(32)
@@ -927,24 +964,24 @@ constexpr int MAX_DEVICES = 64;
 
 // Opt the kernel into its shared-memory size on the current device (once)
 // and return its resident CTAs per SM.
-int prepare(const void* fn, int block, int G) {
+int prepare(const void* fn, int block, int G, bool vtok = false) {
   static std::mutex mu;
-  static int occ[MAX_DEVICES][3][4];  // 0 = not prepared
+  static int occ[MAX_DEVICES][3][4][2];  // 0 = not prepared
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return 0;
   const int bi = block == 16 ? 0 : block == 32 ? 1 : 2;
   const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
   std::lock_guard<std::mutex> lock(mu);
-  if (occ[dev][bi][gi] == 0) {
+  if (occ[dev][bi][gi][vtok ? 1 : 0] == 0) {
     const size_t smem = kernel_smem(G);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return 0;
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, THREADS, smem) != cudaSuccess || n < 1)
       return 0;
-    occ[dev][bi][gi] = n;
+    occ[dev][bi][gi][vtok ? 1 : 0] = n;
   }
-  return occ[dev][bi][gi];
+  return occ[dev][bi][gi][vtok ? 1 : 0];
 }
 
 int sm_count() {
@@ -977,17 +1014,19 @@ extern "C" size_t qkv_paged_decode_workspace_bytes(int32_t n_seq, int32_t q_head
   return o + l;
 }
 
-extern "C" int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int32_t max_splits, const uint16_t* q,
-                                         const uint8_t* k_data, const uint16_t* k_scale, const uint8_t* v_data,
-                                         const uint16_t* v_scale, const int32_t* page_table,
-                                         const int32_t* seq_lens, int32_t n_seq, int32_t q_heads,
-                                         int32_t kv_heads, int32_t head_dim, int32_t block_size,
-                                         int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
-                                         int32_t num_splits, int32_t* device_status, qkv_stream_t stream) {
+extern "C" int qkv_paged_decode_split_f4_v(float* o_parts, float* lse2_parts, int32_t max_splits,
+                                           const uint16_t* q, const uint8_t* k_data, const uint16_t* k_scale,
+                                           const uint8_t* v_data, const uint16_t* v_scale,
+                                           const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
+                                           int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                           int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                                           int32_t num_splits, int32_t v_group, int32_t* device_status,
+                                           qkv_stream_t stream) {
   if (!o_parts || !lse2_parts || !q || !k_data || !k_scale || !v_data || !v_scale || !page_table || !seq_lens)
     return QKV_EINVAL;
   if (n_seq < 0 || q_heads < 1 || kv_heads < 1 || max_pages_per_seq < 1 || num_pages < 1 || max_splits < 1 ||
-      num_splits < 0 || block_size < 1 || !(softmax_scale >= 0.f) || !isfinite(softmax_scale))
+      num_splits < 0 || block_size < 1 || !(softmax_scale >= 0.f) || !isfinite(softmax_scale) ||
+      (v_group != 32 && v_group != head_dim))
     return QKV_EINVAL;
   if (q_heads % kv_heads) return QKV_EINVAL;
   if (!aligned16(q) || !aligned16(k_data) || !aligned16(v_data) || !aligned16(k_scale) || !aligned16(v_scale) ||
@@ -995,7 +1034,8 @@ extern "C" int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int3
     return QKV_EINVAL;
   const int G = q_heads / kv_heads;
   if (head_dim != D) return QKV_EUNSUPPORTED;
-  const void* fn = pick_kernel(block_size, G);
+  const bool vtok = v_group != 32;
+  const void* fn = pick_kernel(block_size, G, vtok);
   if (!fn) return QKV_EUNSUPPORTED;
   const uint64_t cache_rows = (uint64_t)num_pages * kv_heads * block_size;
   if (cache_rows > 0x7fffffffull) return QKV_EUNSUPPORTED;  // TMA row coordinate is int32
@@ -1003,7 +1043,7 @@ extern "C" int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int3
   if (max_splits > 65535 * 16 || n_seq > 65535 || kv_heads > 65535) return QKV_EUNSUPPORTED;
   if (n_seq == 0) return QKV_OK;
 
-  const int occ = prepare(fn, block_size, G);
+  const int occ = prepare(fn, block_size, G, vtok);
   const int sms = sm_count();
   if (occ < 1 || sms < 1) return QKV_ECUDA;
 
@@ -1042,13 +1082,26 @@ extern "C" int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int3
   return QKV_OK;
 }
 
-extern "C" int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
-                                        const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
-                                        const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
-                                        int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
-                                        int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
-                                        int32_t num_splits, int32_t max_splits, void* workspace,
-                                        size_t workspace_bytes, int32_t* device_status, qkv_stream_t stream) {
+extern "C" int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int32_t max_splits, const uint16_t* q,
+                                         const uint8_t* k_data, const uint16_t* k_scale, const uint8_t* v_data,
+                                         const uint16_t* v_scale, const int32_t* page_table,
+                                         const int32_t* seq_lens, int32_t n_seq, int32_t q_heads,
+                                         int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                         int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                                         int32_t num_splits, int32_t* device_status, qkv_stream_t stream) {
+  return qkv_paged_decode_split_f4_v(o_parts, lse2_parts, max_splits, q, k_data, k_scale, v_data, v_scale,
+                                     page_table, seq_lens, n_seq, q_heads, kv_heads, head_dim, block_size,
+                                     max_pages_per_seq, num_pages, softmax_scale, num_splits, 32, device_status,
+                                     stream);
+}
+
+extern "C" int qkv_paged_decode_attn_f4_v(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
+                                          const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
+                                          const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
+                                          int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                          int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                                          int32_t num_splits, int32_t max_splits, int32_t v_group, void* workspace,
+                                          size_t workspace_bytes, int32_t* device_status, qkv_stream_t stream) {
   if (!out || !workspace) return QKV_EINVAL;
   if (((uintptr_t)workspace & 255) || max_splits < 1 || n_seq < 0 || q_heads < 1) return QKV_EINVAL;
   if (workspace_bytes < qkv_paged_decode_workspace_bytes(n_seq, q_heads, head_dim, max_splits)) return QKV_EINVAL;
@@ -1057,9 +1110,23 @@ extern "C" int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const ui
   float* o_parts = reinterpret_cast<float*>(workspace);
   float* lse_parts =
       reinterpret_cast<float*>((char*)workspace + ((rows * max_splits * head_dim * 4 + 255) & ~size_t(255)));
-  int rc = qkv_paged_decode_split_f4(o_parts, lse_parts, max_splits, q, k_data, k_scale, v_data, v_scale,
-                                     page_table, seq_lens, n_seq, q_heads, kv_heads, head_dim, block_size,
-                                     max_pages_per_seq, num_pages, softmax_scale, num_splits, device_status, stream);
+  int rc = qkv_paged_decode_split_f4_v(o_parts, lse_parts, max_splits, q, k_data, k_scale, v_data, v_scale,
+                                       page_table, seq_lens, n_seq, q_heads, kv_heads, head_dim, block_size,
+                                       max_pages_per_seq, num_pages, softmax_scale, num_splits, v_group,
+                                       device_status, stream);
   if (rc != QKV_OK) return rc;
   return qkv_lse_merge(o_parts, lse_parts, max_splits, (int32_t)rows, head_dim, out, lse2_out, stream);
+}
+
+extern "C" int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
+                                        const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
+                                        const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
+                                        int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                        int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                                        int32_t num_splits, int32_t max_splits, void* workspace,
+                                        size_t workspace_bytes, int32_t* device_status, qkv_stream_t stream) {
+  return qkv_paged_decode_attn_f4_v(out, lse2_out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, n_seq,
+                                    q_heads, kv_heads, head_dim, block_size, max_pages_per_seq, num_pages,
+                                    softmax_scale, num_splits, max_splits, 32, workspace, workspace_bytes,
+                                    device_status, stream);
 }

@@ -22,7 +22,8 @@ __global__ void __launch_bounds__(256) rope_kv_write_kernel(
     const int64_t* __restrict__ positions, const int64_t* __restrict__ slots, int n_tok, int q_heads,
     int kv_heads, int head_dim, int rot, const float* __restrict__ cos_tab, const float* __restrict__ sin_tab,
     int64_t tab_start, int64_t tab_len, uint8_t* __restrict__ k_data, __half* __restrict__ k_scale,
-    uint8_t* __restrict__ v_data, __half* __restrict__ v_scale, int block, int64_t num_pages, int32_t* status) {
+    uint8_t* __restrict__ v_data, __half* __restrict__ v_scale, int block, int64_t num_pages, int v_group,
+    int32_t* status) {
   pdl_wait();
   pdl_release();
   const int lane = threadIdx.x & 31;
@@ -111,8 +112,11 @@ __global__ void __launch_bounds__(256) rope_kv_write_kernel(
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
-  amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, 2));
+  // Lanes per scale group: 4 for a 32-value cell; the whole warp for a V
+  // group of head_dim values (lanes past head_dim / 8 hold amax 0).
+  const int group = is_k ? 32 : v_group;
+  const int gl = group == 32 ? 4 : 32;
+  for (int o = 1; o < gl; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, o));
   if (!active) return;
   const __half sh = __float2half_rn(fminf(__fdiv_rn(amax, 7.0f), 65504.0f));
   const float s = __half2float(sh);
@@ -126,27 +130,28 @@ __global__ void __launch_bounds__(256) rope_kv_write_kernel(
   const int64_t page = slot / block, off = slot - page * block;
   const int64_t crow = (page * kv_heads + h) * block + off;
   reinterpret_cast<uint32_t*>((is_k ? k_data : v_data) + crow * (head_dim / 2))[lane] = word;
-  if ((lane & 3) == 0) (is_k ? k_scale : v_scale)[crow * (head_dim / 32) + lane / 4] = sh;
+  if ((lane & (gl - 1)) == 0) (is_k ? k_scale : v_scale)[crow * (head_dim / group) + lane / gl] = sh;
 }
 
 }  // namespace qkv
 
 using namespace qkv;
 
-extern "C" int qkv_rope_kv_write_f4(const uint16_t* q_in, uint16_t* q_out, const uint16_t* k_in,
-                                    const uint16_t* v_in, uint16_t* k_out, const int64_t* positions,
-                                    const int64_t* slot_mapping, int32_t n_tok, int32_t q_heads,
-                                    int32_t kv_heads, int32_t head_dim, int32_t rot_dim, const float* cos_tab,
-                                    const float* sin_tab, int64_t table_pos_start, int64_t table_len,
-                                    uint8_t* k_data, uint16_t* k_scale, uint8_t* v_data, uint16_t* v_scale,
-                                    int32_t block_size, int64_t num_pages, int32_t* device_status,
-                                    qkv_stream_t stream) {
+extern "C" int qkv_rope_kv_write_f4_v(const uint16_t* q_in, uint16_t* q_out, const uint16_t* k_in,
+                                      const uint16_t* v_in, uint16_t* k_out, const int64_t* positions,
+                                      const int64_t* slot_mapping, int32_t n_tok, int32_t q_heads,
+                                      int32_t kv_heads, int32_t head_dim, int32_t rot_dim, const float* cos_tab,
+                                      const float* sin_tab, int64_t table_pos_start, int64_t table_len,
+                                      uint8_t* k_data, uint16_t* k_scale, uint8_t* v_data, uint16_t* v_scale,
+                                      int32_t block_size, int64_t num_pages, int32_t v_group,
+                                      int32_t* device_status, qkv_stream_t stream) {
   if (n_tok == 0) return QKV_OK;
   if (!q_in || !q_out || !k_in || !v_in || !positions || !slot_mapping || !cos_tab || !sin_tab || !k_data ||
       !k_scale || !v_data || !v_scale)
     return QKV_EINVAL;
   if (n_tok < 0 || q_heads < 0 || kv_heads < 1 || head_dim < 32 || head_dim > 256 || head_dim % 32 ||
-      rot_dim < 16 || rot_dim % 16 || rot_dim > head_dim || table_len < 0 || block_size < 1 || num_pages < 1)
+      rot_dim < 16 || rot_dim % 16 || rot_dim > head_dim || table_len < 0 || block_size < 1 || num_pages < 1 ||
+      (v_group != 32 && v_group != head_dim))
     return QKV_EINVAL;
   if (((uintptr_t)k_in | (uintptr_t)v_in | (uintptr_t)k_out) & 15) return QKV_EINVAL;
   if (((uintptr_t)k_data | (uintptr_t)v_data) & 3) return QKV_EINVAL;
@@ -163,14 +168,27 @@ extern "C" int qkv_rope_kv_write_f4(const uint16_t* q_in, uint16_t* q_out, const
   __nv_bfloat16* qo = reinterpret_cast<__nv_bfloat16*>(q_out);
   __half* ks = reinterpret_cast<__half*>(k_scale);
   __half* vs = reinterpret_cast<__half*>(v_scale);
-  int nt = n_tok, hq = q_heads, hkv = kv_heads, hd = head_dim, rd = rot_dim, bs = block_size;
+  int nt = n_tok, hq = q_heads, hkv = kv_heads, hd = head_dim, rd = rot_dim, bs = block_size, vg = v_group;
   void* args[] = {&qi, &qo, &k_in, &v_in, &k_out, &positions, &slot_mapping, &nt, &hq, &hkv, &hd, &rd,
                   &cos_tab, &sin_tab, &table_pos_start, &table_len, &k_data, &ks, &v_data, &vs, &bs, &num_pages,
-                  &device_status};
+                  &vg, &device_status};
   if (launch_pdl((const void*)rope_kv_write_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, args) !=
       cudaSuccess) {
     (void)cudaGetLastError();
     return QKV_ECUDA;
   }
   return QKV_OK;
+}
+
+extern "C" int qkv_rope_kv_write_f4(const uint16_t* q_in, uint16_t* q_out, const uint16_t* k_in,
+                                    const uint16_t* v_in, uint16_t* k_out, const int64_t* positions,
+                                    const int64_t* slot_mapping, int32_t n_tok, int32_t q_heads,
+                                    int32_t kv_heads, int32_t head_dim, int32_t rot_dim, const float* cos_tab,
+                                    const float* sin_tab, int64_t table_pos_start, int64_t table_len,
+                                    uint8_t* k_data, uint16_t* k_scale, uint8_t* v_data, uint16_t* v_scale,
+                                    int32_t block_size, int64_t num_pages, int32_t* device_status,
+                                    qkv_stream_t stream) {
+  return qkv_rope_kv_write_f4_v(q_in, q_out, k_in, v_in, k_out, positions, slot_mapping, n_tok, q_heads, kv_heads,
+                                head_dim, rot_dim, cos_tab, sin_tab, table_pos_start, table_len, k_data, k_scale,
+                                v_data, v_scale, block_size, num_pages, 32, device_status, stream);
 }

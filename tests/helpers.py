@@ -6,12 +6,13 @@ import oracle
 import workloads
 
 
-def oracle_layer(w, layer=0, inputs=None, with_step=True):
+def oracle_layer(w, layer=0, inputs=None, with_step=True, v_group=32):
     """Quantise a workload layer into an oracle cache. Returns (inputs, cache).
     With ``with_step`` the decode step's (unroped) k_new/v_new are written too,
-    at the step slots; rotary is the caller's business."""
+    at the step slots; rotary is the caller's business. ``v_group`` picks the
+    V scale layout (32 per cell, head_dim per token)."""
     x = inputs if inputs is not None else workloads.host_layer(w, layer)
-    cache = oracle.empty_cache(w.num_pages, w.kv_heads, w.block_size, w.head_dim)
+    cache = oracle.empty_cache(w.num_pages, w.kv_heads, w.block_size, w.head_dim, v_group=v_group)
     bad = oracle.kv_write_f4(x["k_cache"], x["v_cache"], x["cache_slots"], cache, w.kv_heads, w.head_dim,
                              w.block_size)
     assert bad == 0

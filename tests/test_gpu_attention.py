@@ -17,8 +17,8 @@ def qkv():
     return q
 
 
-def _dev_cache(qkv, w, x):
-    cache = qkv.PagedF4Cache.allocate(w.num_pages, w.kv_heads, w.block_size, w.head_dim)
+def _dev_cache(qkv, w, x, v_group=32):
+    cache = qkv.PagedF4Cache.allocate(w.num_pages, w.kv_heads, w.block_size, w.head_dim, v_group=v_group)
     cache.write(to_dev(x["k_cache"]), to_dev(x["v_cache"]), to_dev(x["cache_slots"]))
     cache.write(to_dev(x["k_new"]), to_dev(x["v_new"]), to_dev(x["step_slots"]))
     return cache
@@ -83,13 +83,34 @@ def test_decode_attention_matches_oracle(qkv, case):
     _assert_close(out, lse, ref_out, ref_lse)
 
 
+# One V scale per token and head (the PR's own V layout): a subset of the
+# cases above with every block size, ragged tails, empty contexts and splits.
+VTOK_CASES = [CASES[i] for i in (0, 2, 3, 4, 6, 7, 9)]
+
+
+@pytest.mark.parametrize("case", VTOK_CASES, ids=[f"L{c[0]}-B{c[1]}-G{c[2] // c[3]}-S{c[5]}" for c in VTOK_CASES])
+def test_decode_attention_per_token_v_scale(qkv, case):
+    seq_lens, block, hq, hkv, pages, splits = case
+    w = workloads.small("vtok", seq_lens=seq_lens, num_pages=pages, block_size=block, q_heads=hq, kv_heads=hkv,
+                        page_alloc="interleaved" if len(seq_lens) > 1 else "contiguous", head_scale=True)
+    x, ref = oracle_layer(w, v_group=w.head_dim)
+    cache = _dev_cache(qkv, w, x, v_group=w.head_dim)
+    assert cache.v_group == w.head_dim and cache.v_scale.shape[-1] == 1
+    _check_cache_equal(cache, ref)
+    out, lse, st = _run_attn(qkv, w, x, cache, num_splits=splits)
+    assert st == 0
+    ref_out, ref_lse = _oracle_attn(w, x, ref)
+    _assert_close(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("v_group", [32, 256])
 @pytest.mark.parametrize("num_splits", [1, 4, 9])
-def test_split_partials_match_oracle_ranges(qkv, num_splits):
+def test_split_partials_match_oracle_ranges(qkv, num_splits, v_group):
     """Each split's fp32 partial (o, lse2) equals exact attention over that
     split's page range; the fp32 partials meet 2e-3 with no bf16 allowance."""
     w = workloads.small("parts", seq_lens=(900, 130), num_pages=80, block_size=16, head_scale=True)
-    x, ref = oracle_layer(w)
-    cache = _dev_cache(qkv, w, x)
+    x, ref = oracle_layer(w, v_group=v_group)
+    cache = _dev_cache(qkv, w, x, v_group=v_group)
     rows = w.n_seq * w.q_heads
     o_parts = torch.empty((num_splits, rows, 256), dtype=torch.float32, device="cuda")
     l_parts = torch.empty((num_splits, rows), dtype=torch.float32, device="cuda")
@@ -148,10 +169,11 @@ def test_page_permutation_invariance_gpu(qkv):
     assert np.array_equal(out1, out2) and np.array_equal(lse1, lse2)
 
 
-def test_single_token_is_exact_value(qkv):
+@pytest.mark.parametrize("v_group", [32, 256])
+def test_single_token_is_exact_value(qkv, v_group):
     w = workloads.small("one", seq_lens=(1, 1), num_pages=2, block_size=64)
-    x, ref = oracle_layer(w)
-    cache = _dev_cache(qkv, w, x)
+    x, ref = oracle_layer(w, v_group=v_group)
+    cache = _dev_cache(qkv, w, x, v_group=v_group)
     out, lse, st = _run_attn(qkv, w, x, cache)
     ro, rl = _oracle_attn(w, x, ref)
     # p = 1 exactly: the output is the dequantised value, rounded to bf16 once

@@ -94,19 +94,22 @@ def test_rope_position_outside_table(qkv):
     assert np.array_equal(to_host(out, np.uint16)[1], to_host(x, np.uint16)[1])
 
 
-def _write_both(qkv, k, v, slots, num_pages, kv_heads, block, head_dim):
-    cache = qkv.PagedF4Cache.allocate(num_pages, kv_heads, block, head_dim)
+def _write_both(qkv, k, v, slots, num_pages, kv_heads, block, head_dim, v_group=32):
+    cache = qkv.PagedF4Cache.allocate(num_pages, kv_heads, block, head_dim, v_group=v_group)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     cache.write(to_dev(k), to_dev(v), to_dev(slots), device_status=st)
-    ref = oracle.empty_cache(num_pages, kv_heads, block, head_dim)
+    ref = oracle.empty_cache(num_pages, kv_heads, block, head_dim, v_group=v_group)
     bad = oracle.kv_write_f4(k, v, slots, ref, kv_heads, head_dim, block)
     got = (to_host(cache.k_data), to_host(cache.k_scale).view(np.uint16), to_host(cache.v_data),
            to_host(cache.v_scale).view(np.uint16))
     return got, ref, int(st.item()), bad
 
 
-@pytest.mark.parametrize("head_dim", [256, 128, 64])
-def test_kv_write_bitexact(qkv, head_dim):
+@pytest.mark.parametrize("v_group", [32, 0])
+@pytest.mark.parametrize("head_dim", [256, 128, 96, 64])
+def test_kv_write_bitexact(qkv, head_dim, v_group):
+    """v_group 0 stands for head_dim: one V scale per token and head."""
+    v_group = v_group or head_dim
     rng = np.random.default_rng(12)
     n_tok, kv_heads, block, num_pages = 300, 4, 16, 40
     x = rng.standard_normal((2, n_tok, kv_heads, head_dim)) * 10.0 ** rng.uniform(-6, 4, (2, n_tok, kv_heads, 1))
@@ -119,8 +122,9 @@ def test_kv_write_bitexact(qkv, head_dim):
     v = workloads.f32_to_bf16_bits(x[1].astype(np.float32))
     slots = rng.permutation(num_pages * block)[:n_tok].astype(np.int64)
     slots[3] = -1
-    got, ref, st, bad = _write_both(qkv, k, v, slots, num_pages, kv_heads, block, head_dim)
+    got, ref, st, bad = _write_both(qkv, k, v, slots, num_pages, kv_heads, block, head_dim, v_group)
     assert st == 0 and bad == 0
+    assert got[3].shape[-1] == head_dim // v_group
     for a, b in zip(got, ref):
         assert np.array_equal(a, b)
 
@@ -133,9 +137,11 @@ def test_kv_write_bad_slot(qkv):
         assert np.array_equal(a, b)
 
 
+@pytest.mark.parametrize("v_group", [32, 256])
 @pytest.mark.parametrize("amax_bits", [0x3F80, 0x0080, 0x7F7F, 0x3380, 0x0001, 0x4B00])
-def test_kv_write_exhaustive_bf16(qkv, amax_bits):
-    """Every finite bf16 value as one element of a cell whose amax is fixed."""
+def test_kv_write_exhaustive_bf16(qkv, amax_bits, v_group):
+    """Every finite bf16 value as one element of a cell whose amax is fixed
+    (with v_group 256 the V row's amax is the larger of the two)."""
     allb = np.arange(65536, dtype=np.uint16)
     vals = allb[(allb & 0x7F80) != 0x7F80]
     n = vals.size
@@ -143,15 +149,16 @@ def test_kv_write_exhaustive_bf16(qkv, amax_bits):
     k[:, 0, 0] = amax_bits
     k[:, 0, 1] = vals
     k[:, 0, 32 + 7] = vals          # a second cell: the value alone sets amax
-    got, ref, st, bad = _write_both(qkv, k, k, np.arange(n, dtype=np.int64), n // 64 + 1, 1, 64, 256)
+    got, ref, st, bad = _write_both(qkv, k, k, np.arange(n, dtype=np.int64), n // 64 + 1, 1, 64, 256, v_group)
     assert st == 0
     for a, b in zip(got, ref):
         assert np.array_equal(a, b)
 
 
+@pytest.mark.parametrize("v_group", [32, 256])
 @pytest.mark.parametrize("inplace", [False, True])
 @pytest.mark.parametrize("rot", [64, 128, 256])
-def test_rope_kv_write_fused_matches_two_calls(qkv, rot, inplace):
+def test_rope_kv_write_fused_matches_two_calls(qkv, rot, inplace, v_group):
     """The one-launch rotary + F4 write gives the same bits as qkv_rope_apply
     on q and k followed by qkv_kv_write_f4 (and so the oracle parity of those
     two calls carries over)."""
@@ -171,13 +178,13 @@ def test_rope_kv_write_fused_matches_two_calls(qkv, rot, inplace):
     k2 = torch.empty_like(to_dev(k))
     qkv.qkv_rope_apply(to_dev(q), q2, to_dev(pos), c, s, p0, rot)
     qkv.qkv_rope_apply(to_dev(k), k2, to_dev(pos), c, s, p0, rot)
-    ref = qkv.PagedF4Cache.allocate(P, hkv, B, d)
+    ref = qkv.PagedF4Cache.allocate(P, hkv, B, d, v_group=v_group)
     ref.write(k2, to_dev(v), to_dev(slots))
     # one launch
     qi = to_dev(q)
     qo = qi if inplace else torch.empty_like(qi)
     ko = torch.empty_like(to_dev(k))
-    got = qkv.PagedF4Cache.allocate(P, hkv, B, d)
+    got = qkv.PagedF4Cache.allocate(P, hkv, B, d, v_group=v_group)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     qkv.qkv_rope_kv_write_f4(qi, qo, to_dev(k), to_dev(v), to_dev(pos), to_dev(slots), c, s, p0, rot, got.k_data,
                              got.k_scale, got.v_data, got.v_scale, k_out=ko, device_status=st)
