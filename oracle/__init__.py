@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
             "oracle_paged_attention": (None, [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32,
                                               d, vp, vp, i32, i32]),
             "oracle_lse_merge": (None, [vp, vp, i32, i32, i32, vp, vp]),
+            "oracle_gather_kv_f4": (i64, [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i64, i32, vp,
+                                          vp]),
             "oracle_max_threads": (i32, []),
             "oracle_f64_to_f16_array": (None, [vp, vp, i64]),
             "oracle_f16_to_f64_array": (None, [vp, vp, i64]),
@@ -205,6 +207,39 @@ def paged_attention(q, cache, page_table, tok_begin, tok_end, q_heads: int, kv_h
                                  n_seq, q_heads, kv_heads, head_dim, block_size, sc, _p(out), _p(lse2),
                                  n_threads, v_group_of(cache, head_dim))
     return out, lse2
+
+
+def gather_kv_f4(cache, page_table, seq_lens, out_start, kv_heads: int, head_dim: int, block_size: int,
+                 n_out: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray, int]:
+    """Dequantise each sequence's context tokens into contiguous rows:
+    (k_out, v_out) bf16 bits [n_out][kv_heads][head_dim], sequence s at rows
+    out_start[s] .. out_start[s] + seq_lens[s] - 1; plus the number of tokens
+    whose page id was outside the pool (their rows are zero)."""
+    pt = _c(page_table, np.int32); sl = _c(seq_lens, np.int32); st = _c(out_start, np.int64)
+    kd, ks, vd, vs = (np.ascontiguousarray(a) for a in cache)
+    if n_out is None:
+        n_out = int(np.max(st + sl, initial=0))
+    k_out = np.zeros((n_out, kv_heads, head_dim), np.uint16); v_out = np.zeros_like(k_out)
+    bad = lib().oracle_gather_kv_f4(_p(kd), _p(ks), _p(vd), _p(vs), _p(pt), pt.shape[1], _p(sl), _p(st),
+                                    pt.shape[0], kv_heads, head_dim, block_size, kd.shape[0],
+                                    v_group_of(cache, head_dim), _p(k_out), _p(v_out))
+    return k_out, v_out, int(bad)
+
+
+def prefill_attention(q, cache, page_table_row, positions, q_heads: int, kv_heads: int, head_dim: int,
+                      block_size: int, softmax_scale: Optional[float] = None,
+                      n_threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """Causal attention of a chunk of queries of one sequence against its
+    paged cache [CHUNK]: query i (at position positions[i]) attends the
+    cached tokens 0 .. positions[i]. That is paged_attention with one
+    single-query "sequence" per chunk row, all on the same page-table row.
+    Returns (out [n][Hq][D], lse2 [n][Hq])."""
+    pos = _c(positions, np.int64)
+    n = pos.size
+    row = _c(page_table_row, np.int32).reshape(1, -1)
+    pt = np.repeat(row, n, axis=0)
+    return paged_attention(q, cache, pt, np.zeros(n, np.int32), (pos + 1).astype(np.int32), q_heads, kv_heads,
+                           head_dim, block_size, softmax_scale, n_threads)
 
 
 def lse_merge(o_parts, lse2_parts) -> Tuple[np.ndarray, np.ndarray]:

@@ -20,6 +20,9 @@
  *           FreeToken issue #568 "Serving ...'s 1M-token window on one 24 GB
  *           card", proposed solution item 2: partials folded by
  *           log2-sum-exp.
+ *   [GATHER] same PR section 2: gather_kv_cache gains an F4 path (the paged
+ *           cache read back into contiguous rows for prefill attention).
+ *   [CHUNK] same PR section 5: paged prefill runs in chunks of 2048 tokens.
  *
  * Readings where the pages are silent (each one is listed in the design
  * notes): amax/7 scale rounded once to fp16 (RNE, saturating at 65504);
@@ -319,6 +322,40 @@ void oracle_paged_attention(const uint16_t* q, const uint8_t* k_data, const uint
     for (int d = 0; d < head_dim; ++d) o[d] /= z;
     lse2[r] = (m + log(z)) / log(2.0);
   }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Paged -> contiguous gather of the F4 cache [GATHER].                      */
+
+/* For each sequence s and each of its context tokens t < seq_lens[s], every
+ * KV head h and element d:
+ *   k_out[out_start[s] + t][h][d] = bf16((code - 8) * k_scale)
+ *   v_out[...]                    = bf16((code - 8) * v_scale)
+ * The product is exact in double; bf16 rounds to nearest even. A token whose
+ * page-table entry lies outside [0, num_pages) gives zero rows; the return
+ * value counts such tokens. */
+int64_t oracle_gather_kv_f4(const uint8_t* k_data, const uint16_t* k_scale, const uint8_t* v_data,
+                            const uint16_t* v_scale, const int32_t* page_table, int max_pages_per_seq,
+                            const int32_t* seq_lens, const int64_t* out_start, int n_seq, int kv_heads,
+                            int head_dim, int block_size, int64_t num_pages, int v_group, uint16_t* k_out,
+                            uint16_t* v_out) {
+  int64_t bad = 0;
+  for (int s = 0; s < n_seq; ++s) {
+    for (int t = 0; t < seq_lens[s]; ++t) {
+      const int32_t page = page_table[(size_t)s * max_pages_per_seq + t / block_size];
+      const int ok = page >= 0 && page < num_pages;
+      bad += !ok;
+      for (int h = 0; h < kv_heads; ++h) {
+        const size_t dst = ((size_t)(out_start[s] + t) * kv_heads + h) * head_dim;
+        const size_t row = ((size_t)(ok ? page : 0) * kv_heads + h) * block_size + t % block_size;
+        for (int d = 0; d < head_dim; ++d) {
+          k_out[dst + d] = ok ? oracle_f64_to_bf16(deq(k_data, k_scale, row, head_dim, 32, d)) : 0;
+          v_out[dst + d] = ok ? oracle_f64_to_bf16(deq(v_data, v_scale, row, head_dim, v_group, d)) : 0;
+        }
+      }
+    }
+  }
+  return bad;
 }
 
 /* ------------------------------------------------------------------------- */
