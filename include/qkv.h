@@ -291,6 +291,29 @@ QKV_API int qkv_paged_decode_attn_f4_v(uint16_t* out, float* lse2_out, const uin
                                        int32_t v_group, void* workspace, size_t workspace_bytes,
                                        int32_t* device_status, qkv_stream_t stream);
 
+/* Paged -> contiguous gather of the F4 cache ([F4] section 2: gather_kv_cache
+ * with an F4 path, the cache read back for attention outside the paged
+ * kernels).
+ *   k_out, v_out  bf16 [n_out][kv_heads][head_dim]: row out_start[s] + t holds
+ *                 token t of sequence s, t < seq_lens[s], each element
+ *                 bf16((code - 8) * scale) rounded to nearest even (the
+ *                 product is exact). Other rows are not written. 16-byte
+ *                 aligned.
+ *   out_start     int64 [n_seq], the first output row of each sequence.
+ *   page_table, seq_lens, cache and v_group as in qkv_paged_decode_split_f4_v
+ *                 (head_dim a multiple of 32 up to 256, any block_size).
+ * A page id outside [0, num_pages) gives zero rows and QKV_DEV_BAD_PAGE; a
+ * seq_len outside [0, max_pages_per_seq * block_size] is clamped and an
+ * output row outside [0, n_out) skipped, each with QKV_DEV_BAD_SEQLEN.
+ * One thread per 32-value cell; bound by HBM (144 bytes read and 512
+ * written per token, KV head and K or V). */
+QKV_API int qkv_gather_kv_f4(uint16_t* k_out, uint16_t* v_out, int64_t n_out, const uint8_t* k_data,
+                             const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
+                             const int32_t* page_table, const int32_t* seq_lens, const int64_t* out_start,
+                             int32_t n_seq, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                             int32_t max_pages_per_seq, int64_t num_pages, int32_t v_group,
+                             int32_t* device_status, qkv_stream_t stream);
+
 /* Size of the partials array compiled into the library for
  * qkv_paged_decode_attn_f4_static (16 MiB per GPU that loads the library). */
 #define QKV_STATIC_SCRATCH_BYTES (16u << 20)

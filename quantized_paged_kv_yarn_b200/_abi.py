@@ -69,6 +69,8 @@ _SIGS = {
     "qkv_paged_decode_attn_f4_v": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                                                   _i32, _i32, _i32, _i64, _f32, _i32, _i32, _i32, _vp, _sz, _vp,
                                                   _vp]),
+    "qkv_gather_kv_f4": (ctypes.c_int, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+                                        _i32, _i64, _i32, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -256,6 +258,22 @@ def qkv_paged_decode_attn_f4(out, q, k_data, k_scale, v_data, v_scale, page_tabl
         _check("qkv_paged_decode_attn_f4", lib.qkv_paged_decode_attn_f4(*args, *ws, *tail))
     else:
         _check("qkv_paged_decode_attn_f4_v", lib.qkv_paged_decode_attn_f4_v(*args, vg, *ws, *tail))
+
+
+def qkv_gather_kv_f4(k_out, v_out, k_data, k_scale, v_data, v_scale, page_table, seq_lens, out_start,
+                     device_status=None, stream=None):
+    """k_out/v_out bf16 [n_out][kv_heads][head_dim]; out_start int64 [n_seq]."""
+    num_pages, kv_heads, block_size, half = k_data.shape
+    head_dim = 2 * half
+    n_seq = seq_lens.numel()
+    if k_out.shape[1:] != (kv_heads, head_dim) or v_out.shape != k_out.shape:
+        raise ValueError("k_out and v_out must be [n_out][kv_heads][head_dim]")
+    _check("qkv_gather_kv_f4", lib.qkv_gather_kv_f4(
+        _ptr(k_out, "k_out", _U16), _ptr(v_out, "v_out", _U16), k_out.shape[0],
+        *_cache_args(k_data, k_scale, v_data, v_scale), _ptr(page_table, "page_table", (torch.int32,)),
+        _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq), _ptr(out_start, "out_start", (torch.int64,), n_seq),
+        n_seq, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, v_group_of(v_scale, head_dim),
+        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
 
 
 STATIC_SCRATCH_BYTES = 16 << 20
