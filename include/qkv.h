@@ -314,6 +314,33 @@ QKV_API int qkv_gather_kv_f4(uint16_t* k_out, uint16_t* v_out, int64_t n_out, co
                              int32_t max_pages_per_seq, int64_t num_pages, int32_t v_group,
                              int32_t* device_status, qkv_stream_t stream);
 
+/* Chunked causal prefill attention over the paged F4 cache ([F4] section 5:
+ * paged prefill in chunks of 2048 tokens). A chunk of n_q queries of one
+ * sequence occupies cache tokens prefix_len .. prefix_len + n_q - 1, already
+ * written with qkv_kv_write_f4(_v); query i attends the cached tokens
+ * 0 .. prefix_len + i:
+ *   out[i][h] = sum_t softmax_t(softmax_scale * q[i][h] . k^_t) v^_t
+ * with query head h reading KV head h / (q_heads / kv_heads).
+ *   out        bf16 [n_q][q_heads][head_dim]; lse2_out float [n_q][q_heads]
+ *              (log2 sum_t exp(score_t)) or NULL.
+ *   q          bf16 [n_q][q_heads][head_dim], rotary already applied.
+ *   page_table int32 [max_pages_per_seq]: the sequence's row; token t is on
+ *              page page_table[t / block_size]. prefix_len + n_q must not
+ *              exceed max_pages_per_seq * block_size (else QKV_EINVAL).
+ *   cache, v_group, softmax_scale as in qkv_paged_decode_split_f4_v.
+ * Compiled shapes: head_dim 256, q_heads / kv_heads in {1, 2, 4, 8}, any
+ * block_size (else QKV_EUNSUPPORTED). Runs on the tensor cores (tcgen05,
+ * fp16 operands, fp32 accumulators in tensor memory): K and V are
+ * dequantised to fp16 in shared memory, q scaled by a power of two per
+ * row; outputs match exact attention within 2e-3. A page id outside the
+ * pool reads as zero rows and sets QKV_DEV_BAD_PAGE. */
+QKV_API int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
+                                      const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
+                                      const int32_t* page_table, int32_t n_q, int32_t prefix_len,
+                                      int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                      int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                                      int32_t v_group, int32_t* device_status, qkv_stream_t stream);
+
 /* Size of the partials array compiled into the library for
  * qkv_paged_decode_attn_f4_static (16 MiB per GPU that loads the library). */
 #define QKV_STATIC_SCRATCH_BYTES (16u << 20)

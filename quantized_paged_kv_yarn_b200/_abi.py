@@ -71,6 +71,8 @@ _SIGS = {
                                                   _vp]),
     "qkv_gather_kv_f4": (ctypes.c_int, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
                                         _i32, _i64, _i32, _vp, _vp]),
+    "qkv_paged_prefill_attn_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+                                                 _i32, _i32, _i32, _i64, _f32, _i32, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -273,6 +275,22 @@ def qkv_gather_kv_f4(k_out, v_out, k_data, k_scale, v_data, v_scale, page_table,
         *_cache_args(k_data, k_scale, v_data, v_scale), _ptr(page_table, "page_table", (torch.int32,)),
         _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq), _ptr(out_start, "out_start", (torch.int64,), n_seq),
         n_seq, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, v_group_of(v_scale, head_dim),
+        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+
+
+def qkv_paged_prefill_attn_f4(out, q, k_data, k_scale, v_data, v_scale, page_table, prefix_len: int,
+                              kv_heads: int, lse2_out=None, softmax_scale: float = 0.0, device_status=None,
+                              stream=None):
+    """out, q bf16 [n_q][q_heads][head_dim]; page_table int32 [max_pages] (one
+    sequence); the chunk's queries sit at cache tokens prefix_len .. prefix_len + n_q - 1."""
+    n_q, q_heads, head_dim = q.shape
+    num_pages, _, block_size, _ = k_data.shape
+    page_table = page_table.reshape(-1)
+    _check("qkv_paged_prefill_attn_f4", lib.qkv_paged_prefill_attn_f4(
+        _ptr(out, "out", _U16, n_q * q_heads * head_dim), _ptr(lse2_out, "lse2_out", (torch.float32,), n_q * q_heads),
+        _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),
+        _ptr(page_table, "page_table", (torch.int32,)), n_q, int(prefix_len), q_heads, kv_heads, head_dim,
+        block_size, page_table.numel(), num_pages, float(softmax_scale), v_group_of(v_scale, head_dim),
         _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
 
 

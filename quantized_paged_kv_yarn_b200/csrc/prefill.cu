@@ -1,0 +1,612 @@
+// prefill.cu -- chunked causal prefill attention over the paged F4 cache
+// on the sm_100a tensor cores (tcgen05, accumulators in tensor memory).
+//
+// Sources: mistral.rs PR "YaRN rope scaling, 4-bit F4 packed KV cache, and
+// hybrid paged attention for Qwen3.5-Next long-context serving", section 2
+// (the packed cache, values (nibble - 8) * scale) and section 5 (paged
+// prefill in chunks of 2048 tokens). A chunk of n_q queries of one sequence
+// sits at cache tokens prefix_len .. prefix_len + n_q - 1 (already written);
+// query i attends the cached tokens 0 .. prefix_len + i.
+//
+// This is a dense contraction (128 query rows share every dequantised
+// page), so it runs on tcgen05.mma with fp32 accumulators in TMEM:
+//
+//   S[128 x 64]  = Q'[128 x 256] . (K^'hi + K^'lo)[64 x 256]^T   (2 x 16 MMAs, K = 16)
+//   O[128 x 256] += P[128 x 64] . V^'[64 x 256]                  (4 MMAs, N = 256)
+//
+// Rows are (query head of the GQA group, query): 128 = G x (128 / G).
+// One CTA per (128 / G queries, KV head); stages of 64 tokens.
+//
+// Warp roles (512 threads):
+//   warp 0        TMEM allocation; lane 0 issues every MMA and commit
+//   warps 4..7    softmax: thread r owns row r (TMEM lane r): puts its row
+//                 of Q' into tensor memory, reads S, keeps the running max
+//                 and sum, writes P, rescales O when the max moves, and
+//                 writes the output
+//   warps 8..15   dequantisation: each thread turns one token's 64 dims of
+//                 K and of V (32 packed bytes each) into fp16 in a swizzled
+//                 shared tile, prefetching the packed bytes two stages ahead
+//
+// Numerics. With s' = scale * 2^-4 (exact while scale >= 2^-10; the 2^-4
+// keeps 8 * 65504 in range), a K element (code - 8) s' needs up to 14
+// significant bits: it is split into K^'hi = fp16((code - 8) s') and
+// K^'lo = fp16((code - 8) s' - K^'hi), and their sum is exact, so the
+// scores see K exactly (one fp16 rounding of K alone moved scores by up to
+// ~1e-3, more than the attention tolerance allows at short contexts).
+// V^' = fp16((code - 8) s') is rounded once. Q' = fp16(q * 2^e) with a power
+// of two per row (exact for bf16 q in range). The scores and P . V
+// accumulate in fp32; p = 2^(s - m_ref) in fp16 with the reference max moved
+// lazily (only when a score exceeds it by more than 8, so p <= 256).
+//
+// Q' lives in tensor memory (the A operand of Q K^T; row r in lane r, two
+// fp16 per column). Shared-memory tiles use the 128-byte swizzle in the
+// canonical UMMA layouts: a K-major tile is [K / 64 chunks][rows][128 B];
+// the V^' tile, the MN-major B operand of P . V, is
+// [256 dims / 64 chunks][64 tokens][128 B]. Within each 8-dim unit the dims
+// are stored in the order 0,4,1,5,2,6,3,7 (the order in which four nibble
+// masks of a packed word yield them); Q' uses the same order, and the
+// output un-permutes O's columns.
+#include <type_traits>
+
+#include "common.cuh"
+
+namespace qkv {
+namespace prefill {
+
+constexpr int THREADS = 512;
+constexpr int D = 256;
+constexpr int M = 128;          // rows per CTA
+constexpr int NT = 64;          // tokens per stage
+constexpr float TH = 8.f;       // lazy-rescale threshold (log2 units)
+
+// shared-memory map (offsets from a 1024-byte aligned base)
+constexpr int TILE = 4 * NT * 128;              // one [4 chunks][64][128 B] tile: 32 KB
+constexpr int K_OFF = 0;                        // 2 slots x (hi tile, lo tile)
+constexpr int V_OFF = K_OFF + 2 * 2 * TILE;     // 2 slots x tile
+constexpr int P_OFF = V_OFF + 2 * TILE;         // [128][128 B]
+constexpr int BAR_OFF = P_OFF + M * 128;
+constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;  // barriers, flags, alignment slack
+
+// TMEM columns: O 0..255, S slot b at 256 + 64 b, Q' at 384..511
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TQ = 384;
+
+struct Bars {
+  uint64_t kready[2], kfree[2], vready[2], vfree[2], sfull[2], sfree[2];
+  uint64_t pready, odone, qready, drain;
+  uint32_t tmem;
+  int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+struct Params {
+  const uint16_t* q;
+  uint16_t* out;
+  float* lse2;
+  const uint8_t* k_data;
+  const uint16_t* k_scale;
+  const uint8_t* v_data;
+  const uint16_t* v_scale;
+  const int32_t* page_table;
+  int64_t num_pages;
+  int n_q, prefix_len, q_heads, kv_heads, G, QB, block, v_tok;
+  float score_scale;  // softmax_scale * log2(e)
+  int32_t* status;
+};
+
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  // start >> 4 | LBO >> 4 << 16 | SBO >> 4 << 32 | version 1 << 46 | 128-byte swizzle (2) << 61
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// A from tensor memory (row r in lane r), B from shared memory
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+#define QKV_R32(p) \
+  "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3]), "=r"(p[4]), "=r"(p[5]), "=r"(p[6]), "=r"(p[7]), "=r"(p[8]), \
+  "=r"(p[9]), "=r"(p[10]), "=r"(p[11]), "=r"(p[12]), "=r"(p[13]), "=r"(p[14]), "=r"(p[15]), "=r"(p[16]),       \
+  "=r"(p[17]), "=r"(p[18]), "=r"(p[19]), "=r"(p[20]), "=r"(p[21]), "=r"(p[22]), "=r"(p[23]), "=r"(p[24]),      \
+  "=r"(p[25]), "=r"(p[26]), "=r"(p[27]), "=r"(p[28]), "=r"(p[29]), "=r"(p[30]), "=r"(p[31])
+#define QKV_W32(p) \
+  "r"(p[0]), "r"(p[1]), "r"(p[2]), "r"(p[3]), "r"(p[4]), "r"(p[5]), "r"(p[6]), "r"(p[7]), "r"(p[8]), "r"(p[9]), \
+  "r"(p[10]), "r"(p[11]), "r"(p[12]), "r"(p[13]), "r"(p[14]), "r"(p[15]), "r"(p[16]), "r"(p[17]), "r"(p[18]),  \
+  "r"(p[19]), "r"(p[20]), "r"(p[21]), "r"(p[22]), "r"(p[23]), "r"(p[24]), "r"(p[25]), "r"(p[26]), "r"(p[27]),  \
+  "r"(p[28]), "r"(p[29]), "r"(p[30]), "r"(p[31])
+#define QKV_REGLIST32                                                                                           \
+  "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, " \
+  "%23, %24, %25, %26, %27, %28, %29, %30, %31}"
+
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp quarter rule:
+// the address carries lane base 32 * (warp % 4) in its upper half)
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 " QKV_REGLIST32 ", [%32];" : QKV_R32(r) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+               "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+               ::"r"(taddr), QKV_W32(r)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// 2^x (hardware approximation; subnormal results flushed to 0, 2^-inf = 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Byte offset of 16-byte unit u of row r in a [rows][128 B] 128-byte-swizzled chunk.
+__device__ __forceinline__ uint32_t swz(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
+
+// Bounded wait that also gives up once another role has aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > WAIT_LIMIT_NS) return false;
+    }
+  }
+}
+
+// Four fp16 pairs of one packed word (8 codes, low nibble first) times the
+// cell scale s' (fp16 pair): pairs (e0,e4), (e1,e5), (e2,e6), (e3,e7).
+// With LO, also the rounding residual (code - 8) s' - hi (exact, one fma).
+template <bool LO>
+__device__ __forceinline__ void dequant_word(uint32_t w, __half2 s2, uint32_t (&o)[4], uint32_t (&lo)[4]) {
+  const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t x = ((w >> (4 * i)) & 0x000F000Fu) | 0x64006400u;  // fp16 1024 + code, twice
+    const __half2 t = __hsub2(u32_as_h2(x), off);                       // code - 8, exact
+    const __half2 hi = __hmul2(t, s2);
+    o[i] = h2_as_u32(hi);
+    if constexpr (LO) lo[i] = h2_as_u32(__hfma2(t, s2, __hneg2(hi)));
+  }
+}
+
+__device__ __forceinline__ uint32_t bf2_u32(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+struct Raw {
+  uint4 k0, k1, v0, v1;
+  uint32_t ks, vs;
+  int ok;  // 0: outside the context (zero rows), 1: data, 2: bad page (zero rows, flagged)
+};
+
+__global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars& bars = *reinterpret_cast<Bars*>(sm + BAR_OFF);
+  const uint32_t s_base = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  const int kvh = blockIdx.y;
+  const int q0 = blockIdx.x * p.QB;
+  const int q_last = min(p.n_q, q0 + p.QB) - 1;
+  const int kv_len = p.prefix_len + q_last + 1;
+  const int n_st = (kv_len + NT - 1) / NT;
+
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.kready[b], 256);
+      mbar_init(&bars.vready[b], 256);
+      mbar_init(&bars.kfree[b], 1);
+      mbar_init(&bars.vfree[b], 1);
+      mbar_init(&bars.sfull[b], 1);
+      mbar_init(&bars.sfree[b], 128);
+    }
+    mbar_init(&bars.pready, 128);
+    mbar_init(&bars.odone, 1);
+    mbar_init(&bars.qready, 128);
+    mbar_init(&bars.drain, 1);
+    bars.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&bars.tmem)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_wait();
+  pdl_release();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem;
+  volatile int* abort = &bars.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      constexpr uint32_t ID_QK = (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+      constexpr uint32_t ID_PV = (1u << 4) | (1u << 16) | ((uint32_t)(D >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+      const uint32_t sp = s_base + P_OFF;
+      bool ok = wait_bar(&bars.qready, 0, abort);
+      auto pv = [&](int i) -> bool {
+        const int b = i & 1;
+        if (!wait_bar(&bars.pready, (uint32_t)i & 1u, abort)) return false;
+        if (!wait_bar(&bars.vready[b], (uint32_t)(i >> 1) & 1u, abort)) return false;
+        tc_fence_after();
+        const uint32_t sv = s_base + V_OFF + b * TILE;
+#pragma unroll
+        for (int kk = 0; kk < NT / 16; ++kk)
+          umma(tmem, sdesc(sp + 32 * kk, 16, 1024), sdesc(sv + 2048 * kk, NT * 128, 1024), ID_PV,
+               (i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&bars.odone);
+        umma_commit(&bars.vfree[b]);
+        return true;
+      };
+      for (int j = 0; ok && j < n_st; ++j) {
+        const int b = j & 1;
+        if (!wait_bar(&bars.kready[b], (uint32_t)(j >> 1) & 1u, abort)) { ok = false; break; }
+        if (j >= 2 && !wait_bar(&bars.sfree[b], (uint32_t)((j - 2) >> 1) & 1u, abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sk = s_base + K_OFF + b * (2 * TILE);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // K^'hi, then K^'lo into the same accumulator
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t bb = sk + h * TILE + (kk >> 2) * (NT * 128) + 32 * (kk & 3);
+            umma_ts(tmem + 256 + 64 * b, tmem + TQ + 8 * kk, sdesc(bb, 16, 1024), ID_QK,
+                    (h > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&bars.sfull[b]);
+        umma_commit(&bars.kfree[b]);
+        if (j >= 1 && !pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) ok = pv(n_st - 1);
+      if (!ok) {
+        *abort = 1;
+        flag(p.status, QKV_DEV_TIMEOUT);
+      }
+      // every MMA issued so far has completed once this commit lands
+      umma_commit(&bars.drain);
+      mbar_wait_bounded(&bars.drain, 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ softmax
+    const int r = tid - 128;
+    const int hl = r / p.QB, qq = r - hl * p.QB;
+    const int qi = q0 + qq;
+    const bool valid = qi < p.n_q;
+    const int qhead = kvh * p.G + hl;
+    const int lim = p.prefix_len + qi;  // last token this row attends
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+
+    // Q' = fp16(q * 2^e) into tensor memory, dims permuted per 8-dim unit
+    float c_row;
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)qi * p.q_heads + qhead) * D);
+      float amax = 0.f;
+      if (valid) {
+#pragma unroll 4
+        for (int u = 0; u < D / 8; ++u) {
+          const uint4 w = src[u];
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(ws[i] << 16)), fabsf(__uint_as_float(ws[i] & 0xffff0000u))));
+        }
+      }
+      // 2^e with amax * 2^e in [2^13, 2^14); exponent of amax from its bits
+      int e = 0;
+      if (amax > 0.f) e = 13 - (((int)(__float_as_uint(amax) >> 23) & 0xff) - 127);
+      e = max(-100, min(100, e));
+      // 2^e as a product of two normal powers of two (|e| <= 100)
+      const float up = __int_as_float((127 + e / 2) << 23) * __int_as_float((127 + (e - e / 2)) << 23);
+      c_row = p.score_scale * 16.f / up;  // S = S' * 2^(4 - e)
+#pragma unroll 1
+      for (int g = 0; g < 4; ++g) {  // 8 units = 32 columns per store
+        uint32_t o[32];
+#pragma unroll
+        for (int uu = 0; uu < 8; ++uu) {
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (valid) w = src[8 * g + uu];
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+          float f[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(ws[i] << 16) * up;
+            f[2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u) * up;
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[4 * uu + i] = h2_as_u32(__floats2half2_rn(f[i], f[i + 4]));
+        }
+        tmem_st32(tmem + lane_base + TQ + 32 * g, o);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars.qready);
+    }
+
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    const uint32_t prow = s_base + P_OFF;
+    for (int j = 0; j < n_st; ++j) {
+      const int b = j & 1;
+      ok = wait_bar(&bars.sfull[b], (uint32_t)(j >> 1) & 1u, abort);
+      if (!__all_sync(FULL_MASK, ok)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[2][32];
+      tmem_ld32(tmem + lane_base + 256 + 64 * b, sr[0]);
+      tmem_ld32(tmem + lane_base + 256 + 64 * b + 32, sr[1]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars.sfree[b]);
+      float s[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(sr[i >> 5][i & 31]);
+      const int base = j * NT;
+      if (base + NT - 1 > lim) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) s[i] = (base + i <= lim) ? s[i] : -INFINITY;
+      }
+      float smax = s[0];
+#pragma unroll
+      for (int i = 1; i < 64; ++i) smax = fmaxf(smax, s[i]);
+      const float mt = smax * c_row;
+      const bool need = mt > m_ref + TH;
+      const bool any_need = __any_sync(FULL_MASK, need);
+      float alpha = 1.f;
+      if (any_need) {
+        const float m_new = need ? mt : m_ref;
+        alpha = need ? ex2(m_ref - m_new) : 1.f;  // nothing accumulated yet: ex2(-inf) = 0
+        l *= alpha;
+        m_ref = m_new;
+      }
+      // p = 2^(s c - m_ref) as fp16 pairs (token order), summed as rounded
+      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+      uint32_t pw[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float a = ex2(fmaf(s[2 * i], c_row, -mu));
+        const float bq = ex2(fmaf(s[2 * i + 1], c_row, -mu));
+        const __half2 h = __floats2half2_rn(a, bq);
+        const float2 hf = __half22float2(h);
+        l += hf.x + hf.y;
+        pw[i] = h2_as_u32(h);
+      }
+      if (j >= 1) {  // P . V of the previous stage done: P free, O stable
+        ok = wait_bar(&bars.odone, (uint32_t)(j - 1) & 1u, abort);
+        if (!__all_sync(FULL_MASK, ok)) { ok = false; break; }
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sts128(prow + swz(r, u), pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
+      if (any_need && j >= 1) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tmem + lane_base + 32 * c, o);
+        }
+        tmem_wait_st();
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars.pready);
+    }
+
+    // epilogue: O / l, columns un-permuted, bf16 out
+    if (ok) {
+      ok = wait_bar(&bars.odone, (uint32_t)(n_st - 1) & 1u, abort);
+      ok = __all_sync(FULL_MASK, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 16.f / l : 0.f;
+      uint16_t* dst = p.out + ((size_t)qi * p.q_heads + qhead) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + 32 * c, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {  // columns 8u .. 8u+7 hold dims 8u + (0,4,1,5,2,6,3,7)
+            float f[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              f[k] = __uint_as_float(o[8 * u + 2 * k]) * inv;
+              f[k + 4] = __uint_as_float(o[8 * u + 2 * k + 1]) * inv;
+            }
+            reinterpret_cast<uint4*>(dst)[4 * c + u] =
+                make_uint4(bf2_u32(f[0], f[1]), bf2_u32(f[2], f[3]), bf2_u32(f[4], f[5]), bf2_u32(f[6], f[7]));
+          }
+        }
+      }
+      if (valid && p.lse2) p.lse2[(size_t)qi * p.q_heads + qhead] = l > 0.f ? m_ref + log2f(l) : -INFINITY;
+    } else {
+      *abort = 1;
+      flag(p.status, QKV_DEV_TIMEOUT);
+    }
+    tc_fence_before();
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ dequantisation
+    const int d = tid - 256;
+    const int tk = d >> 2, c = d & 3;
+    const size_t row_bytes = D / 2;
+    auto load = [&](int j, Raw& x) {
+      x.ok = 0;
+      if (j >= n_st) return;
+      const int t = j * NT + tk;
+      if (t >= kv_len) return;
+      const int32_t page = p.page_table[t / p.block];
+      if (page < 0 || page >= p.num_pages) {
+        x.ok = 2;
+        return;
+      }
+      const size_t row = ((size_t)page * p.kv_heads + kvh) * p.block + (t % p.block);
+      const uint4* kp = reinterpret_cast<const uint4*>(p.k_data + row * row_bytes + 32 * c);
+      const uint4* vp = reinterpret_cast<const uint4*>(p.v_data + row * row_bytes + 32 * c);
+      x.k0 = __ldg(kp);
+      x.k1 = __ldg(kp + 1);
+      x.v0 = __ldg(vp);
+      x.v1 = __ldg(vp + 1);
+      x.ks = __ldg(reinterpret_cast<const uint32_t*>(p.k_scale + row * 8 + 2 * c));
+      if (p.v_tok) {
+        const uint32_t h = __ldg(p.v_scale + row);
+        x.vs = h | (h << 16);
+      } else {
+        x.vs = __ldg(reinterpret_cast<const uint32_t*>(p.v_scale + row * 8 + 2 * c));
+      }
+      x.ok = 1;
+    };
+    // one token's 64 dims of K (hi and lo tiles) or V into chunk c of a slot
+    auto put = [&](uint32_t chunk_base, const uint4& a, const uint4& bw, uint32_t sc, int okv, auto with_lo) {
+      constexpr bool LO = decltype(with_lo)::value;
+      // s' = scale * 2^-4 per cell (low half: cell 2c, high half: cell 2c + 1)
+      const __half2 s16 = __hmul2(u32_as_h2(sc), __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00)));
+      const __half2 s_lo = __low2half2(s16), s_hi = __high2half2(s16);
+      const uint32_t wd[8] = {a.x, a.y, a.z, a.w, bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        uint32_t o[4] = {0u, 0u, 0u, 0u}, r[4] = {0u, 0u, 0u, 0u};
+        if (okv == 1) dequant_word<LO>(wd[u], u < 4 ? s_lo : s_hi, o, r);
+        sts128(chunk_base + swz(tk, u), o[0], o[1], o[2], o[3]);
+        if constexpr (LO) sts128(chunk_base + TILE + swz(tk, u), r[0], r[1], r[2], r[3]);
+      }
+    };
+    auto process = [&](int j, const Raw& x) -> bool {
+      const int b = j & 1;
+      if (x.ok == 2 && c == 0 && kvh == 0 && ((j * NT + tk) % p.block) == 0) flag(p.status, QKV_DEV_BAD_PAGE);
+      if (j >= 2 && !wait_bar(&bars.kfree[b], (uint32_t)((j - 2) >> 1) & 1u, abort)) return false;
+      put(s_base + K_OFF + b * (2 * TILE) + c * (NT * 128), x.k0, x.k1, x.ks, x.ok, std::true_type{});
+      fence_async_smem();
+      mbar_arrive(&bars.kready[b]);
+      if (j >= 2 && !wait_bar(&bars.vfree[b], (uint32_t)((j - 2) >> 1) & 1u, abort)) return false;
+      put(s_base + V_OFF + b * TILE + c * (NT * 128), x.v0, x.v1, x.vs, x.ok, std::false_type{});
+      fence_async_smem();
+      mbar_arrive(&bars.vready[b]);
+      return true;
+    };
+    Raw ra, rb;
+    load(0, ra);
+    load(1, rb);
+    bool ok = true;
+    for (int j = 0; j < n_st; j += 2) {
+      if (!process(j, ra)) { ok = false; break; }
+      load(j + 2, ra);
+      if (j + 1 < n_st) {
+        if (!process(j + 1, rb)) { ok = false; break; }
+        load(j + 3, rb);
+      }
+    }
+    if (!ok) {
+      *abort = 1;
+      flag(p.status, QKV_DEV_TIMEOUT);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+}  // namespace prefill
+}  // namespace qkv
+
+using namespace qkv;
+
+extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
+                                         const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
+                                         const int32_t* page_table, int32_t n_q, int32_t prefix_len,
+                                         int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                         int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                                         int32_t v_group, int32_t* device_status, qkv_stream_t stream) {
+  if (n_q == 0) return QKV_OK;
+  if (!out || !q || !k_data || !k_scale || !v_data || !v_scale || !page_table) return QKV_EINVAL;
+  if (n_q < 0 || prefix_len < 0 || q_heads < 1 || kv_heads < 1 || q_heads % kv_heads || block_size < 1 ||
+      max_pages_per_seq < 1 || num_pages < 1 || !(softmax_scale >= 0.f) || !isfinite(softmax_scale) ||
+      (v_group != 32 && v_group != head_dim))
+    return QKV_EINVAL;
+  if ((int64_t)prefix_len + n_q > (int64_t)max_pages_per_seq * block_size) return QKV_EINVAL;
+  if (((uintptr_t)out | (uintptr_t)q | (uintptr_t)k_data | (uintptr_t)v_data) & 15) return QKV_EINVAL;
+  if (((uintptr_t)k_scale | (uintptr_t)v_scale | (uintptr_t)lse2_out) & 3) return QKV_EINVAL;
+  const int G = q_heads / kv_heads;
+  if (head_dim != prefill::D || (G != 1 && G != 2 && G != 4 && G != 8)) return QKV_EUNSUPPORTED;
+  if (kv_heads > 65535) return QKV_EUNSUPPORTED;
+
+  prefill::Params p;
+  p.q = q;
+  p.out = out;
+  p.lse2 = lse2_out;
+  p.k_data = k_data;
+  p.k_scale = k_scale;
+  p.v_data = v_data;
+  p.v_scale = v_scale;
+  p.page_table = page_table;
+  p.num_pages = num_pages;
+  p.n_q = n_q;
+  p.prefix_len = prefix_len;
+  p.q_heads = q_heads;
+  p.kv_heads = kv_heads;
+  p.G = G;
+  p.QB = prefill::M / G;
+  p.block = block_size;
+  p.v_tok = v_group != 32;
+  const float sc = softmax_scale > 0.f ? softmax_scale : 0.0625f;  // 1 / sqrt(256)
+  p.score_scale = sc * 1.4426950408889634f;
+  p.status = device_status;
+
+  static bool attr_set[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QKV_ECUDA;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(prefill::paged_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             prefill::SMEM_BYTES) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return QKV_ECUDA;
+    }
+    attr_set[dev] = true;
+  }
+  const dim3 grid((unsigned)((n_q + p.QB - 1) / p.QB), (unsigned)kv_heads);
+  void* args[] = {&p};
+  if (launch_pdl((const void*)prefill::paged_prefill_kernel, grid, dim3(prefill::THREADS), prefill::SMEM_BYTES,
+                 stream, args) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QKV_ECUDA;
+  }
+  return QKV_OK;
+}

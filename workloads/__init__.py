@@ -34,6 +34,7 @@ import numpy as np
 # Stream ids: each tensor of a layer draws from its own seeded stream.
 STREAM_Q, STREAM_K_CACHE, STREAM_V_CACHE, STREAM_K_NEW, STREAM_V_NEW = 0, 1, 2, 3, 4
 STREAM_HEAD_SCALE, STREAM_OUTLIER, STREAM_PAGES = 5, 6, 7
+STREAM_CHUNK_Q = 8
 
 
 @dataclasses.dataclass(frozen=True)
@@ -284,6 +285,25 @@ def device_layer(w: Workload, layer: int, device) -> Dict[str, "object"]:
         "positions": t(np.array(w.step_positions, dtype=np.int64)),
         "page_table_host": pt,
     }
+
+
+def chunk_queries_host(w: Workload, layer: int, n_q: int) -> np.ndarray:
+    """bf16 bits [n_q][Hq][D]: the queries of a prefill chunk (the last n_q
+    tokens of the workload's single sequence), same value recipe as q."""
+    f = _head_factors(w, layer)
+    x = _rng(w.seed, layer, STREAM_CHUNK_Q).standard_normal((n_q, w.q_heads, w.head_dim))
+    return f32_to_bf16_bits((x * f["q"].reshape(1, -1, 1)).astype(np.float32))
+
+
+def chunk_queries_device(w: Workload, layer: int, n_q: int, device):
+    """``chunk_queries_host`` drawn on the device (torch Philox)."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed((w.seed * 1_000_003 + layer) * 64 + STREAM_CHUNK_Q)
+    x = torch.randn((n_q, w.q_heads, w.head_dim), generator=g, device=device, dtype=torch.float32)
+    x = x * torch.tensor(_head_factors(w, layer)["q"], dtype=torch.float32, device=device).view(1, -1, 1)
+    return x.to(torch.bfloat16).view(torch.int16)
 
 
 def yarn_spec(w: Workload) -> Dict[str, float]:
