@@ -8,6 +8,7 @@ launch), the split-KV paged attention and the log2-sum-exp merge -- 1 + 3 x
 layers kernel launches, replayed from a CUDA graph.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --op gather|prefill [--steps K] [--warmup W]
 
 Prints one JSON line (rank 0). ``value`` is the whole-job rate of algorithmic
 K/V bytes (packed data + fp16 scales + page-table entries + q in + out) in
@@ -15,6 +16,13 @@ GB/s, device-timed with CUDA events, max over ranks. Each rank runs its own
 copy of the workload (independent sequences): weak scaling, no collective on
 the data path. ``--impl reference`` times the fp64 CPU oracle on the host
 cores on a bounded sample of the same workload.
+
+``--op`` measures one of the widened rows instead of the decode step, on the
+same workload's layer-0 cache: ``gather`` (the whole context dequantised
+into contiguous bf16 K/V rows; GB/s of algorithmic bytes) or ``prefill`` (a
+2048-query chunk at the end of the context, causal attention over the
+paged F4 cache on the tensor cores; TFLOP/s of the causal attention's
+multiply-adds x 2).
 """
 from __future__ import annotations
 
@@ -50,6 +58,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="host-time budget of the CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--op", choices=["decode", "gather", "prefill"], default="decode",
+                    help="the decode step (default) or one widened row")
+    ap.add_argument("--chunk", type=int, default=2048, help="prefill chunk size (queries)")
     ap.add_argument("--layers", type=int, default=0,
                     help="run fewer layers than the workload has (a smaller case for profiler captures)")
     return ap.parse_args()
@@ -470,6 +481,178 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(result), flush=True)
 
 
+# --------------------------------------------------------------------------- widened rows
+
+def tensor_peak():
+    """Dense fp16/bf16 tensor peak (TFLOP/s): the measured bf16 burst figure
+    (fp16 has the same nominal rate), else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def prefill_flops(prefix: int, n_q: int, q_heads: int, head_dim: int) -> float:
+    """2 x multiply-adds of causal attention of a chunk: query i attends
+    prefix + i + 1 tokens, Q K^T and P V each head_dim per token and head."""
+    tokens = n_q * (prefix + 1) + n_q * (n_q - 1) // 2
+    return 2.0 * 2.0 * tokens * q_heads * head_dim
+
+
+def oracle_op_sample(op: str, w, seconds: float):
+    """The oracle on a bounded host sample of the row: returns (value, unit,
+    cores, sample description)."""
+    import oracle
+    ctx = 16384 if op == "prefill" else 65536
+    s = workloads.Workload(name=w.name + "_sample", n_layers=1, seq_lens=(ctx,), num_pages=-(-ctx // w.block_size),
+                           block_size=w.block_size, q_heads=w.q_heads, kv_heads=w.kv_heads, head_dim=w.head_dim,
+                           head_scale=w.head_scale, k_outlier_frac=w.k_outlier_frac, seed=1)
+    x = workloads.host_layer(s)
+    cache = oracle.empty_cache(s.num_pages, s.kv_heads, s.block_size, s.head_dim)
+    oracle.kv_write_f4(x["k_cache"], x["v_cache"], x["cache_slots"], cache, s.kv_heads, s.head_dim, s.block_size)
+    oracle.kv_write_f4(x["k_new"], x["v_new"], x["step_slots"], cache, s.kv_heads, s.head_dim, s.block_size)
+    pt = x["page_table"]
+    if op == "gather":
+        def run(n):
+            oracle.gather_kv_f4(cache, pt, [n], [0], s.kv_heads, s.head_dim, s.block_size)
+            return n * s.kv_heads * (2 * (s.head_dim // 2 + s.head_dim // 16) + 4 * s.head_dim) + 4 * (n // s.block_size)
+        unit, what = "GB/s", "tokens gathered"
+    else:
+        q = workloads.chunk_queries_host(s, 0, 64)
+
+        def run(n):
+            pos = np.arange(ctx - n, ctx)
+            oracle.prefill_attention(q[:n], cache, pt[0], pos, s.q_heads, s.kv_heads, s.head_dim, s.block_size)
+            return prefill_flops(ctx - n, n, s.q_heads, s.head_dim)
+        unit, what = "TFLOP/s", "chunk queries"
+    n = 1 if op == "prefill" else 1024
+    t0 = time.perf_counter()
+    run(n)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    cap = 64 if op == "prefill" else ctx
+    n = max(1, min(cap, int(n * seconds / dt)))
+    t0 = time.perf_counter()
+    work = run(n)
+    dt = time.perf_counter() - t0
+    scale = 1e9 if unit == "GB/s" else 1e12
+    return work / dt / scale, unit, oracle.max_threads(), f"{n} {what} over a {ctx}-token context, fp64, {dt:.1f} s"
+
+
+def run_op(args, rank, world, local_rank):
+    """Measure the gather or the prefill row on the workload's layer-0 cache."""
+    import torch
+
+    import quantized_paged_kv_yarn_b200 as qkv
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    w = dataclass_replace(workloads.BY_NAME[args.workload], n_layers=1)
+    w = dataclass_replace(w, seed=w.seed + rank)
+    x = workloads.device_layer(w, 0, dev)
+    cache = qkv.PagedF4Cache.allocate(w.num_pages, w.kv_heads, w.block_size, w.head_dim, device=dev)
+    cache.write(x["k_cache"], x["v_cache"], x["cache_slots"])
+    cache.write(x["k_new"], x["v_new"], x["step_slots"])
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ctx = int(sum(w.seq_lens))
+    pt = x["page_table"]
+    if args.op == "gather":
+        lens = x["seq_lens"]
+        start = torch.from_numpy(np.concatenate([[0], np.cumsum(w.seq_lens)[:-1]]).astype(np.int64)).to(dev)
+        k_out = torch.empty((ctx, w.kv_heads, w.head_dim), dtype=torch.int16, device=dev)
+        v_out = torch.empty_like(k_out)
+        h_in = [pt.cpu().pin_memory(), lens.cpu().pin_memory(), start.cpu().pin_memory()]
+        d_in = [pt, lens, start]
+        h_out = [torch.empty(k_out.shape, dtype=k_out.dtype).pin_memory() for _ in range(2)]
+        d_out = [k_out, v_out]
+
+        def call():
+            qkv.qkv_gather_kv_f4(k_out, v_out, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale, pt, lens,
+                                 start, device_status=status)
+        work = ctx * w.kv_heads * (2 * (w.head_dim // 2 + w.head_dim // 16) + 4 * w.head_dim) + 4 * pt.numel()
+        metric, unit, scale = "paged F4 gather to contiguous bf16 K/V GB/s", "GB/s", 1e9
+        peak, peak_kind = hbm_peak()
+        bound, kernel = "hbm", "gather_kv_f4_kernel"
+        cfg = {"workload": w.name, "context_tokens": ctx, "kv_heads": w.kv_heads, "head_dim": w.head_dim,
+               "block_size": w.block_size, "out": "bf16 K and V rows, 1 GiB per 262,144 tokens",
+               "l2": "inputs and outputs larger than L2"}
+    else:
+        n_q = min(args.chunk, ctx)
+        prefix = ctx - n_q
+        q = workloads.chunk_queries_device(w, 0, n_q, dev)
+        out = torch.empty_like(q)
+        row = pt[0].contiguous()
+        h_in, d_in = [q.cpu().pin_memory()], [q]
+        h_out, d_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory()], [out]
+
+        def call():
+            qkv.qkv_paged_prefill_attn_f4(out, q, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale, row,
+                                          prefix, w.kv_heads, device_status=status)
+        work = prefill_flops(prefix, n_q, w.q_heads, w.head_dim)
+        metric, unit, scale = "paged F4 chunked-prefill attention TFLOP/s (causal)", "TFLOP/s", 1e12
+        peak, peak_kind = tensor_peak()
+        bound, kernel = "tensor", "paged_prefill_kernel"
+        cfg = {"workload": w.name, "context_tokens": ctx, "chunk": n_q, "prefix_tokens": prefix,
+               "q_heads": w.q_heads, "kv_heads": w.kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+               "l2": "the layer's 302 MB cache exceeds L2; query blocks of a KV head share pages through it"}
+    cfg["parallelism"] = f"replicas{world}"
+
+    def sync_all():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        call()
+    sync_all()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+    sync_all()
+    ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
+
+    def e2e():
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        call()
+        for h, d in zip(h_out, d_out):
+            h.copy_(d, non_blocking=True)
+    e2e()
+    sync_all()
+    e0.record()
+    for _ in range(args.steps):
+        e2e()
+    e1.record()
+    torch.cuda.synchronize()
+    sync_all()
+    ms_e2e = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
+    if rank != 0:
+        return
+    nb = lambda ts: sum(t.numel() * t.element_size() for t in ts)
+    value = world * work / (ms * 1e-3) / scale
+    achieved = work / (ms * 1e-3) / scale
+    result = {
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u4 cache -> bf16" if args.op == "gather" else "f16 tcgen05, f32 accumulate",
+        "data": "synthetic", "config": cfg, "device_status": int(status.item()),
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                     "traffic": None, "kernel": kernel, "peak_kind": peak_kind, "kernel_ms": ms,
+                     "timing": "CUDA events around back-to-back launches"},
+        "e2e": {"value": world * work / (ms_e2e * 1e-3) / scale, "unit": unit, "h2d_bytes_per_step": nb(h_in),
+                "d2h_bytes_per_step": nb(h_out), "ms_per_step": ms_e2e},
+        "gpu_launches": args.steps, "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, u, cores, sample = oracle_op_sample(args.op, w, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": v, "unit": u, "cores": cores, "kind": "oracle", "sample": sample}
+    print(json.dumps(result), flush=True)
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -485,7 +668,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device(f"cuda:{local_rank}"))
     try:
-        run_ours(args, rank, world, local_rank)
+        if args.op == "decode":
+            run_ours(args, rank, world, local_rank)
+        else:
+            run_op(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
