@@ -328,8 +328,8 @@ QKV_API int qkv_gather_kv_f4(uint16_t* k_out, uint16_t* v_out, int64_t n_out, co
  *              page page_table[t / block_size]. prefix_len + n_q must not
  *              exceed max_pages_per_seq * block_size (else QKV_EINVAL).
  *   cache, v_group, softmax_scale as in qkv_paged_decode_split_f4_v.
- * Compiled shapes: head_dim 256, q_heads / kv_heads in {1, 2, 4, 8}, any
- * block_size (else QKV_EUNSUPPORTED). Runs on the tensor cores (tcgen05,
+ * Compiled shapes: head_dim 256, q_heads / kv_heads in {1, 2, 4, 8}, a
+ * power-of-two block_size (else QKV_EUNSUPPORTED). Runs on the tensor cores (tcgen05,
  * fp16 operands, fp32 accumulators in tensor memory): K and V are
  * dequantised to fp16 in shared memory, q scaled by a power of two per
  * row; outputs match exact attention within 2e-3. A page id outside the

@@ -89,7 +89,7 @@ struct Params {
   const uint16_t* v_scale;
   const int32_t* page_table;
   int64_t num_pages;
-  int n_q, prefix_len, q_heads, kv_heads, G, QB, block, v_tok;
+  int n_q, prefix_len, q_heads, kv_heads, G, QB, block, block_shift, v_tok;
   float score_scale;  // softmax_scale * log2(e)
   int32_t* status;
 };
@@ -166,16 +166,30 @@ __device__ __forceinline__ float ex2(float x) {
 // Byte offset of 16-byte unit u of row r in a [rows][128 B] 128-byte-swizzled chunk.
 __device__ __forceinline__ uint32_t swz(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
-// Bounded wait that also gives up once another role has aborted.
+// try_wait that may suspend the thread (no issue slots) for up to `ns`
+// nanoseconds or until the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait that also gives up once another role has aborted. Waiting
+// threads sleep in the barrier instead of spinning, leaving the issue slots
+// to the warps that do the work.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
-  for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > WAIT_LIMIT_NS) return false;
-    }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > WAIT_LIMIT_NS) return false;
   }
 }
 
@@ -203,7 +217,8 @@ __device__ __forceinline__ uint32_t bf2_u32(float a, float b) {
 struct Raw {
   uint4 k0, k1, v0, v1;
   uint32_t ks, vs;
-  int ok;  // 0: outside the context (zero rows), 1: data, 2: bad page (zero rows, flagged)
+  int ok;         // 0: outside the context (zero rows), 1: data, 2: bad page (zero rows, flagged)
+  int32_t page;   // page id of the stage this set loads next (read one load ahead)
 };
 
 __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params p) {
@@ -256,15 +271,20 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
       constexpr uint32_t ID_PV = (1u << 4) | (1u << 16) | ((uint32_t)(D >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
       const uint32_t sp = s_base + P_OFF;
       bool ok = wait_bar(&bars.qready, 0, abort);
+      // descriptors of slot 0 at offset 0; each MMA adds its byte offset >> 4
+      // to the start-address field (no carry: smem offsets stay below 2^18)
+      const uint64_t dp0 = sdesc(sp, 16, 1024);
+      const uint64_t dv0 = sdesc(s_base + V_OFF, NT * 128, 1024);
+      const uint64_t dk0 = sdesc(s_base + K_OFF, 16, 1024);
       auto pv = [&](int i) -> bool {
         const int b = i & 1;
         if (!wait_bar(&bars.pready, (uint32_t)i & 1u, abort)) return false;
         if (!wait_bar(&bars.vready[b], (uint32_t)(i >> 1) & 1u, abort)) return false;
         tc_fence_after();
-        const uint32_t sv = s_base + V_OFF + b * TILE;
+        const uint64_t dv = dv0 + (uint64_t)((b * TILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < NT / 16; ++kk)
-          umma(tmem, sdesc(sp + 32 * kk, 16, 1024), sdesc(sv + 2048 * kk, NT * 128, 1024), ID_PV,
+          umma(tmem, dp0 + (uint64_t)((32 * kk) >> 4), dv + (uint64_t)((2048 * kk) >> 4), ID_PV,
                (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&bars.odone);
         umma_commit(&bars.vfree[b]);
@@ -275,14 +295,14 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
         if (!wait_bar(&bars.kready[b], (uint32_t)(j >> 1) & 1u, abort)) { ok = false; break; }
         if (j >= 2 && !wait_bar(&bars.sfree[b], (uint32_t)((j - 2) >> 1) & 1u, abort)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sk = s_base + K_OFF + b * (2 * TILE);
+        const uint64_t dk = dk0 + (uint64_t)((b * 2 * TILE) >> 4);
+        const uint32_t ts = tmem + 256 + 64 * b;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // K^'hi, then K^'lo into the same accumulator
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t bb = sk + h * TILE + (kk >> 2) * (NT * 128) + 32 * (kk & 3);
-            umma_ts(tmem + 256 + 64 * b, tmem + TQ + 8 * kk, sdesc(bb, 16, 1024), ID_QK,
-                    (h > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t off = h * TILE + (kk >> 2) * (NT * 128) + 32 * (kk & 3);
+            umma_ts(ts, tmem + TQ + 8 * kk, dk + (uint64_t)(off >> 4), ID_QK, (h > 0 || kk > 0) ? 1u : 0u);
           }
         }
         umma_commit(&bars.sfull[b]);
@@ -465,17 +485,25 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
     const int d = tid - 256;
     const int tk = d >> 2, c = d & 3;
     const size_t row_bytes = D / 2;
-    auto load = [&](int j, Raw& x) {
-      x.ok = 0;
-      if (j >= n_st) return;
+    // page id of this thread's token in stage j (-1 past the context)
+    auto page_of = [&](int j) -> int32_t {
       const int t = j * NT + tk;
-      if (t >= kv_len) return;
-      const int32_t page = p.page_table[t / p.block];
+      return (j < n_st && t < kv_len) ? __ldg(p.page_table + (t >> p.block_shift)) : -1;
+    };
+    // The packed bytes of stage j into x, using the page id read by the
+    // previous load of x; then the page id of stage j + 2 for the next one,
+    // so no data load waits on a page-table read.
+    auto load = [&](int j, Raw& x) {
+      const int32_t page = x.page;
+      x.page = page_of(j + 2);
+      x.ok = 0;
+      const int t = j * NT + tk;
+      if (j >= n_st || t >= kv_len) return;
       if (page < 0 || page >= p.num_pages) {
         x.ok = 2;
         return;
       }
-      const size_t row = ((size_t)page * p.kv_heads + kvh) * p.block + (t % p.block);
+      const size_t row = ((size_t)page * p.kv_heads + kvh) * p.block + (t & (p.block - 1));
       const uint4* kp = reinterpret_cast<const uint4*>(p.k_data + row * row_bytes + 32 * c);
       const uint4* vp = reinterpret_cast<const uint4*>(p.v_data + row * row_bytes + 32 * c);
       x.k0 = __ldg(kp);
@@ -508,7 +536,7 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
     };
     auto process = [&](int j, const Raw& x) -> bool {
       const int b = j & 1;
-      if (x.ok == 2 && c == 0 && kvh == 0 && ((j * NT + tk) % p.block) == 0) flag(p.status, QKV_DEV_BAD_PAGE);
+      if (x.ok == 2 && c == 0 && kvh == 0 && ((j * NT + tk) & (p.block - 1)) == 0) flag(p.status, QKV_DEV_BAD_PAGE);
       if (j >= 2 && !wait_bar(&bars.kfree[b], (uint32_t)((j - 2) >> 1) & 1u, abort)) return false;
       put(s_base + K_OFF + b * (2 * TILE) + c * (NT * 128), x.k0, x.k1, x.ks, x.ok, std::true_type{});
       fence_async_smem();
@@ -520,6 +548,8 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
       return true;
     };
     Raw ra, rb;
+    ra.page = page_of(0);
+    rb.page = page_of(1);
     load(0, ra);
     load(1, rb);
     bool ok = true;
@@ -566,6 +596,7 @@ extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const u
   if (((uintptr_t)k_scale | (uintptr_t)v_scale | (uintptr_t)lse2_out) & 3) return QKV_EINVAL;
   const int G = q_heads / kv_heads;
   if (head_dim != prefill::D || (G != 1 && G != 2 && G != 4 && G != 8)) return QKV_EUNSUPPORTED;
+  if (block_size & (block_size - 1)) return QKV_EUNSUPPORTED;  // pages of a power-of-two size
   if (kv_heads > 65535) return QKV_EUNSUPPORTED;
 
   prefill::Params p;
@@ -585,6 +616,8 @@ extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const u
   p.G = G;
   p.QB = prefill::M / G;
   p.block = block_size;
+  p.block_shift = 0;
+  while ((1 << p.block_shift) < block_size) ++p.block_shift;
   p.v_tok = v_group != 32;
   const float sc = softmax_scale > 0.f ? softmax_scale : 0.0625f;  // 1 / sqrt(256)
   p.score_scale = sc * 1.4426950408889634f;
