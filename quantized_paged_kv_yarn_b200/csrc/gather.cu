@@ -26,10 +26,10 @@ __global__ void __launch_bounds__(256) gather_kv_f4_kernel(
   const int s = blockIdx.y;
   const int cells = head_dim / 32;
   // thread -> (token t, head h, K or V, cell c), cells fastest
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int per_tok = kv_heads * 2 * cells;
-  const int64_t t = i / per_tok;
-  int rem = (int)(i - t * per_tok);
+  const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;  // < 2^31 (checked on the host)
+  const uint32_t per_tok = (uint32_t)(kv_heads * 2 * cells);
+  const int t = (int)(i / per_tok);
+  int rem = (int)(i - (uint32_t)t * per_tok);
   const int h = rem / (2 * cells);
   rem -= h * 2 * cells;
   const int which = rem / cells, c = rem - which * cells;
@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(256) gather_kv_f4_kernel(
     if (t % block == 0 && rem == 0 && h == 0) flag(status, QKV_DEV_BAD_PAGE);
     const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) dst[j] = z;
+    for (int j = 0; j < 4; ++j) __stcs(dst + j, z);
     return;
   }
   const int64_t row = ((int64_t)page * kv_heads + h) * block + t % block;
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(256) gather_kv_f4_kernel(
       const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
       o[e] = *reinterpret_cast<const uint32_t*>(&p);
     }
-    dst[j] = make_uint4(o[0], o[1], o[2], o[3]);
+    __stcs(dst + j, make_uint4(o[0], o[1], o[2], o[3]));  // streaming: the rows are not read back here
   }
 }
 
@@ -95,7 +95,7 @@ extern "C" int qkv_gather_kv_f4(uint16_t* k_out, uint16_t* v_out, int64_t n_out,
   if (((uintptr_t)k_scale | (uintptr_t)v_scale) & 1) return QKV_EINVAL;
   const int64_t threads = (int64_t)max_pages_per_seq * block_size * kv_heads * 2 * (head_dim / 32);
   const int64_t blocks = (threads + 255) / 256;
-  if (blocks > 0x7fffffff) return QKV_EUNSUPPORTED;
+  if (threads > 0x7fffffff) return QKV_EUNSUPPORTED;
   __half* ks = reinterpret_cast<__half*>(const_cast<uint16_t*>(k_scale));
   __half* vs = reinterpret_cast<__half*>(const_cast<uint16_t*>(v_scale));
   int mp = max_pages_per_seq, kvh = kv_heads, hd = head_dim, bs = block_size, vg = v_group;
