@@ -38,8 +38,11 @@
 // accumulate in fp32; p = 2^(s - m_ref) in fp16 with the reference max moved
 // lazily (only when a score exceeds it by more than 8, so p <= 256).
 //
-// Q' lives in tensor memory (the A operand of Q K^T; row r in lane r, two
-// fp16 per column). Shared-memory tiles use the 128-byte swizzle in the
+// Q' and P live in tensor memory (the A operands; row r in lane r, two fp16
+// per column); P of a stage overwrites the first half of the S columns it
+// was computed from, which the next Q K^T into that slot may overwrite only
+// after the P . V reading it (issued earlier by the same thread, and the
+// tensor core keeps one thread's MMAs in order). Shared-memory tiles use the 128-byte swizzle in the
 // canonical UMMA layouts: a K-major tile is [K / 64 chunks][rows][128 B];
 // the V^' tile, the MN-major B operand of P . V, is
 // [256 dims / 64 chunks][64 tokens][128 B]. Within each 8-dim unit the dims
@@ -63,16 +66,16 @@ constexpr float TH = 8.f;       // lazy-rescale threshold (log2 units)
 constexpr int TILE = 4 * NT * 128;              // one [4 chunks][64][128 B] tile: 32 KB
 constexpr int K_OFF = 0;                        // 2 slots x (hi tile, lo tile)
 constexpr int V_OFF = K_OFF + 2 * 2 * TILE;     // 2 slots x tile
-constexpr int P_OFF = V_OFF + 2 * TILE;         // [128][128 B]
-constexpr int BAR_OFF = P_OFF + M * 128;
+constexpr int BAR_OFF = V_OFF + 2 * TILE;
 constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;  // barriers, flags, alignment slack
 
-// TMEM columns: O 0..255, S slot b at 256 + 64 b, Q' at 384..511
+// TMEM columns: O 0..255, S slot b at 256 + 64 b (P of that stage, fp16,
+// overwrites its first 32 columns once S is read), Q' at 384..511
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TQ = 384;
 
 struct Bars {
-  uint64_t kready[2], kfree[2], vready[2], vfree[2], sfull[2], sfree[2];
+  uint64_t kready[2], kfree[2], vready[2], vfree[2], sfull[2];
   uint64_t pready, odone, qready, drain;
   uint32_t tmem;
   int abort;
@@ -98,13 +101,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
   // start >> 4 | LBO >> 4 << 16 | SBO >> 4 << 32 | version 1 << 46 | 128-byte swizzle (2) << 61
   return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
          (1ull << 46) | (2ull << 61);
-}
-
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc));
 }
 
 // A from tensor memory (row r in lane r), B from shared memory
@@ -214,6 +210,26 @@ __device__ __forceinline__ uint32_t bf2_u32(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// Loads issued where they stand in the program (volatile: the compiler may
+// not sink them to their first use, which would expose their latency).
+__device__ __forceinline__ uint4 ldg_early16(const void* ptr) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(ptr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_early4(const void* ptr) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(ptr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg_early2(const void* ptr) {
+  unsigned short v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(ptr));
+  return v;
+}
+
 struct Raw {
   uint4 k0, k1, v0, v1;
   uint32_t ks, vs;
@@ -241,7 +257,6 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
       mbar_init(&bars.kfree[b], 1);
       mbar_init(&bars.vfree[b], 1);
       mbar_init(&bars.sfull[b], 1);
-      mbar_init(&bars.sfree[b], 128);
     }
     mbar_init(&bars.pready, 128);
     mbar_init(&bars.odone, 1);
@@ -269,11 +284,9 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
     if (lane == 0) {
       constexpr uint32_t ID_QK = (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
       constexpr uint32_t ID_PV = (1u << 4) | (1u << 16) | ((uint32_t)(D >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-      const uint32_t sp = s_base + P_OFF;
       bool ok = wait_bar(&bars.qready, 0, abort);
       // descriptors of slot 0 at offset 0; each MMA adds its byte offset >> 4
       // to the start-address field (no carry: smem offsets stay below 2^18)
-      const uint64_t dp0 = sdesc(sp, 16, 1024);
       const uint64_t dv0 = sdesc(s_base + V_OFF, NT * 128, 1024);
       const uint64_t dk0 = sdesc(s_base + K_OFF, 16, 1024);
       auto pv = [&](int i) -> bool {
@@ -283,9 +296,9 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
         tc_fence_after();
         const uint64_t dv = dv0 + (uint64_t)((b * TILE) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < NT / 16; ++kk)
-          umma(tmem, dp0 + (uint64_t)((32 * kk) >> 4), dv + (uint64_t)((2048 * kk) >> 4), ID_PV,
-               (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < NT / 16; ++kk)  // A = P in tensor memory (S slot b)
+          umma_ts(tmem, tmem + 256 + 64 * b + 8 * kk, dv + (uint64_t)((2048 * kk) >> 4), ID_PV,
+                  (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&bars.odone);
         umma_commit(&bars.vfree[b]);
         return true;
@@ -293,7 +306,9 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
       for (int j = 0; ok && j < n_st; ++j) {
         const int b = j & 1;
         if (!wait_bar(&bars.kready[b], (uint32_t)(j >> 1) & 1u, abort)) { ok = false; break; }
-        if (j >= 2 && !wait_bar(&bars.sfree[b], (uint32_t)((j - 2) >> 1) & 1u, abort)) { ok = false; break; }
+        // S slot b is free again: P . V of stage j - 2, which read P from it,
+        // was issued (after its pready) before this Q K^T, and the tensor
+        // core runs one thread's MMAs in order
         tc_fence_after();
         const uint64_t dk = dk0 + (uint64_t)((b * 2 * TILE) >> 4);
         const uint32_t ts = tmem + 256 + 64 * b;
@@ -377,7 +392,6 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
 
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    const uint32_t prow = s_base + P_OFF;
     for (int j = 0; j < n_st; ++j) {
       const int b = j & 1;
       ok = wait_bar(&bars.sfull[b], (uint32_t)(j >> 1) & 1u, abort);
@@ -387,8 +401,6 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
       tmem_ld32(tmem + lane_base + 256 + 64 * b, sr[0]);
       tmem_ld32(tmem + lane_base + 256 + 64 * b + 32, sr[1]);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars.sfree[b]);
       float s[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(sr[i >> 5][i & 31]);
@@ -422,14 +434,12 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
         l += hf.x + hf.y;
         pw[i] = h2_as_u32(h);
       }
-      if (j >= 1) {  // P . V of the previous stage done: P free, O stable
+      // P into the first 32 columns of S slot b (its S is in registers)
+      tmem_st32(tmem + lane_base + 256 + 64 * b, pw);
+      if (any_need && j >= 1) {  // rescale O once P . V of the previous stage is done
         ok = wait_bar(&bars.odone, (uint32_t)(j - 1) & 1u, abort);
         if (!__all_sync(FULL_MASK, ok)) { ok = false; break; }
         tc_fence_after();
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) sts128(prow + swz(r, u), pw[4 * u], pw[4 * u + 1], pw[4 * u + 2], pw[4 * u + 3]);
-      if (any_need && j >= 1) {
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -439,9 +449,8 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tmem + lane_base + 32 * c, o);
         }
-        tmem_wait_st();
       }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars.pready);
     }
@@ -488,7 +497,7 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
     // page id of this thread's token in stage j (-1 past the context)
     auto page_of = [&](int j) -> int32_t {
       const int t = j * NT + tk;
-      return (j < n_st && t < kv_len) ? __ldg(p.page_table + (t >> p.block_shift)) : -1;
+      return (j < n_st && t < kv_len) ? (int32_t)ldg_early4(p.page_table + (t >> p.block_shift)) : -1;
     };
     // The packed bytes of stage j into x, using the page id read by the
     // previous load of x; then the page id of stage j + 2 for the next one,
@@ -506,16 +515,16 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
       const size_t row = ((size_t)page * p.kv_heads + kvh) * p.block + (t & (p.block - 1));
       const uint4* kp = reinterpret_cast<const uint4*>(p.k_data + row * row_bytes + 32 * c);
       const uint4* vp = reinterpret_cast<const uint4*>(p.v_data + row * row_bytes + 32 * c);
-      x.k0 = __ldg(kp);
-      x.k1 = __ldg(kp + 1);
-      x.v0 = __ldg(vp);
-      x.v1 = __ldg(vp + 1);
-      x.ks = __ldg(reinterpret_cast<const uint32_t*>(p.k_scale + row * 8 + 2 * c));
+      x.k0 = ldg_early16(kp);
+      x.k1 = ldg_early16(kp + 1);
+      x.v0 = ldg_early16(vp);
+      x.v1 = ldg_early16(vp + 1);
+      x.ks = ldg_early4(p.k_scale + row * 8 + 2 * c);
       if (p.v_tok) {
-        const uint32_t h = __ldg(p.v_scale + row);
+        const uint32_t h = ldg_early2(p.v_scale + row);
         x.vs = h | (h << 16);
       } else {
-        x.vs = __ldg(reinterpret_cast<const uint32_t*>(p.v_scale + row * 8 + 2 * c));
+        x.vs = ldg_early4(p.v_scale + row * 8 + 2 * c);
       }
       x.ok = 1;
     };
