@@ -95,25 +95,25 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(source: str = "decode_split.cu") -> str:
     h = hashlib.sha256()
-    for name in ("decode_split.cu", "common.cuh"):
+    for name in (source, "common.cuh"):
         with open(os.path.join(ROOT, "quantized_paged_kv_yarn_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per split-kernel launch from the committed ncu summary, if
+def profiled_traffic(workload: str, kernel: str = "paged_decode_split", source: str = "decode_split.cu"):
+    """DRAM bytes per launch of a kernel from its committed ncu summary, if
     it was taken from the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"paged_decode_split_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         text = open(path).read()
     except OSError:
         return None
     m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
     m_traffic = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not m_hash or not m_traffic or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_traffic or m_hash.group(1) != kernel_source_hash(source):
         return None
     return int(m_traffic.group(1))
 
@@ -633,6 +633,7 @@ def run_op(args, rank, world, local_rank):
     if rank != 0:
         return
     nb = lambda ts: sum(t.numel() * t.element_size() for t in ts)
+    profile_of = {"gather": ("gather_kv_f4", "gather.cu"), "prefill": ("paged_prefill", "prefill.cu")}
     value = world * work / (ms * 1e-3) / scale
     achieved = work / (ms * 1e-3) / scale
     result = {
@@ -641,7 +642,8 @@ def run_op(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "u4 cache -> bf16" if args.op == "gather" else "f16 tcgen05, f32 accumulate",
         "data": "synthetic", "config": cfg, "device_status": int(status.item()),
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                     "traffic": None, "kernel": kernel, "peak_kind": peak_kind, "kernel_ms": ms,
+                     "traffic": profiled_traffic(w.name, *profile_of[args.op]), "kernel": kernel,
+                     "peak_kind": peak_kind, "kernel_ms": ms,
                      "timing": "CUDA events around back-to-back launches"},
         "e2e": {"value": world * work / (ms_e2e * 1e-3) / scale, "unit": unit, "h2d_bytes_per_step": nb(h_in),
                 "d2h_bytes_per_step": nb(h_out), "ms_per_step": ms_e2e},
