@@ -1,5 +1,6 @@
 // prefill.cu -- chunked causal prefill attention over the paged F4 cache
-// on the sm_100a tensor cores (tcgen05, accumulators in tensor memory).
+// on the sm_100a tensor cores (tcgen05, CTA pairs, accumulators in tensor
+// memory).
 //
 // Sources: mistral.rs PR "YaRN rope scaling, 4-bit F4 packed KV cache, and
 // hybrid paged attention for Qwen3.5-Next long-context serving", section 2
@@ -8,24 +9,35 @@
 // sits at cache tokens prefix_len .. prefix_len + n_q - 1 (already written);
 // query i attends the cached tokens 0 .. prefix_len + i.
 //
-// This is a dense contraction (128 query rows share every dequantised
-// page), so it runs on tcgen05.mma with fp32 accumulators in TMEM:
+// This is a dense contraction (256 query rows share every dequantised
+// page), so it runs on tcgen05.mma with fp32 accumulators in TMEM, issued
+// for a pair of CTAs on two SMs (cta_group::2, M = 256):
 //
-//   S[128 x 64]  = Q'[128 x 256] . (K^'hi + K^'lo)[64 x 256]^T   (2 x 16 MMAs, K = 16)
-//   O[128 x 256] += P[128 x 64] . V^'[64 x 256]                  (4 MMAs, N = 256)
+//   S[256 x 64]  = Q'[256 x 256] . (K^'hi + K^'lo)[64 x 256]^T   (2 x 16 MMAs, K = 16)
+//   O[256 x 256] += P[256 x 64] . V^'[64 x 256]                  (4 MMAs, N = 256)
 //
-// Rows are (query head of the GQA group, query): 128 = G x (128 / G).
-// One CTA per (128 / G queries, KV head); stages of 64 tokens.
+// Rows are (query head of the GQA group, query): 256 = G x (256 / G); CTA
+// rank r of the pair owns rows 128 r .. 128 r + 127 (its lanes of Q', S, P
+// and O). The B operands are split by N: of each 64-token stage, rank r
+// dequantises the K of tokens 32 r .. 32 r + 31 (all 256 dims) and the V of
+// dims 128 r .. 128 r + 127 (all 64 tokens) into its own shared memory, so
+// each SM writes and the tensor core reads half of every tile, and the
+// shared-memory pipe (the bound of a one-SM version) carries half the bytes.
+// One pair per (256 / G queries, KV head).
 //
-// Warp roles (512 threads):
-//   warp 0        TMEM allocation; lane 0 issues every MMA and commit
-//   warps 4..7    softmax: thread r owns row r (TMEM lane r): puts its row
-//                 of Q' into tensor memory, reads S, keeps the running max
-//                 and sum, writes P, rescales O when the max moves, and
+// Warp roles (512 threads per CTA):
+//   warp 0        TMEM allocation (both CTAs); in rank 0, lane 0 issues every
+//                 MMA and commit of the pair
+//   warps 4..7    softmax: thread r owns row r of its CTA (TMEM lane r): puts
+//                 its row of Q' into tensor memory, reads S, keeps the running
+//                 max and sum, writes P, rescales O when the max moves, and
 //                 writes the output
-//   warps 8..15   dequantisation: each thread turns one token's 64 dims of
-//                 K and of V (32 packed bytes each) into fp16 in a swizzled
-//                 shared tile, prefetching the packed bytes two stages ahead
+//   warps 8..11   K dequantisation: one token's 64 dims of K per thread
+//   warps 12..15  V dequantisation: one token's 64 of this CTA's 128 dims
+//                 Packed bytes are read two stages ahead, page ids one
+//                 load ahead of those.
+// Producers signal rank 0's barriers (a remote arrive from rank 1); the MMA
+// thread's commits arrive on both CTAs' barriers (multicast).
 //
 // Numerics. With s' = scale * 2^-4 (exact while scale >= 2^-10; the 2^-4
 // keeps 8 * 65504 in range), a K element (code - 8) s' needs up to 14
@@ -42,13 +54,13 @@
 // per column); P of a stage overwrites the first half of the S columns it
 // was computed from, which the next Q K^T into that slot may overwrite only
 // after the P . V reading it (issued earlier by the same thread, and the
-// tensor core keeps one thread's MMAs in order). Shared-memory tiles use the 128-byte swizzle in the
-// canonical UMMA layouts: a K-major tile is [K / 64 chunks][rows][128 B];
-// the V^' tile, the MN-major B operand of P . V, is
-// [256 dims / 64 chunks][64 tokens][128 B]. Within each 8-dim unit the dims
-// are stored in the order 0,4,1,5,2,6,3,7 (the order in which four nibble
-// masks of a packed word yield them); Q' uses the same order, and the
-// output un-permutes O's columns.
+// tensor core keeps one thread's MMAs in order). Shared-memory tiles use the
+// 128-byte swizzle in the canonical UMMA layouts: the K^' tiles (K-major)
+// are [4 chunks of 64 dims][32 tokens][128 B]; the V^' tile, the MN-major
+// B operand of P . V, is [2 chunks of 64 dims][64 tokens][128 B]. Within
+// each 8-dim unit the dims are stored in the order 0,4,1,5,2,6,3,7 (the
+// order in which four nibble masks of a packed word yield them); Q' uses the
+// same order, and the output un-permutes O's columns.
 #include <type_traits>
 
 #include "common.cuh"
@@ -58,25 +70,33 @@ namespace prefill {
 
 constexpr int THREADS = 512;
 constexpr int D = 256;
-constexpr int M = 128;          // rows per CTA
+constexpr int M = 256;          // rows per CTA pair
+constexpr int ML = 128;         // rows per CTA
 constexpr int NT = 64;          // tokens per stage
+constexpr int NTL = NT / 2;     // K tokens per CTA per stage
+constexpr int NS = 3;           // shared-memory slots of K^ and V^
 constexpr float TH = 8.f;       // lazy-rescale threshold (log2 units)
 
 // shared-memory map (offsets from a 1024-byte aligned base)
-constexpr int TILE = 4 * NT * 128;              // one [4 chunks][64][128 B] tile: 32 KB
-constexpr int K_OFF = 0;                        // 2 slots x (hi tile, lo tile)
-constexpr int V_OFF = K_OFF + 2 * 2 * TILE;     // 2 slots x tile
-constexpr int BAR_OFF = V_OFF + 2 * TILE;
+constexpr int KT = 4 * NTL * 128;               // one K^ tile (hi or lo): [4][32][128 B] = 16 KB
+constexpr int VT = 2 * NT * 128;                // one V^ tile: [2][64][128 B] = 16 KB
+constexpr int K_OFF = 0;                        // NS slots x (hi, lo)
+constexpr int V_OFF = K_OFF + NS * 2 * KT;      // NS slots
+constexpr int BAR_OFF = V_OFF + NS * VT;
 constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;  // barriers, flags, alignment slack
+static_assert(SMEM_BYTES > 116 * 1024, "one CTA per SM: TMEM is allocated whole");
 
-// TMEM columns: O 0..255, S slot b at 256 + 64 b (P of that stage, fp16,
-// overwrites its first 32 columns once S is read), Q' at 384..511
+// TMEM columns (each CTA, its 128 rows): O 0..255, S slot b at 256 + 64 b
+// (P of that stage, fp16, overwrites its first 32 columns once S is read),
+// Q' at 384..511
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TQ = 384;
 
 struct Bars {
-  uint64_t kready[2], kfree[2], vready[2], vfree[2], sfull[2];
-  uint64_t pready, odone, qready, drain;
+  // signalled by producers of both CTAs, waited on in rank 0
+  uint64_t kready[NS], vready[NS], pready, qready;
+  // signalled by the MMA commits of the pair, waited on in each CTA
+  uint64_t kfree[NS], vfree[NS], sfull[2], odone, drain;
   uint32_t tmem;
   int abort;
 };
@@ -103,17 +123,42 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
          (1ull << 46) | (2ull << 61);
 }
 
-// A from tensor memory (row r in lane r), B from shared memory
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+// Pair MMA: A from tensor memory (row r of each CTA in its lane r), B from
+// both CTAs' shared memory at the same offset (each holds N / 2 columns).
+__device__ __forceinline__ void umma2_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                         uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
 }
 
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
+// Arrive, once the pair's MMAs issued so far are done, on the barrier at
+// this offset in both CTAs.
+__device__ __forceinline__ void umma2_commit_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((unsigned short)3)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// All threads of both CTAs.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on rank 0's copy of a barrier (release at cluster scope).
+__device__ __forceinline__ void arrive_rank0(uint64_t* bar) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(remote) : "r"(smem_u32(bar)));
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -162,13 +207,14 @@ __device__ __forceinline__ float ex2(float x) {
 // Byte offset of 16-byte unit u of row r in a [rows][128 B] 128-byte-swizzled chunk.
 __device__ __forceinline__ uint32_t swz(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
-// try_wait that may suspend the thread (no issue slots) for up to `ns`
+// try_wait (acquire at cluster scope: producers of the other CTA release to
+// it) that may suspend the thread, using no issue slots, for up to `ns`
 // nanoseconds or until the phase completes.
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
@@ -176,11 +222,9 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Bounded wait that also gives up once another role has aborted. Waiting
-// threads sleep in the barrier instead of spinning, leaving the issue slots
-// to the warps that do the work.
+// Bounded wait that also gives up once another role of this CTA has
+// aborted. Waiting threads sleep in the barrier instead of spinning.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
@@ -230,58 +274,62 @@ __device__ __forceinline__ uint32_t ldg_early2(const void* ptr) {
   return v;
 }
 
+// One dequantising thread's packed bytes of one stage.
 struct Raw {
-  uint4 k0, k1, v0, v1;
-  uint32_t ks, vs;
+  uint4 a, b;     // 32 packed bytes: 64 dims
+  uint32_t sc;    // fp16 scales of the two 32-dim cells (or the token's V scale, twice)
   int ok;         // 0: outside the context (zero rows), 1: data, 2: bad page (zero rows, flagged)
   int32_t page;   // page id of the stage this set loads next (read one load ahead)
 };
 
-__global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    paged_prefill_kernel(const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars& bars = *reinterpret_cast<Bars*>(sm + BAR_OFF);
   const uint32_t s_base = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rank = (int)cluster_rank();
 
   const int kvh = blockIdx.y;
-  const int q0 = blockIdx.x * p.QB;
-  const int q_last = min(p.n_q, q0 + p.QB) - 1;
+  const int QB2 = p.QB;  // queries per pair
+  const int q0 = (blockIdx.x >> 1) * QB2;
+  const int q_last = min(p.n_q, q0 + QB2) - 1;
   const int kv_len = p.prefix_len + q_last + 1;
   const int n_st = (kv_len + NT - 1) / NT;
 
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars.kready[b], 256);
-      mbar_init(&bars.vready[b], 256);
+    for (int b = 0; b < NS; ++b) {
+      mbar_init(&bars.kready[b], 2 * 128);
+      mbar_init(&bars.vready[b], 2 * 128);
       mbar_init(&bars.kfree[b], 1);
       mbar_init(&bars.vfree[b], 1);
-      mbar_init(&bars.sfull[b], 1);
     }
-    mbar_init(&bars.pready, 128);
+    for (int b = 0; b < 2; ++b) mbar_init(&bars.sfull[b], 1);
+    mbar_init(&bars.pready, 2 * 128);
+    mbar_init(&bars.qready, 2 * 128);
     mbar_init(&bars.odone, 1);
-    mbar_init(&bars.qready, 128);
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
     fence_barrier_init();
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&bars.tmem)),
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&bars.tmem)),
                  "r"(TMEM_COLS)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   pdl_wait();
   pdl_release();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
   const uint32_t tmem = bars.tmem;
   volatile int* abort = &bars.abort;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issue (rank 0)
+    if (rank == 0 && lane == 0) {
       constexpr uint32_t ID_QK = (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
       constexpr uint32_t ID_PV = (1u << 4) | (1u << 16) | ((uint32_t)(D >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
       bool ok = wait_bar(&bars.qready, 0, abort);
@@ -290,38 +338,38 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
       const uint64_t dv0 = sdesc(s_base + V_OFF, NT * 128, 1024);
       const uint64_t dk0 = sdesc(s_base + K_OFF, 16, 1024);
       auto pv = [&](int i) -> bool {
-        const int b = i & 1;
+        const int b = i % NS, u = i / NS, sb = i & 1;
         if (!wait_bar(&bars.pready, (uint32_t)i & 1u, abort)) return false;
-        if (!wait_bar(&bars.vready[b], (uint32_t)(i >> 1) & 1u, abort)) return false;
+        if (!wait_bar(&bars.vready[b], (uint32_t)u & 1u, abort)) return false;
         tc_fence_after();
-        const uint64_t dv = dv0 + (uint64_t)((b * TILE) >> 4);
+        const uint64_t dv = dv0 + (uint64_t)((b * VT) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < NT / 16; ++kk)  // A = P in tensor memory (S slot b)
-          umma_ts(tmem, tmem + 256 + 64 * b + 8 * kk, dv + (uint64_t)((2048 * kk) >> 4), ID_PV,
-                  (i > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&bars.odone);
-        umma_commit(&bars.vfree[b]);
+        for (int kk = 0; kk < NT / 16; ++kk)  // A = P in tensor memory (S slot sb)
+          umma2_ts(tmem, tmem + 256 + 64 * sb + 8 * kk, dv + (uint64_t)((2048 * kk) >> 4), ID_PV,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+        umma2_commit_both(&bars.odone);
+        umma2_commit_both(&bars.vfree[b]);
         return true;
       };
       for (int j = 0; ok && j < n_st; ++j) {
-        const int b = j & 1;
-        if (!wait_bar(&bars.kready[b], (uint32_t)(j >> 1) & 1u, abort)) { ok = false; break; }
-        // S slot b is free again: P . V of stage j - 2, which read P from it,
+        const int b = j % NS, u = j / NS, sb = j & 1;
+        if (!wait_bar(&bars.kready[b], (uint32_t)u & 1u, abort)) { ok = false; break; }
+        // S slot sb is free again: P . V of stage j - 2, which read P from it,
         // was issued (after its pready) before this Q K^T, and the tensor
         // core runs one thread's MMAs in order
         tc_fence_after();
-        const uint64_t dk = dk0 + (uint64_t)((b * 2 * TILE) >> 4);
-        const uint32_t ts = tmem + 256 + 64 * b;
+        const uint64_t dk = dk0 + (uint64_t)((b * 2 * KT) >> 4);
+        const uint32_t ts = tmem + 256 + 64 * sb;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // K^'hi, then K^'lo into the same accumulator
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = h * TILE + (kk >> 2) * (NT * 128) + 32 * (kk & 3);
-            umma_ts(ts, tmem + TQ + 8 * kk, dk + (uint64_t)(off >> 4), ID_QK, (h > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t off = h * KT + (kk >> 2) * (NTL * 128) + 32 * (kk & 3);
+            umma2_ts(ts, tmem + TQ + 8 * kk, dk + (uint64_t)(off >> 4), ID_QK, (h > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit(&bars.sfull[b]);
-        umma_commit(&bars.kfree[b]);
+        umma2_commit_both(&bars.sfull[sb]);
+        umma2_commit_both(&bars.kfree[b]);
         if (j >= 1 && !pv(j - 1)) { ok = false; break; }
       }
       if (ok) ok = pv(n_st - 1);
@@ -329,15 +377,17 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
         *abort = 1;
         flag(p.status, QKV_DEV_TIMEOUT);
       }
-      // every MMA issued so far has completed once this commit lands
-      umma_commit(&bars.drain);
-      mbar_wait_bounded(&bars.drain, 0);
+      // every MMA issued so far has completed once this commit lands (both CTAs)
+      umma2_commit_both(&bars.drain);
     }
+    // both CTAs: the pair's MMAs, which write this CTA's tensor memory, are done
+    if (lane == 0) mbar_wait_bounded(&bars.drain, 0);
     __syncwarp();
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ softmax
     const int r = tid - 128;
-    const int hl = r / p.QB, qq = r - hl * p.QB;
+    const int R = ML * rank + r;  // row of the pair
+    const int hl = R / QB2, qq = R - hl * QB2;
     const int qi = q0 + qq;
     const bool valid = qi < p.n_q;
     const int qhead = kvh * p.G + hl;
@@ -387,19 +437,19 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars.qready);
+      arrive_rank0(&bars.qready);
     }
 
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_st; ++j) {
-      const int b = j & 1;
-      ok = wait_bar(&bars.sfull[b], (uint32_t)(j >> 1) & 1u, abort);
+      const int sb = j & 1;
+      ok = wait_bar(&bars.sfull[sb], (uint32_t)(j >> 1) & 1u, abort);
       if (!__all_sync(FULL_MASK, ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[2][32];
-      tmem_ld32(tmem + lane_base + 256 + 64 * b, sr[0]);
-      tmem_ld32(tmem + lane_base + 256 + 64 * b + 32, sr[1]);
+      tmem_ld32(tmem + lane_base + 256 + 64 * sb, sr[0]);
+      tmem_ld32(tmem + lane_base + 256 + 64 * sb + 32, sr[1]);
       tmem_wait_ld();
       float s[64];
 #pragma unroll
@@ -434,8 +484,8 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
         l += hf.x + hf.y;
         pw[i] = h2_as_u32(h);
       }
-      // P into the first 32 columns of S slot b (its S is in registers)
-      tmem_st32(tmem + lane_base + 256 + 64 * b, pw);
+      // P into the first 32 columns of S slot sb (its S is in registers)
+      tmem_st32(tmem + lane_base + 256 + 64 * sb, pw);
       if (any_need && j >= 1) {  // rescale O once P . V of the previous stage is done
         ok = wait_bar(&bars.odone, (uint32_t)(j - 1) & 1u, abort);
         if (!__all_sync(FULL_MASK, ok)) { ok = false; break; }
@@ -452,7 +502,7 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars.pready);
+      arrive_rank0(&bars.pready);
     }
 
     // epilogue: O / l, columns un-permuted, bf16 out
@@ -491,8 +541,18 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
     tc_fence_before();
   } else if (warp >= 8) {
     // ------------------------------------------------------------ dequantisation
-    const int d = tid - 256;
-    const int tk = d >> 2, c = d & 3;
+    const bool is_k = warp < 12;
+    const int d = is_k ? tid - 256 : tid - 384;  // 0..127
+    // K: token 32 rank + d / 4 of the stage, dims 64 (d % 4) .. + 63
+    // V: token d / 2 of the stage, dims 128 rank + 64 (d % 2) .. + 63
+    const int tk = is_k ? NTL * rank + (d >> 2) : (d >> 1);
+    const int trow = is_k ? (d >> 2) : (d >> 1);  // row in this CTA's tile
+    const int chunk = is_k ? (d & 3) : (d & 1);
+    const int byte_off = is_k ? 32 * chunk : 64 * rank + 32 * chunk;  // in the 128-byte packed row
+    const int cell = byte_off / 16;                                    // first 32-dim cell
+    const uint8_t* data = is_k ? p.k_data : p.v_data;
+    const uint16_t* scales = is_k ? p.k_scale : p.v_scale;
+    const bool per_tok = !is_k && p.v_tok;
     const size_t row_bytes = D / 2;
     // page id of this thread's token in stage j (-1 past the context)
     auto page_of = [&](int j) -> int32_t {
@@ -513,47 +573,46 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
         return;
       }
       const size_t row = ((size_t)page * p.kv_heads + kvh) * p.block + (t & (p.block - 1));
-      const uint4* kp = reinterpret_cast<const uint4*>(p.k_data + row * row_bytes + 32 * c);
-      const uint4* vp = reinterpret_cast<const uint4*>(p.v_data + row * row_bytes + 32 * c);
-      x.k0 = ldg_early16(kp);
-      x.k1 = ldg_early16(kp + 1);
-      x.v0 = ldg_early16(vp);
-      x.v1 = ldg_early16(vp + 1);
-      x.ks = ldg_early4(p.k_scale + row * 8 + 2 * c);
-      if (p.v_tok) {
-        const uint32_t h = ldg_early2(p.v_scale + row);
-        x.vs = h | (h << 16);
+      const uint4* src = reinterpret_cast<const uint4*>(data + row * row_bytes + byte_off);
+      x.a = ldg_early16(src);
+      x.b = ldg_early16(src + 1);
+      if (per_tok) {
+        const uint32_t h = ldg_early2(scales + row);
+        x.sc = h | (h << 16);
       } else {
-        x.vs = ldg_early4(p.v_scale + row * 8 + 2 * c);
+        x.sc = ldg_early4(scales + row * 8 + cell);
       }
       x.ok = 1;
     };
-    // one token's 64 dims of K (hi and lo tiles) or V into chunk c of a slot
-    auto put = [&](uint32_t chunk_base, const uint4& a, const uint4& bw, uint32_t sc, int okv, auto with_lo) {
+    // one token's 64 dims into chunk `chunk` of a tile slot (K: hi and lo tiles)
+    auto put = [&](uint32_t chunk_base, const Raw& x, auto with_lo) {
       constexpr bool LO = decltype(with_lo)::value;
-      // s' = scale * 2^-4 per cell (low half: cell 2c, high half: cell 2c + 1)
-      const __half2 s16 = __hmul2(u32_as_h2(sc), __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00)));
+      // s' = scale * 2^-4 per cell (low half: first cell, high half: second)
+      const __half2 s16 = __hmul2(u32_as_h2(x.sc), __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00)));
       const __half2 s_lo = __low2half2(s16), s_hi = __high2half2(s16);
-      const uint32_t wd[8] = {a.x, a.y, a.z, a.w, bw.x, bw.y, bw.z, bw.w};
+      const uint32_t wd[8] = {x.a.x, x.a.y, x.a.z, x.a.w, x.b.x, x.b.y, x.b.z, x.b.w};
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         uint32_t o[4] = {0u, 0u, 0u, 0u}, r[4] = {0u, 0u, 0u, 0u};
-        if (okv == 1) dequant_word<LO>(wd[u], u < 4 ? s_lo : s_hi, o, r);
-        sts128(chunk_base + swz(tk, u), o[0], o[1], o[2], o[3]);
-        if constexpr (LO) sts128(chunk_base + TILE + swz(tk, u), r[0], r[1], r[2], r[3]);
+        if (x.ok == 1) dequant_word<LO>(wd[u], u < 4 ? s_lo : s_hi, o, r);
+        sts128(chunk_base + swz(trow, u), o[0], o[1], o[2], o[3]);
+        if constexpr (LO) sts128(chunk_base + KT + swz(trow, u), r[0], r[1], r[2], r[3]);
       }
     };
     auto process = [&](int j, const Raw& x) -> bool {
-      const int b = j & 1;
-      if (x.ok == 2 && c == 0 && kvh == 0 && ((j * NT + tk) & (p.block - 1)) == 0) flag(p.status, QKV_DEV_BAD_PAGE);
-      if (j >= 2 && !wait_bar(&bars.kfree[b], (uint32_t)((j - 2) >> 1) & 1u, abort)) return false;
-      put(s_base + K_OFF + b * (2 * TILE) + c * (NT * 128), x.k0, x.k1, x.ks, x.ok, std::true_type{});
-      fence_async_smem();
-      mbar_arrive(&bars.kready[b]);
-      if (j >= 2 && !wait_bar(&bars.vfree[b], (uint32_t)((j - 2) >> 1) & 1u, abort)) return false;
-      put(s_base + V_OFF + b * TILE + c * (NT * 128), x.v0, x.v1, x.vs, x.ok, std::false_type{});
-      fence_async_smem();
-      mbar_arrive(&bars.vready[b]);
+      const int b = j % NS, u = j / NS;
+      if (x.ok == 2 && chunk == 0 && kvh == 0 && ((j * NT + tk) & (p.block - 1)) == 0) flag(p.status, QKV_DEV_BAD_PAGE);
+      if (is_k) {
+        if (u >= 1 && !wait_bar(&bars.kfree[b], (uint32_t)(u - 1) & 1u, abort)) return false;
+        put(s_base + K_OFF + b * (2 * KT) + chunk * (NTL * 128), x, std::true_type{});
+        fence_async_smem();
+        arrive_rank0(&bars.kready[b]);
+      } else {
+        if (u >= 1 && !wait_bar(&bars.vfree[b], (uint32_t)(u - 1) & 1u, abort)) return false;
+        put(s_base + V_OFF + b * VT + chunk * (NT * 128), x, std::false_type{});
+        fence_async_smem();
+        arrive_rank0(&bars.vready[b]);
+      }
       return true;
     };
     Raw ra, rb;
@@ -576,10 +635,11 @@ __global__ void __launch_bounds__(THREADS, 1) paged_prefill_kernel(const Params 
     }
   }
 
-  __syncthreads();
+  tc_fence_before();
+  cluster_sync();  // every role of both CTAs is done with tensor memory
   if (warp == 0) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
   }
 }
 
@@ -643,7 +703,8 @@ extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const u
     }
     attr_set[dev] = true;
   }
-  const dim3 grid((unsigned)((n_q + p.QB - 1) / p.QB), (unsigned)kv_heads);
+  // one CTA pair (a cluster of two, compiled in) per (256 / G queries, KV head)
+  const dim3 grid(2u * (unsigned)((n_q + p.QB - 1) / p.QB), (unsigned)kv_heads);
   void* args[] = {&p};
   if (launch_pdl((const void*)prefill::paged_prefill_kernel, grid, dim3(prefill::THREADS), prefill::SMEM_BYTES,
                  stream, args) != cudaSuccess) {
