@@ -329,11 +329,12 @@ QKV_API int qkv_gather_kv_f4(uint16_t* k_out, uint16_t* v_out, int64_t n_out, co
  *              exceed max_pages_per_seq * block_size (else QKV_EINVAL).
  *   cache, v_group, softmax_scale as in qkv_paged_decode_split_f4_v.
  * Compiled shapes: head_dim 256, q_heads / kv_heads in {1, 2, 4, 8}, a
- * power-of-two block_size (else QKV_EUNSUPPORTED). Runs on the tensor cores (tcgen05,
- * fp16 operands, fp32 accumulators in tensor memory): K and V are
- * dequantised to fp16 in shared memory, q scaled by a power of two per
- * row; outputs match exact attention within 2e-3. A page id outside the
- * pool reads as zero rows and sets QKV_DEV_BAD_PAGE. */
+ * power-of-two block_size (else QKV_EUNSUPPORTED). Runs on the tensor cores
+ * (tcgen05 on clusters of two CTAs, fp16 operands, fp32 accumulators in
+ * tensor memory): K (as exact hi + lo halves) and V are dequantised to fp16
+ * in shared memory, q scaled by a power of two per row; outputs match
+ * exact attention within 2e-3. A page id outside the pool reads as zero
+ * rows and sets QKV_DEV_BAD_PAGE. */
 QKV_API int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
                                       const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
                                       const int32_t* page_table, int32_t n_q, int32_t prefix_len,
