@@ -278,6 +278,35 @@ QKV_API int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint1
                              void* workspace, size_t workspace_bytes, int32_t* device_status,
                              qkv_stream_t stream);
 
+/* One decode step of a layer in two launches: a2 + a3 + a4 in the split
+ * pass, then a5. The split kernel rotates each sequence's q itself (NEOX on
+ * the first rot_dim dims, rounded to bf16 as qkv_rope_apply rounds), and the
+ * CTA whose split holds a sequence's last page first writes the step's new
+ * k (rotated) and v into the cache at slot_mapping[s] (F4, as
+ * qkv_kv_write_f4(_v)), so out, lse2_out and the cache bytes equal those of
+ * qkv_rope_kv_write_f4 followed by qkv_paged_decode_attn_f4(_v).
+ *   q            bf16 [n_seq][q_heads][head_dim], NOT rotated (read only).
+ *   k_new, v_new bf16 [n_seq][kv_heads][head_dim]: the step's new token, the
+ *                last of each sequence's seq_lens[s] tokens (16-byte aligned).
+ *   positions    int64 [n_seq]: rotary position of each step token.
+ *   slot_mapping int64 [n_seq]: cache slot of token seq_lens[s] - 1 (< 0:
+ *                not written).
+ *   cos_tab, sin_tab, table_pos_start, table_len, rot_dim: as in
+ *                qkv_rope_apply (a position outside the table leaves q and k
+ *                unrotated and sets QKV_DEV_BAD_POSITION).
+ *   the rest as in qkv_paged_decode_attn_f4_v (v_group 32 or head_dim).
+ * A slot past the pool sets QKV_DEV_BAD_SLOT and skips the write. */
+QKV_API int qkv_decode_step_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint16_t* k_new,
+                               const uint16_t* v_new, const int64_t* positions, const int64_t* slot_mapping,
+                               const float* cos_tab, const float* sin_tab, int64_t table_pos_start,
+                               int64_t table_len, int32_t rot_dim, uint8_t* k_data, uint16_t* k_scale,
+                               uint8_t* v_data, uint16_t* v_scale, const int32_t* page_table,
+                               const int32_t* seq_lens, int32_t n_seq, int32_t q_heads, int32_t kv_heads,
+                               int32_t head_dim, int32_t block_size, int32_t max_pages_per_seq,
+                               int64_t num_pages, float softmax_scale, int32_t num_splits, int32_t max_splits,
+                               int32_t v_group, void* workspace, size_t workspace_bytes, int32_t* device_status,
+                               qkv_stream_t stream);
+
 /* qkv_paged_decode_attn_f4 over a cache written with qkv_kv_write_f4_v
  * (v_group 32 or head_dim). */
 QKV_API int qkv_paged_decode_attn_f4_v(uint16_t* out, float* lse2_out, const uint16_t* q,

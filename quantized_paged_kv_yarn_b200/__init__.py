@@ -19,6 +19,7 @@ from ._abi import (  # noqa: F401
     DEV_TIMEOUT,
     exported_symbols,
     lib,
+    qkv_decode_step_f4,
     qkv_gather_kv_f4,
     qkv_kv_write_f4,
     qkv_lse_merge,

@@ -73,6 +73,9 @@ _SIGS = {
                                         _i32, _i64, _i32, _vp, _vp]),
     "qkv_paged_prefill_attn_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
                                                  _i32, _i32, _i32, _i64, _f32, _i32, _vp, _vp]),
+    "qkv_decode_step_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _vp, _vp,
+                                          _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _f32, _i32,
+                                          _i32, _i32, _vp, _sz, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -291,6 +294,29 @@ def qkv_paged_prefill_attn_f4(out, q, k_data, k_scale, v_data, v_scale, page_tab
         _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),
         _ptr(page_table, "page_table", (torch.int32,)), n_q, int(prefix_len), q_heads, kv_heads, head_dim,
         block_size, page_table.numel(), num_pages, float(softmax_scale), v_group_of(v_scale, head_dim),
+        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+
+
+def qkv_decode_step_f4(out, q, k_new, v_new, positions, slot_mapping, cos_tab, sin_tab, table_pos_start: int,
+                       rot_dim: int, k_data, k_scale, v_data, v_scale, page_table, seq_lens, kv_heads: int, workspace,
+                       max_splits: int, lse2_out=None, softmax_scale: float = 0.0, num_splits: int = 0,
+                       device_status=None, stream=None):
+    """One layer's decode step (rotary, F4 write of the new k/v, attention,
+    merge) in two launches; q unrotated. Shapes as in qkv_rope_kv_write_f4
+    and qkv_paged_decode_attn_f4."""
+    n_seq, q_heads, head_dim = q.shape
+    num_pages, _, block_size, _ = k_data.shape
+    half = rot_dim // 2
+    _check("qkv_decode_step_f4", lib.qkv_decode_step_f4(
+        _ptr(out, "out", _U16, n_seq * q_heads * head_dim), _ptr(lse2_out, "lse2_out", (torch.float32,)),
+        _ptr(q, "q", _U16), _ptr(k_new, "k_new", _U16, n_seq * kv_heads * head_dim),
+        _ptr(v_new, "v_new", _U16, n_seq * kv_heads * head_dim), _ptr(positions, "positions", (torch.int64,), n_seq),
+        _ptr(slot_mapping, "slot_mapping", (torch.int64,), n_seq), _ptr(cos_tab, "cos_tab", (torch.float32,)),
+        _ptr(sin_tab, "sin_tab", (torch.float32,)), int(table_pos_start), cos_tab.numel() // half, int(rot_dim),
+        *_cache_args(k_data, k_scale, v_data, v_scale), _ptr(page_table, "page_table", (torch.int32,)),
+        _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq), n_seq, q_heads, kv_heads, head_dim, block_size,
+        page_table.shape[1], num_pages, float(softmax_scale), int(num_splits), int(max_splits),
+        v_group_of(v_scale, head_dim), _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
 
 

@@ -71,6 +71,17 @@ class DecodeAttention:
         nbytes = _abi.qkv_paged_decode_workspace_bytes(n_seq, q_heads, head_dim, self.max_splits)
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
 
+    def step(self, out, q, k_new, v_new, positions, slot_mapping, cos_tab, sin_tab, table_pos_start: int,
+             rot_dim: int, cache: PagedF4Cache, page_table, seq_lens, lse2_out=None, softmax_scale=0.0,
+             num_splits=0, device_status=None, stream=None):
+        """The layer's whole decode step (rotary, F4 write of the new token,
+        attention, merge) in two launches; q unrotated."""
+        _abi.qkv_decode_step_f4(out, q, k_new, v_new, positions, slot_mapping, cos_tab, sin_tab, table_pos_start,
+                                rot_dim, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale, page_table,
+                                seq_lens, self.kv_heads, self.workspace, self.max_splits, lse2_out=lse2_out,
+                                softmax_scale=softmax_scale, num_splits=num_splits, device_status=device_status,
+                                stream=stream)
+
     def __call__(self, out, q, cache: PagedF4Cache, page_table, seq_lens, lse2_out=None, softmax_scale=0.0,
                  num_splits=0, device_status=None, stream=None):
         _abi.qkv_paged_decode_attn_f4(out, q, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale,

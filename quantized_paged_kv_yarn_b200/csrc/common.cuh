@@ -64,6 +64,79 @@ __device__ __forceinline__ float rot_second(float x0, float x1, float c, float s
   return __fmaf_rn(x1, c, __fmul_rn(x0, s));
 }
 
+// Row helpers for one K or V head row of a token spread over a warp: lane l
+// holds elements 8 l .. 8 l + 7 (lanes past head_dim / 8 hold zeros). All
+// 32 lanes must call them.
+
+// NEOX rotation of dims [0, rot) in place, rounded to bf16 as qkv_rope_apply
+// rounds its output; the partner of dim j < rot / 2 is j + rot / 2, which sits
+// rot / 16 lanes away (rot is a multiple of 16). cos_row / sin_row: the
+// position's table row.
+__device__ __forceinline__ void rope_row_bf16(float (&x)[8], int lane, int rot, const float* cos_row,
+                                              const float* sin_row) {
+  const int half = rot / 2, dl = half / 8;
+  float y[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float other = __shfl_sync(0xffffffffu, x[i], lane < dl ? lane + dl : lane - dl);
+    y[i] = x[i];
+    const int j = lane * 8 + i;
+    if (j < rot) {
+      const int jj = j < half ? j : j - half;
+      const float c = cos_row[jj], s = sin_row[jj];
+      y[i] = __bfloat162float(__float2bfloat16_rn(j < half ? rot_first(x[i], other, c, s)
+                                                           : rot_second(other, x[i], c, s)));
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = y[i];
+}
+
+// F4 quantise-write of the row (as qkv_kv_write_f4): scale = fp16(amax / 7)
+// per `group` values (32, or head_dim: one scale for the row), codes
+// rint(x / scale) clamped to [-8, 7] + 8, low nibble first. data_row: the
+// row's head_dim / 2 packed bytes; scale_row: its head_dim / group scales.
+// (Both divisions are IEEE; the results are exact, as argued in kv_write.cu.)
+__device__ __forceinline__ void f4_write_row(const float (&x)[8], int lane, int head_dim, int group,
+                                             uint8_t* data_row, __half* scale_row) {
+  const bool active = lane * 8 < head_dim;
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  // lanes per scale group: 4 for a 32-value cell; the whole warp for a group
+  // of head_dim values (lanes past head_dim / 8 hold amax 0)
+  const int gl = group == 32 ? 4 : 32;
+  for (int o = 1; o < gl; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (!active) return;
+  const __half sh = __float2half_rn(fminf(__fdiv_rn(amax, 7.0f), 65504.0f));
+  const float s = __half2float(sh);
+  uint32_t word = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int code = 8;
+    if (s != 0.f) code = (int)fminf(7.f, fmaxf(-8.f, rintf(__fdiv_rn(x[i], s)))) + 8;
+    word |= (uint32_t)code << (4 * i);
+  }
+  reinterpret_cast<uint32_t*>(data_row)[lane] = word;
+  if ((lane & (gl - 1)) == 0) scale_row[lane / gl] = sh;
+}
+
+// Row of 8 bf16 per lane as float (zeros past head_dim).
+__device__ __forceinline__ void load_row8(const uint16_t* row, int lane, int head_dim, float (&x)[8]) {
+  if (lane * 8 < head_dim) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(row + lane * 8);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = 0.f;
+  }
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -128,6 +128,30 @@ struct Params {
   int n_seq, q_heads, kv_heads, max_pages, max_splits, num_splits, target;
   float score_scale;  // softmax_scale * log2(e)
 };
+// The decode step's inputs (qkv_decode_step_f4): q is unrotated; the kernel
+// rotates it and writes the step's new K (rotated) and V into the cache
+// first. Only the fused instances take them: a larger parameter block made
+// ptxas compile the plain kernel's loop 1.2 us slower.
+struct StepFields {
+  int rot, v_group;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  const int64_t* positions;
+  const int64_t* slots;
+  const float* cos_tab;
+  const float* sin_tab;
+  int64_t tab_start, tab_len;
+  uint8_t* k_data_w;
+  uint8_t* v_data_w;
+  __half* k_scale_w;
+  __half* v_scale_w;
+};
+template <bool FUSE>
+struct KParams : Params {};
+template <>
+struct KParams<true> : Params {
+  StepFields st;
+};
 }  // namespace split
 
 using namespace split;
@@ -246,10 +270,10 @@ __device__ void plan(const Params& p, int seq, int split, int block, int& S, int
   pg1 = muldiv((uint32_t)split + 1, n, (uint32_t)S);
 }
 
-template <int BLOCK, int G, bool VTOK>
+template <int BLOCK, int G, bool VTOK, bool FUSE>
 __global__ void __launch_bounds__(THREADS, 1)
     paged_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                              const Params p) {
+                              const KParams<FUSE> p) {
   static_assert(STAGE_TOK % BLOCK == 0, "pages must tile a stage");
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "query heads per KV head");
   constexpr int HQ = Cfg<G>::HQ;
@@ -299,6 +323,53 @@ __global__ void __launch_bounds__(THREADS, 1)
   // probability rows of absent query heads (G < 8) are read as zeros
   for (int i = threadIdx.x % GTHREADS; i < (int)(sizeof(gs.prob) / 4); i += GTHREADS)
     reinterpret_cast<uint32_t*>(&gs.prob[0][0][0])[i] = 0u;
+  // Decode step: the CTA's query heads, rotated (bf16), in group 0's last V
+  // slot, which is first written by the copy of its local stage 2, issued in
+  // the main loop, after the q set-up has read them (8 KiB, 1024-aligned).
+  uint16_t(*qrot)[D] = reinterpret_cast<uint16_t(*)[D]>(&sm.grp[0].v[NSV - 1][0]);
+  static_assert(8 * D * 2 <= STAGE_TOK * ROW_BYTES, "qrot fits a V slot");
+  if constexpr (FUSE) {
+    // The decode step's rotary and F4 write inside this launch (as
+    // qkv_rope_kv_write_f4 computes them): warp h < G rotates query head h
+    // into shared memory; the CTA whose split holds the sequence's last
+    // page writes the new token's K (rotated, warp 8) and V (warp 9) into the
+    // cache before any of its copies starts.
+    const int half = p.st.rot / 2;
+    const int64_t ti = p.st.positions[seq] - p.st.tab_start;
+    const bool pos_ok = ti >= 0 && ti < p.st.tab_len;
+    const float* crow = p.st.cos_tab + (pos_ok ? ti : 0) * half;
+    const float* srow = p.st.sin_tab + (pos_ok ? ti : 0) * half;
+    if (!pos_ok && threadIdx.x == 0 && split == 0 && kvh == 0) flag(p.status, QKV_DEV_BAD_POSITION);
+    if (warp < G) {
+      float x[8];
+      load_row8(p.q + (size_t)(row0 + warp) * D, lane, D, x);
+      if (pos_ok) rope_row_bf16(x, lane, p.st.rot, crow, srow);
+      uint4 o;  // the rotated values are bf16-exact
+      o.x = (__float_as_uint(x[0]) >> 16) | (__float_as_uint(x[1]) & 0xffff0000u);
+      o.y = (__float_as_uint(x[2]) >> 16) | (__float_as_uint(x[3]) & 0xffff0000u);
+      o.z = (__float_as_uint(x[4]) >> 16) | (__float_as_uint(x[5]) & 0xffff0000u);
+      o.w = (__float_as_uint(x[6]) >> 16) | (__float_as_uint(x[7]) & 0xffff0000u);
+      *reinterpret_cast<uint4*>(&qrot[warp][8 * lane]) = o;
+    }
+    const int last_pg = (L - 1) / BLOCK;
+    if (L > 0 && last_pg >= pg0 && last_pg < pg1 && (warp == 8 || warp == 9)) {
+      const bool is_k = warp == 8;
+      const int64_t slot = p.st.slots[seq];
+      if (slot >= p.num_pages * BLOCK) {
+        if (lane == 0 && is_k) flag(p.status, QKV_DEV_BAD_SLOT);
+      } else if (slot >= 0) {
+        float x[8];
+        load_row8((is_k ? p.st.k_new : p.st.v_new) + ((size_t)seq * p.kv_heads + kvh) * D, lane, D, x);
+        if (is_k && pos_ok) rope_row_bf16(x, lane, p.st.rot, crow, srow);
+        const int group = is_k ? 32 : p.st.v_group;
+        const int64_t crw = ((slot / BLOCK) * p.kv_heads + kvh) * BLOCK + slot % BLOCK;
+        f4_write_row(x, lane, D, group, (is_k ? p.st.k_data_w : p.st.v_data_w) + crw * ROW_BYTES,
+                     (is_k ? p.st.k_scale_w : p.st.v_scale_w) + crw * (D / group));
+        // the copies of this CTA (async proxy) read these bytes after the barrier
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
+    }
+  }
   __syncthreads();
 
   // ------------------------------------------------------------ copy issue
@@ -416,8 +487,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int pp = 0; pp < PAIRS; ++pp) {
         if (col_ok) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(p.q + (size_t)(row0 + 4 * hq + hl) * D +
-                                                            32 * (2 * pp + par) + 8 * t);
+          uint4 raw;
+          if constexpr (FUSE)  // rotated in shared memory
+            raw = *reinterpret_cast<const uint4*>(&qrot[4 * hq + hl][32 * (2 * pp + par) + 8 * t]);
+          else
+            raw = *reinterpret_cast<const uint4*>(p.q + (size_t)(row0 + 4 * hq + hl) * D +
+                                                  32 * (2 * pp + par) + 8 * t);
           const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -938,20 +1013,23 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, int block) {
 }
 
 template <int BLOCK, int G>
-const void* kernel_ptr(bool vtok) {
-  return vtok ? reinterpret_cast<const void*>(&paged_decode_split_kernel<BLOCK, G, true>)
-              : reinterpret_cast<const void*>(&paged_decode_split_kernel<BLOCK, G, false>);
+const void* kernel_ptr(bool vtok, bool fuse) {
+  if (fuse)
+    return vtok ? reinterpret_cast<const void*>(&paged_decode_split_kernel<BLOCK, G, true, true>)
+                : reinterpret_cast<const void*>(&paged_decode_split_kernel<BLOCK, G, false, true>);
+  return vtok ? reinterpret_cast<const void*>(&paged_decode_split_kernel<BLOCK, G, true, false>)
+              : reinterpret_cast<const void*>(&paged_decode_split_kernel<BLOCK, G, false, false>);
 }
 
 size_t kernel_smem(int G) { return G > 4 ? smem_bytes<2>() : smem_bytes<1>(); }
 
-const void* pick_kernel(int block, int G, bool vtok = false) {
+const void* pick_kernel(int block, int G, bool vtok = false, bool fuse = false) {
 #define QKV_PICK(B)                         \
   if (block == B) {                         \
-    if (G == 1) return kernel_ptr<B, 1>(vtok);  \
-    if (G == 2) return kernel_ptr<B, 2>(vtok);  \
-    if (G == 4) return kernel_ptr<B, 4>(vtok);  \
-    if (G == 8) return kernel_ptr<B, 8>(vtok);  \
+    if (G == 1) return kernel_ptr<B, 1>(vtok, fuse);  \
+    if (G == 2) return kernel_ptr<B, 2>(vtok, fuse);  \
+    if (G == 4) return kernel_ptr<B, 4>(vtok, fuse);  \
+    if (G == 8) return kernel_ptr<B, 8>(vtok, fuse);  \
   }
   QKV_PICK(16)
   QKV_PICK(32)
@@ -964,24 +1042,25 @@ constexpr int MAX_DEVICES = 64;
 
 // Opt the kernel into its shared-memory size on the current device (once)
 // and return its resident CTAs per SM.
-int prepare(const void* fn, int block, int G, bool vtok = false) {
+int prepare(const void* fn, int block, int G, bool vtok = false, bool fuse = false) {
   static std::mutex mu;
-  static int occ[MAX_DEVICES][3][4][2];  // 0 = not prepared
+  static int occ[MAX_DEVICES][3][4][4];  // [vtok + 2 fuse]; 0 = not prepared
+  const int vi = (vtok ? 1 : 0) + (fuse ? 2 : 0);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return 0;
   const int bi = block == 16 ? 0 : block == 32 ? 1 : 2;
   const int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3;
   std::lock_guard<std::mutex> lock(mu);
-  if (occ[dev][bi][gi][vtok ? 1 : 0] == 0) {
+  if (occ[dev][bi][gi][vi] == 0) {
     const size_t smem = kernel_smem(G);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return 0;
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, THREADS, smem) != cudaSuccess || n < 1)
       return 0;
-    occ[dev][bi][gi][vtok ? 1 : 0] = n;
+    occ[dev][bi][gi][vi] = n;
   }
-  return occ[dev][bi][gi][vtok ? 1 : 0];
+  return occ[dev][bi][gi][vi];
 }
 
 int sm_count() {
@@ -1014,14 +1093,24 @@ extern "C" size_t qkv_paged_decode_workspace_bytes(int32_t n_seq, int32_t q_head
   return o + l;
 }
 
-extern "C" int qkv_paged_decode_split_f4_v(float* o_parts, float* lse2_parts, int32_t max_splits,
-                                           const uint16_t* q, const uint8_t* k_data, const uint16_t* k_scale,
-                                           const uint8_t* v_data, const uint16_t* v_scale,
-                                           const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
-                                           int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
-                                           int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
-                                           int32_t num_splits, int32_t v_group, int32_t* device_status,
-                                           qkv_stream_t stream) {
+// The decode step's inputs of the fused launch (qkv_decode_step_f4).
+struct StepArgs {
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  const int64_t* positions;
+  const int64_t* slots;
+  const float* cos_tab;
+  const float* sin_tab;
+  int64_t tab_start, tab_len;
+  int rot;
+};
+
+static int split_impl(float* o_parts, float* lse2_parts, int32_t max_splits, const uint16_t* q,
+                      const uint8_t* k_data, const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
+                      const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq, int32_t q_heads,
+                      int32_t kv_heads, int32_t head_dim, int32_t block_size, int32_t max_pages_per_seq,
+                      int64_t num_pages, float softmax_scale, int32_t num_splits, int32_t v_group,
+                      int32_t* device_status, qkv_stream_t stream, const StepArgs* step) {
   if (!o_parts || !lse2_parts || !q || !k_data || !k_scale || !v_data || !v_scale || !page_table || !seq_lens)
     return QKV_EINVAL;
   if (n_seq < 0 || q_heads < 1 || kv_heads < 1 || max_pages_per_seq < 1 || num_pages < 1 || max_splits < 1 ||
@@ -1035,7 +1124,7 @@ extern "C" int qkv_paged_decode_split_f4_v(float* o_parts, float* lse2_parts, in
   const int G = q_heads / kv_heads;
   if (head_dim != D) return QKV_EUNSUPPORTED;
   const bool vtok = v_group != 32;
-  const void* fn = pick_kernel(block_size, G, vtok);
+  const void* fn = pick_kernel(block_size, G, vtok, step != nullptr);
   if (!fn) return QKV_EUNSUPPORTED;
   const uint64_t cache_rows = (uint64_t)num_pages * kv_heads * block_size;
   if (cache_rows > 0x7fffffffull) return QKV_EUNSUPPORTED;  // TMA row coordinate is int32
@@ -1043,7 +1132,7 @@ extern "C" int qkv_paged_decode_split_f4_v(float* o_parts, float* lse2_parts, in
   if (max_splits > 65535 * 16 || n_seq > 65535 || kv_heads > 65535) return QKV_EUNSUPPORTED;
   if (n_seq == 0) return QKV_OK;
 
-  const int occ = prepare(fn, block_size, G, vtok);
+  const int occ = prepare(fn, block_size, G, vtok, step != nullptr);
   const int sms = sm_count();
   if (occ < 1 || sms < 1) return QKV_ECUDA;
 
@@ -1070,16 +1159,47 @@ extern "C" int qkv_paged_decode_split_f4_v(float* o_parts, float* lse2_parts, in
   p.target = std::max(1, occ * sms / kv_heads);
   const float sc = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
   p.score_scale = sc * 1.4426950408889634f;
+  KParams<true> pf;  // the fused instances' parameters: Params + the step's inputs
+  static_cast<Params&>(pf) = p;
+  if (step) {
+    pf.st.rot = step->rot;
+    pf.st.v_group = v_group;
+    pf.st.k_new = step->k_new;
+    pf.st.v_new = step->v_new;
+    pf.st.positions = step->positions;
+    pf.st.slots = step->slots;
+    pf.st.cos_tab = step->cos_tab;
+    pf.st.sin_tab = step->sin_tab;
+    pf.st.tab_start = step->tab_start;
+    pf.st.tab_len = step->tab_len;
+    pf.st.k_data_w = const_cast<uint8_t*>(k_data);
+    pf.st.v_data_w = const_cast<uint8_t*>(v_data);
+    pf.st.k_scale_w = reinterpret_cast<__half*>(const_cast<uint16_t*>(k_scale));
+    pf.st.v_scale_w = reinterpret_cast<__half*>(const_cast<uint16_t*>(v_scale));
+  }
 
   // Slots past the plan's split count still get lse2 = -inf: the grid
   // covers every slot the merge reads.
   dim3 grid((unsigned)max_splits, (unsigned)n_seq, (unsigned)kv_heads);
-  void* args[] = {(void*)&tm_k, (void*)&tm_v, (void*)&p};
+  void* args[] = {(void*)&tm_k, (void*)&tm_v, step ? (void*)&pf : (void*)&p};
   if (launch_pdl(fn, grid, dim3(THREADS), kernel_smem(G), stream, args) != cudaSuccess) {
     (void)cudaGetLastError();
     return QKV_ECUDA;
   }
   return QKV_OK;
+}
+
+extern "C" int qkv_paged_decode_split_f4_v(float* o_parts, float* lse2_parts, int32_t max_splits,
+                                           const uint16_t* q, const uint8_t* k_data, const uint16_t* k_scale,
+                                           const uint8_t* v_data, const uint16_t* v_scale,
+                                           const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
+                                           int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                           int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                                           int32_t num_splits, int32_t v_group, int32_t* device_status,
+                                           qkv_stream_t stream) {
+  return split_impl(o_parts, lse2_parts, max_splits, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, n_seq,
+                    q_heads, kv_heads, head_dim, block_size, max_pages_per_seq, num_pages, softmax_scale, num_splits,
+                    v_group, device_status, stream, nullptr);
 }
 
 extern "C" int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int32_t max_splits, const uint16_t* q,
@@ -1114,6 +1234,34 @@ extern "C" int qkv_paged_decode_attn_f4_v(uint16_t* out, float* lse2_out, const 
                                        page_table, seq_lens, n_seq, q_heads, kv_heads, head_dim, block_size,
                                        max_pages_per_seq, num_pages, softmax_scale, num_splits, v_group,
                                        device_status, stream);
+  if (rc != QKV_OK) return rc;
+  return qkv_lse_merge(o_parts, lse_parts, max_splits, (int32_t)rows, head_dim, out, lse2_out, stream);
+}
+
+extern "C" int qkv_decode_step_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint16_t* k_new,
+                                  const uint16_t* v_new, const int64_t* positions, const int64_t* slot_mapping,
+                                  const float* cos_tab, const float* sin_tab, int64_t table_pos_start,
+                                  int64_t table_len, int32_t rot_dim, uint8_t* k_data, uint16_t* k_scale,
+                                  uint8_t* v_data, uint16_t* v_scale, const int32_t* page_table,
+                                  const int32_t* seq_lens, int32_t n_seq, int32_t q_heads, int32_t kv_heads,
+                                  int32_t head_dim, int32_t block_size, int32_t max_pages_per_seq, int64_t num_pages,
+                                  float softmax_scale, int32_t num_splits, int32_t max_splits, int32_t v_group,
+                                  void* workspace, size_t workspace_bytes, int32_t* device_status,
+                                  qkv_stream_t stream) {
+  if (!out || !workspace || !k_new || !v_new || !positions || !slot_mapping || !cos_tab || !sin_tab) return QKV_EINVAL;
+  if (((uintptr_t)workspace & 255) || max_splits < 1 || n_seq < 0 || q_heads < 1) return QKV_EINVAL;
+  if (rot_dim < 16 || rot_dim % 16 || rot_dim > head_dim || table_len < 0) return QKV_EINVAL;
+  if (((uintptr_t)k_new | (uintptr_t)v_new) & 15) return QKV_EINVAL;
+  if (workspace_bytes < qkv_paged_decode_workspace_bytes(n_seq, q_heads, head_dim, max_splits)) return QKV_EINVAL;
+  if (n_seq == 0) return QKV_OK;
+  const size_t rows = (size_t)n_seq * q_heads;
+  float* o_parts = reinterpret_cast<float*>(workspace);
+  float* lse_parts =
+      reinterpret_cast<float*>((char*)workspace + ((rows * max_splits * head_dim * 4 + 255) & ~size_t(255)));
+  const StepArgs step = {k_new, v_new, positions, slot_mapping, cos_tab, sin_tab, table_pos_start, table_len, rot_dim};
+  int rc = split_impl(o_parts, lse_parts, max_splits, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens,
+                      n_seq, q_heads, kv_heads, head_dim, block_size, max_pages_per_seq, num_pages, softmax_scale,
+                      num_splits, v_group, device_status, stream, &step);
   if (rc != QKV_OK) return rc;
   return qkv_lse_merge(o_parts, lse_parts, max_splits, (int32_t)rows, head_dim, out, lse2_out, stream);
 }

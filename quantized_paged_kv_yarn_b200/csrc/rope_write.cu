@@ -59,41 +59,12 @@ __global__ void __launch_bounds__(256) rope_kv_write_kernel(
   // ---- one k or v head row: lane l holds elements 8l .. 8l+7
   const bool is_k = kind < q_heads + kv_heads;
   const int h = is_k ? kind - q_heads : kind - q_heads - kv_heads;
-  const bool active = lane * 8 < head_dim;
-  const uint16_t* src = (is_k ? k_in : v_in) + (tok * kv_heads + h) * head_dim;
   float x[8];
-  if (active) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(src + lane * 8);
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x[2 * i] = __uint_as_float(w[i] << 16);
-      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = 0.f;
-  }
+  load_row8((is_k ? k_in : v_in) + (tok * kv_heads + h) * head_dim, lane, head_dim, x);
   if (is_k) {
-    // Rotate dims [0, rot): the partner of dim j < half is j + half, which
-    // sits half / 8 lanes away (rot is a multiple of 16).
-    const int dl = half / 8;
-    float y[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float other = __shfl_sync(FULL_MASK, x[i], lane < dl ? lane + dl : lane - dl);
-      y[i] = x[i];
-      const int j = lane * 8 + i;
-      if (pos_ok && j < rot) {
-        const int jj = j < half ? j : j - half;
-        const float c = cos_tab[row * half + jj], s = sin_tab[row * half + jj];
-        y[i] = __bfloat162float(__float2bfloat16_rn(j < half ? rot_first(x[i], other, c, s) : rot_second(other, x[i], c, s)));
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = y[i];
+    if (pos_ok) rope_row_bf16(x, lane, rot, cos_tab + row * half, sin_tab + row * half);
     if (!pos_ok && lane == 0 && h == 0) flag(status, QKV_DEV_BAD_POSITION);
-    if (k_out && active) {
+    if (k_out && lane * 8 < head_dim) {
       uint4 o;
       uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
@@ -109,28 +80,11 @@ __global__ void __launch_bounds__(256) rope_kv_write_kernel(
     if (lane == 0 && is_k && h == 0) flag(status, QKV_DEV_BAD_SLOT);
     return;
   }
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
-  // Lanes per scale group: 4 for a 32-value cell; the whole warp for a V
-  // group of head_dim values (lanes past head_dim / 8 hold amax 0).
   const int group = is_k ? 32 : v_group;
-  const int gl = group == 32 ? 4 : 32;
-  for (int o = 1; o < gl; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL_MASK, amax, o));
-  if (!active) return;
-  const __half sh = __float2half_rn(fminf(__fdiv_rn(amax, 7.0f), 65504.0f));
-  const float s = __half2float(sh);
-  uint32_t word = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int code = 8;
-    if (s != 0.f) code = (int)fminf(7.f, fmaxf(-8.f, rintf(__fdiv_rn(x[i], s)))) + 8;
-    word |= (uint32_t)code << (4 * i);
-  }
   const int64_t page = slot / block, off = slot - page * block;
   const int64_t crow = (page * kv_heads + h) * block + off;
-  reinterpret_cast<uint32_t*>((is_k ? k_data : v_data) + crow * (head_dim / 2))[lane] = word;
-  if ((lane & (gl - 1)) == 0) (is_k ? k_scale : v_scale)[crow * (head_dim / group) + lane / gl] = sh;
+  f4_write_row(x, lane, head_dim, group, (is_k ? k_data : v_data) + crow * (head_dim / 2),
+               (is_k ? k_scale : v_scale) + crow * (head_dim / group));
 }
 
 }  // namespace qkv
