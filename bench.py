@@ -581,12 +581,15 @@ def run_op(args, rank, world, local_rank):
         q = workloads.chunk_queries_device(w, 0, n_q, dev)
         out = torch.empty_like(q)
         row = pt[0].contiguous()
+        # room for the automatic context split (up to 8 parts, folded by the merge)
+        ws = torch.empty(qkv.qkv_paged_prefill_workspace_bytes(n_q, w.q_heads, w.head_dim, 8), dtype=torch.uint8,
+                         device=dev)
         h_in, d_in = [q.cpu().pin_memory()], [q]
         h_out, d_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory()], [out]
 
         def call():
             qkv.qkv_paged_prefill_attn_f4(out, q, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale, row,
-                                          prefix, w.kv_heads, device_status=status)
+                                          prefix, w.kv_heads, workspace=ws, device_status=status)
         work = prefill_flops(prefix, n_q, w.q_heads, w.head_dim)
         metric, unit, scale = "paged F4 chunked-prefill attention TFLOP/s (causal)", "TFLOP/s", 1e12
         peak, peak_kind = tensor_peak()

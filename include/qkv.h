@@ -357,6 +357,15 @@ QKV_API int qkv_gather_kv_f4(uint16_t* k_out, uint16_t* v_out, int64_t n_out, co
  *              page page_table[t / block_size]. prefix_len + n_q must not
  *              exceed max_pages_per_seq * block_size (else QKV_EINVAL).
  *   cache, v_group, softmax_scale as in qkv_paged_decode_split_f4_v.
+ *   num_splits parts of each query block's context (each part's partials go
+ *              to the workspace and a log2-sum-exp merge folds them): 1 for
+ *              none (workspace may be NULL), 0 for automatic (the fewest
+ *              parts, up to 8, that fill the GPU's waves of CTA pairs, within
+ *              the workspace given; 1 without one). QKV_EINVAL when a part
+ *              would have no 64-token stage or the workspace is too small.
+ *   workspace  device buffer (256-byte aligned) of at least
+ *              qkv_paged_prefill_workspace_bytes(n_q, q_heads, head_dim,
+ *              num_splits) bytes, owned by the caller.
  * Compiled shapes: head_dim 256, q_heads / kv_heads in {1, 2, 4, 8}, a
  * power-of-two block_size (else QKV_EUNSUPPORTED). Runs on the tensor cores
  * (tcgen05 on clusters of two CTAs, fp16 operands, fp32 accumulators in
@@ -369,7 +378,14 @@ QKV_API int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const uint
                                       const int32_t* page_table, int32_t n_q, int32_t prefix_len,
                                       int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
                                       int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
-                                      int32_t v_group, int32_t* device_status, qkv_stream_t stream);
+                                      int32_t v_group, int32_t num_splits, void* workspace,
+                                      size_t workspace_bytes, int32_t* device_status, qkv_stream_t stream);
+
+/* Workspace bytes of qkv_paged_prefill_attn_f4 for num_splits parts (0 for
+ * one part; the automatic choice never needs more than 8 parts' worth).
+ * Host-only. */
+QKV_API size_t qkv_paged_prefill_workspace_bytes(int32_t n_q, int32_t q_heads, int32_t head_dim,
+                                                 int32_t num_splits);
 
 /* Size of the partials array compiled into the library for
  * qkv_paged_decode_attn_f4_static (16 MiB per GPU that loads the library). */

@@ -30,6 +30,7 @@ from ._abi import (  # noqa: F401
     qkv_paged_decode_split_f4,
     qkv_paged_decode_workspace_bytes,
     qkv_paged_prefill_attn_f4,
+    qkv_paged_prefill_workspace_bytes,
     qkv_rope_apply,
     qkv_rope_kv_write_f4,
     qkv_status_string,

@@ -72,7 +72,8 @@ _SIGS = {
     "qkv_gather_kv_f4": (ctypes.c_int, [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
                                         _i32, _i64, _i32, _vp, _vp]),
     "qkv_paged_prefill_attn_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
-                                                 _i32, _i32, _i32, _i64, _f32, _i32, _vp, _vp]),
+                                                 _i32, _i32, _i32, _i64, _f32, _i32, _i32, _vp, _sz, _vp, _vp]),
+    "qkv_paged_prefill_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "qkv_decode_step_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _vp, _vp,
                                           _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _f32, _i32,
                                           _i32, _i32, _vp, _sz, _vp, _vp]),
@@ -281,20 +282,27 @@ def qkv_gather_kv_f4(k_out, v_out, k_data, k_scale, v_data, v_scale, page_table,
         _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
 
 
+def qkv_paged_prefill_workspace_bytes(n_q: int, q_heads: int, head_dim: int, num_splits: int) -> int:
+    return lib.qkv_paged_prefill_workspace_bytes(int(n_q), int(q_heads), int(head_dim), int(num_splits))
+
+
 def qkv_paged_prefill_attn_f4(out, q, k_data, k_scale, v_data, v_scale, page_table, prefix_len: int,
-                              kv_heads: int, lse2_out=None, softmax_scale: float = 0.0, device_status=None,
-                              stream=None):
+                              kv_heads: int, lse2_out=None, softmax_scale: float = 0.0, num_splits: int = 0,
+                              workspace=None, device_status=None, stream=None):
     """out, q bf16 [n_q][q_heads][head_dim]; page_table int32 [max_pages] (one
-    sequence); the chunk's queries sit at cache tokens prefix_len .. prefix_len + n_q - 1."""
+    sequence); the chunk's queries sit at cache tokens prefix_len .. prefix_len + n_q - 1.
+    workspace: a uint8 CUDA tensor (qkv_paged_prefill_workspace_bytes) or None."""
     n_q, q_heads, head_dim = q.shape
     num_pages, _, block_size, _ = k_data.shape
     page_table = page_table.reshape(-1)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("qkv_paged_prefill_attn_f4", lib.qkv_paged_prefill_attn_f4(
         _ptr(out, "out", _U16, n_q * q_heads * head_dim), _ptr(lse2_out, "lse2_out", (torch.float32,), n_q * q_heads),
         _ptr(q, "q", _U16), *_cache_args(k_data, k_scale, v_data, v_scale),
         _ptr(page_table, "page_table", (torch.int32,)), n_q, int(prefix_len), q_heads, kv_heads, head_dim,
         block_size, page_table.numel(), num_pages, float(softmax_scale), v_group_of(v_scale, head_dim),
-        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+        int(num_splits), _ptr(workspace, "workspace"), ws_bytes, _ptr(device_status, "device_status", (torch.int32,)),
+        _stream(stream)))
 
 
 def qkv_decode_step_f4(out, q, k_new, v_new, positions, slot_mapping, cos_tab, sin_tab, table_pos_start: int,

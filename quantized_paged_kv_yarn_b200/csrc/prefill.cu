@@ -115,6 +115,12 @@ struct Params {
   int n_q, prefix_len, q_heads, kv_heads, G, QB, block, block_shift, v_tok;
   float score_scale;  // softmax_scale * log2(e)
   int32_t* status;
+  // Context split in n_splits parts (blockIdx.z): with n_splits > 1 each
+  // part writes its normalised partial output (fp32) and lse2 to o_part /
+  // lse_part [part][n_q * q_heads], which the log2-sum-exp merge folds.
+  int n_splits;
+  float* o_part;
+  float* lse_part;
 };
 
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
@@ -296,7 +302,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int q0 = (blockIdx.x >> 1) * QB2;
   const int q_last = min(p.n_q, q0 + QB2) - 1;
   const int kv_len = p.prefix_len + q_last + 1;
-  const int n_st = (kv_len + NT - 1) / NT;
+  // this part's stages st0 .. st0 + n_st - 1 of the pair's context (the
+  // host keeps n_splits <= the stage count, so every part has a stage)
+  const int n_all = (kv_len + NT - 1) / NT;
+  const int st0 = (int)((int64_t)blockIdx.z * n_all / p.n_splits);
+  const int n_st = (int)((int64_t)(blockIdx.z + 1) * n_all / p.n_splits) - st0;
 
   if (tid == 0) {
     for (int b = 0; b < NS; ++b) {
@@ -454,7 +464,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       float s[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(sr[i >> 5][i & 31]);
-      const int base = j * NT;
+      const int base = (st0 + j) * NT;
       if (base + NT - 1 > lim) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) s[i] = (base + i <= lim) ? s[i] : -INFINITY;
@@ -505,7 +515,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       arrive_rank0(&bars.pready);
     }
 
-    // epilogue: O / l, columns un-permuted, bf16 out
+    // epilogue: O / l, columns un-permuted; bf16 out, or this part's fp32 partial
     if (ok) {
       ok = wait_bar(&bars.odone, (uint32_t)(n_st - 1) & 1u, abort);
       ok = __all_sync(FULL_MASK, ok);
@@ -513,7 +523,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? 16.f / l : 0.f;
-      uint16_t* dst = p.out + ((size_t)qi * p.q_heads + qhead) * D;
+      const size_t row = (size_t)qi * p.q_heads + qhead;
+      const bool part = p.n_splits > 1;
+      uint16_t* dst = p.out + row * D;
+      float* pdst = part ? p.o_part + ((size_t)blockIdx.z * p.n_q * p.q_heads + row) * D : nullptr;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -528,12 +541,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               f[k] = __uint_as_float(o[8 * u + 2 * k]) * inv;
               f[k + 4] = __uint_as_float(o[8 * u + 2 * k + 1]) * inv;
             }
-            reinterpret_cast<uint4*>(dst)[4 * c + u] =
-                make_uint4(bf2_u32(f[0], f[1]), bf2_u32(f[2], f[3]), bf2_u32(f[4], f[5]), bf2_u32(f[6], f[7]));
+            if (part) {
+              reinterpret_cast<float4*>(pdst)[2 * (4 * c + u)] = make_float4(f[0], f[1], f[2], f[3]);
+              reinterpret_cast<float4*>(pdst)[2 * (4 * c + u) + 1] = make_float4(f[4], f[5], f[6], f[7]);
+            } else {
+              reinterpret_cast<uint4*>(dst)[4 * c + u] =
+                  make_uint4(bf2_u32(f[0], f[1]), bf2_u32(f[2], f[3]), bf2_u32(f[4], f[5]), bf2_u32(f[6], f[7]));
+            }
           }
         }
       }
-      if (valid && p.lse2) p.lse2[(size_t)qi * p.q_heads + qhead] = l > 0.f ? m_ref + log2f(l) : -INFINITY;
+      const float lse = l > 0.f ? m_ref + log2f(l) : -INFINITY;
+      if (valid && part) p.lse_part[(size_t)blockIdx.z * p.n_q * p.q_heads + row] = lse;
+      else if (valid && p.lse2) p.lse2[row] = lse;
     } else {
       *abort = 1;
       flag(p.status, QKV_DEV_TIMEOUT);
@@ -556,7 +576,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const size_t row_bytes = D / 2;
     // page id of this thread's token in stage j (-1 past the context)
     auto page_of = [&](int j) -> int32_t {
-      const int t = j * NT + tk;
+      const int t = (st0 + j) * NT + tk;
       return (j < n_st && t < kv_len) ? (int32_t)ldg_early4(p.page_table + (t >> p.block_shift)) : -1;
     };
     // The packed bytes of stage j into x, using the page id read by the
@@ -566,7 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const int32_t page = x.page;
       x.page = page_of(j + 2);
       x.ok = 0;
-      const int t = j * NT + tk;
+      const int t = (st0 + j) * NT + tk;
       if (j >= n_st || t >= kv_len) return;
       if (page < 0 || page >= p.num_pages) {
         x.ok = 2;
@@ -601,7 +621,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     };
     auto process = [&](int j, const Raw& x) -> bool {
       const int b = j % NS, u = j / NS;
-      if (x.ok == 2 && chunk == 0 && kvh == 0 && ((j * NT + tk) & (p.block - 1)) == 0) flag(p.status, QKV_DEV_BAD_PAGE);
+      if (x.ok == 2 && chunk == 0 && kvh == 0 && (((st0 + j) * NT + tk) & (p.block - 1)) == 0)
+        flag(p.status, QKV_DEV_BAD_PAGE);
       if (is_k) {
         if (u >= 1 && !wait_bar(&bars.kfree[b], (uint32_t)(u - 1) & 1u, abort)) return false;
         put(s_base + K_OFF + b * (2 * KT) + chunk * (NTL * 128), x, std::true_type{});
@@ -648,25 +669,68 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
 using namespace qkv;
 
+extern "C" size_t qkv_paged_prefill_workspace_bytes(int32_t n_q, int32_t q_heads, int32_t head_dim,
+                                                   int32_t num_splits) {
+  if (n_q < 0 || q_heads < 1 || head_dim < 1 || num_splits < 1) return 0;
+  if (num_splits == 1) return 0;
+  const size_t rows = (size_t)n_q * q_heads;
+  const size_t o = (rows * num_splits * head_dim * 4 + 255) & ~size_t(255);
+  const size_t l = (rows * num_splits * 4 + 255) & ~size_t(255);
+  return o + l;
+}
+
 extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
                                          const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
                                          const int32_t* page_table, int32_t n_q, int32_t prefix_len,
                                          int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
                                          int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
-                                         int32_t v_group, int32_t* device_status, qkv_stream_t stream) {
+                                         int32_t v_group, int32_t num_splits, void* workspace,
+                                         size_t workspace_bytes, int32_t* device_status, qkv_stream_t stream) {
   if (n_q == 0) return QKV_OK;
   if (!out || !q || !k_data || !k_scale || !v_data || !v_scale || !page_table) return QKV_EINVAL;
   if (n_q < 0 || prefix_len < 0 || q_heads < 1 || kv_heads < 1 || q_heads % kv_heads || block_size < 1 ||
       max_pages_per_seq < 1 || num_pages < 1 || !(softmax_scale >= 0.f) || !isfinite(softmax_scale) ||
-      (v_group != 32 && v_group != head_dim))
+      (v_group != 32 && v_group != head_dim) || num_splits < 0 || num_splits > 64)
     return QKV_EINVAL;
   if ((int64_t)prefix_len + n_q > (int64_t)max_pages_per_seq * block_size) return QKV_EINVAL;
   if (((uintptr_t)out | (uintptr_t)q | (uintptr_t)k_data | (uintptr_t)v_data) & 15) return QKV_EINVAL;
   if (((uintptr_t)k_scale | (uintptr_t)v_scale | (uintptr_t)lse2_out) & 3) return QKV_EINVAL;
+  if ((uintptr_t)workspace & 255) return QKV_EINVAL;
   const int G = q_heads / kv_heads;
   if (head_dim != prefill::D || (G != 1 && G != 2 && G != 4 && G != 8)) return QKV_EUNSUPPORTED;
   if (block_size & (block_size - 1)) return QKV_EUNSUPPORTED;  // pages of a power-of-two size
   if (kv_heads > 65535) return QKV_EUNSUPPORTED;
+
+  const int QB = prefill::M / G;
+  const int pairs_x = (n_q + QB - 1) / QB;
+  // the smallest context of a pair (the first query block) bounds the parts
+  const int min_stages = (prefix_len + (n_q < QB ? n_q : QB) + prefill::NT - 1) / prefill::NT;
+  int S = num_splits;
+  if (S == 0) {
+    // automatic: the fewest parts that fill the waves of CTA pairs (one CTA
+    // per SM) to 95 %, within the workspace given
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess)
+      return QKV_ECUDA;
+    const int slots = sms / 2 > 0 ? sms / 2 : 1;
+    const int pairs = pairs_x * kv_heads;
+    S = 1;
+    double best = 0.0;
+    for (int c = 1; c <= 8 && c <= min_stages; ++c) {
+      if (c > 1 && workspace_bytes < qkv_paged_prefill_workspace_bytes(n_q, q_heads, head_dim, c)) break;
+      const int units = pairs * c, waves = (units + slots - 1) / slots;
+      const double eff = (double)units / ((double)waves * slots);
+      if (eff > best + 1e-9) {
+        best = eff;
+        S = c;
+      }
+      if (eff >= 0.95) break;
+    }
+  }
+  if (S > min_stages) return QKV_EINVAL;  // a part without a stage
+  if (S > 1 && (!workspace || workspace_bytes < qkv_paged_prefill_workspace_bytes(n_q, q_heads, head_dim, S)))
+    return QKV_EINVAL;
 
   prefill::Params p;
   p.q = q;
@@ -683,7 +747,7 @@ extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const u
   p.q_heads = q_heads;
   p.kv_heads = kv_heads;
   p.G = G;
-  p.QB = prefill::M / G;
+  p.QB = QB;
   p.block = block_size;
   p.block_shift = 0;
   while ((1 << p.block_shift) < block_size) ++p.block_shift;
@@ -691,6 +755,12 @@ extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const u
   const float sc = softmax_scale > 0.f ? softmax_scale : 0.0625f;  // 1 / sqrt(256)
   p.score_scale = sc * 1.4426950408889634f;
   p.status = device_status;
+  const size_t rows = (size_t)n_q * q_heads;
+  p.n_splits = S;
+  p.o_part = S > 1 ? reinterpret_cast<float*>(workspace) : nullptr;
+  p.lse_part = S > 1 ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                                ((rows * S * head_dim * 4 + 255) & ~size_t(255)))
+                     : nullptr;
 
   static bool attr_set[64];
   int dev = 0;
@@ -703,13 +773,14 @@ extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const u
     }
     attr_set[dev] = true;
   }
-  // one CTA pair (a cluster of two, compiled in) per (256 / G queries, KV head)
-  const dim3 grid(2u * (unsigned)((n_q + p.QB - 1) / p.QB), (unsigned)kv_heads);
+  // one CTA pair (a cluster of two, compiled in) per (256 / G queries, KV head, part)
+  const dim3 grid(2u * (unsigned)pairs_x, (unsigned)kv_heads, (unsigned)S);
   void* args[] = {&p};
   if (launch_pdl((const void*)prefill::paged_prefill_kernel, grid, dim3(prefill::THREADS), prefill::SMEM_BYTES,
                  stream, args) != cudaSuccess) {
     (void)cudaGetLastError();
     return QKV_ECUDA;
   }
-  return QKV_OK;
+  if (S == 1) return QKV_OK;
+  return qkv_lse_merge(p.o_part, p.lse_part, S, (int32_t)rows, head_dim, out, lse2_out, stream);
 }

@@ -31,15 +31,18 @@ def _setup(qkv, L, n_q, block, hq, hkv, v_group=256, pages=None, seed=0, head_sc
     return w, x, ref, cache, q
 
 
-def _run(qkv, w, x, cache, q, prefix, page_table=None, softmax_scale=0.0):
+def _run(qkv, w, x, cache, q, prefix, page_table=None, softmax_scale=0.0, num_splits=1, ws_splits=0):
     n_q = q.shape[0]
     out = torch.full((n_q, w.q_heads, 256), 0x7FC1, dtype=torch.int16, device="cuda")
     lse = torch.empty((n_q, w.q_heads), dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     pt = x["page_table"][0] if page_table is None else page_table
+    nb = qkv.qkv_paged_prefill_workspace_bytes(n_q, w.q_heads, 256, ws_splits) if ws_splits > 1 else 0
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda") if nb else None
     qkv.qkv_paged_prefill_attn_f4(out, to_dev(q), cache.k_data, cache.k_scale, cache.v_data, cache.v_scale,
                                   to_dev(np.ascontiguousarray(pt)), prefix, w.kv_heads, lse2_out=lse,
-                                  softmax_scale=softmax_scale, device_status=st)
+                                  softmax_scale=softmax_scale, num_splits=num_splits, workspace=ws,
+                                  device_status=st)
     return to_host(out, np.uint16), to_host(lse), int(st.item())
 
 
@@ -70,6 +73,18 @@ def test_prefill_matches_oracle(qkv, case, v_group):
     out, lse, st = _run(qkv, w, x, cache, q, prefix)
     assert st == 0
     ro, rl = oracle.prefill_attention(q, ref, x["page_table"][0], np.arange(prefix, L), hq, hkv, 256, block)
+    _check(out, lse, ro, rl)
+
+
+@pytest.mark.parametrize("splits", [(2, 2), (3, 3), (0, 8)], ids=["S2", "S3", "auto"])
+def test_prefill_context_split(qkv, splits):
+    """Each query block's context in parts, partials folded by the merge."""
+    num_splits, ws_splits = splits
+    L, n_q = 1600, 257
+    w, x, ref, cache, q = _setup(qkv, L, n_q, 32, 16, 4, 32)
+    out, lse, st = _run(qkv, w, x, cache, q, L - n_q, num_splits=num_splits, ws_splits=ws_splits)
+    assert st == 0
+    ro, rl = oracle.prefill_attention(q, ref, x["page_table"][0], np.arange(L - n_q, L), 16, 4, 256, 32)
     _check(out, lse, ro, rl)
 
 
@@ -105,4 +120,10 @@ def test_prefill_argument_errors(qkv):
     w, x, ref, cache, q = _setup(qkv, 100, 10, 64, 16, 4)
     with pytest.raises(qkv.QkvError) as e:         # prefix + n_q past the page-table row
         _run(qkv, w, x, cache, q, 10 ** 6)
+    assert e.value.code == 1
+    with pytest.raises(qkv.QkvError) as e:         # 3 parts of a 2-stage context
+        _run(qkv, w, x, cache, q, 90, num_splits=3, ws_splits=3)
+    assert e.value.code == 1
+    with pytest.raises(qkv.QkvError) as e:         # 2 parts without a workspace
+        _run(qkv, w, x, cache, q, 90, num_splits=2)
     assert e.value.code == 1
