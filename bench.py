@@ -8,7 +8,7 @@ launch), the split-KV paged attention and the log2-sum-exp merge -- 1 + 3 x
 layers kernel launches, replayed from a CUDA graph.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-    python bench.py --op gather|prefill [--steps K] [--warmup W]
+    python bench.py --op gather|prefill|tier|tier_prefill [--steps K] [--warmup W]
 
 Prints one JSON line (rank 0). ``value`` is the whole-job rate of algorithmic
 K/V bytes (packed data + fp16 scales + page-table entries + q in + out) in
@@ -22,7 +22,13 @@ same workload's layer-0 cache: ``gather`` (the whole context dequantised
 into contiguous bf16 K/V rows; GB/s of algorithmic bytes) or ``prefill`` (a
 2048-query chunk at the end of the context, causal attention over the
 paged F4 cache on the tensor cores; TFLOP/s of the causal attention's
-multiply-adds x 2).
+multiply-adds x 2) or ``tier`` (decode attention with all but the last
+``--device-pages`` pages of the context in a pinned host pool, staged over
+the host link through a ``--window-pages`` device window; GB/s of host-tier
+bytes, against the link's pinned host-to-device copy rate measured in the
+same run) or ``tier_prefill`` (the prefill chunk with the same host tier:
+the host pages staged window by window, attended there, folded with the
+device part's causal pass; TFLOP/s as for ``prefill``).
 """
 from __future__ import annotations
 
@@ -58,9 +64,11 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="host-time budget of the CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
-    ap.add_argument("--op", choices=["decode", "gather", "prefill"], default="decode",
+    ap.add_argument("--op", choices=["decode", "gather", "prefill", "tier", "tier_prefill"], default="decode",
                     help="the decode step (default) or one widened row")
     ap.add_argument("--chunk", type=int, default=2048, help="prefill chunk size (queries)")
+    ap.add_argument("--window-pages", type=int, default=2048, help="host tier: device window (pages)")
+    ap.add_argument("--device-pages", type=int, default=64, help="host tier: newest pages kept on the device")
     ap.add_argument("--layers", type=int, default=0,
                     help="run fewer layers than the workload has (a smaller case for profiler captures)")
     return ap.parse_args()
@@ -493,6 +501,27 @@ def tensor_peak():
         return 1590.0, "fallback"
 
 
+def link_peak(nbytes: int, dev):
+    """Host-to-device rate of the link (GB/s): the copy engines moving a
+    pinned host buffer of nbytes into device memory, best of three, timed
+    with CUDA events in this run."""
+    import torch
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    d.copy_(h, non_blocking=True)
+    torch.cuda.synchronize()
+    best = 0.0
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        d.copy_(h, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        best = max(best, nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del h, d
+    return best, "measured in this run: pinned host-to-device copy (copy engines)"
+
+
 def prefill_flops(prefix: int, n_q: int, q_heads: int, head_dim: int) -> float:
     """2 x multiply-adds of causal attention of a chunk: query i attends
     prefix + i + 1 tokens, Q K^T and P V each head_dim per token and head."""
@@ -504,7 +533,8 @@ def oracle_op_sample(op: str, w, seconds: float):
     """The oracle on a bounded host sample of the row: returns (value, unit,
     cores, sample description)."""
     import oracle
-    ctx = 16384 if op == "prefill" else 65536
+    is_prefill = op in ("prefill", "tier_prefill")
+    ctx = 16384 if is_prefill else 65536
     s = workloads.Workload(name=w.name + "_sample", n_layers=1, seq_lens=(ctx,), num_pages=-(-ctx // w.block_size),
                            block_size=w.block_size, q_heads=w.q_heads, kv_heads=w.kv_heads, head_dim=w.head_dim,
                            head_scale=w.head_scale, k_outlier_frac=w.k_outlier_frac, seed=1)
@@ -518,19 +548,36 @@ def oracle_op_sample(op: str, w, seconds: float):
             oracle.gather_kv_f4(cache, pt, [n], [0], s.kv_heads, s.head_dim, s.block_size)
             return n * s.kv_heads * (2 * (s.head_dim // 2 + s.head_dim // 16) + 4 * s.head_dim) + 4 * (n // s.block_size)
         unit, what = "GB/s", "tokens gathered"
+    elif op == "tier":
+        page_bytes = s.kv_heads * s.block_size * 2 * (s.head_dim // 2 + s.head_dim // 16)
+        q = x["q"]
+
+        def run(n):
+            hp = max(1, n // s.block_size)        # host pages; the newest page stays on the device
+            dl = min(ctx, hp * s.block_size + s.block_size) - hp * s.block_size
+            oracle.tiered_attention(q, cache, pt[:, :hp], [hp * s.block_size], cache, pt[:, hp:], [dl],
+                                    s.q_heads, s.kv_heads, s.head_dim, s.block_size)
+            return hp * page_bytes
+        unit, what = "GB/s", "host-tier tokens attended"
     else:
         q = workloads.chunk_queries_host(s, 0, 64)
+        hp = ctx // s.block_size - 2           # tier_prefill: all but the last two pages on the host
 
         def run(n):
             pos = np.arange(ctx - n, ctx)
-            oracle.prefill_attention(q[:n], cache, pt[0], pos, s.q_heads, s.kv_heads, s.head_dim, s.block_size)
+            if op == "tier_prefill":
+                H = hp * s.block_size
+                oracle.tiered_prefill_attention(q[:n], cache, pt[0, :hp], H, cache, pt[0, hp:], pos - H, s.q_heads,
+                                                s.kv_heads, s.head_dim, s.block_size)
+            else:
+                oracle.prefill_attention(q[:n], cache, pt[0], pos, s.q_heads, s.kv_heads, s.head_dim, s.block_size)
             return prefill_flops(ctx - n, n, s.q_heads, s.head_dim)
         unit, what = "TFLOP/s", "chunk queries"
-    n = 1 if op == "prefill" else 1024
+    n = 1 if is_prefill else 1024
     t0 = time.perf_counter()
     run(n)
     dt = max(time.perf_counter() - t0, 1e-4)
-    cap = 64 if op == "prefill" else ctx
+    cap = 64 if is_prefill else (ctx - s.block_size if op == "tier" else ctx)
     n = max(1, min(cap, int(n * seconds / dt)))
     t0 = time.perf_counter()
     work = run(n)
@@ -555,6 +602,7 @@ def run_op(args, rank, world, local_rank):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     ctx = int(sum(w.seq_lens))
     pt = x["page_table"]
+    launches_per_call, kernel_override = 1, None
     if args.op == "gather":
         lens = x["seq_lens"]
         start = torch.from_numpy(np.concatenate([[0], np.cumsum(w.seq_lens)[:-1]]).astype(np.int64)).to(dev)
@@ -575,6 +623,91 @@ def run_op(args, rank, world, local_rank):
         cfg = {"workload": w.name, "context_tokens": ctx, "kv_heads": w.kv_heads, "head_dim": w.head_dim,
                "block_size": w.block_size, "out": "bf16 K and V rows, 1 GiB per 262,144 tokens",
                "l2": "inputs and outputs larger than L2"}
+    elif args.op == "tier":
+        if w.n_seq != 1:
+            raise SystemExit("--op tier measures a single-sequence workload")
+        B = w.block_size
+        n_host = -(-ctx // B) - args.device_pages
+        host = qkv.PagedF4Cache.allocate(w.num_pages, w.kv_heads, B, w.head_dim, pinned=True)
+        for a, b in zip((host.k_data, host.k_scale, host.v_data, host.v_scale),
+                        (cache.k_data, cache.k_scale, cache.v_data, cache.v_scale)):
+            a.copy_(b)
+        hpt, dpt = pt[:, :n_host].contiguous(), pt[:, n_host:].contiguous()
+        host_lens = np.array([n_host * B], np.int32)
+        dev_lens = torch.tensor([ctx - n_host * B], dtype=torch.int32, device=dev)
+        att = qkv.TieredDecodeAttention(w.q_heads, w.kv_heads, w.head_dim, B, n_host, args.window_pages,
+                                        device=dev)
+        q = x["q"]
+        out = torch.empty_like(q)
+        h_in, d_in = [q.cpu().pin_memory()], [q]
+        h_out, d_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory()], [out]
+
+        def call():
+            att(out, q, cache, dpt, dev_lens, host, hpt, host_lens, device_status=status)
+        page_bytes = w.kv_heads * B * 2 * (w.head_dim // 2 + w.head_dim // 32 * 2)
+        work = n_host * page_bytes
+        launches_per_call = 2 * -(-n_host // args.window_pages) + 2
+        metric, unit, scale = "host-tier decode: host-placed F4 K/V read over the host link, GB/s", "GB/s", 1e9
+        peak, peak_kind = link_peak(work, dev)
+        bound, kernel = "link", "stage_pages_f4_kernel"
+        cfg = {"workload": w.name + "_host_tier", "context_tokens": ctx, "host_tokens": n_host * B,
+               "device_tokens": ctx - n_host * B, "window_pages": args.window_pages, "q_heads": w.q_heads,
+               "kv_heads": w.kv_heads, "head_dim": w.head_dim, "block_size": B,
+               "host_pool": "pinned host memory read in place by the staging kernel",
+               "l2": "host-tier bytes cross the link once per step; the window (151 MB) exceeds L2"}
+        # the staging kernel alone: one full window of host pages
+        wn = min(args.window_pages, n_host)
+        win = qkv.PagedF4Cache.allocate(wn, w.kv_heads, B, w.head_dim, device=dev)
+        ids = hpt[0, :wn].contiguous()
+
+        def stage_only():
+            qkv.qkv_stage_pages_f4(win.k_data, win.k_scale, win.v_data, win.v_scale, host.k_data, host.k_scale,
+                                   host.v_data, host.v_scale, ids, device_status=status)
+        stage_only()
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(3):
+            stage_only()
+        s1.record()
+        torch.cuda.synchronize()
+        stage_ms = s0.elapsed_time(s1) / 3
+        kernel_override = (wn * page_bytes, stage_ms)
+    elif args.op == "tier_prefill":
+        B = w.block_size
+        n_host = -(-ctx // B) - args.device_pages
+        n_q = min(args.chunk, ctx - n_host * B)
+        prefix = ctx - n_host * B - n_q                 # device tokens before the chunk
+        host = qkv.PagedF4Cache.allocate(w.num_pages, w.kv_heads, B, w.head_dim, pinned=True)
+        for a, b in zip((host.k_data, host.k_scale, host.v_data, host.v_scale),
+                        (cache.k_data, cache.k_scale, cache.v_data, cache.v_scale)):
+            a.copy_(b)
+        hrow, drow = pt[0, :n_host].contiguous(), pt[0, n_host:].contiguous()
+        q = workloads.chunk_queries_device(w, 0, n_q, dev)
+        out = torch.empty_like(q)
+        ppl = 4
+        ws = torch.empty(qkv.qkv_paged_prefill_tiered_workspace_bytes(n_q, w.q_heads, w.kv_heads, w.head_dim, B, 32,
+                                                                      n_host, args.window_pages, ppl),
+                         dtype=torch.uint8, device=dev)
+        h_in, d_in = [q.cpu().pin_memory()], [q]
+        h_out, d_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory()], [out]
+
+        def call():
+            qkv.qkv_paged_prefill_attn_f4_tiered(out, q, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale,
+                                                 drow, prefix, host.k_data, host.k_scale, host.v_data,
+                                                 host.v_scale, hrow, n_host * B, w.kv_heads, args.window_pages,
+                                                 ppl, ws, device_status=status)
+        work = prefill_flops(n_host * B + prefix, n_q, w.q_heads, w.head_dim)
+        windows = -(-n_host // args.window_pages)
+        launches_per_call = 2 * windows + 1 + 1            # stage + prefill per window, the device pass, the merge
+        metric, unit, scale = "host-tier chunked prefill TFLOP/s (causal, host pages staged)", "TFLOP/s", 1e12
+        peak, peak_kind = tensor_peak()
+        bound, kernel = "tensor", "paged_prefill_kernel"
+        cfg = {"workload": w.name + "_host_tier", "context_tokens": ctx, "chunk": n_q, "host_tokens": n_host * B,
+               "device_tokens": ctx - n_host * B, "window_pages": args.window_pages, "parts_per_launch": ppl,
+               "q_heads": w.q_heads, "kv_heads": w.kv_heads, "head_dim": w.head_dim, "block_size": B,
+               "host_pool": "pinned host memory read in place by the staging kernel",
+               "l2": "the host tier and the window exceed L2"}
     else:
         n_q = min(args.chunk, ctx)
         prefix = ctx - n_q
@@ -591,6 +724,8 @@ def run_op(args, rank, world, local_rank):
             qkv.qkv_paged_prefill_attn_f4(out, q, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale, row,
                                           prefix, w.kv_heads, workspace=ws, device_status=status)
         work = prefill_flops(prefix, n_q, w.q_heads, w.head_dim)
+        parts = qkv.qkv_paged_prefill_auto_splits(n_q, prefix, w.q_heads, w.kv_heads, w.head_dim, ws.numel())
+        launches_per_call = 2 if parts > 1 else 1         # the kernel, and the merge of its parts
         metric, unit, scale = "paged F4 chunked-prefill attention TFLOP/s (causal)", "TFLOP/s", 1e12
         peak, peak_kind = tensor_peak()
         bound, kernel = "tensor", "paged_prefill_kernel"
@@ -636,21 +771,29 @@ def run_op(args, rank, world, local_rank):
     if rank != 0:
         return
     nb = lambda ts: sum(t.numel() * t.element_size() for t in ts)
-    profile_of = {"gather": ("gather_kv_f4", "gather.cu"), "prefill": ("paged_prefill", "prefill.cu")}
+    profile_of = {"gather": ("gather_kv_f4", "gather.cu"), "prefill": ("paged_prefill", "prefill.cu"),
+                  "tier": ("stage_pages_f4", "host_tier.cu"), "tier_prefill": ("paged_prefill", "prefill.cu")}
     value = world * work / (ms * 1e-3) / scale
     achieved = work / (ms * 1e-3) / scale
+    kernel_ms = ms
+    if kernel_override is not None:
+        achieved = kernel_override[0] / (kernel_override[1] * 1e-3) / scale
+        kernel_ms = kernel_override[1]
     result = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "u4 cache -> bf16" if args.op == "gather" else "f16 tcgen05, f32 accumulate",
+        "vs_baseline": None,
+        "dtype": {"gather": "u4 cache -> bf16", "prefill": "f16 tcgen05, f32 accumulate",
+                  "tier": "u4 cache bytes (staged), f16 mma, f32 accumulate",
+                  "tier_prefill": "f16 tcgen05, f32 accumulate"}[args.op],
         "data": "synthetic", "config": cfg, "device_status": int(status.item()),
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                      "traffic": profiled_traffic(w.name, *profile_of[args.op]), "kernel": kernel,
-                     "peak_kind": peak_kind, "kernel_ms": ms,
+                     "peak_kind": peak_kind, "kernel_ms": kernel_ms,
                      "timing": "CUDA events around back-to-back launches"},
         "e2e": {"value": world * work / (ms_e2e * 1e-3) / scale, "unit": unit, "h2d_bytes_per_step": nb(h_in),
                 "d2h_bytes_per_step": nb(h_out), "ms_per_step": ms_e2e},
-        "gpu_launches": args.steps, "clocks": clk.summary(),
+        "gpu_launches": args.steps * launches_per_call, "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
         v, u, cores, sample = oracle_op_sample(args.op, w, args.cpu_seconds)

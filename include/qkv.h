@@ -387,6 +387,13 @@ QKV_API int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const uint
 QKV_API size_t qkv_paged_prefill_workspace_bytes(int32_t n_q, int32_t q_heads, int32_t head_dim,
                                                  int32_t num_splits);
 
+/* The part count qkv_paged_prefill_attn_f4 chooses with num_splits 0 and a
+ * workspace of workspace_bytes (1: one launch, no merge; k > 1: k parts and
+ * the merge, two launches). 0 for shapes the prefill does not compile.
+ * Host-only; asks the current device for its SM count. */
+QKV_API int32_t qkv_paged_prefill_auto_splits(int32_t n_q, int32_t prefix_len, int32_t q_heads,
+                                              int32_t kv_heads, int32_t head_dim, size_t workspace_bytes);
+
 /* Size of the partials array compiled into the library for
  * qkv_paged_decode_attn_f4_static (16 MiB per GPU that loads the library). */
 #define QKV_STATIC_SCRATCH_BYTES (16u << 20)
@@ -419,6 +426,125 @@ QKV_API int qkv_paged_decode_attn_f4_static(uint16_t* out, float* lse2_out, cons
                                             int32_t max_pages_per_seq, int64_t num_pages,
                                             float softmax_scale, int32_t num_splits,
                                             int32_t* device_status, qkv_stream_t stream);
+
+/* [TIER] Copy pages of one F4 pool into consecutive pages of another: the
+ * host tier's pages into a device window. FreeToken issue #568, proposed
+ * solution item 2 (host-placed K/V: the K/V of a long context kept in host
+ * RAM and read over the host link; a prefill stages its pages into a device
+ * window).
+ *   dst_*       destination pool (layout as in qkv_kv_write_f4_v) of
+ *               dst_num_pages pages; pages dst_page0 .. dst_page0 + n_pages - 1
+ *               are overwritten. Device memory, 16-byte aligned.
+ *   src_*       source pool of src_num_pages pages with the same kv_heads,
+ *               block_size, head_dim and v_group: pinned host memory mapped
+ *               into the device's address space (cudaHostAlloc, or
+ *               cudaHostRegister with the mapped flag) or device memory,
+ *               16-byte aligned. The kernel reads it in place, each byte
+ *               once, with 16-byte loads.
+ *   src_pages   int32 [n_pages], device or mapped pinned host memory: the
+ *               source page of destination page dst_page0 + i.
+ * The bytes are copied unchanged. A source page id outside [0,
+ * src_num_pages) zero-fills its destination page and sets QKV_DEV_BAD_PAGE.
+ * EINVAL: a null or misaligned pointer; a source pointer that is pageable
+ * host memory (the call asks the driver what each pointer is); n_pages < 0;
+ * a destination range outside the pool; head_dim not a multiple of 32 up to
+ * 256; v_group not 32 or head_dim; a per-page scale slab that is not a
+ * multiple of 16 bytes (kv_heads * block_size * head_dim / v_group * 2). */
+QKV_API int qkv_stage_pages_f4(uint8_t* dst_k_data, uint16_t* dst_k_scale, uint8_t* dst_v_data,
+                               uint16_t* dst_v_scale, int64_t dst_num_pages, int64_t dst_page0,
+                               const uint8_t* src_k_data, const uint16_t* src_k_scale,
+                               const uint8_t* src_v_data, const uint16_t* src_v_scale,
+                               int64_t src_num_pages, const int32_t* src_pages, int32_t n_pages,
+                               int32_t kv_heads, int32_t head_dim, int32_t block_size, int32_t v_group,
+                               int32_t* device_status, qkv_stream_t stream);
+
+/* Workspace bytes of qkv_paged_decode_attn_f4_tiered: the window (window_pages
+ * pages of the F4 layout), its page table, and the partials of one sequence,
+ * (ceil(max_host_pages_per_seq / window_pages) + 1) * max_splits parts of
+ * q_heads * (head_dim + 1) floats; each region 256-byte aligned. 0 for
+ * invalid sizes. Host-only. */
+QKV_API size_t qkv_paged_decode_tiered_workspace_bytes(int32_t q_heads, int32_t kv_heads, int32_t head_dim,
+                                                       int32_t block_size, int32_t v_group,
+                                                       int32_t max_host_pages_per_seq, int32_t window_pages,
+                                                       int32_t max_splits);
+
+/* [TIER] + a4 + a5: decode attention of one layer whose context sits partly in
+ * a host-placed tier. FreeToken issue #568, proposed solution item 2: the
+ * host K/V read over the host link, the parts folded by log2-sum-exp.
+ * Context of sequence s, in order: host_lens[s] tokens in the host pool
+ * (token i in page host_page_table[s][i / block_size]), then seq_lens[s]
+ * tokens in the device pool (token i in page page_table[s][i / block_size]).
+ *   q, out, lse2_out, the device pool, page_table, seq_lens, softmax_scale,
+ *               v_group: as in qkv_paged_decode_attn_f4_v.
+ *   host_*      the host pool (host_num_pages pages, same shape), pinned and
+ *               mapped as for qkv_stage_pages_f4.
+ *   host_page_table  int32 [n_seq][max_host_pages_per_seq], device or
+ *               mapped pinned host memory.
+ *   host_lens   int32 [n_seq] in HOST memory, read by this call on the CPU to
+ *               plan the windows: multiples of block_size, at most
+ *               max_host_pages_per_seq * block_size (EINVAL otherwise).
+ *   window_pages  device pages per window; workspace as sized by
+ *               qkv_paged_decode_tiered_workspace_bytes, 256-byte aligned.
+ *   max_splits  split slots per window and for the device part
+ *               (qkv_paged_decode_auto_splits fills the device).
+ * Per sequence, per window of its host pages: qkv_stage_pages_f4 into the
+ * window, then the split pass over the window; then the split pass over the
+ * device pages and qkv_lse_merge of all the parts. Launch count per sequence:
+ * 2 * ceil(host pages / window_pages) + 2. The host tier's bytes cross the
+ * link once per call. Data-dependent errors as in the two kernels. */
+QKV_API int qkv_paged_decode_attn_f4_tiered(
+    uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data, const uint16_t* k_scale,
+    const uint8_t* v_data, const uint16_t* v_scale, const int32_t* page_table, const int32_t* seq_lens,
+    int32_t max_pages_per_seq, int64_t num_pages, const uint8_t* host_k_data, const uint16_t* host_k_scale,
+    const uint8_t* host_v_data, const uint16_t* host_v_scale, int64_t host_num_pages,
+    const int32_t* host_page_table, int32_t max_host_pages_per_seq, const int32_t* host_lens, int32_t n_seq,
+    int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size, int32_t v_group,
+    float softmax_scale, int32_t window_pages, int32_t max_splits, void* workspace, size_t workspace_bytes,
+    int32_t* device_status, qkv_stream_t stream);
+
+/* Workspace bytes of qkv_paged_prefill_attn_f4_tiered: the window and its
+ * page table, then fp32 partials for (ceil(max_host_pages / window_pages) +
+ * 1) * parts_per_launch parts of n_q * q_heads * (head_dim + 1) floats; each
+ * region 256-byte aligned. 0 for invalid sizes. Host-only. */
+QKV_API size_t qkv_paged_prefill_tiered_workspace_bytes(int32_t n_q, int32_t q_heads, int32_t kv_heads,
+                                                        int32_t head_dim, int32_t block_size, int32_t v_group,
+                                                        int32_t max_host_pages, int32_t window_pages,
+                                                        int32_t parts_per_launch);
+
+/* [TIER] + [CHUNK]: causal attention of a chunk of queries of one sequence
+ * whose oldest tokens sit in a host-placed tier. FreeToken issue #568,
+ * proposed solution item 2: a prefill stages the host pages into a device
+ * window, attends it there, and the parts are folded by log2-sum-exp.
+ * The sequence's context, in order: host_len tokens in the host pool (token
+ * i in page host_page_table[i / block_size]), then the device tokens of
+ * page_table (the row, as in qkv_paged_prefill_attn_f4). The chunk's queries
+ * sit at device tokens prefix_len .. prefix_len + n_q - 1 (already written):
+ * query i attends all host_len host tokens and device tokens 0 ..
+ * prefix_len + i.
+ *   out, lse2_out, q, the device pool, page_table, n_q, prefix_len,
+ *               softmax_scale, v_group: as in qkv_paged_prefill_attn_f4
+ *               (head_dim 256, power-of-two block_size).
+ *   host_*      the host pool (host_num_pages pages, same shape), pinned and
+ *               mapped as for qkv_stage_pages_f4; host_page_table int32
+ *               [host_len / block_size], device or mapped pinned memory.
+ *   host_len    whole pages (EINVAL otherwise).
+ *   window_pages  device pages per window.
+ *   parts_per_launch  upper bound of the context split of each prefill
+ *               launch (the automatic count fills the device's waves).
+ *   workspace   qkv_paged_prefill_tiered_workspace_bytes(n_q, ..., host_len
+ *               / block_size, window_pages, parts_per_launch) bytes or more,
+ *               256-byte aligned.
+ * Per window: qkv_stage_pages_f4 of its host pages, then the prefill kernel
+ * over the window with every query seeing every token; then the causal
+ * prefill over the device pages; qkv_lse_merge of all the fp32 parts. */
+QKV_API int qkv_paged_prefill_attn_f4_tiered(
+    uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data, const uint16_t* k_scale,
+    const uint8_t* v_data, const uint16_t* v_scale, const int32_t* page_table, int32_t n_q, int32_t prefix_len,
+    int32_t max_pages_per_seq, int64_t num_pages, const uint8_t* host_k_data, const uint16_t* host_k_scale,
+    const uint8_t* host_v_data, const uint16_t* host_v_scale, int64_t host_num_pages,
+    const int32_t* host_page_table, int32_t host_len, int32_t q_heads, int32_t kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t v_group, float softmax_scale, int32_t window_pages, int32_t parts_per_launch,
+    void* workspace, size_t workspace_bytes, int32_t* device_status, qkv_stream_t stream);
 
 /* Static text for a return code. */
 QKV_API const char* qkv_status_string(int status);

@@ -242,6 +242,68 @@ def prefill_attention(q, cache, page_table_row, positions, q_heads: int, kv_head
                            head_dim, block_size, softmax_scale, n_threads)
 
 
+def tiered_attention(q, host_cache, host_page_table, host_lens, dev_cache, dev_page_table, dev_lens,
+                     q_heads: int, kv_heads: int, head_dim: int, block_size: int,
+                     softmax_scale: Optional[float] = None, n_threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """Exact decode attention over a context held in two pools [TIER]
+    (FreeToken issue #568, proposed solution item 2: the K/V of a long
+    context kept in host RAM beside the device's pages). The context of
+    sequence s is host_lens[s] tokens walked through host_page_table[s] in
+    the host pool, then dev_lens[s] tokens walked through dev_page_table[s] in
+    the device pool. host_lens are whole pages. Written as paged_attention
+    over one pool holding both (device page ids shifted past the host pool's
+    pages) and one page-table row per sequence: host pages, then device pages.
+    Returns (out [n_seq][Hq][D], lse2 [n_seq][Hq])."""
+    hl = np.asarray(host_lens, np.int64); dl = np.asarray(dev_lens, np.int64)
+    hpt = np.asarray(host_page_table, np.int64); dpt = np.asarray(dev_page_table, np.int64)
+    if np.any(hl % block_size):
+        raise ValueError("host_lens must be whole pages")
+    n_host_pages = host_cache[0].shape[0]
+    pool = tuple(np.concatenate([np.ascontiguousarray(h), np.ascontiguousarray(d)]) for h, d in
+                 zip(host_cache, dev_cache))
+    n_seq = hl.size
+    width = hpt.shape[1] + dpt.shape[1]
+    pt = np.zeros((n_seq, width), np.int32)
+    for s in range(n_seq):
+        nh = int(hl[s]) // block_size
+        nd = -(-int(dl[s]) // block_size)
+        pt[s, :nh] = hpt[s, :nh]
+        pt[s, nh:nh + nd] = dpt[s, :nd] + n_host_pages
+    return paged_attention(q, pool, pt, np.zeros(n_seq, np.int32), (hl + dl).astype(np.int32), q_heads, kv_heads,
+                           head_dim, block_size, softmax_scale, n_threads)
+
+
+def _two_pool_row(host_cache, host_row, host_len: int, dev_cache, dev_row, dev_tokens: int, block_size: int):
+    """One pool holding both (device page ids shifted past the host pool's
+    pages) and the page-table row: host pages, then device pages."""
+    if host_len % block_size:
+        raise ValueError("host_len must be whole pages")
+    pool = tuple(np.concatenate([np.ascontiguousarray(h), np.ascontiguousarray(d)]) for h, d in
+                 zip(host_cache, dev_cache))
+    nh, nd = host_len // block_size, -(-dev_tokens // block_size)
+    row = np.zeros(max(1, nh + nd), np.int32)
+    row[:nh] = np.asarray(host_row, np.int64)[:nh]
+    row[nh:nh + nd] = np.asarray(dev_row, np.int64)[:nd] + host_cache[0].shape[0]
+    return pool, row
+
+
+def tiered_prefill_attention(q, host_cache, host_row, host_len: int, dev_cache, dev_row, positions, q_heads: int,
+                             kv_heads: int, head_dim: int, block_size: int, softmax_scale: Optional[float] = None,
+                             n_threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """Causal attention of a chunk of queries of one sequence whose first
+    host_len tokens (whole pages, row host_row) sit in the host pool [TIER]
+    (FreeToken issue #568, proposed solution item 2: a prefill over host-placed
+    K/V). Query i sits at device token positions[i] of dev_row and attends
+    all host tokens and device tokens 0 .. positions[i]: prefill_attention
+    over the sequence's whole context (host tokens first) at position
+    host_len + positions[i]. Returns (out [n][Hq][D], lse2 [n][Hq])."""
+    pos = np.asarray(positions, np.int64)
+    pool, row = _two_pool_row(host_cache, host_row, host_len, dev_cache, dev_row, int(pos.max(initial=-1)) + 1,
+                              block_size)
+    return prefill_attention(q, pool, row, host_len + pos, q_heads, kv_heads, head_dim, block_size, softmax_scale,
+                             n_threads)
+
+
 def lse_merge(o_parts, lse2_parts) -> Tuple[np.ndarray, np.ndarray]:
     """o_parts [n_parts][rows][D], lse2_parts [n_parts][rows] -> (out, lse2)."""
     o = _c(o_parts, np.float64); l = _c(lse2_parts, np.float64)

@@ -25,17 +25,23 @@ from ._abi import (  # noqa: F401
     qkv_lse_merge,
     qkv_paged_decode_attn_f4,
     qkv_paged_decode_attn_f4_static,
+    qkv_paged_decode_attn_f4_tiered,
+    qkv_paged_decode_tiered_workspace_bytes,
     STATIC_SCRATCH_BYTES,
     qkv_paged_decode_auto_splits,
     qkv_paged_decode_split_f4,
     qkv_paged_decode_workspace_bytes,
     qkv_paged_prefill_attn_f4,
+    qkv_paged_prefill_attn_f4_tiered,
+    qkv_paged_prefill_auto_splits,
+    qkv_paged_prefill_tiered_workspace_bytes,
     qkv_paged_prefill_workspace_bytes,
     qkv_rope_apply,
     qkv_rope_kv_write_f4,
+    qkv_stage_pages_f4,
     qkv_status_string,
     qkv_yarn_auto_factor,
     qkv_yarn_rope_table,
     v_group_of,
 )
-from .cache import DecodeAttention, PagedF4Cache  # noqa: F401
+from .cache import DecodeAttention, PagedF4Cache, TieredDecodeAttention  # noqa: F401

@@ -6,6 +6,7 @@ import math
 import os
 from typing import Optional
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -77,6 +78,17 @@ _SIGS = {
     "qkv_decode_step_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _vp, _vp,
                                           _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _f32, _i32,
                                           _i32, _i32, _vp, _sz, _vp, _vp]),
+    "qkv_stage_pages_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _i32, _i32,
+                                          _i32, _i32, _i32, _vp, _vp]),
+    "qkv_paged_decode_tiered_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32]),
+    "qkv_paged_decode_attn_f4_tiered": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _vp,
+                                                       _vp, _vp, _vp, _i64, _vp, _i32, _vp, _i32, _i32, _i32, _i32,
+                                                       _i32, _i32, _f32, _i32, _i32, _vp, _sz, _vp, _vp]),
+    "qkv_paged_prefill_auto_splits": (_i32, [_i32, _i32, _i32, _i32, _i32, _sz]),
+    "qkv_paged_prefill_tiered_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32]),
+    "qkv_paged_prefill_attn_f4_tiered": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                                                        _i64, _vp, _vp, _vp, _vp, _i64, _vp, _i32, _i32, _i32, _i32,
+                                                        _i32, _i32, _f32, _i32, _i32, _vp, _sz, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -348,3 +360,116 @@ def qkv_paged_decode_attn_f4_static(out, q, k_data, k_scale, v_data, v_scale, pa
         _ptr(page_table, "page_table", (torch.int32,)), _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq), n_seq,
         q_heads, kv_heads, head_dim, block_size, page_table.shape[1], num_pages, float(softmax_scale),
         int(num_splits), _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+
+
+def _hptr(t: torch.Tensor, name: str, dtypes=None, numel=None):
+    """A device tensor, or a pinned (page-locked) host tensor that kernels
+    read in place over the host link."""
+    if isinstance(t, torch.Tensor) and not t.is_cuda:
+        if not t.is_pinned():
+            raise ValueError(f"{name}: a host tensor must be pinned (page-locked)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous")
+        if dtypes is not None and t.dtype not in dtypes:
+            raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
+        if numel is not None and t.numel() < numel:
+            raise ValueError(f"{name}: has {t.numel()} elements, needs {numel}")
+        return t.data_ptr()
+    return _ptr(t, name, dtypes, numel)
+
+
+def _pool_args(k_data, k_scale, v_data, v_scale, host: bool):
+    f = _hptr if host else _ptr
+    return (f(k_data, "k_data", (torch.uint8,)), f(k_scale, "k_scale", _U16), f(v_data, "v_data", (torch.uint8,)),
+            f(v_scale, "v_scale", _U16))
+
+
+def qkv_stage_pages_f4(dst_k_data, dst_k_scale, dst_v_data, dst_v_scale, src_k_data, src_k_scale, src_v_data,
+                       src_v_scale, src_pages, dst_page0: int = 0, device_status=None, stream=None):
+    """Copy source pages src_pages[i] (int32, device or pinned host) into
+    destination pages dst_page0 + i. The source pool may be pinned host
+    memory (read over the host link) or device memory."""
+    num_pages, kv_heads, block_size, half = dst_k_data.shape
+    head_dim = 2 * half
+    if tuple(src_k_data.shape[1:]) != (kv_heads, block_size, half) or src_v_scale.shape[1:] != dst_v_scale.shape[1:]:
+        raise ValueError("source and destination pools must have the same page shape")
+    n = src_pages.numel()
+    _check("qkv_stage_pages_f4", lib.qkv_stage_pages_f4(
+        *_pool_args(dst_k_data, dst_k_scale, dst_v_data, dst_v_scale, False), num_pages, int(dst_page0),
+        *_pool_args(src_k_data, src_k_scale, src_v_data, src_v_scale, True), src_k_data.shape[0],
+        _hptr(src_pages, "src_pages", (torch.int32,)), n, kv_heads, head_dim, block_size,
+        v_group_of(dst_v_scale, head_dim), _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+
+
+def qkv_paged_decode_tiered_workspace_bytes(q_heads: int, kv_heads: int, head_dim: int, block_size: int,
+                                            v_group: int, max_host_pages_per_seq: int, window_pages: int,
+                                            max_splits: int) -> int:
+    return lib.qkv_paged_decode_tiered_workspace_bytes(int(q_heads), int(kv_heads), int(head_dim), int(block_size),
+                                                       int(v_group), int(max_host_pages_per_seq), int(window_pages),
+                                                       int(max_splits))
+
+
+def qkv_paged_decode_attn_f4_tiered(out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, host_k_data,
+                                    host_k_scale, host_v_data, host_v_scale, host_page_table, host_lens,
+                                    kv_heads: int, window_pages: int, max_splits: int, workspace, lse2_out=None,
+                                    softmax_scale: float = 0.0, device_status=None, stream=None):
+    """Decode attention over host_lens[s] tokens of the pinned host pool
+    (pages host_page_table[s]) followed by seq_lens[s] tokens of the device
+    pool (pages page_table[s]). host_lens: host integers (a list, numpy array
+    or CPU tensor), whole pages. workspace: a uint8 CUDA tensor of
+    qkv_paged_decode_tiered_workspace_bytes(...) bytes."""
+    n_seq, q_heads, head_dim = q.shape
+    num_pages, _, block_size, _ = k_data.shape
+    hl = np.ascontiguousarray(np.asarray(host_lens.cpu() if isinstance(host_lens, torch.Tensor) else host_lens,
+                                         dtype=np.int32))
+    if hl.size != n_seq:
+        raise ValueError(f"host_lens: {hl.size} entries for {n_seq} sequences")
+    _check("qkv_paged_decode_attn_f4_tiered", lib.qkv_paged_decode_attn_f4_tiered(
+        _ptr(out, "out", _U16, n_seq * q_heads * head_dim), _ptr(lse2_out, "lse2_out", (torch.float32,), n_seq * q_heads),
+        _ptr(q, "q", _U16), *_pool_args(k_data, k_scale, v_data, v_scale, False),
+        _ptr(page_table, "page_table", (torch.int32,)), _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq),
+        page_table.shape[1], num_pages, *_pool_args(host_k_data, host_k_scale, host_v_data, host_v_scale, True),
+        host_k_data.shape[0], _hptr(host_page_table, "host_page_table", (torch.int32,), n_seq),
+        host_page_table.shape[1], hl.ctypes.data, n_seq, q_heads, kv_heads, head_dim, block_size,
+        v_group_of(v_scale, head_dim), float(softmax_scale), int(window_pages), int(max_splits),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+
+
+def qkv_paged_prefill_auto_splits(n_q: int, prefix_len: int, q_heads: int, kv_heads: int, head_dim: int,
+                                  workspace_bytes: int) -> int:
+    return lib.qkv_paged_prefill_auto_splits(int(n_q), int(prefix_len), int(q_heads), int(kv_heads), int(head_dim),
+                                             int(workspace_bytes))
+
+
+def qkv_paged_prefill_tiered_workspace_bytes(n_q: int, q_heads: int, kv_heads: int, head_dim: int, block_size: int,
+                                             v_group: int, max_host_pages: int, window_pages: int,
+                                             parts_per_launch: int) -> int:
+    return lib.qkv_paged_prefill_tiered_workspace_bytes(int(n_q), int(q_heads), int(kv_heads), int(head_dim),
+                                                        int(block_size), int(v_group), int(max_host_pages),
+                                                        int(window_pages), int(parts_per_launch))
+
+
+def qkv_paged_prefill_attn_f4_tiered(out, q, k_data, k_scale, v_data, v_scale, page_table, prefix_len: int,
+                                     host_k_data, host_k_scale, host_v_data, host_v_scale, host_page_table,
+                                     host_len: int, kv_heads: int, window_pages: int, parts_per_launch: int,
+                                     workspace, lse2_out=None, softmax_scale: float = 0.0, device_status=None,
+                                     stream=None):
+    """Chunked causal prefill of one sequence whose first host_len tokens
+    (whole pages, pages host_page_table) sit in the pinned host pool; the rest
+    of its context, the chunk included, in the device pool (row page_table,
+    the chunk at device tokens prefix_len .. prefix_len + n_q - 1)."""
+    n_q, q_heads, head_dim = q.shape
+    num_pages, _, block_size, _ = k_data.shape
+    page_table = page_table.reshape(-1)
+    host_page_table = host_page_table.reshape(-1)
+    _check("qkv_paged_prefill_attn_f4_tiered", lib.qkv_paged_prefill_attn_f4_tiered(
+        _ptr(out, "out", _U16, n_q * q_heads * head_dim), _ptr(lse2_out, "lse2_out", (torch.float32,), n_q * q_heads),
+        _ptr(q, "q", _U16), *_pool_args(k_data, k_scale, v_data, v_scale, False),
+        _ptr(page_table, "page_table", (torch.int32,)), n_q, int(prefix_len), page_table.numel(), num_pages,
+        *_pool_args(host_k_data, host_k_scale, host_v_data, host_v_scale, True), host_k_data.shape[0],
+        _hptr(host_page_table, "host_page_table", (torch.int32,), int(host_len) // block_size), int(host_len),
+        q_heads, kv_heads, head_dim, block_size, v_group_of(v_scale, head_dim), float(softmax_scale),
+        int(window_pages), int(parts_per_launch), _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _ptr(device_status, "device_status", (torch.int32,)),
+        _stream(stream)))

@@ -25,12 +25,14 @@ class PagedF4Cache:
 
     @classmethod
     def allocate(cls, num_pages: int, kv_heads: int, block_size: int, head_dim: int, device="cuda",
-                 v_group: int = 32):
+                 v_group: int = 32, pinned: bool = False):
+        """pinned=True: a host-placed pool in page-locked host memory (device
+        "cpu"), which the tier's kernels read in place over the host link."""
         if v_group not in (32, head_dim):
             raise ValueError(f"v_group must be 32 or head_dim ({head_dim}), got {v_group}")
-        d = lambda: torch.zeros((num_pages, kv_heads, block_size, head_dim // 2), dtype=torch.uint8, device=device)
-        s = lambda g: torch.zeros((num_pages, kv_heads, block_size, head_dim // g), dtype=torch.float16,
-                                  device=device)
+        kw = dict(device="cpu", pin_memory=True) if pinned else dict(device=device)
+        d = lambda: torch.zeros((num_pages, kv_heads, block_size, head_dim // 2), dtype=torch.uint8, **kw)
+        s = lambda g: torch.zeros((num_pages, kv_heads, block_size, head_dim // g), dtype=torch.float16, **kw)
         return cls(d(), s(32), d(), s(v_group))
 
     @property
@@ -88,3 +90,29 @@ class DecodeAttention:
                                       page_table, seq_lens, self.kv_heads, self.workspace, self.max_splits,
                                       lse2_out=lse2_out, softmax_scale=softmax_scale, num_splits=num_splits,
                                       device_status=device_status, stream=stream)
+
+
+class TieredDecodeAttention:
+    """Decode attention over a context split between a pinned host pool (the
+    older tokens, whole pages) and the device pool, with the window and
+    partials workspace sized once."""
+
+    def __init__(self, q_heads: int, kv_heads: int, head_dim: int, block_size: int, max_host_pages_per_seq: int,
+                 window_pages: int, v_group: int = 32, max_splits: int = 0, device="cuda"):
+        self.kv_heads = kv_heads
+        self.window_pages = window_pages
+        self.max_splits = max_splits or max(1, _abi.qkv_paged_decode_auto_splits(kv_heads, block_size))
+        nbytes = _abi.qkv_paged_decode_tiered_workspace_bytes(q_heads, kv_heads, head_dim, block_size, v_group,
+                                                              max_host_pages_per_seq, window_pages, self.max_splits)
+        if nbytes == 0:
+            raise ValueError("invalid tiered-decode sizes")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+    def __call__(self, out, q, cache: PagedF4Cache, page_table, seq_lens, host: PagedF4Cache, host_page_table,
+                 host_lens, lse2_out=None, softmax_scale=0.0, device_status=None, stream=None):
+        _abi.qkv_paged_decode_attn_f4_tiered(out, q, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale,
+                                             page_table, seq_lens, host.k_data, host.k_scale, host.v_data,
+                                             host.v_scale, host_page_table, host_lens, self.kv_heads,
+                                             self.window_pages, self.max_splits, self.workspace, lse2_out=lse2_out,
+                                             softmax_scale=softmax_scale, device_status=device_status,
+                                             stream=stream)

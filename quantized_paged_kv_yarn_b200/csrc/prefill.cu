@@ -61,6 +61,7 @@
 // each 8-dim unit the dims are stored in the order 0,4,1,5,2,6,3,7 (the
 // order in which four nibble masks of a packed word yield them); Q' uses the
 // same order, and the output un-permutes O's columns.
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
@@ -113,6 +114,7 @@ struct Params {
   const int32_t* page_table;
   int64_t num_pages;
   int n_q, prefix_len, q_heads, kv_heads, G, QB, block, block_shift, v_tok;
+  int kv_limit;  // tokens past this one are not attended (a window pass: every query sees all of them)
   float score_scale;  // softmax_scale * log2(e)
   int32_t* status;
   // Context split in n_splits parts (blockIdx.z): with n_splits > 1 each
@@ -301,7 +303,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int QB2 = p.QB;  // queries per pair
   const int q0 = (blockIdx.x >> 1) * QB2;
   const int q_last = min(p.n_q, q0 + QB2) - 1;
-  const int kv_len = p.prefix_len + q_last + 1;
+  const int kv_len = min(p.prefix_len + q_last + 1, p.kv_limit);
   // this part's stages st0 .. st0 + n_st - 1 of the pair's context (the
   // host keeps n_splits <= the stage count, so every part has a stage)
   const int n_all = (kv_len + NT - 1) / NT;
@@ -401,7 +403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int qi = q0 + qq;
     const bool valid = qi < p.n_q;
     const int qhead = kvh * p.G + hl;
-    const int lim = p.prefix_len + qi;  // last token this row attends
+    const int lim = min(p.prefix_len + qi, p.kv_limit - 1);  // last token this row attends
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
     // Q' = fp16(q * 2^e) into tensor memory, dims permuted per 8-dim unit
@@ -524,7 +526,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const float inv = l > 0.f ? 16.f / l : 0.f;
       const size_t row = (size_t)qi * p.q_heads + qhead;
-      const bool part = p.n_splits > 1;
+      const bool part = p.o_part != nullptr;
       uint16_t* dst = p.out + row * D;
       float* pdst = part ? p.o_part + ((size_t)blockIdx.z * p.n_q * p.q_heads + row) * D : nullptr;
 #pragma unroll 1
@@ -679,58 +681,78 @@ extern "C" size_t qkv_paged_prefill_workspace_bytes(int32_t n_q, int32_t q_heads
   return o + l;
 }
 
-extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
-                                         const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
-                                         const int32_t* page_table, int32_t n_q, int32_t prefix_len,
-                                         int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
-                                         int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
-                                         int32_t v_group, int32_t num_splits, void* workspace,
-                                         size_t workspace_bytes, int32_t* device_status, qkv_stream_t stream) {
-  if (n_q == 0) return QKV_OK;
-  if (!out || !q || !k_data || !k_scale || !v_data || !v_scale || !page_table) return QKV_EINVAL;
-  if (n_q < 0 || prefix_len < 0 || q_heads < 1 || kv_heads < 1 || q_heads % kv_heads || block_size < 1 ||
-      max_pages_per_seq < 1 || num_pages < 1 || !(softmax_scale >= 0.f) || !isfinite(softmax_scale) ||
-      (v_group != 32 && v_group != head_dim) || num_splits < 0 || num_splits > 64)
+namespace qkv {
+
+// The automatic part count: the fewest parts (at most max_parts and the
+// stage count of the shortest pair) that fill the waves of CTA pairs (one
+// CTA per SM) to 95 %. -1 when the device cannot be queried.
+static int prefill_auto_parts(int pairs, int min_stages, int max_parts) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                 cudaSuccess) {
+    (void)cudaGetLastError();
+    return -1;
+  }
+  const int slots = sms / 2 > 0 ? sms / 2 : 1;
+  int S = 1;
+  double best = 0.0;
+  for (int c = 1; c <= max_parts && c <= min_stages; ++c) {
+    const int units = pairs * c, waves = (units + slots - 1) / slots;
+    const double eff = (double)units / ((double)waves * slots);
+    if (eff > best + 1e-9) {
+      best = eff;
+      S = c;
+    }
+    if (eff >= 0.95) break;
+  }
+  return S;
+}
+
+// Validation and launch of the prefill kernel. Query i of the chunk attends
+// tokens 0 .. min(prefix_len + i, kv_limit - 1) of the page-table row.
+// num_splits 0: automatic, at most max_parts parts. With o_part set, every
+// part writes its fp32 partial and lse2 to o_part / lse_part [part][n_q *
+// q_heads] (the caller merges); without, num_splits must come out 1 and the
+// kernel writes out and lse2 itself. *parts_used gets the part count.
+int prefill_run(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data, const uint16_t* k_scale,
+                const uint8_t* v_data, const uint16_t* v_scale, const int32_t* page_table, int32_t n_q,
+                int32_t prefix_len, int32_t kv_limit, int32_t q_heads, int32_t kv_heads, int32_t head_dim,
+                int32_t block_size, int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                int32_t v_group, int32_t num_splits, int32_t max_parts, float* o_part, float* lse_part,
+                int32_t* device_status, cudaStream_t stream, int* parts_used) {
+  if (!q || !k_data || !k_scale || !v_data || !v_scale || !page_table || (!o_part && !out)) return QKV_EINVAL;
+  if (n_q < 0 || prefix_len < 0 || kv_limit < 1 || q_heads < 1 || kv_heads < 1 || q_heads % kv_heads ||
+      block_size < 1 || max_pages_per_seq < 1 || num_pages < 1 || !(softmax_scale >= 0.f) ||
+      !isfinite(softmax_scale) || (v_group != 32 && v_group != head_dim) || num_splits < 0 || num_splits > 64 ||
+      max_parts < 1)
     return QKV_EINVAL;
-  if ((int64_t)prefix_len + n_q > (int64_t)max_pages_per_seq * block_size) return QKV_EINVAL;
-  if (((uintptr_t)out | (uintptr_t)q | (uintptr_t)k_data | (uintptr_t)v_data) & 15) return QKV_EINVAL;
-  if (((uintptr_t)k_scale | (uintptr_t)v_scale | (uintptr_t)lse2_out) & 3) return QKV_EINVAL;
-  if ((uintptr_t)workspace & 255) return QKV_EINVAL;
+  const int64_t span = std::min<int64_t>((int64_t)prefix_len + n_q, kv_limit);
+  if (span > (int64_t)max_pages_per_seq * block_size) return QKV_EINVAL;
+  if (((uintptr_t)out | (uintptr_t)q | (uintptr_t)k_data | (uintptr_t)v_data | (uintptr_t)o_part) & 15)
+    return QKV_EINVAL;
+  if (((uintptr_t)k_scale | (uintptr_t)v_scale | (uintptr_t)lse2_out | (uintptr_t)lse_part) & 3) return QKV_EINVAL;
+  if (o_part && !lse_part) return QKV_EINVAL;
   const int G = q_heads / kv_heads;
   if (head_dim != prefill::D || (G != 1 && G != 2 && G != 4 && G != 8)) return QKV_EUNSUPPORTED;
   if (block_size & (block_size - 1)) return QKV_EUNSUPPORTED;  // pages of a power-of-two size
   if (kv_heads > 65535) return QKV_EUNSUPPORTED;
+  if (n_q == 0) {
+    *parts_used = 0;
+    return QKV_OK;
+  }
 
   const int QB = prefill::M / G;
   const int pairs_x = (n_q + QB - 1) / QB;
   // the smallest context of a pair (the first query block) bounds the parts
-  const int min_stages = (prefix_len + (n_q < QB ? n_q : QB) + prefill::NT - 1) / prefill::NT;
+  const int64_t first_span = std::min<int64_t>((int64_t)prefix_len + (n_q < QB ? n_q : QB), kv_limit);
+  const int min_stages = (int)((first_span + prefill::NT - 1) / prefill::NT);
   int S = num_splits;
   if (S == 0) {
-    // automatic: the fewest parts that fill the waves of CTA pairs (one CTA
-    // per SM) to 95 %, within the workspace given
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
-                                                   cudaSuccess)
-      return QKV_ECUDA;
-    const int slots = sms / 2 > 0 ? sms / 2 : 1;
-    const int pairs = pairs_x * kv_heads;
-    S = 1;
-    double best = 0.0;
-    for (int c = 1; c <= 8 && c <= min_stages; ++c) {
-      if (c > 1 && workspace_bytes < qkv_paged_prefill_workspace_bytes(n_q, q_heads, head_dim, c)) break;
-      const int units = pairs * c, waves = (units + slots - 1) / slots;
-      const double eff = (double)units / ((double)waves * slots);
-      if (eff > best + 1e-9) {
-        best = eff;
-        S = c;
-      }
-      if (eff >= 0.95) break;
-    }
+    S = prefill_auto_parts(pairs_x * kv_heads, min_stages, max_parts);
+    if (S < 0) return QKV_ECUDA;
   }
-  if (S > min_stages) return QKV_EINVAL;  // a part without a stage
-  if (S > 1 && (!workspace || workspace_bytes < qkv_paged_prefill_workspace_bytes(n_q, q_heads, head_dim, S)))
-    return QKV_EINVAL;
+  if (S > min_stages || S > max_parts) return QKV_EINVAL;  // a part without a stage, or no room for it
+  if (!o_part && S != 1) return QKV_EINVAL;
 
   prefill::Params p;
   p.q = q;
@@ -744,6 +766,7 @@ extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const u
   p.num_pages = num_pages;
   p.n_q = n_q;
   p.prefix_len = prefix_len;
+  p.kv_limit = kv_limit;
   p.q_heads = q_heads;
   p.kv_heads = kv_heads;
   p.G = G;
@@ -755,12 +778,9 @@ extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const u
   const float sc = softmax_scale > 0.f ? softmax_scale : 0.0625f;  // 1 / sqrt(256)
   p.score_scale = sc * 1.4426950408889634f;
   p.status = device_status;
-  const size_t rows = (size_t)n_q * q_heads;
   p.n_splits = S;
-  p.o_part = S > 1 ? reinterpret_cast<float*>(workspace) : nullptr;
-  p.lse_part = S > 1 ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
-                                                ((rows * S * head_dim * 4 + 255) & ~size_t(255)))
-                     : nullptr;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
 
   static bool attr_set[64];
   int dev = 0;
@@ -781,6 +801,64 @@ extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const u
     (void)cudaGetLastError();
     return QKV_ECUDA;
   }
-  if (S == 1) return QKV_OK;
-  return qkv_lse_merge(p.o_part, p.lse_part, S, (int32_t)rows, head_dim, out, lse2_out, stream);
+  *parts_used = S;
+  return QKV_OK;
+}
+
+// Parts the one-call entry may use within workspace_bytes (at most 8).
+static int prefill_max_parts(int32_t n_q, int32_t q_heads, int32_t head_dim, size_t workspace_bytes) {
+  int c = 1;
+  while (c < 8 && workspace_bytes >= qkv_paged_prefill_workspace_bytes(n_q, q_heads, head_dim, c + 1)) ++c;
+  return c;
+}
+
+}  // namespace qkv
+
+extern "C" int32_t qkv_paged_prefill_auto_splits(int32_t n_q, int32_t prefix_len, int32_t q_heads,
+                                                 int32_t kv_heads, int32_t head_dim, size_t workspace_bytes) {
+  if (n_q < 1 || prefix_len < 0 || q_heads < 1 || kv_heads < 1 || q_heads % kv_heads || head_dim != prefill::D)
+    return 0;
+  const int G = q_heads / kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
+  const int QB = prefill::M / G;
+  const int min_stages = (prefix_len + (n_q < QB ? n_q : QB) + prefill::NT - 1) / prefill::NT;
+  const int S = prefill_auto_parts((n_q + QB - 1) / QB * kv_heads, min_stages,
+                                   prefill_max_parts(n_q, q_heads, head_dim, workspace_bytes));
+  return S < 0 ? 0 : S;
+}
+
+extern "C" int qkv_paged_prefill_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
+                                         const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
+                                         const int32_t* page_table, int32_t n_q, int32_t prefix_len,
+                                         int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                         int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                                         int32_t v_group, int32_t num_splits, void* workspace,
+                                         size_t workspace_bytes, int32_t* device_status, qkv_stream_t stream) {
+  if (n_q == 0) return QKV_OK;
+  if (!out) return QKV_EINVAL;
+  if ((uintptr_t)workspace & 255) return QKV_EINVAL;
+  if (n_q < 0 || q_heads < 1 || head_dim < 1) return QKV_EINVAL;
+  const int max_parts = prefill_max_parts(n_q, q_heads, head_dim, workspace ? workspace_bytes : 0);
+  if (num_splits > 1 && (!workspace || workspace_bytes < qkv_paged_prefill_workspace_bytes(n_q, q_heads, head_dim,
+                                                                                            num_splits)))
+    return QKV_EINVAL;
+  const int cap = num_splits > 0 ? num_splits : max_parts;
+  // run as one part unless the plan splits; a split run writes partials into the workspace
+  const size_t rows = (size_t)n_q * q_heads;
+  float* o_part = reinterpret_cast<float*>(workspace);
+  float* lse_part = workspace ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                                          ((rows * cap * head_dim * 4 + 255) & ~size_t(255)))
+                              : nullptr;
+  int S = num_splits;
+  if (S == 0) {
+    S = qkv_paged_prefill_auto_splits(n_q, prefix_len, q_heads, kv_heads, head_dim, workspace ? workspace_bytes : 0);
+    if (S < 1) S = 1;  // invalid shapes are reported by the run below
+  }
+  int used = 0;
+  const int rc = prefill_run(out, lse2_out, q, k_data, k_scale, v_data, v_scale, page_table, n_q, prefix_len,
+                             0x7fffffff, q_heads, kv_heads, head_dim, block_size, max_pages_per_seq, num_pages,
+                             softmax_scale, v_group, S, S > 1 ? cap : 1, S > 1 ? o_part : nullptr,
+                             S > 1 ? lse_part : nullptr, device_status, stream, &used);
+  if (rc || used <= 1) return rc;
+  return qkv_lse_merge(o_part, lse_part, used, (int32_t)rows, head_dim, out, lse2_out, stream);
 }

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 from conftest import ROOT, read_golden
@@ -102,3 +103,52 @@ def test_invalid_arguments_rejected_before_launch(qkv):
     need = qkv.qkv_paged_decode_workspace_bytes(1, 16, 256, 4)
     assert L.qkv_paged_decode_attn_f4(*wa(FAKE, need - 1)) == 1
     assert L.qkv_paged_decode_attn_f4(*wa(ctypes.c_void_p(4096 + 16), need)) == 1
+
+
+def test_tier_workspace_bytes(qkv):
+    """Window (four page arrays), page table, count, then (windows + 1) *
+    max_splits parts of q_heads * (head_dim + 1) floats, 256-byte aligned."""
+    a = lambda x: (x + 255) // 256 * 256
+    hq, hkv, d, blk, vg, max_host, win, ms = 16, 4, 256, 64, 32, 4096, 2048, 37
+    rows = hkv * blk
+    parts = (-(-max_host // win) + 1) * ms
+    want = (2 * a(win * rows * d // 2) + a(win * rows * d // 32 * 2) + a(win * rows * d // vg * 2) + a(win * 4) + 256
+            + a(parts * hq * d * 4) + a(parts * hq * 4))
+    assert qkv.qkv_paged_decode_tiered_workspace_bytes(hq, hkv, d, blk, vg, max_host, win, ms) == want
+    # per-token V scales shrink the V-scale window
+    assert (qkv.qkv_paged_decode_tiered_workspace_bytes(hq, hkv, d, blk, d, max_host, win, ms)
+            == want - a(win * rows * d // 32 * 2) + a(win * rows * 2))
+    assert qkv.qkv_paged_decode_tiered_workspace_bytes(hq, hkv, d, blk, 48, max_host, win, ms) == 0
+    assert qkv.qkv_paged_decode_tiered_workspace_bytes(hq, hkv, d, blk, vg, max_host, 0, ms) == 0
+
+
+def test_tier_invalid_arguments_rejected_before_launch(qkv):
+    L = qkv.lib
+    i64 = ctypes.c_int64
+    # staging: destination range past the pool, bad head_dim, pageable source
+    st = lambda n, page0, d=256, src=FAKE: (FAKE, FAKE, FAKE, FAKE, i64(8), i64(page0), src, FAKE, FAKE, FAKE, i64(8),
+                                            FAKE, n, 4, d, 64, 32, NUL, NUL)
+    assert L.qkv_stage_pages_f4(*st(4, 5)) == 1
+    assert L.qkv_stage_pages_f4(*st(4, -1)) == 1
+    assert L.qkv_stage_pages_f4(*st(4, 0, d=48)) == 1
+    assert L.qkv_stage_pages_f4(*st(0, 0)) == 0                         # nothing to do
+    pageable = np.zeros(1 << 16, np.uint8)
+    assert L.qkv_stage_pages_f4(*st(4, 0, src=ctypes.c_void_p(pageable.ctypes.data))) == 1
+    # tiered decode: host lengths not whole pages or past the table, workspace too small
+    need = qkv.qkv_paged_decode_tiered_workspace_bytes(16, 4, 256, 64, 32, 4, 2, 4)
+
+    def td(host_lens, ws_bytes, host=FAKE):
+        hl = np.asarray(host_lens, np.int32)
+        return (FAKE, NUL, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, i64(64), host, FAKE, FAKE, FAKE, i64(16),
+                FAKE, 4, ctypes.c_void_p(hl.ctypes.data), len(hl), 16, 4, 256, 64, 32, ctypes.c_float(0.0), 2, 4,
+                ctypes.c_void_p(1 << 20), ws_bytes, NUL, NUL), hl
+    a, keep = td([64], need)
+    assert L.qkv_paged_decode_attn_f4_tiered(*a) == 1              # FAKE host pool: not device-accessible
+    a, keep = td([40], need)                                        # not whole pages
+    assert L.qkv_paged_decode_attn_f4_tiered(*a) == 1
+    a, keep = td([5 * 64], need)                                    # past max_host_pages_per_seq
+    assert L.qkv_paged_decode_attn_f4_tiered(*a) == 1
+    a, keep = td([64], need - 1)                                    # workspace too small
+    assert L.qkv_paged_decode_attn_f4_tiered(*a) == 1
+    a, keep = td([64], need, host=ctypes.c_void_p(pageable.ctypes.data))   # pageable host pool
+    assert L.qkv_paged_decode_attn_f4_tiered(*a) == 1
