@@ -686,17 +686,13 @@ def run_op(args, rank, world, local_rank):
         q = workloads.chunk_queries_device(w, 0, n_q, dev)
         out = torch.empty_like(q)
         ppl = 4
-        ws = torch.empty(qkv.qkv_paged_prefill_tiered_workspace_bytes(n_q, w.q_heads, w.kv_heads, w.head_dim, B, 32,
-                                                                      n_host, args.window_pages, ppl),
-                         dtype=torch.uint8, device=dev)
+        att = qkv.TieredPrefillAttention(n_q, w.q_heads, w.kv_heads, w.head_dim, B, n_host, args.window_pages,
+                                         parts_per_launch=ppl, device=dev)
         h_in, d_in = [q.cpu().pin_memory()], [q]
         h_out, d_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory()], [out]
 
         def call():
-            qkv.qkv_paged_prefill_attn_f4_tiered(out, q, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale,
-                                                 drow, prefix, host.k_data, host.k_scale, host.v_data,
-                                                 host.v_scale, hrow, n_host * B, w.kv_heads, args.window_pages,
-                                                 ppl, ws, device_status=status)
+            att(out, q, cache, drow, prefix, host, hrow, n_host * B, device_status=status)
         work = prefill_flops(n_host * B + prefix, n_q, w.q_heads, w.head_dim)
         windows = -(-n_host // args.window_pages)
         launches_per_call = 2 * windows + 1 + 1            # stage + prefill per window, the device pass, the merge
@@ -707,6 +703,7 @@ def run_op(args, rank, world, local_rank):
                "device_tokens": ctx - n_host * B, "window_pages": args.window_pages, "parts_per_launch": ppl,
                "q_heads": w.q_heads, "kv_heads": w.kv_heads, "head_dim": w.head_dim, "block_size": B,
                "host_pool": "pinned host memory read in place by the staging kernel",
+               "staging": "in order with the attention on one stream",
                "l2": "the host tier and the window exceed L2"}
     else:
         n_q = min(args.chunk, ctx)

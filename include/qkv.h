@@ -536,7 +536,10 @@ QKV_API size_t qkv_paged_prefill_tiered_workspace_bytes(int32_t n_q, int32_t q_h
  *               256-byte aligned.
  * Per window: qkv_stage_pages_f4 of its host pages, then the prefill kernel
  * over the window with every query seeing every token; then the causal
- * prefill over the device pages; qkv_lse_merge of all the fp32 parts. */
+ * prefill over the device pages; qkv_lse_merge of all the fp32 parts. The
+ * staging of a window and the attention run one after the other on
+ * `stream` (the staging is bound by the host link, the attention by the
+ * tensor cores; they are not overlapped). */
 QKV_API int qkv_paged_prefill_attn_f4_tiered(
     uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data, const uint16_t* k_scale,
     const uint8_t* v_data, const uint16_t* v_scale, const int32_t* page_table, int32_t n_q, int32_t prefix_len,

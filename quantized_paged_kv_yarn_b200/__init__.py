@@ -44,4 +44,4 @@ from ._abi import (  # noqa: F401
     qkv_yarn_rope_table,
     v_group_of,
 )
-from .cache import DecodeAttention, PagedF4Cache, TieredDecodeAttention  # noqa: F401
+from .cache import DecodeAttention, PagedF4Cache, TieredDecodeAttention, TieredPrefillAttention  # noqa: F401

@@ -116,3 +116,28 @@ class TieredDecodeAttention:
                                              self.window_pages, self.max_splits, self.workspace, lse2_out=lse2_out,
                                              softmax_scale=softmax_scale, device_status=device_status,
                                              stream=stream)
+
+
+class TieredPrefillAttention:
+    """Chunked prefill of one sequence whose oldest pages sit in a pinned host
+    pool, with the window and partials workspace sized once."""
+
+    def __init__(self, n_q: int, q_heads: int, kv_heads: int, head_dim: int, block_size: int, max_host_pages: int,
+                 window_pages: int, v_group: int = 32, parts_per_launch: int = 4, device="cuda"):
+        self.kv_heads = kv_heads
+        self.window_pages = window_pages
+        self.parts_per_launch = parts_per_launch
+        nbytes = _abi.qkv_paged_prefill_tiered_workspace_bytes(n_q, q_heads, kv_heads, head_dim, block_size, v_group,
+                                                               max_host_pages, window_pages, parts_per_launch)
+        if nbytes == 0:
+            raise ValueError("invalid tiered-prefill sizes")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+    def __call__(self, out, q, cache: PagedF4Cache, page_table, prefix_len: int, host: PagedF4Cache,
+                 host_page_table, host_len: int, lse2_out=None, softmax_scale=0.0, device_status=None, stream=None):
+        _abi.qkv_paged_prefill_attn_f4_tiered(out, q, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale,
+                                              page_table, prefix_len, host.k_data, host.k_scale, host.v_data,
+                                              host.v_scale, host_page_table, host_len, self.kv_heads,
+                                              self.window_pages, self.parts_per_launch, self.workspace,
+                                              lse2_out=lse2_out, softmax_scale=softmax_scale,
+                                              device_status=device_status, stream=stream)

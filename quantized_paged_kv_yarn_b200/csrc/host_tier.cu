@@ -39,42 +39,53 @@ struct StageParams {
 constexpr int STAGE_THREADS = 256;
 constexpr int STAGE_UNROLL = 4;  // loads in flight per thread before its stores
 
-// One CTA per destination page: the source page id is read once, then each
-// array's slab is copied with STAGE_UNROLL independent 16-byte loads per
-// thread ahead of the stores (the link's latency is microseconds; the bytes
-// in flight across the grid keep it busy).
+// A persistent grid of one CTA per SM at most (256 threads, no shared
+// memory). Each CTA walks destination pages i = blockIdx.x, + gridDim.x, ...:
+// the source page id is read once, then each array's slab is copied with
+// STAGE_UNROLL independent 16-byte loads per thread ahead of the stores (the
+// link's latency is microseconds; a few MB in flight across the grid keep it
+// busy).
+//
+// Unlike the other kernels it does not let its successor start early: the
+// attention kernels that follow it would otherwise sit on the same SMs while
+// its loads of host memory are outstanding. (With a prefill kernel running
+// beside a live staging grid -- staging on a second stream -- a bounded wait
+// of the prefill ran out once in three chunk-layers at full size; the
+// library therefore never overlaps the two.)
 __global__ void __launch_bounds__(STAGE_THREADS) stage_pages_f4_kernel(const StageParams p) {
   pdl_wait();
-  pdl_release();
-  const int i = blockIdx.x;
-  if (p.tab_out && i == 0) {
-    for (int j = threadIdx.x; j < p.n_pages; j += STAGE_THREADS) p.tab_out[j] = j;
-    if (threadIdx.x == 0) *p.len_out = p.len_value;
+  if (blockIdx.x == 0) {
+    if (p.tab_out)
+      for (int j = threadIdx.x; j < p.n_pages; j += STAGE_THREADS) p.tab_out[j] = j;
+    if (p.len_out && threadIdx.x == 0) *p.len_out = p.len_value;
   }
-  const int32_t page = p.src_pages[i];
-  const bool bad = page < 0 || page >= p.src_num_pages;
-  if (bad && threadIdx.x == 0) flag(p.status, QKV_DEV_BAD_PAGE);
 #pragma unroll 1
-  for (int a = 0; a < 4; ++a) {
-    const int64_t n = p.slab[a];
-    uint4* d = p.dst[a] + (p.dst_page0 + i) * n;
-    if (bad) {
-      for (int64_t u = threadIdx.x; u < n; u += STAGE_THREADS) d[u] = make_uint4(0, 0, 0, 0);
-      continue;
-    }
-    const uint4* s = p.src[a] + (int64_t)page * n;
+  for (int i = blockIdx.x; i < p.n_pages; i += gridDim.x) {
+    const int32_t page = p.src_pages[i];
+    const bool bad = page < 0 || page >= p.src_num_pages;
+    if (bad && threadIdx.x == 0) flag(p.status, QKV_DEV_BAD_PAGE);
 #pragma unroll 1
-    for (int64_t u0 = threadIdx.x; u0 < n; u0 += STAGE_THREADS * STAGE_UNROLL) {
-      uint4 v[STAGE_UNROLL];
-#pragma unroll
-      for (int k = 0; k < STAGE_UNROLL; ++k) {
-        const int64_t u = u0 + (int64_t)k * STAGE_THREADS;
-        if (u < n) v[k] = s[u];
+    for (int a = 0; a < 4; ++a) {
+      const int64_t n = p.slab[a];
+      uint4* d = p.dst[a] + (p.dst_page0 + i) * n;
+      if (bad) {
+        for (int64_t u = threadIdx.x; u < n; u += STAGE_THREADS) d[u] = make_uint4(0, 0, 0, 0);
+        continue;
       }
+      const uint4* s = p.src[a] + (int64_t)page * n;
+#pragma unroll 1
+      for (int64_t u0 = threadIdx.x; u0 < n; u0 += STAGE_THREADS * STAGE_UNROLL) {
+        uint4 v[STAGE_UNROLL];
 #pragma unroll
-      for (int k = 0; k < STAGE_UNROLL; ++k) {
-        const int64_t u = u0 + (int64_t)k * STAGE_THREADS;
-        if (u < n) d[u] = v[k];
+        for (int k = 0; k < STAGE_UNROLL; ++k) {
+          const int64_t u = u0 + (int64_t)k * STAGE_THREADS;
+          if (u < n) v[k] = s[u];
+        }
+#pragma unroll
+        for (int k = 0; k < STAGE_UNROLL; ++k) {
+          const int64_t u = u0 + (int64_t)k * STAGE_THREADS;
+          if (u < n) d[u] = v[k];
+        }
       }
     }
   }
@@ -138,9 +149,15 @@ int stage_impl(void* const dst[4], int64_t dst_num_pages, int64_t dst_page0, con
   p.len_value = len_value;
   p.n_pages = n_pages;
   (void)dst_num_pages;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                 cudaSuccess || sms < 1) {
+    (void)cudaGetLastError();
+    return QKV_ECUDA;
+  }
   void* args[] = {&p};
-  if (launch_pdl((const void*)stage_pages_f4_kernel, dim3((unsigned)n_pages), dim3(STAGE_THREADS), 0, stream,
-                 args) != cudaSuccess) {
+  if (launch_pdl((const void*)stage_pages_f4_kernel, dim3((unsigned)std::min(n_pages, sms)), dim3(STAGE_THREADS), 0,
+                 stream, args) != cudaSuccess) {
     (void)cudaGetLastError();
     return QKV_ECUDA;
   }
@@ -382,7 +399,6 @@ extern "C" int qkv_paged_prefill_attn_f4_tiered(
   void* win[4];
   for (int a = 0; a < 4; ++a) win[a] = ws + L.win[a];
   int32_t* tab = reinterpret_cast<int32_t*>(ws + L.tab);
-  int32_t* len = reinterpret_cast<int32_t*>(ws + L.len);
   float* o = reinterpret_cast<float*>(ws + L.o);
   float* lse = reinterpret_cast<float*>(ws + L.lse);
   Slabs sl;
@@ -394,7 +410,7 @@ extern "C" int qkv_paged_prefill_attn_f4_tiered(
   for (int32_t c0 = 0; c0 < n_host; c0 += window_pages) {
     const int32_t n = std::min(window_pages, n_host - c0);
     int rc = stage_impl(win, window_pages, 0, src, host_num_pages, static_cast<const int32_t*>(hpt) + c0, n, sl, tab,
-                        len, n * block_size, device_status, stream);
+                        nullptr, 0, device_status, stream);
     if (rc) return rc;
     // every query of the chunk sees every token of the window
     rc = prefill_run(out, nullptr, q, static_cast<const uint8_t*>(win[0]), static_cast<const uint16_t*>(win[1]),

@@ -4,7 +4,7 @@ link) byte for byte, and qkv_paged_decode_attn_f4_tiered (the older whole
 pages of each sequence in the host pool, the rest in the device pool)
 against the oracle's attention over the two pools, for several sequences,
 windows smaller and larger than the host part, empty tiers, both V scale
-layouts and three query-group sizes."""
+layouts and three query-group sizes; and the tiered prefill."""
 import numpy as np
 import pytest
 import torch
@@ -196,15 +196,12 @@ def test_tiered_prefill_matches_oracle(qkv, case, v_group):
     hrow, drow = np.ascontiguousarray(row[:max(hp, 1)]), np.ascontiguousarray(row[hp:])
     prefix = dev_tokens - n_q
     q = workloads.chunk_queries_host(w, 0, n_q)
-    nb = qkv.qkv_paged_prefill_tiered_workspace_bytes(n_q, hq, hkv, 256, block, v_group, hp, window, ppl)
-    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    att = qkv.TieredPrefillAttention(n_q, hq, hkv, 256, block, hp, window, v_group=v_group, parts_per_launch=ppl)
     out = torch.full((n_q, hq, 256), 0x7FC1, dtype=torch.int16, device="cuda")
     lse = torch.empty((n_q, hq), dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    qkv.qkv_paged_prefill_attn_f4_tiered(out, to_dev(q), dev.k_data, dev.k_scale, dev.v_data, dev.v_scale,
-                                         to_dev(drow), prefix, host.k_data, host.k_scale, host.v_data, host.v_scale,
-                                         torch.from_numpy(hrow).pin_memory(), hp * block, hkv, window, ppl, ws,
-                                         lse2_out=lse, device_status=st)
+    att(out, to_dev(q), dev, to_dev(drow), prefix, host, torch.from_numpy(hrow).pin_memory(), hp * block,
+        lse2_out=lse, device_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     ro, rl = oracle.tiered_prefill_attention(q, ref, hrow, hp * block, ref, drow, np.arange(prefix, dev_tokens), hq,
