@@ -152,3 +152,28 @@ def test_tier_invalid_arguments_rejected_before_launch(qkv):
     assert L.qkv_paged_decode_attn_f4_tiered(*a) == 1
     a, keep = td([64], need, host=ctypes.c_void_p(pageable.ctypes.data))   # pageable host pool
     assert L.qkv_paged_decode_attn_f4_tiered(*a) == 1
+
+
+def test_prefill_tier_workspace_bytes_and_refusals(qkv):
+    a = lambda x: (x + 255) // 256 * 256
+    n_q, hq, hkv, d, blk, vg, max_host, win, ppl = 2048, 16, 4, 256, 64, 32, 4032, 2048, 4
+    rows = hkv * blk
+    parts = (-(-max_host // win) + 1) * ppl
+    want = (2 * a(win * rows * d // 2) + 2 * a(win * rows * d // 32 * 2) + a(win * 4) + 256
+            + a(parts * n_q * hq * d * 4) + a(parts * n_q * hq * 4))
+    assert qkv.qkv_paged_prefill_tiered_workspace_bytes(n_q, hq, hkv, d, blk, vg, max_host, win, ppl) == want
+    assert qkv.qkv_paged_prefill_tiered_workspace_bytes(n_q, hq, hkv, d, blk, vg, max_host, win, 65) == 0
+    assert qkv.qkv_paged_prefill_tiered_workspace_bytes(0, hq, hkv, d, blk, vg, max_host, win, ppl) == 0
+    L = qkv.lib
+    i64 = ctypes.c_int64
+    need = qkv.qkv_paged_prefill_tiered_workspace_bytes(64, 16, 4, 256, 64, 32, 2, 2, 2)
+    pageable = np.zeros(1 << 16, np.uint8)
+
+    def tp(host_len, ws_bytes, host=FAKE):
+        return (FAKE, NUL, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 0, 4, i64(64), host, FAKE, FAKE, FAKE, i64(16),
+                FAKE, host_len, 16, 4, 256, 64, 32, ctypes.c_float(0.0), 2, 2, ctypes.c_void_p(1 << 20), ws_bytes,
+                NUL, NUL)
+    assert L.qkv_paged_prefill_attn_f4_tiered(*tp(40, need)) == 1          # host part not whole pages
+    assert L.qkv_paged_prefill_attn_f4_tiered(*tp(128, need - 1)) == 1     # workspace too small
+    assert L.qkv_paged_prefill_attn_f4_tiered(*tp(128, need)) == 1         # FAKE host pool: not device-accessible
+    assert L.qkv_paged_prefill_attn_f4_tiered(*tp(128, need, ctypes.c_void_p(pageable.ctypes.data))) == 1
