@@ -768,8 +768,10 @@ def run_op(args, rank, world, local_rank):
     if rank != 0:
         return
     nb = lambda ts: sum(t.numel() * t.element_size() for t in ts)
+    # committed ncu summaries of each op's dominant kernel in this launch configuration (the tiered
+    # prefill's window passes have none: its traffic is reported as unknown)
     profile_of = {"gather": ("gather_kv_f4", "gather.cu"), "prefill": ("paged_prefill", "prefill.cu"),
-                  "tier": ("stage_pages_f4", "host_tier.cu"), "tier_prefill": ("paged_prefill", "prefill.cu")}
+                  "tier": ("stage_pages_f4", "host_tier.cu")}
     value = world * work / (ms * 1e-3) / scale
     achieved = work / (ms * 1e-3) / scale
     kernel_ms = ms
@@ -785,9 +787,12 @@ def run_op(args, rank, world, local_rank):
                   "tier_prefill": "f16 tcgen05, f32 accumulate"}[args.op],
         "data": "synthetic", "config": cfg, "device_status": int(status.item()),
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                     "traffic": profiled_traffic(w.name, *profile_of[args.op]), "kernel": kernel,
+                     "traffic": profiled_traffic(w.name, *profile_of[args.op]) if args.op in profile_of else None,
+                     "kernel": kernel,
                      "peak_kind": peak_kind, "kernel_ms": kernel_ms,
-                     "timing": "CUDA events around back-to-back launches"},
+                     "timing": ("CUDA events around back-to-back calls (staging, window passes, device pass, "
+                                "merge)" if args.op == "tier_prefill" else
+                                "CUDA events around back-to-back launches")},
         "e2e": {"value": world * work / (ms_e2e * 1e-3) / scale, "unit": unit, "h2d_bytes_per_step": nb(h_in),
                 "d2h_bytes_per_step": nb(h_out), "ms_per_step": ms_e2e},
         "gpu_launches": args.steps * launches_per_call, "clocks": clk.summary(),
