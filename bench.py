@@ -2,10 +2,12 @@
 """Decode-step benchmark of the paged F4 attention hot path on B200.
 
 One step = one decode token for every sequence of the workload through all
-its full-attention layers: the YaRN table row(s) of the step positions, the
-partial rotary of q and of the new key with the F4 write of the new K/V (one
-launch), the split-KV paged attention and the log2-sum-exp merge -- 1 + 3 x
-layers kernel launches, replayed from a CUDA graph.
+its full-attention layers: the YaRN table row(s) of the step positions, then
+per layer the split launch of the decode step (partial rotary of q and of the
+new key, F4 write of the new K/V, split-KV paged attention) and the
+log2-sum-exp merge -- 1 + 2 x layers kernel launches, replayed from a CUDA
+graph (``--two-call``: the rotary and write as a launch of their own before
+the attention, 1 + 3 x layers).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --op gather|prefill|tier|tier_prefill [--steps K] [--warmup W]
@@ -64,6 +66,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="host-time budget of the CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--two-call", action="store_true",
+                    help="decode step as rotary + F4 write, then split pass + merge (three launches per layer) "
+                         "instead of the fused step (two)")
     ap.add_argument("--op", choices=["decode", "gather", "prefill", "tier", "tier_prefill"], default="decode",
                     help="the decode step (default) or one widened row")
     ap.add_argument("--chunk", type=int, default=2048, help="prefill chunk size (queries)")
@@ -134,7 +139,7 @@ class ClockSampler:
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device, period_s: float = 0.005):
+    def __init__(self, device, period_s: float = 0.001):
         self.period = period_s
         self.samples, self.reasons, self.ok = [], set(), False
         self.max_mhz = None
@@ -184,10 +189,11 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- CPU oracle sample
 
-def oracle_step_sample(w: workloads.Workload, n_tok: int, seed: int = 1):
+def oracle_step_sample(w: workloads.Workload, n_tok: int, seed: int = 1, n_threads: int = 0):
     """Build a host sample of the workload (same recipe, first ``n_tok``
     context tokens of the first sequence) and return a callable that runs one
-    oracle decode step on it, plus the algorithmic bytes that step covers."""
+    oracle decode step on it with ``n_threads`` threads (0: all host cores),
+    plus the algorithmic bytes that step covers and the thread count."""
     import oracle
     s = workloads.Workload(name=w.name + "_sample", n_layers=1, seq_lens=(n_tok,),
                            num_pages=-(-n_tok // w.block_size), block_size=w.block_size, q_heads=w.q_heads,
@@ -205,15 +211,16 @@ def oracle_step_sample(w: workloads.Workload, n_tok: int, seed: int = 1):
         k = oracle.rope_apply_bf16(x["k_new"], x["positions"], spec)
         oracle.kv_write_f4(k, x["v_new"], x["step_slots"], cache, s.kv_heads, s.head_dim, s.block_size)
         return oracle.paged_attention(q, cache, x["page_table"], [0], x["seq_lens"], s.q_heads, s.kv_heads,
-                                      s.head_dim, s.block_size)
+                                      s.head_dim, s.block_size, n_threads=threads)
 
-    return step, s.algorithmic_bytes_per_layer(), oracle.max_threads()
+    threads = n_threads if n_threads > 0 else oracle.max_threads()
+    return step, s.algorithmic_bytes_per_layer(), threads
 
 
-def calibrate_sample(w, seconds: float):
+def calibrate_sample(w, seconds: float, n_threads: int = 0):
     """Token count whose oracle step takes about ``seconds`` on this host."""
     probe = min(2048, w.seq_lens[0])
-    step, _, _ = oracle_step_sample(w, probe)
+    step, _, _ = oracle_step_sample(w, probe, n_threads=n_threads)
     t0 = time.perf_counter()
     step()
     dt = max(time.perf_counter() - t0, 1e-4)
@@ -222,14 +229,22 @@ def calibrate_sample(w, seconds: float):
 
 
 def cpu_baseline(w, seconds: float):
-    n_tok = calibrate_sample(w, seconds)
-    step, nbytes, cores = oracle_step_sample(w, n_tok)
-    t0 = time.perf_counter()
-    step()
-    dt = time.perf_counter() - t0
-    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"one layer, first sequence, {n_tok} of {w.seq_lens[0]} context tokens "
-                      f"(rotary + F4 write of the new token + exact attention, fp64), {dt:.1f} s"}
+    """The oracle on all host cores (the reported baseline) and on one core,
+    each on a bounded sample of about ``seconds`` of host time."""
+    runs = {}
+    for n_threads in (0, 1):
+        n_tok = calibrate_sample(w, seconds / 2, n_threads)
+        step, nbytes, cores = oracle_step_sample(w, n_tok, n_threads=n_threads)
+        t0 = time.perf_counter()
+        step()
+        dt = time.perf_counter() - t0
+        runs[n_threads] = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                           "sample": f"one layer, first sequence, {n_tok} of {w.seq_lens[0]} context tokens "
+                                     f"(rotary + F4 write of the new token + exact attention, fp64), {dt:.1f} s "
+                                     f"on {cores} thread{'s' if cores > 1 else ''}"}
+    out = runs[0]
+    out["single_thread"] = runs[1]
+    return out
 
 
 # --------------------------------------------------------------------------- reference arm
@@ -270,7 +285,7 @@ def config_of(w, args):
 # --------------------------------------------------------------------------- our arm
 
 class Bench:
-    def __init__(self, w: workloads.Workload, device, seed_offset: int):
+    def __init__(self, w: workloads.Workload, device, seed_offset: int, two_call: bool = False):
         import torch
 
         import quantized_paged_kv_yarn_b200 as qkv
@@ -300,9 +315,14 @@ class Bench:
         self.cos = torch.empty((self.n_rows, w.rot_dim // 2), dtype=torch.float32, device=device)
         self.sin = torch.empty_like(self.cos)
         self.params = qkv.YarnParams.make(**workloads.yarn_spec(w))
-        self.att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size)
+        # a fixed split count (the 1M-token workload's 148) sizes the workspace; 0: the automatic plan
+        self.att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size,
+                                       max_splits=w.num_splits)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
-        self.launches_per_step = 1 + 3 * self.L
+        self.two_call = two_call
+        # the split launch merges its own partials unless the plan is too wide (then a merge launch follows)
+        self.folds = qkv.decode_folds(self.att.max_splits, w.n_seq, w.q_heads, w.kv_heads)
+        self.launches_per_step = 1 + ((2 if two_call else 1) + (0 if self.folds else 1)) * self.L
         # host side of the end-to-end measurement (pinned)
         self.h_q = [t.cpu().pin_memory() for t in self.q_raw]
         self.h_kn = [t.cpu().pin_memory() for t in self.kn_raw]
@@ -315,6 +335,13 @@ class Bench:
         q.qkv_yarn_rope_table(self.params, self.pos0, self.n_rows, self.cos, self.sin)
         for l in range(self.L):
             c = self.caches[l]
+            if not self.two_call:
+                # a2 + a3 + a4 in the split launch (rotary of q, rotary and F4 write of the
+                # new token, split attention), then a5
+                self.att.step(self.out[l], self.q_raw[l], self.kn_raw[l], self.vn[l], self.positions,
+                              self.step_slots, self.cos, self.sin, self.pos0, w.rot_dim, c, self.page_table,
+                              self.seq_lens, num_splits=w.num_splits, device_status=self.status)
+                continue
             # a2 + a3 in one launch: rotary of q and of the new k, F4 write of k and v
             q.qkv_rope_kv_write_f4(self.q_raw[l], self.q_rot[l], self.kn_raw[l], self.vn[l], self.positions,
                                    self.step_slots, self.cos, self.sin, self.pos0, w.rot_dim, c.k_data, c.k_scale,
@@ -346,11 +373,13 @@ class Bench:
         return g
 
     def split_kernel_ms(self, rounds: int):
-        """Average duration of the split-pass kernel: CUDA events on its
-        stream around `rounds` passes over the layers' caches (each cache is
-        larger than L2, so every launch reads HBM), launched back to back as
-        in the step; also the per-launch times with events around every
-        launch (these include each launch's own start-up gap)."""
+        """Average duration of the split-pass kernel as the step runs it (with
+        its partials folded in the launch when the plan allows, else alone):
+        CUDA events on its stream around `rounds` passes over the layers'
+        caches (each cache is larger than L2, so every launch reads HBM),
+        launched back to back as in the step; also the per-launch times with
+        events around every launch (these include each launch's own start-up
+        gap)."""
         torch, qkv, w = self.torch, self.qkv, self.w
         rows = w.n_seq * w.q_heads
         ms = self.att.max_splits
@@ -360,9 +389,23 @@ class Bench:
 
         def launch(l):
             c = self.caches[l]
-            qkv.qkv_paged_decode_split_f4(o_parts, l_parts, self.q_rot[l], c.k_data, c.k_scale, c.v_data,
-                                          c.v_scale, self.page_table, self.seq_lens, w.kv_heads,
-                                          num_splits=w.num_splits)
+            if self.folds:  # one launch: the split pass with its fold
+                if self.two_call:
+                    self.att(self.out[l], self.q_rot[l], c, self.page_table, self.seq_lens,
+                             num_splits=w.num_splits)
+                else:
+                    self.att.step(self.out[l], self.q_raw[l], self.kn_raw[l], self.vn[l], self.positions,
+                                  self.step_slots, self.cos, self.sin, self.pos0, w.rot_dim, c, self.page_table,
+                                  self.seq_lens, num_splits=w.num_splits)
+            elif self.two_call:
+                qkv.qkv_paged_decode_split_f4(o_parts, l_parts, self.q_rot[l], c.k_data, c.k_scale, c.v_data,
+                                              c.v_scale, self.page_table, self.seq_lens, w.kv_heads,
+                                              num_splits=w.num_splits)
+            else:  # the step's split launch: rotary, F4 write of the new token, split attention
+                qkv.qkv_decode_step_split_f4(o_parts, l_parts, self.q_raw[l], self.kn_raw[l], self.vn[l],
+                                             self.positions, self.step_slots, self.cos, self.sin, self.pos0,
+                                             w.rot_dim, c.k_data, c.k_scale, c.v_data, c.v_scale, self.page_table,
+                                             self.seq_lens, w.kv_heads, num_splits=w.num_splits)
 
         for l in range(self.L):  # warm
             launch(l)
@@ -400,7 +443,7 @@ def run_ours(args, rank, world, local_rank):
     w = workloads.BY_NAME[args.workload]
     if args.layers:
         w = dataclass_replace(w, n_layers=args.layers)
-    b = Bench(w, dev, seed_offset=rank)
+    b = Bench(w, dev, seed_offset=rank, two_call=args.two_call)
 
     def barrier():
         if world > 1:
@@ -459,7 +502,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_value = whole_job_gbps(step_bytes, ms_e2e, world)
     peak, peak_kind = hbm_peak()
     out_bytes = 2 * w.n_seq * w.q_heads * w.head_dim
-    split_bytes = per_layer - out_bytes  # the merge writes out
+    split_bytes = per_layer if b.folds else per_layer - out_bytes  # without the fold the merge writes out
     achieved = split_bytes / (split_ms_mean * 1e-3) / 1e9
     traffic = profiled_traffic(w.name)
     bi, bo = b.io_bytes()
@@ -475,7 +518,9 @@ def run_ours(args, rank, world, local_rank):
         "device_status": status,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "paged_decode_split_kernel", "peak_kind": f"{peak_kind} (copy bandwidth)",
+                     "kernel": "paged_decode_split_kernel" + ("" if args.two_call else " (decode-step instance)")
+                               + (", partials folded in the launch" if b.folds else ""),
+                     "peak_kind": f"{peak_kind} (copy bandwidth)",
                      "kernel_ms": split_ms_mean, "kernel_ms_isolated": split_ms_each,
                      "timing": "CUDA events around back-to-back launches over the layers' caches",
                      "algorithmic_bytes_per_launch": split_bytes},

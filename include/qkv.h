@@ -200,8 +200,15 @@ QKV_API int qkv_rope_kv_write_f4_v(const uint16_t* q_in, uint16_t* q_out, const 
  * CUDA device is present. */
 QKV_API int32_t qkv_paged_decode_auto_splits(int32_t kv_heads, int32_t block_size);
 
-/* Bytes of workspace qkv_paged_decode_attn_f4 needs: max_splits *
- * n_seq * q_heads * (head_dim + 1) floats, rounded up to 256 bytes. */
+/* Bytes of the fold's ticket counters at the start of a decode workspace:
+ * one 32-bit counter per (sequence, KV head), so a fold needs
+ * n_seq * kv_heads <= 1024. */
+#define QKV_DECODE_FOLD_TICKET_BYTES 4096
+
+/* Bytes of workspace qkv_paged_decode_attn_f4 needs:
+ * QKV_DECODE_FOLD_TICKET_BYTES of ticket counters, max_splits * n_seq *
+ * q_heads * head_dim floats (o_parts) and max_splits * n_seq * q_heads
+ * floats (lse2_parts), each part rounded up to 256 bytes. */
 QKV_API size_t qkv_paged_decode_workspace_bytes(int32_t n_seq, int32_t q_heads, int32_t head_dim,
                                         int32_t max_splits);
 
@@ -213,8 +220,9 @@ QKV_API size_t qkv_paged_decode_workspace_bytes(int32_t n_seq, int32_t q_heads, 
  *             in page page_table[s][i / block_size] at offset i % block_size.
  *   seq_lens  int32 [n_seq], context tokens of each sequence.
  *   softmax_scale  0 selects 1/sqrt(head_dim).
- *   num_splits  > 0: every sequence is cut into min(num_splits, max_splits)
- *             splits; 0: the plan balances pages over the device (splits of
+ *   num_splits  > 0: every sequence is cut into exactly num_splits splits
+ *             (EINVAL when num_splits > max_splits: the count is never cut
+ *             to fit); 0: the plan balances pages over the device (splits of
  *             about sum(pages) / auto_splits pages each, at most max_splits
  *             per sequence). Split i of a sequence with n pages covers pages
  *             [i*n/S, (i+1)*n/S).
@@ -255,19 +263,43 @@ QKV_API int qkv_paged_decode_split_f4_v(float* o_parts, float* lse2_parts, int32
  *   out       bf16 [rows][head_dim] (nearest even); lse2_out float [rows] or NULL.
  * Per row: M = max_i lse2_i; w_i = 2^(lse2_i - M); out = sum_i w_i o_i /
  * sum_i w_i; lse2 = M + log2 sum_i w_i. Parts with lse2 = -inf carry no
- * weight and their o rows are not read; a row without any gives out = 0 and
- * lse2 = -inf.
+ * weight: their o rows may be read but never enter the result (they may
+ * hold anything, NaN included); a row without any weighted part gives
+ * out = 0 and lse2 = -inf.
  * EINVAL: null pointer, n_parts < 1, rows < 0, head_dim not a multiple of 4
  * or > 1024. */
 QKV_API int qkv_lse_merge(const float* o_parts, const float* lse2_parts, int32_t n_parts, int32_t rows,
                   int32_t head_dim, uint16_t* out, float* lse2_out, qkv_stream_t stream);
 
+/* Largest max_splits * (q_heads / kv_heads) for which the decode attention
+ * folds the split partials inside the split launch (the last CTA of each
+ * (sequence, KV head) to finish merges them, when also n_seq * kv_heads * 4
+ * <= QKV_DECODE_FOLD_TICKET_BYTES); otherwise a merge launch follows. */
+#define QKV_DECODE_FOLD_MAX_ROWS 320
+
 /* a4 + a5: the decode attention of one layer. Runs the split pass into
  * `workspace` (see qkv_paged_decode_workspace_bytes) and merges it into
- * `out` (bf16 [n_seq][q_heads][head_dim]) and `lse2_out` (float
- * [n_seq][q_heads] or NULL). Arguments and errors as in the two calls;
- * EINVAL also when workspace_bytes is too small or workspace is not
- * 256-byte aligned. */
+ * `out` (bf16 [n_seq][q_heads][head_dim], 4-byte aligned) and `lse2_out`
+ * (float [n_seq][q_heads] or NULL), with the arithmetic of qkv_lse_merge:
+ * in the split launch itself when max_splits * (q_heads / kv_heads) <=
+ * QKV_DECODE_FOLD_MAX_ROWS and n_seq * kv_heads * 4 <=
+ * QKV_DECODE_FOLD_TICKET_BYTES (one launch), else by a qkv_lse_merge launch.
+ * Arguments and errors as in the two calls; EINVAL also when workspace_bytes
+ * is too small or workspace is not 256-byte aligned. The workspace starts
+ * with the fold's ticket counters (QKV_DECODE_FOLD_TICKET_BYTES); after the
+ * call it holds the split pass's o_parts (float [max_splits][n_seq *
+ * q_heads][head_dim], from offset QKV_DECODE_FOLD_TICKET_BYTES) and
+ * lse2_parts (float [max_splits][n_seq * q_heads], from the next 256-byte
+ * boundary). The counters must be zero before the first call with a
+ * workspace (zero-fill it once); every call, aborted ones included, leaves
+ * them at zero, whatever its shapes. Calls that overlap on the GPU must not
+ * share a workspace.
+ * Programmatic dependent launch: the split launch may start while the
+ * kernel ahead of it in the stream still runs (when that kernel allows
+ * it), and reads the page table, the sequence lengths and the cache pages
+ * before that kernel completes; q is read after. A kernel that lets its
+ * successor start early must therefore not write those (this library's
+ * cache writers never let their successor start early). */
 QKV_API int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q,
                              const uint8_t* k_data, const uint16_t* k_scale,
                              const uint8_t* v_data, const uint16_t* v_scale,
@@ -278,8 +310,9 @@ QKV_API int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint1
                              void* workspace, size_t workspace_bytes, int32_t* device_status,
                              qkv_stream_t stream);
 
-/* One decode step of a layer in two launches: a2 + a3 + a4 in the split
- * pass, then a5. The split kernel rotates each sequence's q itself (NEOX on
+/* One decode step of a layer: a2 + a3 + a4 in the split launch, a5 in it
+ * too or in a merge launch (as in qkv_paged_decode_attn_f4). The split
+ * kernel rotates each sequence's q itself (NEOX on
  * the first rot_dim dims, rounded to bf16 as qkv_rope_apply rounds), and the
  * CTA whose split holds a sequence's last page first writes the step's new
  * k (rotated) and v into the cache at slot_mapping[s] (F4, as
@@ -295,7 +328,12 @@ QKV_API int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint1
  *                qkv_rope_apply (a position outside the table leaves q and k
  *                unrotated and sets QKV_DEV_BAD_POSITION).
  *   the rest as in qkv_paged_decode_attn_f4_v (v_group 32 or head_dim).
- * A slot past the pool sets QKV_DEV_BAD_SLOT and skips the write. */
+ * A slot past the pool sets QKV_DEV_BAD_SLOT and skips the write.
+ * Besides what qkv_paged_decode_attn_f4 reads early, positions,
+ * slot_mapping and the cos/sin tables are read before the kernel ahead in
+ * the stream completes (q, k_new and v_new after): the step's metadata must
+ * not be written by a kernel that lets its successor start early (the
+ * library's table kernel never does). */
 QKV_API int qkv_decode_step_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint16_t* k_new,
                                const uint16_t* v_new, const int64_t* positions, const int64_t* slot_mapping,
                                const float* cos_tab, const float* sin_tab, int64_t table_pos_start,
@@ -306,6 +344,22 @@ QKV_API int qkv_decode_step_f4(uint16_t* out, float* lse2_out, const uint16_t* q
                                int64_t num_pages, float softmax_scale, int32_t num_splits, int32_t max_splits,
                                int32_t v_group, void* workspace, size_t workspace_bytes, int32_t* device_status,
                                qkv_stream_t stream);
+
+/* The split pass of qkv_decode_step_f4 alone (a2 + a3 + a4 in one launch):
+ * rotates q, writes the step's new token into the cache and writes the
+ * partials like qkv_paged_decode_split_f4_v, for a caller that merges them
+ * itself (qkv_lse_merge). Arguments as in qkv_decode_step_f4, with o_parts /
+ * lse2_parts / max_splits as in qkv_paged_decode_split_f4. */
+QKV_API int qkv_decode_step_split_f4(float* o_parts, float* lse2_parts, int32_t max_splits, const uint16_t* q,
+                                     const uint16_t* k_new, const uint16_t* v_new, const int64_t* positions,
+                                     const int64_t* slot_mapping, const float* cos_tab, const float* sin_tab,
+                                     int64_t table_pos_start, int64_t table_len, int32_t rot_dim,
+                                     uint8_t* k_data, uint16_t* k_scale, uint8_t* v_data, uint16_t* v_scale,
+                                     const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
+                                     int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                     int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                                     int32_t num_splits, int32_t v_group, int32_t* device_status,
+                                     qkv_stream_t stream);
 
 /* qkv_paged_decode_attn_f4 over a cache written with qkv_kv_write_f4_v
  * (v_group 32 or head_dim). */
@@ -412,11 +466,17 @@ QKV_API int32_t qkv_paged_prefill_auto_splits(int32_t n_q, int32_t prefix_len, i
  *     256 at a B200's automatic 37 splits: up to 27 sequences).
  *   - The first call on a device resolves the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture. The address is cached with the identity of
+ *     the device's CUDA context: after cudaDeviceReset (or any new context
+ *     on the device) the next call resolves it again, so make that call
+ *     outside capture as well; a call whose launch fails drops the cached
+ *     address.
  *   - Every call on a device shares the one array and it keeps the last
- *     call's contents (nothing in it needs to start at zero). Calls whose
- *     kernels overlap on the GPU -- on different streams, or from different
- *     host threads -- race on it: order them on one stream. */
+ *     call's contents. It is zero when the library is loaded; the ticket
+ *     counters of the in-launch fold must be zero before a call and every
+ *     call leaves them at zero. Calls whose kernels overlap on the GPU -- on
+ *     different streams, or from different host threads -- race on it:
+ *     order them on one stream. */
 QKV_API int qkv_paged_decode_attn_f4_static(uint16_t* out, float* lse2_out, const uint16_t* q,
                                             const uint8_t* k_data, const uint16_t* k_scale,
                                             const uint8_t* v_data, const uint16_t* v_scale,

@@ -78,6 +78,9 @@ _SIGS = {
     "qkv_decode_step_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _vp, _vp,
                                           _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _f32, _i32,
                                           _i32, _i32, _vp, _sz, _vp, _vp]),
+    "qkv_decode_step_split_f4": (ctypes.c_int, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32,
+                                                _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64,
+                                                _f32, _i32, _i32, _vp, _vp]),
     "qkv_stage_pages_f4": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _i32, _i32,
                                           _i32, _i32, _i32, _vp, _vp]),
     "qkv_paged_decode_tiered_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32]),
@@ -322,7 +325,8 @@ def qkv_decode_step_f4(out, q, k_new, v_new, positions, slot_mapping, cos_tab, s
                        max_splits: int, lse2_out=None, softmax_scale: float = 0.0, num_splits: int = 0,
                        device_status=None, stream=None):
     """One layer's decode step (rotary, F4 write of the new k/v, attention,
-    merge) in two launches; q unrotated. Shapes as in qkv_rope_kv_write_f4
+    merge) in one launch (two when the partials are merged by a launch of their
+    own, see QKV_DECODE_FOLD_MAX_ROWS); q unrotated. Shapes as in qkv_rope_kv_write_f4
     and qkv_paged_decode_attn_f4."""
     n_seq, q_heads, head_dim = q.shape
     num_pages, _, block_size, _ = k_data.shape
@@ -340,7 +344,39 @@ def qkv_decode_step_f4(out, q, k_new, v_new, positions, slot_mapping, cos_tab, s
         _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
 
 
+def qkv_decode_step_split_f4(o_parts, lse2_parts, q, k_new, v_new, positions, slot_mapping, cos_tab, sin_tab,
+                             table_pos_start: int, rot_dim: int, k_data, k_scale, v_data, v_scale, page_table,
+                             seq_lens, kv_heads: int, softmax_scale: float = 0.0, num_splits: int = 0,
+                             device_status=None, stream=None):
+    """The decode step's split pass alone (rotary, F4 write of the new k/v,
+    partials); o_parts / lse2_parts as in qkv_paged_decode_split_f4."""
+    n_seq, q_heads, head_dim = q.shape
+    max_splits = o_parts.shape[0]
+    num_pages, _, block_size, _ = k_data.shape
+    half = rot_dim // 2
+    _check("qkv_decode_step_split_f4", lib.qkv_decode_step_split_f4(
+        _ptr(o_parts, "o_parts", (torch.float32,), max_splits * n_seq * q_heads * head_dim),
+        _ptr(lse2_parts, "lse2_parts", (torch.float32,), max_splits * n_seq * q_heads), max_splits,
+        _ptr(q, "q", _U16), _ptr(k_new, "k_new", _U16, n_seq * kv_heads * head_dim),
+        _ptr(v_new, "v_new", _U16, n_seq * kv_heads * head_dim), _ptr(positions, "positions", (torch.int64,), n_seq),
+        _ptr(slot_mapping, "slot_mapping", (torch.int64,), n_seq), _ptr(cos_tab, "cos_tab", (torch.float32,)),
+        _ptr(sin_tab, "sin_tab", (torch.float32,)), int(table_pos_start), cos_tab.numel() // half, int(rot_dim),
+        *_cache_args(k_data, k_scale, v_data, v_scale), _ptr(page_table, "page_table", (torch.int32,)),
+        _ptr(seq_lens, "seq_lens", (torch.int32,), n_seq), n_seq, q_heads, kv_heads, head_dim, block_size,
+        page_table.shape[1], num_pages, float(softmax_scale), int(num_splits), v_group_of(v_scale, head_dim),
+        _ptr(device_status, "device_status", (torch.int32,)), _stream(stream)))
+
+
 STATIC_SCRATCH_BYTES = 16 << 20
+DECODE_FOLD_MAX_ROWS = 320  # QKV_DECODE_FOLD_MAX_ROWS
+DECODE_FOLD_TICKET_BYTES = 4096  # QKV_DECODE_FOLD_TICKET_BYTES
+
+
+def decode_folds(max_splits: int, n_seq: int, q_heads: int, kv_heads: int) -> bool:
+    """Whether the decode attention merges its partials inside the split
+    launch (else a merge launch follows)."""
+    return (max_splits * (q_heads // kv_heads) <= DECODE_FOLD_MAX_ROWS
+            and n_seq * kv_heads * 4 <= DECODE_FOLD_TICKET_BYTES)
 
 
 def qkv_paged_decode_attn_f4_static(out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, kv_heads: int,

@@ -28,10 +28,17 @@ constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;
 
 // Programmatic dependent launch. Every kernel of the library is launched
 // with programmatic stream serialization allowed, so it may be scheduled
-// while its predecessor in the stream is still running. It calls
-// pdl_wait() before touching any global memory -- the wait returns once the
-// predecessor grid has completed and its writes are visible -- and then
-// pdl_release() so its own successor may be scheduled early in turn.
+// while its predecessor in the stream is still running. On every path, and
+// before it reads anything a kernel ahead of it may write, it calls
+// pdl_wait(), which returns once the predecessor grid has completed and its
+// writes are visible (so a grid's completion implies its predecessors').
+// pdl_release() lets the successor be scheduled: kernels call it at their
+// start, except those that write the K/V cache (the F4 writes and the
+// staging of host pages) or the rotary table, which leave it to their
+// completion. The split pass of decode attention reads the page table, the
+// sequence lengths, cache pages and (the decode step's) positions, slots
+// and rotary table before it waits; that is safe because no kernel that
+// released its successor early writes them.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
@@ -72,8 +79,26 @@ __device__ __forceinline__ float rot_second(float x0, float x1, float c, float s
 // rounds its output; the partner of dim j < rot / 2 is j + rot / 2, which sits
 // rot / 16 lanes away (rot is a multiple of 16). cos_row / sin_row: the
 // position's table row.
-__device__ __forceinline__ void rope_row_bf16(float (&x)[8], int lane, int rot, const float* cos_row,
-                                              const float* sin_row) {
+// The table values lane l needs for the rotation of its 8 elements (as
+// rope_row_bf16_cs uses them); lanes past rot / 8 load nothing.
+__device__ __forceinline__ void rope_load_cs(int lane, int rot, const float* cos_row, const float* sin_row,
+                                             float (&c)[8], float (&s)[8]) {
+  const int half = rot / 2;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int j = lane * 8 + i;
+    c[i] = s[i] = 0.f;
+    if (j < rot) {
+      const int jj = j < half ? j : j - half;
+      c[i] = cos_row[jj];
+      s[i] = sin_row[jj];
+    }
+  }
+}
+
+// rope_row_bf16 with the table values already loaded (rope_load_cs).
+__device__ __forceinline__ void rope_row_bf16_cs(float (&x)[8], int lane, int rot, const float (&c)[8],
+                                                 const float (&s)[8]) {
   const int half = rot / 2, dl = half / 8;
   float y[8];
 #pragma unroll
@@ -81,15 +106,19 @@ __device__ __forceinline__ void rope_row_bf16(float (&x)[8], int lane, int rot, 
     const float other = __shfl_sync(0xffffffffu, x[i], lane < dl ? lane + dl : lane - dl);
     y[i] = x[i];
     const int j = lane * 8 + i;
-    if (j < rot) {
-      const int jj = j < half ? j : j - half;
-      const float c = cos_row[jj], s = sin_row[jj];
-      y[i] = __bfloat162float(__float2bfloat16_rn(j < half ? rot_first(x[i], other, c, s)
-                                                           : rot_second(other, x[i], c, s)));
-    }
+    if (j < rot)
+      y[i] = __bfloat162float(__float2bfloat16_rn(j < half ? rot_first(x[i], other, c[i], s[i])
+                                                           : rot_second(other, x[i], c[i], s[i])));
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) x[i] = y[i];
+}
+
+__device__ __forceinline__ void rope_row_bf16(float (&x)[8], int lane, int rot, const float* cos_row,
+                                              const float* sin_row) {
+  float c[8], s[8];
+  rope_load_cs(lane, rot, cos_row, sin_row, c, s);
+  rope_row_bf16_cs(x, lane, rot, c, s);
 }
 
 // F4 quantise-write of the row (as qkv_kv_write_f4): scale = fp16(amax / 7)

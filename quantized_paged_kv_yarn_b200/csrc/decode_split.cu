@@ -109,6 +109,7 @@ struct __align__(1024) Smem {
   float gl[GROUPS][8];            // per group and head: softmax sum
   int next;                       // next stage of the split to claim
   int abort_flag;
+  int fold_last;                  // this CTA took the last ticket of its (sequence, KV head)
 };
 template <int HQ>
 constexpr size_t smem_bytes() {
@@ -127,6 +128,13 @@ struct Params {
   int64_t num_pages;
   int n_seq, q_heads, kv_heads, max_pages, max_splits, num_splits, target;
   float score_scale;  // softmax_scale * log2(e)
+  // Fold of the partials inside the launch (null out: the caller merges):
+  // the last CTA of each (sequence, KV head) to finish, found by a ticket
+  // counter per (sequence, KV head), merges its splits' partials into out /
+  // lse2_final.
+  __nv_bfloat16* out;
+  float* lse2_final;
+  unsigned int* tickets;  // [n_seq * kv_heads], zero between launches
 };
 // The decode step's inputs (qkv_decode_step_f4): q is unrotated; the kernel
 // rotates it and writes the step's new K (rotated) and V into the cache
@@ -230,7 +238,104 @@ __device__ __forceinline__ int muldiv(uint32_t a, uint32_t b, uint32_t c) {
   return (ab >> 32) == 0 ? (int)((uint32_t)ab / c) : (int)(ab / c);
 }
 
-// Split plan. Fixed: min(num_splits, max_splits) splits per sequence.
+// Ticket of a CTA that has written its partial: true for the last of the
+// S CTAs of its (sequence, KV head). The counter is zero before the launch
+// and the last CTA sets it back to zero for the next one. One atomic add
+// per CTA (a compare-and-swap loop here serialised the CTAs that finish
+// together: ~16 us at 37 splits).
+__device__ __forceinline__ bool take_ticket(unsigned int* counter, int S) {
+  const unsigned int old = atomicAdd(counter, 1u);
+  const bool last = old + 1u == (unsigned int)S;
+  if (last) atomicExch(counter, 0u);
+  return last;
+}
+
+// The fold of the S partials (o, lse2) of the G query rows row0 .. row0 +
+// G - 1 into bf16 out and lse2_out, by the last CTA of a (sequence, KV
+// head): the merge qkv_lse_merge computes (M = max lse2, weights 2^(lse2 -
+// M), out = sum w o / sum w, lse2 = M + log2 sum w). All THREADS threads
+// call it; sbuf is idle shared memory of at least fold_smem_floats(S, G).
+// Thread (slice sl, element e) sums parts sl, sl + SL, ... of float4 e of
+// the G rows; the first rows' loads are in flight with the lse2 loads.
+constexpr int FOLD_MAX_ROWS = QKV_DECODE_FOLD_MAX_ROWS;  // S * G
+template <int G>
+__device__ __noinline__ void fold_parts(const float* o_parts, const float* lse_parts, int rows, int row0, int S,
+                                        __nv_bfloat16* out, float* lse2_out, float* sbuf) {
+  constexpr int NV = G * (D / 4);   // float4 of one part's G rows
+  constexpr int SL = THREADS / NV;  // slices of the parts
+  constexpr int B = 8;              // part rows in flight per thread
+  const int e = threadIdx.x % NV, sl = threadIdx.x / NV;
+  const int h = e / (D / 4), d4 = e % (D / 4);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float* ls = sbuf;                                               // [S][G]: lse2, then weights
+  float* mh = sbuf + FOLD_MAX_ROWS;                               // [G] max lse2
+  float4* accs = reinterpret_cast<float4*>(sbuf + FOLD_MAX_ROWS + 8);  // [SL][NV]
+  const int mine = (S - sl + SL - 1) / SL;  // parts sl + SL k, k < mine
+  float4 x[B];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < B; ++u) {
+      x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k0 + u < mine)
+        x[u] = __ldcg(reinterpret_cast<const float4*>(o_parts + ((size_t)(sl + SL * (k0 + u)) * rows + row0 + h) * D) +
+                      d4);
+    }
+  };
+  load(0);
+  for (int j = threadIdx.x; j < S * G; j += THREADS) ls[j] = __ldcg(lse_parts + (size_t)(j / G) * rows + row0 + j % G);
+  __syncthreads();
+  if (warp < G) {  // warp h: the max of head h's lse2
+    float m = -INFINITY;
+    for (int i = lane; i < S; i += 32) m = fmaxf(m, ls[i * G + warp]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, o));
+    if (lane == 0) mh[warp] = m;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < S * G; j += THREADS) {
+    const float l = ls[j];
+    ls[j] = l == -INFINITY ? 0.f : exp2f(l - mh[j % G]);
+  }
+  __syncthreads();
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k0 = 0; k0 < mine; k0 += B) {
+    if (k0 > 0) load(k0);
+#pragma unroll
+    for (int u = 0; u < B; ++u) {
+      if (k0 + u < mine) {
+        const float w = ls[(sl + SL * (k0 + u)) * G + h];
+        if (w != 0.f) {  // a part without weight may hold anything
+          a.x = fmaf(w, x[u].x, a.x);
+          a.y = fmaf(w, x[u].y, a.y);
+          a.z = fmaf(w, x[u].z, a.z);
+          a.w = fmaf(w, x[u].w, a.w);
+        }
+      }
+    }
+  }
+  accs[sl * NV + e] = a;
+  __syncthreads();
+  if (sl == 0) {
+#pragma unroll
+    for (int s2 = 1; s2 < SL; ++s2) {
+      const float4 b = accs[s2 * NV + e];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    float W = 0.f;
+    for (int i = 0; i < S; ++i) W += ls[i * G + h];
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + (size_t)(row0 + h) * D + 4 * d4);
+    dst[0] = __floats2bfloat162_rn(a.x * inv, a.y * inv);
+    dst[1] = __floats2bfloat162_rn(a.z * inv, a.w * inv);
+    if (d4 == 0 && lse2_out) lse2_out[row0 + h] = W > 0.f ? mh[h] + log2f(W) : -INFINITY;
+  }
+}
+
+// Split plan. Fixed: num_splits splits per sequence (the host refuses a
+// count above max_splits).
 // Automatic: pages are cut into pieces of about total pages / target, so the
 // grid holds at most `target` busy CTAs per KV head whatever the mix of
 // lengths. Split i of a sequence with n pages covers [i*n/S, (i+1)*n/S).
@@ -244,7 +349,7 @@ __device__ void plan(const Params& p, int seq, int split, int block, int& S, int
   L = seq_len_of(p, seq, block, split == 0 && blockIdx.z == 0);
   const uint32_t n = cdiv((uint32_t)L, (uint32_t)block);
   if (p.num_splits > 0) {
-    S = min(p.num_splits, p.max_splits);
+    S = p.num_splits;
   } else {
     // Pieces of P pages with sum_s ceil(n_s / P) <= target, so the busy CTAs
     // fit the resident slots in one wave.
@@ -286,8 +391,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   SmemT& sm = *reinterpret_cast<SmemT*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  pdl_wait();
-  pdl_release();
+  // Programmatic dependent launch. The kernel lets its successor launch at
+  // once (the fused instance: once the CTA that writes the step's new token
+  // has written it), and does everything that reads no output of the
+  // kernels ahead of it before it waits for them: the split plan (sequence
+  // lengths), the page ids and the first two stages' copies of every group.
+  // Kernels ahead of it that let their successors start early write none of
+  // these: the library's writers of the cache never do, and the fused
+  // instance's own write is ordered before the copies of its stage below.
+  if constexpr (!FUSE) pdl_release();
   const int split = blockIdx.x, seq = blockIdx.y, kvh = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = warp / GWARPS, gw = warp % GWARPS;  // group, warp within the group
@@ -300,12 +412,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   int S, pg0, pg1, L;
   plan(p, seq, split, BLOCK, S, pg0, pg1, L);
   if (split >= S) {  // unused slot of the plan
+    if constexpr (FUSE) pdl_release();
+    pdl_wait();  // the workspace may still be read by the kernels ahead
     if (threadIdx.x < G) lse_out[threadIdx.x] = -INFINITY;
     return;
   }
   const int t_begin = pg0 * BLOCK;
   const int t_end = min(pg1 * BLOCK, L);
   const int n_it = t_end > t_begin ? (t_end - t_begin + STAGE_TOK - 1) / STAGE_TOK : 0;
+  // Decode step: this CTA's split holds the sequence's last page, where the
+  // step's new token goes; that page's stage (the split's last) is copied
+  // only after the write.
+  const int last_pg = (L - 1) / BLOCK;
+  const bool writes_token = FUSE && L > 0 && last_pg >= pg0 && last_pg < pg1;
+  if constexpr (FUSE) {
+    if (!writes_token) pdl_release();
+  }
 
   if (threadIdx.x == 0) {
     for (int q = 0; q < GROUPS; ++q) {
@@ -323,54 +445,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   // probability rows of absent query heads (G < 8) are read as zeros
   for (int i = threadIdx.x % GTHREADS; i < (int)(sizeof(gs.prob) / 4); i += GTHREADS)
     reinterpret_cast<uint32_t*>(&gs.prob[0][0][0])[i] = 0u;
-  // Decode step: the CTA's query heads, rotated (bf16), in group 0's last V
-  // slot, which is first written by the copy of its local stage 2, issued in
-  // the main loop, after the q set-up has read them (8 KiB, 1024-aligned).
-  uint16_t(*qrot)[D] = reinterpret_cast<uint16_t(*)[D]>(&sm.grp[0].v[NSV - 1][0]);
-  static_assert(8 * D * 2 <= STAGE_TOK * ROW_BYTES, "qrot fits a V slot");
-  if constexpr (FUSE) {
-    // The decode step's rotary and F4 write inside this launch (as
-    // qkv_rope_kv_write_f4 computes them): warp h < G rotates query head h
-    // into shared memory; the CTA whose split holds the sequence's last
-    // page writes the new token's K (rotated, warp 8) and V (warp 9) into the
-    // cache before any of its copies starts.
-    const int half = p.st.rot / 2;
-    const int64_t ti = p.st.positions[seq] - p.st.tab_start;
-    const bool pos_ok = ti >= 0 && ti < p.st.tab_len;
-    const float* crow = p.st.cos_tab + (pos_ok ? ti : 0) * half;
-    const float* srow = p.st.sin_tab + (pos_ok ? ti : 0) * half;
-    if (!pos_ok && threadIdx.x == 0 && split == 0 && kvh == 0) flag(p.status, QKV_DEV_BAD_POSITION);
-    if (warp < G) {
-      float x[8];
-      load_row8(p.q + (size_t)(row0 + warp) * D, lane, D, x);
-      if (pos_ok) rope_row_bf16(x, lane, p.st.rot, crow, srow);
-      uint4 o;  // the rotated values are bf16-exact
-      o.x = (__float_as_uint(x[0]) >> 16) | (__float_as_uint(x[1]) & 0xffff0000u);
-      o.y = (__float_as_uint(x[2]) >> 16) | (__float_as_uint(x[3]) & 0xffff0000u);
-      o.z = (__float_as_uint(x[4]) >> 16) | (__float_as_uint(x[5]) & 0xffff0000u);
-      o.w = (__float_as_uint(x[6]) >> 16) | (__float_as_uint(x[7]) & 0xffff0000u);
-      *reinterpret_cast<uint4*>(&qrot[warp][8 * lane]) = o;
-    }
-    const int last_pg = (L - 1) / BLOCK;
-    if (L > 0 && last_pg >= pg0 && last_pg < pg1 && (warp == 8 || warp == 9)) {
-      const bool is_k = warp == 8;
-      const int64_t slot = p.st.slots[seq];
-      if (slot >= p.num_pages * BLOCK) {
-        if (lane == 0 && is_k) flag(p.status, QKV_DEV_BAD_SLOT);
-      } else if (slot >= 0) {
-        float x[8];
-        load_row8((is_k ? p.st.k_new : p.st.v_new) + ((size_t)seq * p.kv_heads + kvh) * D, lane, D, x);
-        if (is_k && pos_ok) rope_row_bf16(x, lane, p.st.rot, crow, srow);
-        const int group = is_k ? 32 : p.st.v_group;
-        const int64_t crw = ((slot / BLOCK) * p.kv_heads + kvh) * BLOCK + slot % BLOCK;
-        f4_write_row(x, lane, D, group, (is_k ? p.st.k_data_w : p.st.v_data_w) + crw * ROW_BYTES,
-                     (is_k ? p.st.k_scale_w : p.st.v_scale_w) + crw * (D / group));
-        // the copies of this CTA (async proxy) read these bytes after the barrier
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-      }
-    }
-  }
-  __syncthreads();
+  __syncthreads();  // barriers initialised
 
   // ------------------------------------------------------------ copy issue
   // Stage R of the split holds tokens t_begin + 64 R ... + 63, i.e. 64 /
@@ -464,11 +539,74 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     atomicMax(&gs.issued, j + 1);
   };
-  // local stage 0 now, 1 after the q set-up (so that every group's first
-  // stage is queued at the memory ahead of the second ones); stage j + 2
-  // follows at the group barrier of stage j
+  // Local stages 0 and 1 of every group now, before the wait (unless the
+  // stage holds the page of the step's new token); stage j + 2 follows at
+  // the group barrier of stage j.
   claim(gw);
-  if (gw == 0) issue(0, true);
+  const bool first_copy = gw < 2;  // this warp issues a first stage
+  const bool defer = writes_token && held == n_it - 1;
+  if (first_copy && !defer) issue(gw, true);
+  // Decode step: the step's position, rotary table values and slot are
+  // metadata, read before the wait like the page table; q and the new k and
+  // v are the step's activations, read after it.
+  float rc[8] = {}, rs[8] = {};  // table values of this lane's 8 rotated dims
+  bool pos_ok = false;
+  int64_t slot = -1;
+  if constexpr (FUSE) {
+    const int half = p.st.rot / 2;
+    const int64_t ti = p.st.positions[seq] - p.st.tab_start;
+    pos_ok = ti >= 0 && ti < p.st.tab_len;
+    if (!pos_ok && threadIdx.x == 0 && split == 0 && kvh == 0) flag(p.status, QKV_DEV_BAD_POSITION);
+    if (pos_ok && (warp < G || warp == 8))
+      rope_load_cs(lane, p.st.rot, p.st.cos_tab + ti * half, p.st.sin_tab + ti * half, rc, rs);
+    if (writes_token && (warp == 8 || warp == 9)) slot = p.st.slots[seq];
+  }
+  pdl_wait();
+  // Decode step: the CTA's query heads, rotated (bf16), in group 0's last V
+  // slot, which is first written by the copy of its local stage 2, issued in
+  // the main loop, after the q set-up has read them (8 KiB, 1024-aligned).
+  uint16_t(*qrot)[D] = reinterpret_cast<uint16_t(*)[D]>(&sm.grp[0].v[NSV - 1][0]);
+  static_assert(8 * D * 2 <= STAGE_TOK * ROW_BYTES, "qrot fits a V slot");
+  if constexpr (FUSE) {
+    // The decode step's rotary and F4 write inside this launch (as
+    // qkv_rope_kv_write_f4 computes them): warp h < G rotates query head h
+    // into shared memory; the CTA whose split holds the sequence's last
+    // page writes the new token's K (rotated, warp 8) and V (warp 9) into the
+    // cache before any of its copies starts.
+    if (warp < G) {
+      float x[8];
+      load_row8(p.q + (size_t)(row0 + warp) * D, lane, D, x);
+      if (pos_ok) rope_row_bf16_cs(x, lane, p.st.rot, rc, rs);
+      uint4 o;  // the rotated values are bf16-exact
+      o.x = (__float_as_uint(x[0]) >> 16) | (__float_as_uint(x[1]) & 0xffff0000u);
+      o.y = (__float_as_uint(x[2]) >> 16) | (__float_as_uint(x[3]) & 0xffff0000u);
+      o.z = (__float_as_uint(x[4]) >> 16) | (__float_as_uint(x[5]) & 0xffff0000u);
+      o.w = (__float_as_uint(x[6]) >> 16) | (__float_as_uint(x[7]) & 0xffff0000u);
+      *reinterpret_cast<uint4*>(&qrot[warp][8 * lane]) = o;
+    }
+    if (writes_token && (warp == 8 || warp == 9)) {
+      const bool is_k = warp == 8;
+      if (slot >= p.num_pages * BLOCK) {
+        if (lane == 0 && is_k) flag(p.status, QKV_DEV_BAD_SLOT);
+      } else if (slot >= 0) {
+        float x[8];
+        load_row8((is_k ? p.st.k_new : p.st.v_new) + ((size_t)seq * p.kv_heads + kvh) * D, lane, D, x);
+        if (is_k && pos_ok) rope_row_bf16_cs(x, lane, p.st.rot, rc, rs);
+        const int group = is_k ? 32 : p.st.v_group;
+        const int64_t crw = ((slot / BLOCK) * p.kv_heads + kvh) * BLOCK + slot % BLOCK;
+        f4_write_row(x, lane, D, group, (is_k ? p.st.k_data_w : p.st.v_data_w) + crw * ROW_BYTES,
+                     (is_k ? p.st.k_scale_w : p.st.v_scale_w) + crw * (D / group));
+        // the copies of this CTA (async proxy) read these bytes after the
+        // barrier; the kernels after this one may read them once it lets
+        // them start
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+      }
+    }
+  }
+  __syncthreads();
+  if (writes_token) pdl_release();
+  if (first_copy && defer) issue(gw, true);
 
   // ------------------------------------------------------------ q as the B operand
   // Column n of the Q K^T tile is (query head n >> 1 of the quad, cell
@@ -549,7 +687,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
   }
-  if (gw == 1) issue(1, true);
   __syncthreads();
 
   // ------------------------------------------------------------ main loop
@@ -881,98 +1018,109 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait_bounded(&q.vfull[r % NSV], (r / NSV) & 1)) flag(p.status, QKV_DEV_TIMEOUT);
     }
     if (threadIdx.x < G) lse_out[threadIdx.x] = -INFINITY;
-    return;
-  }
-  float2* vsp = reinterpret_cast<float2*>(&gs.vs[0][0]);
-  vsp[gw * 32 + lane] = make_float2(vsum[0], vsum[1]);
-  bar_sync(bar_id);
-  // the group's softmax sum and exponent reference per head
-  if (gw == 0 && g == 0) {
+  } else {
+    float2* vsp = reinterpret_cast<float2*>(&gs.vs[0][0]);
+    vsp[gw * 32 + lane] = make_float2(vsum[0], vsum[1]);
+    bar_sync(bar_id);
+    // the group's softmax sum and exponent reference per head
+    if (gw == 0 && g == 0) {
 #pragma unroll
-    for (int hq = 0; hq < HQ; ++hq) {
-      const int h = 4 * hq + t;
-      float Ls = 0.f;
+      for (int hq = 0; hq < HQ; ++hq) {
+        const int h = 4 * hq + t;
+        float Ls = 0.f;
 #pragma unroll
-      for (int w = 0; w < GWARPS; ++w) Ls += gs.wl[w][h];
-      sm.gl[grp][h] = Ls;
-      sm.gm[grp][h] = m_ref[hq];
-    }
-  }
-  // Undo the subnormal encoding of V: rows 0-7 carry 2^-24 * sum(n p s),
-  // rows 8-15 2^-20 * sum(n p s); the -8 offset is 8 * sum(p s) per cell.
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    const int cell = 2 * gw + c;
-    float b0 = 0.f, b1 = 0.f;
-    if constexpr (VTOK) {  // the warp's own sum covers every token and cell
-      b0 = vsum[0];
-      b1 = vsum[1];
-    } else {
-#pragma unroll
-      for (int w = 0; w < GWARPS; ++w) {
-        const float2 v = vsp[w * 32 + 4 * cell + t];
-        b0 += v.x;
-        b1 += v.y;
+        for (int w = 0; w < GWARPS; ++w) Ls += gs.wl[w][h];
+        sm.gl[grp][h] = Ls;
+        sm.gm[grp][h] = m_ref[hq];
       }
     }
-    b0 *= 8.f;
-    b1 *= 8.f;
+    // Undo the subnormal encoding of V: rows 0-7 carry 2^-24 * sum(n p s),
+    // rows 8-15 2^-20 * sum(n p s); the -8 offset is 8 * sum(p s) per cell.
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      acc[c][k][0] = fmaf(acc[c][k][0], 16777216.f, -b0);
-      acc[c][k][1] = fmaf(acc[c][k][1], 16777216.f, -b1);
-      acc[c][k][2] = fmaf(acc[c][k][2], 1048576.f, -b0);
-      acc[c][k][3] = fmaf(acc[c][k][3], 1048576.f, -b1);
+    for (int c = 0; c < 2; ++c) {
+      const int cell = 2 * gw + c;
+      float b0 = 0.f, b1 = 0.f;
+      if constexpr (VTOK) {  // the warp's own sum covers every token and cell
+        b0 = vsum[0];
+        b1 = vsum[1];
+      } else {
+#pragma unroll
+        for (int w = 0; w < GWARPS; ++w) {
+          const float2 v = vsp[w * 32 + 4 * cell + t];
+          b0 += v.x;
+          b1 += v.y;
+        }
+      }
+      b0 *= 8.f;
+      b1 *= 8.f;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        acc[c][k][0] = fmaf(acc[c][k][0], 16777216.f, -b0);
+        acc[c][k][1] = fmaf(acc[c][k][1], 16777216.f, -b1);
+        acc[c][k][2] = fmaf(acc[c][k][2], 1048576.f, -b0);
+        acc[c][k][3] = fmaf(acc[c][k][3], 1048576.f, -b1);
+      }
     }
-  }
-  __syncthreads();
-  // Fold the groups: weights 2^(m_ref of the group - M) per head.
-  float* slab = reinterpret_cast<float*>(&sm.grp[0].k[0][0]);  // [group][head][dim], in idle rings
+    __syncthreads();
+    // Fold the groups: weights 2^(m_ref of the group - M) per head.
+    float* slab = reinterpret_cast<float*>(&sm.grp[0].k[0][0]);  // [group][head][dim], in idle rings
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int h = 2 * t + j;
-    if (h < G) {
+    for (int j = 0; j < 2; ++j) {
+      const int h = 2 * t + j;
+      if (h < G) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < GROUPS; ++q)
+          if (sm.gl[q][h] > 0.f) M = fmaxf(M, sm.gm[q][h]);
+        const float f = (sm.gl[grp][h] > 0.f) ? exp2f(sm.gm[grp][h] - M) : 0.f;
+        float* dst = slab + ((size_t)grp * G + h) * D + 4 * g;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const float4 o = make_float4(f * acc[c][0][j], f * acc[c][0][j + 2], f * acc[c][1][j], f * acc[c][1][j + 2]);
+          *reinterpret_cast<float4*>(dst + 32 * (2 * gw + c)) = o;
+        }
+      }
+    }
+    __syncthreads();
+    // Sum the groups, normalise, write the partial of this split.
+    for (int e = threadIdx.x; e < G * (D / 4); e += THREADS) {
+      const int h = e / (D / 4), d4 = e % (D / 4);
       float M = -INFINITY;
 #pragma unroll
       for (int q = 0; q < GROUPS; ++q)
         if (sm.gl[q][h] > 0.f) M = fmaxf(M, sm.gm[q][h]);
-      const float f = (sm.gl[grp][h] > 0.f) ? exp2f(sm.gm[grp][h] - M) : 0.f;
-      float* dst = slab + ((size_t)grp * G + h) * D + 4 * g;
+      float Ls = 0.f;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const float4 o = make_float4(f * acc[c][0][j], f * acc[c][0][j + 2], f * acc[c][1][j], f * acc[c][1][j + 2]);
-        *reinterpret_cast<float4*>(dst + 32 * (2 * gw + c)) = o;
+      for (int q = 0; q < GROUPS; ++q) {
+        const float f = (sm.gl[q][h] > 0.f) ? exp2f(sm.gm[q][h] - M) : 0.f;
+        Ls = fmaf(f, sm.gl[q][h], Ls);
+        const float4 x = *reinterpret_cast<const float4*>(slab + ((size_t)q * G + h) * D + 4 * d4);
+        o.x += x.x;
+        o.y += x.y;
+        o.z += x.z;
+        o.w += x.w;
       }
+      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+      o.x *= inv;
+      o.y *= inv;
+      o.z *= inv;
+      o.w *= inv;
+      *reinterpret_cast<float4*>(p.o_parts + ((size_t)split * rows + row0 + h) * D + 4 * d4) = o;
+      if (d4 == 0) lse_out[h] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
     }
   }
+  if (p.out == nullptr) return;
+  // The fold: every CTA's partial is visible before it takes its ticket;
+  // the last CTA of the (sequence, KV head) merges them.
+  __threadfence();
   __syncthreads();
-  // Sum the groups, normalise, write the partial of this split.
-  for (int e = threadIdx.x; e < G * (D / 4); e += THREADS) {
-    const int h = e / (D / 4), d4 = e % (D / 4);
-    float M = -INFINITY;
-#pragma unroll
-    for (int q = 0; q < GROUPS; ++q)
-      if (sm.gl[q][h] > 0.f) M = fmaxf(M, sm.gm[q][h]);
-    float Ls = 0.f;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int q = 0; q < GROUPS; ++q) {
-      const float f = (sm.gl[q][h] > 0.f) ? exp2f(sm.gm[q][h] - M) : 0.f;
-      Ls = fmaf(f, sm.gl[q][h], Ls);
-      const float4 x = *reinterpret_cast<const float4*>(slab + ((size_t)q * G + h) * D + 4 * d4);
-      o.x += x.x;
-      o.y += x.y;
-      o.z += x.z;
-      o.w += x.w;
-    }
-    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-    o.x *= inv;
-    o.y *= inv;
-    o.z *= inv;
-    o.w *= inv;
-    *reinterpret_cast<float4*>(p.o_parts + ((size_t)split * rows + row0 + h) * D + 4 * d4) = o;
-    if (d4 == 0) lse_out[h] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
-  }
+  if (threadIdx.x == 0) sm.fold_last = take_ticket(p.tickets + (size_t)seq * p.kv_heads + kvh, S) ? 1 : 0;
+  __syncthreads();
+  if (sm.fold_last == 0) return;
+  __threadfence();
+  fold_parts<G>(p.o_parts, p.lse2_parts, rows, row0, S, p.out, p.lse2_final,
+                reinterpret_cast<float*>(&sm.grp[0].k[0][0]));
 }
 
 }  // namespace qkv
@@ -1084,13 +1232,28 @@ extern "C" int32_t qkv_paged_decode_auto_splits(int32_t kv_heads, int32_t block_
   return (int32_t)std::max(1, occ * sms / kv_heads);
 }
 
+// Workspace of the one-call decode attention: the fold's ticket counters in
+// a fixed first QKV_DECODE_FOLD_TICKET_BYTES (so a workspace reused with
+// other shapes, or the library's static array, keeps them where every call
+// leaves them at zero), then o_parts and lse2_parts, each from a 256-byte
+// boundary.
+struct DecodeWs {
+  size_t o, lse, tickets, total;
+};
+DecodeWs decode_ws(int64_t n_seq, int64_t q_heads, int64_t head_dim, int64_t max_splits) {
+  const size_t rows = (size_t)n_seq * q_heads;
+  DecodeWs w;
+  w.tickets = 0;
+  w.o = QKV_DECODE_FOLD_TICKET_BYTES;
+  w.lse = w.o + ((rows * max_splits * head_dim * 4 + 255) & ~size_t(255));
+  w.total = w.lse + ((rows * max_splits * 4 + 255) & ~size_t(255));
+  return w;
+}
+
 extern "C" size_t qkv_paged_decode_workspace_bytes(int32_t n_seq, int32_t q_heads, int32_t head_dim,
                                                    int32_t max_splits) {
   if (n_seq < 0 || q_heads < 0 || head_dim < 0 || max_splits < 0) return 0;
-  const size_t rows = (size_t)n_seq * q_heads * max_splits;
-  const size_t o = (rows * head_dim * 4 + 255) & ~size_t(255);
-  const size_t l = (rows * 4 + 255) & ~size_t(255);
-  return o + l;
+  return decode_ws(n_seq, q_heads, head_dim, max_splits).total;
 }
 
 // The decode step's inputs of the fused launch (qkv_decode_step_f4).
@@ -1110,11 +1273,14 @@ static int split_impl(float* o_parts, float* lse2_parts, int32_t max_splits, con
                       const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq, int32_t q_heads,
                       int32_t kv_heads, int32_t head_dim, int32_t block_size, int32_t max_pages_per_seq,
                       int64_t num_pages, float softmax_scale, int32_t num_splits, int32_t v_group,
-                      int32_t* device_status, qkv_stream_t stream, const StepArgs* step) {
+                      int32_t* device_status, qkv_stream_t stream, const StepArgs* step,
+                      uint16_t* fold_out = nullptr, float* fold_lse2 = nullptr,
+                      unsigned int* tickets = nullptr) {
   if (!o_parts || !lse2_parts || !q || !k_data || !k_scale || !v_data || !v_scale || !page_table || !seq_lens)
     return QKV_EINVAL;
   if (n_seq < 0 || q_heads < 1 || kv_heads < 1 || max_pages_per_seq < 1 || num_pages < 1 || max_splits < 1 ||
-      num_splits < 0 || block_size < 1 || !(softmax_scale >= 0.f) || !isfinite(softmax_scale) ||
+      num_splits < 0 || num_splits > max_splits || block_size < 1 || !(softmax_scale >= 0.f) ||
+      !isfinite(softmax_scale) ||
       (v_group != 32 && v_group != head_dim))
     return QKV_EINVAL;
   if (q_heads % kv_heads) return QKV_EINVAL;
@@ -1159,6 +1325,9 @@ static int split_impl(float* o_parts, float* lse2_parts, int32_t max_splits, con
   p.target = std::max(1, occ * sms / kv_heads);
   const float sc = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
   p.score_scale = sc * 1.4426950408889634f;
+  p.out = reinterpret_cast<__nv_bfloat16*>(fold_out);
+  p.lse2_final = fold_lse2;
+  p.tickets = tickets;
   KParams<true> pf;  // the fused instances' parameters: Params + the step's inputs
   static_cast<Params&>(pf) = p;
   if (step) {
@@ -1215,6 +1384,39 @@ extern "C" int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int3
                                      stream);
 }
 
+// a4 + a5 (+ a2 + a3 with step): the split pass into the workspace; its
+// partials folded inside the launch when max_splits * G is at most
+// QKV_DECODE_FOLD_MAX_ROWS, else by a merge launch.
+static int attn_impl(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
+                     const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
+                     const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq, int32_t q_heads,
+                     int32_t kv_heads, int32_t head_dim, int32_t block_size, int32_t max_pages_per_seq,
+                     int64_t num_pages, float softmax_scale, int32_t num_splits, int32_t max_splits, int32_t v_group,
+                     void* workspace, size_t workspace_bytes, int32_t* device_status, qkv_stream_t stream,
+                     const StepArgs* step) {
+  if (!out || !workspace) return QKV_EINVAL;
+  if (((uintptr_t)workspace & 255) || max_splits < 1 || n_seq < 0 || q_heads < 1 || kv_heads < 1 ||
+      head_dim < 1)
+    return QKV_EINVAL;
+  if (((uintptr_t)out & 3) || ((uintptr_t)lse2_out & 3)) return QKV_EINVAL;
+  const DecodeWs L = decode_ws(n_seq, q_heads, head_dim, max_splits);
+  if (workspace_bytes < L.total) return QKV_EINVAL;
+  if (n_seq == 0) return QKV_OK;
+  const size_t rows = (size_t)n_seq * q_heads;
+  char* ws = static_cast<char*>(workspace);
+  float* o_parts = reinterpret_cast<float*>(ws + L.o);
+  float* lse_parts = reinterpret_cast<float*>(ws + L.lse);
+  const bool fold = q_heads % kv_heads == 0 && (int64_t)max_splits * (q_heads / kv_heads) <= QKV_DECODE_FOLD_MAX_ROWS &&
+                    (int64_t)n_seq * kv_heads * 4 <= QKV_DECODE_FOLD_TICKET_BYTES;
+  int rc = split_impl(o_parts, lse_parts, max_splits, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens,
+                      n_seq, q_heads, kv_heads, head_dim, block_size, max_pages_per_seq, num_pages, softmax_scale,
+                      num_splits, v_group, device_status, stream, step, fold ? out : nullptr,
+                      fold ? lse2_out : nullptr,
+                      fold ? reinterpret_cast<unsigned int*>(ws + L.tickets) : nullptr);
+  if (rc != QKV_OK || fold) return rc;
+  return qkv_lse_merge(o_parts, lse_parts, max_splits, (int32_t)rows, head_dim, out, lse2_out, stream);
+}
+
 extern "C" int qkv_paged_decode_attn_f4_v(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
                                           const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
                                           const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
@@ -1222,20 +1424,28 @@ extern "C" int qkv_paged_decode_attn_f4_v(uint16_t* out, float* lse2_out, const 
                                           int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
                                           int32_t num_splits, int32_t max_splits, int32_t v_group, void* workspace,
                                           size_t workspace_bytes, int32_t* device_status, qkv_stream_t stream) {
-  if (!out || !workspace) return QKV_EINVAL;
-  if (((uintptr_t)workspace & 255) || max_splits < 1 || n_seq < 0 || q_heads < 1) return QKV_EINVAL;
-  if (workspace_bytes < qkv_paged_decode_workspace_bytes(n_seq, q_heads, head_dim, max_splits)) return QKV_EINVAL;
-  if (n_seq == 0) return QKV_OK;
-  const size_t rows = (size_t)n_seq * q_heads;
-  float* o_parts = reinterpret_cast<float*>(workspace);
-  float* lse_parts =
-      reinterpret_cast<float*>((char*)workspace + ((rows * max_splits * head_dim * 4 + 255) & ~size_t(255)));
-  int rc = qkv_paged_decode_split_f4_v(o_parts, lse_parts, max_splits, q, k_data, k_scale, v_data, v_scale,
-                                       page_table, seq_lens, n_seq, q_heads, kv_heads, head_dim, block_size,
-                                       max_pages_per_seq, num_pages, softmax_scale, num_splits, v_group,
-                                       device_status, stream);
-  if (rc != QKV_OK) return rc;
-  return qkv_lse_merge(o_parts, lse_parts, max_splits, (int32_t)rows, head_dim, out, lse2_out, stream);
+  return attn_impl(out, lse2_out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, n_seq, q_heads, kv_heads,
+                   head_dim, block_size, max_pages_per_seq, num_pages, softmax_scale, num_splits, max_splits, v_group,
+                   workspace, workspace_bytes, device_status, stream, nullptr);
+}
+
+extern "C" int qkv_decode_step_split_f4(float* o_parts, float* lse2_parts, int32_t max_splits, const uint16_t* q,
+                                        const uint16_t* k_new, const uint16_t* v_new, const int64_t* positions,
+                                        const int64_t* slot_mapping, const float* cos_tab, const float* sin_tab,
+                                        int64_t table_pos_start, int64_t table_len, int32_t rot_dim,
+                                        uint8_t* k_data, uint16_t* k_scale, uint8_t* v_data, uint16_t* v_scale,
+                                        const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq,
+                                        int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                        int32_t max_pages_per_seq, int64_t num_pages, float softmax_scale,
+                                        int32_t num_splits, int32_t v_group, int32_t* device_status,
+                                        qkv_stream_t stream) {
+  if (!k_new || !v_new || !positions || !slot_mapping || !cos_tab || !sin_tab) return QKV_EINVAL;
+  if (rot_dim < 16 || rot_dim % 16 || rot_dim > head_dim || table_len < 0) return QKV_EINVAL;
+  if (((uintptr_t)k_new | (uintptr_t)v_new) & 15) return QKV_EINVAL;
+  const StepArgs step = {k_new, v_new, positions, slot_mapping, cos_tab, sin_tab, table_pos_start, table_len, rot_dim};
+  return split_impl(o_parts, lse2_parts, max_splits, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, n_seq,
+                    q_heads, kv_heads, head_dim, block_size, max_pages_per_seq, num_pages, softmax_scale, num_splits,
+                    v_group, device_status, stream, &step);
 }
 
 extern "C" int qkv_decode_step_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint16_t* k_new,
@@ -1248,22 +1458,13 @@ extern "C" int qkv_decode_step_f4(uint16_t* out, float* lse2_out, const uint16_t
                                   float softmax_scale, int32_t num_splits, int32_t max_splits, int32_t v_group,
                                   void* workspace, size_t workspace_bytes, int32_t* device_status,
                                   qkv_stream_t stream) {
-  if (!out || !workspace || !k_new || !v_new || !positions || !slot_mapping || !cos_tab || !sin_tab) return QKV_EINVAL;
-  if (((uintptr_t)workspace & 255) || max_splits < 1 || n_seq < 0 || q_heads < 1) return QKV_EINVAL;
+  if (!k_new || !v_new || !positions || !slot_mapping || !cos_tab || !sin_tab) return QKV_EINVAL;
   if (rot_dim < 16 || rot_dim % 16 || rot_dim > head_dim || table_len < 0) return QKV_EINVAL;
   if (((uintptr_t)k_new | (uintptr_t)v_new) & 15) return QKV_EINVAL;
-  if (workspace_bytes < qkv_paged_decode_workspace_bytes(n_seq, q_heads, head_dim, max_splits)) return QKV_EINVAL;
-  if (n_seq == 0) return QKV_OK;
-  const size_t rows = (size_t)n_seq * q_heads;
-  float* o_parts = reinterpret_cast<float*>(workspace);
-  float* lse_parts =
-      reinterpret_cast<float*>((char*)workspace + ((rows * max_splits * head_dim * 4 + 255) & ~size_t(255)));
   const StepArgs step = {k_new, v_new, positions, slot_mapping, cos_tab, sin_tab, table_pos_start, table_len, rot_dim};
-  int rc = split_impl(o_parts, lse_parts, max_splits, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens,
-                      n_seq, q_heads, kv_heads, head_dim, block_size, max_pages_per_seq, num_pages, softmax_scale,
-                      num_splits, v_group, device_status, stream, &step);
-  if (rc != QKV_OK) return rc;
-  return qkv_lse_merge(o_parts, lse_parts, max_splits, (int32_t)rows, head_dim, out, lse2_out, stream);
+  return attn_impl(out, lse2_out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, n_seq, q_heads, kv_heads,
+                   head_dim, block_size, max_pages_per_seq, num_pages, softmax_scale, num_splits, max_splits, v_group,
+                   workspace, workspace_bytes, device_status, stream, &step);
 }
 
 extern "C" int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,

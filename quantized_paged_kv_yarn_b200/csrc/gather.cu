@@ -21,8 +21,8 @@ __global__ void __launch_bounds__(256) gather_kv_f4_kernel(
     const int32_t* __restrict__ seq_lens, const int64_t* __restrict__ out_start, int kv_heads, int head_dim,
     int block, int64_t num_pages, int v_group, int64_t n_out, uint16_t* __restrict__ k_out,
     uint16_t* __restrict__ v_out, int32_t* status) {
-  pdl_wait();
   pdl_release();
+  pdl_wait();
   const int s = blockIdx.y;
   const int cells = head_dim / 32;
   // thread -> (token t, head h, K or V, cell c), cells fastest

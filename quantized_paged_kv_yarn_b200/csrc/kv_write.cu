@@ -30,8 +30,7 @@ __global__ void __launch_bounds__(256) kv_write_f4_kernel(
     int n_tok, uint8_t* __restrict__ k_data, __half* __restrict__ k_scale, uint8_t* __restrict__ v_data,
     __half* __restrict__ v_scale, int kv_heads, int head_dim, int block, int64_t num_pages, int v_group,
     int32_t* status) {
-  pdl_wait();
-  pdl_release();
+  pdl_wait();  // writes the cache: no early start of its successor
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (item >= (int64_t)n_tok * kv_heads * 2) return;

@@ -14,11 +14,13 @@
 namespace qkv {
 
 // One CTA per (row, 64-dim chunk); 16 warps split the parts (warp w takes
-// parts w, w + 16, ...). A warp first loads the lse2 of up to 32 of its
-// parts with one load per lane, takes their max and weights, then issues the
-// loads of all those parts' 64-dim rows (2 dims per lane) before using them,
-// so a row costs two dependent global-latency rounds per 32 x 16 parts. The
-// warps' (max, weight sum, weighted sum) are combined in shared memory.
+// parts w, w + 16, ...). A warp loads the lse2 of up to 32 of its parts (one
+// per lane) together with the 64-dim rows (2 dims per lane) of the first 8 of
+// them, before their weights are known: the rows of parts without weight are
+// selected away, never multiplied, so whatever they hold is harmless. With
+// up to 8 parts per warp (128 per row) the fold costs one global-latency
+// round. The warps' (max, weight sum, weighted sum) are combined in shared
+// memory.
 constexpr int MERGE_WARPS = 16;
 constexpr int MERGE_THREADS = MERGE_WARPS * 32;
 constexpr int MERGE_DIMS = 64;
@@ -29,8 +31,8 @@ __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* _
                                                                   int n_parts, int rows, int head_dim,
                                                                   __nv_bfloat16* __restrict__ out,
                                                                   float* __restrict__ lse2_out) {
-  pdl_wait();
   pdl_release();
+  pdl_wait();
   __shared__ float wm[MERGE_WARPS], wsum[MERGE_WARPS];
   __shared__ float2 wacc[MERGE_WARPS][32];
   const int row = blockIdx.x;
@@ -44,6 +46,18 @@ __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* _
   for (int base = warp; base < n_parts; base += MERGE_WARPS * 32) {
     // lane j holds part base + 16 j of this round
     const int my = base + MERGE_WARPS * lane;
+    const int cnt = min(32, (n_parts - base + MERGE_WARPS - 1) / MERGE_WARPS);
+    auto load_rows = [&](int j0, float2 (&x)[MERGE_BATCH]) {
+#pragma unroll
+      for (int u = 0; u < MERGE_BATCH; ++u) {
+        const int j = j0 + u;
+        x[u] = make_float2(0.f, 0.f);
+        if (j < cnt && dim_ok)
+          x[u] = *reinterpret_cast<const float2*>(o_parts + ((size_t)(base + MERGE_WARPS * j) * rows + row) * head_dim + d);
+      }
+    };
+    float2 x[MERGE_BATCH];
+    load_rows(0, x);
     const float l = my < n_parts ? lse2_parts[(size_t)my * rows + row] : -INFINITY;
     float mr = l;
 #pragma unroll
@@ -60,23 +74,14 @@ __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* _
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsr += __shfl_xor_sync(FULL_MASK, wsr, o);
     ws += wsr;
-    const int cnt = min(32, (n_parts - base + MERGE_WARPS - 1) / MERGE_WARPS);
     for (int j0 = 0; j0 < cnt; j0 += MERGE_BATCH) {
-      float2 x[MERGE_BATCH];
-      float w[MERGE_BATCH];
+      if (j0 > 0) load_rows(j0, x);
 #pragma unroll
       for (int u = 0; u < MERGE_BATCH; ++u) {
-        const int j = j0 + u;
-        w[u] = __shfl_sync(FULL_MASK, wt, j & 31);
-        x[u] = make_float2(0.f, 0.f);
-        if (j < cnt && w[u] != 0.f && dim_ok)
-          x[u] = *reinterpret_cast<const float2*>(o_parts + ((size_t)(base + MERGE_WARPS * j) * rows + row) * head_dim + d);
-      }
-#pragma unroll
-      for (int u = 0; u < MERGE_BATCH; ++u) {
-        if (j0 + u < cnt) {
-          acc.x = fmaf(w[u], x[u].x, acc.x);
-          acc.y = fmaf(w[u], x[u].y, acc.y);
+        const float w = __shfl_sync(FULL_MASK, wt, (j0 + u) & 31);
+        if (j0 + u < cnt && w != 0.f) {
+          acc.x = fmaf(w, x[u].x, acc.x);
+          acc.y = fmaf(w, x[u].y, acc.y);
         }
       }
     }

@@ -42,8 +42,7 @@ __device__ double yarn_theta(const YarnDev& p, int j, double* mscale) {
 __global__ void __launch_bounds__(256) yarn_table_kernel(YarnDev p, int64_t pos_start, int64_t n_pos,
                                                          float* __restrict__ cos_out,
                                                          float* __restrict__ sin_out) {
-  pdl_wait();
-  pdl_release();
+  pdl_wait();  // the decode step reads the table before it waits: no early start of the successor
   __shared__ double s_theta[MAX_ROT_HALF];
   __shared__ double s_ms;
   const int half = p.rot / 2;
@@ -75,8 +74,8 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const __nv_bfloat16* x_
                                                          const float* __restrict__ sin_tab,
                                                          int64_t tab_start, int64_t tab_len,
                                                          int32_t* status) {
-  pdl_wait();
   pdl_release();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (item >= (int64_t)n_tok * n_heads) return;

@@ -24,8 +24,7 @@ __global__ void __launch_bounds__(256) rope_kv_write_kernel(
     int64_t tab_start, int64_t tab_len, uint8_t* __restrict__ k_data, __half* __restrict__ k_scale,
     uint8_t* __restrict__ v_data, __half* __restrict__ v_scale, int block, int64_t num_pages, int v_group,
     int32_t* status) {
-  pdl_wait();
-  pdl_release();
+  pdl_wait();  // writes the cache: no early start of its successor
   const int lane = threadIdx.x & 31;
   const int per_tok = q_heads + 2 * kv_heads;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);

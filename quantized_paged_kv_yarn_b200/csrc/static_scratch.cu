@@ -12,8 +12,14 @@
 // The array is a file-scope __device__ variable: every GPU that loads the
 // library holds QKV_STATIC_SCRATCH_BYTES of it until the process exits. In
 // host code its name is only a host-side handle, not a device address, so
-// the address is resolved with cudaGetSymbolAddress once per device (on the
-// first call made with that device current) and cached.
+// the address is resolved with cudaGetSymbolAddress on the first call made
+// with a device current, and cached for that device together with the
+// identity of its CUDA context. A later call under another context of the
+// device (after cudaDeviceReset, or once the primary context was released
+// and created again, the module and its array are loaded anew) resolves the
+// address again, and a failed launch drops the cached address.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -23,23 +29,66 @@ namespace {
 __device__ __align__(256) unsigned char g_static_scratch[QKV_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
+
+struct Resolved {
+  void* addr;               // device address of g_static_scratch
+  unsigned long long ctx;   // unique id of the context it belongs to
+};
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices];  // device address of g_static_scratch, per device
+Resolved g_scratch[kMaxDevices];
+
+using CtxGetCurrent = PFN_cuCtxGetCurrent_v4000;
+using CtxGetId = PFN_cuCtxGetId_v12000;
+
+// Unique id of the calling thread's current context (0 when it cannot be
+// read: the cached address is then never trusted).
+unsigned long long current_context_id() {
+  static CtxGetCurrent get_current = nullptr;
+  static CtxGetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of the array on the current device, or nullptr.
-void* static_scratch_address() {
-  int dev = -1;
+void* static_scratch_address(int& dev) {
+  dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  // cudaGetSymbolAddress makes the device's primary context current if none
+  // is; the context id is read after it
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
-      (void)cudaGetLastError();
-      return nullptr;
-    }
-    g_scratch_addr[dev] = p;
+  unsigned long long ctx = current_context_id();
+  Resolved& r = g_scratch[dev];
+  if (r.addr && ctx != 0 && r.ctx == ctx) return r.addr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+    (void)cudaGetLastError();
+    r = Resolved{nullptr, 0};
+    return nullptr;
   }
-  return g_scratch_addr[dev];
+  ctx = current_context_id();
+  r = Resolved{p, ctx};
+  return p;
+}
+
+void forget_static_scratch(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_scratch[dev] = Resolved{nullptr, 0};
 }
 
 }  // namespace
@@ -58,13 +107,17 @@ extern "C" int qkv_paged_decode_attn_f4_static(uint16_t* out, float* lse2_out, c
   if (max_splits < 1) return QKV_EUNSUPPORTED;
   const size_t need = qkv_paged_decode_workspace_bytes(n_seq, q_heads, head_dim, max_splits);
   if (need == 0 || need > (size_t)QKV_STATIC_SCRATCH_BYTES) return QKV_EINVAL;  // partials do not fit
-  void* scratch = static_scratch_address();
+  int dev = -1;
+  void* scratch = static_scratch_address(dev);
   if (!scratch) return QKV_ECUDA;
-  // Nothing in the array has to start at zero: the split pass writes the
-  // lse2 of every slot the merge reads, and the o row of every slot whose
-  // lse2 is finite.
-  return qkv_paged_decode_attn_f4(out, lse2_out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, n_seq,
-                                  q_heads, kv_heads, head_dim, block_size, max_pages_per_seq, num_pages,
-                                  softmax_scale, num_splits, max_splits, scratch, (size_t)QKV_STATIC_SCRATCH_BYTES,
-                                  device_status, stream);
+  // The array is zero when the library is loaded. The partials need no
+  // clearing (the split pass writes the lse2 of every slot it reads back, and
+  // the o row of every slot whose lse2 is finite); the fold's ticket
+  // counters must start at zero, and every call leaves them at zero.
+  const int rc = qkv_paged_decode_attn_f4(out, lse2_out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens,
+                                          n_seq, q_heads, kv_heads, head_dim, block_size, max_pages_per_seq,
+                                          num_pages, softmax_scale, num_splits, max_splits, scratch,
+                                          (size_t)QKV_STATIC_SCRATCH_BYTES, device_status, stream);
+  if (rc == QKV_ECUDA) forget_static_scratch(dev);  // the next call resolves the address again
+  return rc;
 }

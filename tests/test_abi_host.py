@@ -52,8 +52,19 @@ def test_status_strings(qkv):
 def test_workspace_bytes(qkv):
     n = qkv.qkv_paged_decode_workspace_bytes(3, 16, 256, 74)
     rows = 3 * 16 * 74
-    assert n == ((rows * 256 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    a = lambda x: (x + 255) // 256 * 256
+    assert n == 4096 + a(rows * 256 * 4) + a(rows * 4)   # fold tickets, o_parts, lse2_parts
     assert qkv.qkv_paged_decode_workspace_bytes(-1, 16, 256, 4) == 0
+
+
+def test_fold_limit_mirrors_header(qkv):
+    src = open(HEADER).read()
+    m = re.search(r"#define QKV_DECODE_FOLD_MAX_ROWS (\d+)", src)
+    assert m and int(m.group(1)) == qkv.DECODE_FOLD_MAX_ROWS
+    m = re.search(r"#define QKV_DECODE_FOLD_TICKET_BYTES (\d+)", src)
+    assert m and int(m.group(1)) == qkv.DECODE_FOLD_TICKET_BYTES
+    assert qkv.decode_folds(37, 1, 16, 4) and not qkv.decode_folds(148, 1, 16, 4)
+    assert not qkv.decode_folds(37, 257, 16, 4)
 
 
 FAKE = ctypes.c_void_p(4096)  # never dereferenced: validation fails first
@@ -89,6 +100,8 @@ def test_invalid_arguments_rejected_before_launch(qkv):
     assert L.qkv_paged_decode_split_f4(*args(16, 4, 256, 128)) == 2    # block 128
     assert L.qkv_paged_decode_split_f4(*args(16, 3, 256, 64)) == 1     # 16 % 3
     assert L.qkv_paged_decode_split_f4(*args(16, 4, 256, 64, 0)) == 1  # max_splits 0
+    a = list(args(16, 4, 256, 64, 4)); a[18] = 5                       # num_splits above max_splits
+    assert L.qkv_paged_decode_split_f4(*a) == 1
     a = list(args(16, 4, 256, 64)); a[3] = NUL
     assert L.qkv_paged_decode_split_f4(*a) == 1
     a = list(args(16, 4, 256, 64)); a[4] = ctypes.c_void_p(4100)       # cache not 16-byte aligned

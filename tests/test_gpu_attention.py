@@ -32,7 +32,9 @@ def _check_cache_equal(cache, ref):
 
 
 def _run_attn(qkv, w, x, cache, num_splits=0, max_splits=0, softmax_scale=0.0):
-    att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size, max_splits=max_splits)
+    # a fixed split count needs that many workspace slots
+    att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size,
+                              max_splits=max_splits or num_splits)
     out = torch.empty((w.n_seq, w.q_heads, w.head_dim), dtype=torch.int16, device="cuda")
     lse = torch.empty((w.n_seq, w.q_heads), dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -133,13 +135,20 @@ def test_split_partials_match_oracle_ranges(qkv, num_splits, v_group):
         assert np.max(np.abs(l_parts[i][fin] - rl[fin]), initial=0.0) <= 2e-4
 
 
-def test_lse_merge_matches_oracle(qkv):
-    rng = np.random.default_rng(21)
-    n, rows, d = 37, 48, 256
+# part counts: the automatic plan's 37 on a B200, the 1M-token workload's 148
+# (>= 128 weighted parts per row), and 600, past the merge's first round of
+# 512 parts (16 warps x 32 lanes) into its second
+@pytest.mark.parametrize("n", [37, 148, 600])
+def test_lse_merge_matches_oracle(qkv, n):
+    rng = np.random.default_rng(21 + n)
+    rows, d = 48, 256
     o = rng.standard_normal((n, rows, d)).astype(np.float32)
     l = (rng.standard_normal((n, rows)) * 30).astype(np.float32)
     l[rng.random((n, rows)) < 0.2] = -np.inf
     l[:, 5] = -np.inf                     # a row without any weighted part
+    if n > 512:
+        l[:512, 7] = -np.inf              # weighted parts only in the second round
+        l[600 - 3, 9] = 400.0             # the row's maximum in the second round
     o[np.isinf(l)] = np.nan               # unweighted parts are never read
     out = torch.empty((rows, d), dtype=torch.int16, device="cuda")
     lo = torch.empty(rows, dtype=torch.float32, device="cuda")
@@ -153,6 +162,45 @@ def test_lse_merge_matches_oracle(qkv):
     fin = np.isfinite(ref_l)
     assert np.max(np.abs(lo[fin] - ref_l[fin])) <= 1e-5 * np.max(np.abs(ref_l[fin]))
     assert np.all(got[5] == 0)
+    # rows with at least 128 weighted parts are covered at n >= 148
+    assert np.max(np.isfinite(l).sum(0)) >= min(n, 128) * 0.7
+
+
+def test_split_count_above_workspace_refused(qkv):
+    """A fixed split count larger than the workspace's split slots is an
+    argument error, never silently reduced."""
+    w = workloads.small("toomany", seq_lens=(640,), num_pages=10, block_size=64)
+    x, _ = oracle_layer(w)
+    cache = _dev_cache(qkv, w, x)
+    att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size, max_splits=4)
+    out = torch.empty((w.n_seq, w.q_heads, w.head_dim), dtype=torch.int16, device="cuda")
+    with pytest.raises(qkv.QkvError) as e:
+        att(out, to_dev(x["q"]), cache, to_dev(x["page_table"]), to_dev(x["seq_lens"]), num_splits=5)
+    assert e.value.code == 1
+
+
+@pytest.mark.parametrize("v_group", [32, 256])
+def test_148_splits_all_weighted(qkv, v_group):
+    """The 1M-token workload's plan shape at a size the oracle finishes: 148
+    splits of every sequence, each holding pages (so every query row merges
+    148 weighted parts), checked part by part and after the merge."""
+    S = 148
+    w = workloads.small("s148", seq_lens=(S * 2 * 64 - 17, S * 64 + 5), num_pages=S * 3 + 1, block_size=64,
+                        head_scale=True, page_alloc="interleaved", k_outlier_frac=0.01)
+    x, ref = oracle_layer(w, v_group=v_group)
+    cache = _dev_cache(qkv, w, x, v_group=v_group)
+    att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size, max_splits=S)
+    out = torch.empty((w.n_seq, w.q_heads, w.head_dim), dtype=torch.int16, device="cuda")
+    lse = torch.empty((w.n_seq, w.q_heads), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    att(out, to_dev(x["q"]), cache, to_dev(x["page_table"]), to_dev(x["seq_lens"]), lse2_out=lse, num_splits=S,
+        device_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    _, l_parts = att.partials(w.n_seq, w.q_heads, w.head_dim)
+    assert np.all(np.isfinite(to_host(l_parts)).sum(0) == S)
+    ref_out, ref_lse = _oracle_attn(w, x, ref)
+    _assert_close(to_host(out, np.uint16), to_host(lse), ref_out, ref_lse)
 
 
 def test_page_permutation_invariance_gpu(qkv):
@@ -242,3 +290,6 @@ def test_workspace_reuse_across_calls(qkv):
         assert int(st.item()) == 0
         ref_out, ref_lse = _oracle_attn(w, x, ref)
         _assert_close(to_host(out, np.uint16), to_host(lse), ref_out, ref_lse)
+        # the in-launch fold left its ticket counters at zero for the next call
+        assert qkv.decode_folds(16, w.n_seq, w.q_heads, w.kv_heads)
+        assert int(att.workspace[:qkv.DECODE_FOLD_TICKET_BYTES].count_nonzero()) == 0

@@ -42,12 +42,21 @@ def test_fullsize_layer0(qkv, name):
     qkv.qkv_rope_kv_write_f4(x["q"], q_rot, x["k_new"], x["v_new"], x["positions"], x["step_slots"], cos, sin, p0,
                              w.rot_dim, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale, k_out=k_rot,
                              device_status=st)
-    att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size)
+    # the workload's own split plan: a fixed count sizes the workspace (148 at
+    # 1,048,576 tokens), otherwise the automatic plan
+    att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size, max_splits=w.num_splits)
     out = torch.empty_like(x["q"])
     lse = torch.empty((w.n_seq, w.q_heads), dtype=torch.float32, device=dev)
     att(out, q_rot, cache, x["page_table"], x["seq_lens"], lse2_out=lse, num_splits=w.num_splits, device_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
+    _, l_parts = att.partials(w.n_seq, w.q_heads, w.head_dim)
+    weighted = np.isfinite(to_host(l_parts)).sum(0)       # parts merged per query row
+    if w.num_splits:
+        assert att.max_splits == w.num_splits
+        assert np.all(weighted == w.num_splits), weighted
+    else:
+        assert np.all(weighted >= 1)
 
     # oracle: the same generated inputs, on the host
     h = {k: to_host(v, np.uint16) if v.dtype == torch.int16 else to_host(v)

@@ -41,7 +41,8 @@ def _both(qkv, w, x, v_group, spec, num_splits=0, positions=None, slots=None, ta
         cache = qkv.PagedF4Cache.allocate(w.num_pages, w.kv_heads, w.block_size, w.head_dim, v_group=v_group)
         cache.write(to_dev(x["k_cache"]), to_dev(x["v_cache"]), to_dev(x["cache_slots"]))
         caches.append(cache)
-    att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size, max_splits=40)
+    att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size,
+                              max_splits=max(40, num_splits))
     outs = []
     # two calls
     st = torch.zeros(1, dtype=torch.int32, device="cuda")

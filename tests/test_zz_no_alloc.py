@@ -4,16 +4,19 @@ Some callers can't call cudaMalloc -- a plugin running inside a host engine
 that owns all device memory, or a runtime whose memory budget is fixed at
 start-up -- so they cannot hand the library a partials workspace.
 qkv_paged_decode_attn_f4_static keeps the partials in an array compiled into
-the library instead. These tests call it through the C ABI and check it
-against the workspace entry point, twice in a row on different inputs (the
-array keeps the previous call's contents), and check that a problem too large
-for the array is refused."""
+the library instead. These tests call it through the C ABI: twice in a row
+on one stream with different inputs (the array keeps the previous call's
+contents), each call bit-identical to the workspace entry point on the same
+inputs (same kernels, same split plan) and within the attention tolerance
+of the fp64 oracle; with no device memory allocated by the calls; and a
+problem too large for the array is refused."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
-from helpers import attn_within, to_dev, to_host
+from helpers import attn_within, oracle_layer, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -24,12 +27,12 @@ def qkv():
     return q
 
 
-def _inputs(qkv, w):
-    x = workloads.host_layer(w)
+def _cache(qkv, w):
+    x, ref = oracle_layer(w)
     cache = qkv.PagedF4Cache.allocate(w.num_pages, w.kv_heads, w.block_size, w.head_dim)
     cache.write(to_dev(x["k_cache"]), to_dev(x["v_cache"]), to_dev(x["cache_slots"]))
     cache.write(to_dev(x["k_new"]), to_dev(x["v_new"]), to_dev(x["step_slots"]))
-    return x, cache
+    return x, ref, cache
 
 
 def _outputs(w):
@@ -38,41 +41,72 @@ def _outputs(w):
     return out, lse
 
 
+def _free_device_bytes():
+    free, _ = torch.cuda.mem_get_info()
+    return free
+
+
 CALLS = [
     workloads.small("noalloc_a", seq_lens=(3000, 1000, 17), num_pages=80, block_size=64, head_scale=True),
     workloads.small("noalloc_b", seq_lens=(5000,), num_pages=320, block_size=16, q_heads=8, kv_heads=4, seed=7),
 ]
 
 
-def test_static_scratch_matches_workspace_entry_point(qkv):
-    for w in CALLS:  # two calls in a row through the shared array
-        x, cache = _inputs(qkv, w)
-        q, pt, sl = to_dev(x["q"]), to_dev(x["page_table"]), to_dev(x["seq_lens"])
-        st = torch.zeros(1, dtype=torch.int32, device="cuda")
-
-        ref_out, ref_lse = _outputs(w)
-        att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size)
-        att(ref_out, q, cache, pt, sl, lse2_out=ref_lse, device_status=st)
-
+def test_static_scratch_two_calls_match_workspace_and_oracle(qkv):
+    prepared = []
+    for w in CALLS:
+        x, ref, cache = _cache(qkv, w)
+        dev = {k: to_dev(x[k]) for k in ("q", "page_table", "seq_lens")}
         out, lse = _outputs(w)
         out.fill_(-1)
         lse.fill_(float("nan"))
-        qkv.qkv_paged_decode_attn_f4_static(out, q, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale, pt,
-                                            sl, w.kv_heads, lse2_out=lse, device_status=st)
+        prepared.append((w, x, ref, cache, dev, out, lse))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def both_calls():
+        # the two calls back to back on one stream, one synchronisation after them
+        for w, x, ref, cache, dev, out, lse in prepared:
+            qkv.qkv_paged_decode_attn_f4_static(out, dev["q"], cache.k_data, cache.k_scale, cache.v_data,
+                                                cache.v_scale, dev["page_table"], dev["seq_lens"], w.kv_heads,
+                                                lse2_out=lse, device_status=st)
+        torch.cuda.synchronize()
+
+    # the first round also loads the library's kernels and its array onto the
+    # device (module loading is the driver's, not the call's); the second
+    # round must leave device memory exactly as it found it
+    both_calls()
+    for *_, out, lse in prepared:
+        out.fill_(-1)
+        lse.fill_(float("nan"))
+    torch.cuda.synchronize()
+    alloc0, free0 = torch.cuda.memory_allocated(), _free_device_bytes()
+    both_calls()
+    assert int(st.item()) == 0
+    assert torch.cuda.memory_allocated() == alloc0
+    assert _free_device_bytes() == free0
+
+    for w, x, ref, cache, dev, out, lse in prepared:
+        # the workspace entry point with the same split plan (automatic, same slot count)
+        att = qkv.DecodeAttention(w.n_seq, w.q_heads, w.kv_heads, w.head_dim, w.block_size)
+        ref_out, ref_lse = _outputs(w)
+        att(ref_out, dev["q"], cache, dev["page_table"], dev["seq_lens"], lse2_out=ref_lse, device_status=st)
         torch.cuda.synchronize()
         assert int(st.item()) == 0
-
-        ref = workloads.bf16_bits_to_f32(to_host(ref_out, np.uint16)).astype(np.float64)
-        err, bound = attn_within(to_host(out, np.uint16), ref)
+        assert torch.equal(out, ref_out), w.name
+        assert torch.equal(lse.view(torch.int32), ref_lse.view(torch.int32)), w.name
+        # and the fp64 oracle
+        ro, rl = oracle.paged_attention(x["q"], ref, x["page_table"], np.zeros(w.n_seq, np.int32), x["seq_lens"],
+                                        w.q_heads, w.kv_heads, w.head_dim, w.block_size)
+        err, bound = attn_within(to_host(out, np.uint16), ro)
         assert np.all(err <= bound), f"{w.name}: max err {err.max():.3e}"
-        got_l, ref_l = to_host(lse), to_host(ref_lse)
+        got_l = to_host(lse)
         assert np.all(np.isfinite(got_l))
-        assert np.max(np.abs(got_l - ref_l)) <= 2e-4
+        assert np.max(np.abs(got_l - rl)) <= 2e-4
 
 
 def test_static_scratch_refuses_oversize(qkv):
     w = workloads.small("noalloc_big", seq_lens=(64,) * 4, num_pages=8, block_size=64)
-    x, cache = _inputs(qkv, w)
+    x, _, cache = _cache(qkv, w)
     out, lse = _outputs(w)
     need = qkv.qkv_paged_decode_workspace_bytes(w.n_seq, w.q_heads, w.head_dim, 400)
     assert need > qkv.STATIC_SCRATCH_BYTES
