@@ -320,9 +320,7 @@ class Bench:
                                        max_splits=w.num_splits)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.two_call = two_call
-        # the split launch merges its own partials unless the plan is too wide (then a merge launch follows)
-        self.folds = qkv.decode_folds(self.att.max_splits, w.n_seq, w.q_heads, w.kv_heads)
-        self.launches_per_step = 1 + ((2 if two_call else 1) + (0 if self.folds else 1)) * self.L
+        self.launches_per_step = 1 + (3 if two_call else 2) * self.L
         # host side of the end-to-end measurement (pinned)
         self.h_q = [t.cpu().pin_memory() for t in self.q_raw]
         self.h_kn = [t.cpu().pin_memory() for t in self.kn_raw]
@@ -373,8 +371,7 @@ class Bench:
         return g
 
     def split_kernel_ms(self, rounds: int):
-        """Average duration of the split-pass kernel as the step runs it (with
-        its partials folded in the launch when the plan allows, else alone):
+        """Average duration of the split-pass kernel as the step runs it:
         CUDA events on its stream around `rounds` passes over the layers'
         caches (each cache is larger than L2, so every launch reads HBM),
         launched back to back as in the step; also the per-launch times with
@@ -389,15 +386,7 @@ class Bench:
 
         def launch(l):
             c = self.caches[l]
-            if self.folds:  # one launch: the split pass with its fold
-                if self.two_call:
-                    self.att(self.out[l], self.q_rot[l], c, self.page_table, self.seq_lens,
-                             num_splits=w.num_splits)
-                else:
-                    self.att.step(self.out[l], self.q_raw[l], self.kn_raw[l], self.vn[l], self.positions,
-                                  self.step_slots, self.cos, self.sin, self.pos0, w.rot_dim, c, self.page_table,
-                                  self.seq_lens, num_splits=w.num_splits)
-            elif self.two_call:
+            if self.two_call:
                 qkv.qkv_paged_decode_split_f4(o_parts, l_parts, self.q_rot[l], c.k_data, c.k_scale, c.v_data,
                                               c.v_scale, self.page_table, self.seq_lens, w.kv_heads,
                                               num_splits=w.num_splits)
@@ -502,7 +491,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_value = whole_job_gbps(step_bytes, ms_e2e, world)
     peak, peak_kind = hbm_peak()
     out_bytes = 2 * w.n_seq * w.q_heads * w.head_dim
-    split_bytes = per_layer if b.folds else per_layer - out_bytes  # without the fold the merge writes out
+    split_bytes = per_layer - out_bytes  # the merge writes out
     achieved = split_bytes / (split_ms_mean * 1e-3) / 1e9
     traffic = profiled_traffic(w.name)
     bi, bo = b.io_bytes()
@@ -518,8 +507,7 @@ def run_ours(args, rank, world, local_rank):
         "device_status": status,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "paged_decode_split_kernel" + ("" if args.two_call else " (decode-step instance)")
-                               + (", partials folded in the launch" if b.folds else ""),
+                     "kernel": "paged_decode_split_kernel" + ("" if args.two_call else " (decode-step instance)"),
                      "peak_kind": f"{peak_kind} (copy bandwidth)",
                      "kernel_ms": split_ms_mean, "kernel_ms_isolated": split_ms_each,
                      "timing": "CUDA events around back-to-back launches over the layers' caches",

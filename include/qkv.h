@@ -200,15 +200,9 @@ QKV_API int qkv_rope_kv_write_f4_v(const uint16_t* q_in, uint16_t* q_out, const 
  * CUDA device is present. */
 QKV_API int32_t qkv_paged_decode_auto_splits(int32_t kv_heads, int32_t block_size);
 
-/* Bytes of the fold's ticket counters at the start of a decode workspace:
- * one 32-bit counter per (sequence, KV head), so a fold needs
- * n_seq * kv_heads <= 1024. */
-#define QKV_DECODE_FOLD_TICKET_BYTES 4096
-
-/* Bytes of workspace qkv_paged_decode_attn_f4 needs:
- * QKV_DECODE_FOLD_TICKET_BYTES of ticket counters, max_splits * n_seq *
- * q_heads * head_dim floats (o_parts) and max_splits * n_seq * q_heads
- * floats (lse2_parts), each part rounded up to 256 bytes. */
+/* Bytes of workspace qkv_paged_decode_attn_f4 needs: max_splits *
+ * n_seq * q_heads * head_dim floats (o_parts) and max_splits * n_seq *
+ * q_heads floats (lse2_parts), each rounded up to 256 bytes. */
 QKV_API size_t qkv_paged_decode_workspace_bytes(int32_t n_seq, int32_t q_heads, int32_t head_dim,
                                         int32_t max_splits);
 
@@ -271,29 +265,15 @@ QKV_API int qkv_paged_decode_split_f4_v(float* o_parts, float* lse2_parts, int32
 QKV_API int qkv_lse_merge(const float* o_parts, const float* lse2_parts, int32_t n_parts, int32_t rows,
                   int32_t head_dim, uint16_t* out, float* lse2_out, qkv_stream_t stream);
 
-/* Largest max_splits * (q_heads / kv_heads) for which the decode attention
- * folds the split partials inside the split launch (the last CTA of each
- * (sequence, KV head) to finish merges them, when also n_seq * kv_heads * 4
- * <= QKV_DECODE_FOLD_TICKET_BYTES); otherwise a merge launch follows. */
-#define QKV_DECODE_FOLD_MAX_ROWS 320
-
 /* a4 + a5: the decode attention of one layer. Runs the split pass into
  * `workspace` (see qkv_paged_decode_workspace_bytes) and merges it into
- * `out` (bf16 [n_seq][q_heads][head_dim], 4-byte aligned) and `lse2_out`
- * (float [n_seq][q_heads] or NULL), with the arithmetic of qkv_lse_merge:
- * in the split launch itself when max_splits * (q_heads / kv_heads) <=
- * QKV_DECODE_FOLD_MAX_ROWS and n_seq * kv_heads * 4 <=
- * QKV_DECODE_FOLD_TICKET_BYTES (one launch), else by a qkv_lse_merge launch.
- * Arguments and errors as in the two calls; EINVAL also when workspace_bytes
- * is too small or workspace is not 256-byte aligned. The workspace starts
- * with the fold's ticket counters (QKV_DECODE_FOLD_TICKET_BYTES); after the
- * call it holds the split pass's o_parts (float [max_splits][n_seq *
- * q_heads][head_dim], from offset QKV_DECODE_FOLD_TICKET_BYTES) and
- * lse2_parts (float [max_splits][n_seq * q_heads], from the next 256-byte
- * boundary). The counters must be zero before the first call with a
- * workspace (zero-fill it once); every call, aborted ones included, leaves
- * them at zero, whatever its shapes. Calls that overlap on the GPU must not
- * share a workspace.
+ * `out` (bf16 [n_seq][q_heads][head_dim]) and `lse2_out` (float
+ * [n_seq][q_heads] or NULL). Arguments and errors as in the two calls;
+ * EINVAL also when workspace_bytes is too small or workspace is not
+ * 256-byte aligned. After the call the workspace holds the split pass's
+ * o_parts (float [max_splits][n_seq * q_heads][head_dim], from offset 0)
+ * and lse2_parts (float [max_splits][n_seq * q_heads], from the next
+ * 256-byte boundary); it needs no initialisation.
  * Programmatic dependent launch: the split launch may start while the
  * kernel ahead of it in the stream still runs (when that kernel allows
  * it), and reads the page table, the sequence lengths and the cache pages
@@ -310,9 +290,8 @@ QKV_API int qkv_paged_decode_attn_f4(uint16_t* out, float* lse2_out, const uint1
                              void* workspace, size_t workspace_bytes, int32_t* device_status,
                              qkv_stream_t stream);
 
-/* One decode step of a layer: a2 + a3 + a4 in the split launch, a5 in it
- * too or in a merge launch (as in qkv_paged_decode_attn_f4). The split
- * kernel rotates each sequence's q itself (NEOX on
+/* One decode step of a layer in two launches: a2 + a3 + a4 in the split
+ * pass, then a5. The split kernel rotates each sequence's q itself (NEOX on
  * the first rot_dim dims, rounded to bf16 as qkv_rope_apply rounds), and the
  * CTA whose split holds a sequence's last page first writes the step's new
  * k (rotated) and v into the cache at slot_mapping[s] (F4, as
@@ -472,11 +451,9 @@ QKV_API int32_t qkv_paged_prefill_auto_splits(int32_t n_q, int32_t prefix_len, i
  *     outside capture as well; a call whose launch fails drops the cached
  *     address.
  *   - Every call on a device shares the one array and it keeps the last
- *     call's contents. It is zero when the library is loaded; the ticket
- *     counters of the in-launch fold must be zero before a call and every
- *     call leaves them at zero. Calls whose kernels overlap on the GPU -- on
- *     different streams, or from different host threads -- race on it:
- *     order them on one stream. */
+ *     call's contents (nothing in it needs to start at zero). Calls whose
+ *     kernels overlap on the GPU -- on different streams, or from different
+ *     host threads -- race on it: order them on one stream. */
 QKV_API int qkv_paged_decode_attn_f4_static(uint16_t* out, float* lse2_out, const uint16_t* q,
                                             const uint8_t* k_data, const uint16_t* k_scale,
                                             const uint8_t* v_data, const uint16_t* v_scale,

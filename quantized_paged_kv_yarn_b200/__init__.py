@@ -29,9 +29,6 @@ from ._abi import (  # noqa: F401
     qkv_paged_decode_attn_f4_tiered,
     qkv_paged_decode_tiered_workspace_bytes,
     STATIC_SCRATCH_BYTES,
-    DECODE_FOLD_MAX_ROWS,
-    DECODE_FOLD_TICKET_BYTES,
-    decode_folds,
     qkv_paged_decode_auto_splits,
     qkv_paged_decode_split_f4,
     qkv_paged_decode_workspace_bytes,

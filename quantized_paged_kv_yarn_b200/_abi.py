@@ -325,8 +325,7 @@ def qkv_decode_step_f4(out, q, k_new, v_new, positions, slot_mapping, cos_tab, s
                        max_splits: int, lse2_out=None, softmax_scale: float = 0.0, num_splits: int = 0,
                        device_status=None, stream=None):
     """One layer's decode step (rotary, F4 write of the new k/v, attention,
-    merge) in one launch (two when the partials are merged by a launch of their
-    own, see QKV_DECODE_FOLD_MAX_ROWS); q unrotated. Shapes as in qkv_rope_kv_write_f4
+    merge) in two launches; q unrotated. Shapes as in qkv_rope_kv_write_f4
     and qkv_paged_decode_attn_f4."""
     n_seq, q_heads, head_dim = q.shape
     num_pages, _, block_size, _ = k_data.shape
@@ -368,15 +367,6 @@ def qkv_decode_step_split_f4(o_parts, lse2_parts, q, k_new, v_new, positions, sl
 
 
 STATIC_SCRATCH_BYTES = 16 << 20
-DECODE_FOLD_MAX_ROWS = 320  # QKV_DECODE_FOLD_MAX_ROWS
-DECODE_FOLD_TICKET_BYTES = 4096  # QKV_DECODE_FOLD_TICKET_BYTES
-
-
-def decode_folds(max_splits: int, n_seq: int, q_heads: int, kv_heads: int) -> bool:
-    """Whether the decode attention merges its partials inside the split
-    launch (else a merge launch follows)."""
-    return (max_splits * (q_heads // kv_heads) <= DECODE_FOLD_MAX_ROWS
-            and n_seq * kv_heads * 4 <= DECODE_FOLD_TICKET_BYTES)
 
 
 def qkv_paged_decode_attn_f4_static(out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens, kv_heads: int,

@@ -71,8 +71,7 @@ class DecodeAttention:
         self.kv_heads = kv_heads
         self.max_splits = max_splits or max(1, _abi.qkv_paged_decode_auto_splits(kv_heads, block_size))
         nbytes = _abi.qkv_paged_decode_workspace_bytes(n_seq, q_heads, head_dim, self.max_splits)
-        # zero-filled once: the fold's ticket counters start at zero (calls leave them so)
-        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
 
     def partials(self, n_seq: int, q_heads: int, head_dim: int):
         """Views of the workspace as the split pass leaves it after a call:
@@ -80,9 +79,8 @@ class DecodeAttention:
         float [max_splits][n_seq * q_heads] (-inf for a split slot that held
         no tokens), the layout include/qkv.h gives for the workspace."""
         rows = n_seq * q_heads * self.max_splits
-        o0 = _abi.DECODE_FOLD_TICKET_BYTES
-        l0 = o0 + (rows * head_dim * 4 + 255) // 256 * 256
-        o = self.workspace[o0:o0 + rows * head_dim * 4].view(torch.float32)
+        l0 = (rows * head_dim * 4 + 255) // 256 * 256
+        o = self.workspace[:rows * head_dim * 4].view(torch.float32)
         lse = self.workspace[l0:l0 + rows * 4].view(torch.float32)
         return o.view(self.max_splits, n_seq * q_heads, head_dim), lse.view(self.max_splits, n_seq * q_heads)
 
@@ -90,8 +88,7 @@ class DecodeAttention:
              rot_dim: int, cache: PagedF4Cache, page_table, seq_lens, lse2_out=None, softmax_scale=0.0,
              num_splits=0, device_status=None, stream=None):
         """The layer's whole decode step (rotary, F4 write of the new token,
-        attention, merge) in one launch (two when the partials need a merge
-        launch); q unrotated."""
+        attention, merge) in two launches; q unrotated."""
         _abi.qkv_decode_step_f4(out, q, k_new, v_new, positions, slot_mapping, cos_tab, sin_tab, table_pos_start,
                                 rot_dim, cache.k_data, cache.k_scale, cache.v_data, cache.v_scale, page_table,
                                 seq_lens, self.kv_heads, self.workspace, self.max_splits, lse2_out=lse2_out,

@@ -109,7 +109,6 @@ struct __align__(1024) Smem {
   float gl[GROUPS][8];            // per group and head: softmax sum
   int next;                       // next stage of the split to claim
   int abort_flag;
-  int fold_last;                  // this CTA took the last ticket of its (sequence, KV head)
 };
 template <int HQ>
 constexpr size_t smem_bytes() {
@@ -128,13 +127,6 @@ struct Params {
   int64_t num_pages;
   int n_seq, q_heads, kv_heads, max_pages, max_splits, num_splits, target;
   float score_scale;  // softmax_scale * log2(e)
-  // Fold of the partials inside the launch (null out: the caller merges):
-  // the last CTA of each (sequence, KV head) to finish, found by a ticket
-  // counter per (sequence, KV head), merges its splits' partials into out /
-  // lse2_final.
-  __nv_bfloat16* out;
-  float* lse2_final;
-  unsigned int* tickets;  // [n_seq * kv_heads], zero between launches
 };
 // The decode step's inputs (qkv_decode_step_f4): q is unrotated; the kernel
 // rotates it and writes the step's new K (rotated) and V into the cache
@@ -238,102 +230,6 @@ __device__ __forceinline__ int muldiv(uint32_t a, uint32_t b, uint32_t c) {
   return (ab >> 32) == 0 ? (int)((uint32_t)ab / c) : (int)(ab / c);
 }
 
-// Ticket of a CTA that has written its partial: true for the last of the
-// S CTAs of its (sequence, KV head). The counter is zero before the launch
-// and the last CTA sets it back to zero for the next one. One atomic add
-// per CTA (a compare-and-swap loop here serialised the CTAs that finish
-// together: ~16 us at 37 splits).
-__device__ __forceinline__ bool take_ticket(unsigned int* counter, int S) {
-  const unsigned int old = atomicAdd(counter, 1u);
-  const bool last = old + 1u == (unsigned int)S;
-  if (last) atomicExch(counter, 0u);
-  return last;
-}
-
-// The fold of the S partials (o, lse2) of the G query rows row0 .. row0 +
-// G - 1 into bf16 out and lse2_out, by the last CTA of a (sequence, KV
-// head): the merge qkv_lse_merge computes (M = max lse2, weights 2^(lse2 -
-// M), out = sum w o / sum w, lse2 = M + log2 sum w). All THREADS threads
-// call it; sbuf is idle shared memory of at least fold_smem_floats(S, G).
-// Thread (slice sl, element e) sums parts sl, sl + SL, ... of float4 e of
-// the G rows; the first rows' loads are in flight with the lse2 loads.
-constexpr int FOLD_MAX_ROWS = QKV_DECODE_FOLD_MAX_ROWS;  // S * G
-template <int G>
-__device__ __noinline__ void fold_parts(const float* o_parts, const float* lse_parts, int rows, int row0, int S,
-                                        __nv_bfloat16* out, float* lse2_out, float* sbuf) {
-  constexpr int NV = G * (D / 4);   // float4 of one part's G rows
-  constexpr int SL = THREADS / NV;  // slices of the parts
-  constexpr int B = 8;              // part rows in flight per thread
-  const int e = threadIdx.x % NV, sl = threadIdx.x / NV;
-  const int h = e / (D / 4), d4 = e % (D / 4);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float* ls = sbuf;                                               // [S][G]: lse2, then weights
-  float* mh = sbuf + FOLD_MAX_ROWS;                               // [G] max lse2
-  float4* accs = reinterpret_cast<float4*>(sbuf + FOLD_MAX_ROWS + 8);  // [SL][NV]
-  const int mine = (S - sl + SL - 1) / SL;  // parts sl + SL k, k < mine
-  float4 x[B];
-  auto load = [&](int k0) {
-#pragma unroll
-    for (int u = 0; u < B; ++u) {
-      x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (k0 + u < mine)
-        x[u] = __ldcg(reinterpret_cast<const float4*>(o_parts + ((size_t)(sl + SL * (k0 + u)) * rows + row0 + h) * D) +
-                      d4);
-    }
-  };
-  load(0);
-  for (int j = threadIdx.x; j < S * G; j += THREADS) ls[j] = __ldcg(lse_parts + (size_t)(j / G) * rows + row0 + j % G);
-  __syncthreads();
-  if (warp < G) {  // warp h: the max of head h's lse2
-    float m = -INFINITY;
-    for (int i = lane; i < S; i += 32) m = fmaxf(m, ls[i * G + warp]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, o));
-    if (lane == 0) mh[warp] = m;
-  }
-  __syncthreads();
-  for (int j = threadIdx.x; j < S * G; j += THREADS) {
-    const float l = ls[j];
-    ls[j] = l == -INFINITY ? 0.f : exp2f(l - mh[j % G]);
-  }
-  __syncthreads();
-  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int k0 = 0; k0 < mine; k0 += B) {
-    if (k0 > 0) load(k0);
-#pragma unroll
-    for (int u = 0; u < B; ++u) {
-      if (k0 + u < mine) {
-        const float w = ls[(sl + SL * (k0 + u)) * G + h];
-        if (w != 0.f) {  // a part without weight may hold anything
-          a.x = fmaf(w, x[u].x, a.x);
-          a.y = fmaf(w, x[u].y, a.y);
-          a.z = fmaf(w, x[u].z, a.z);
-          a.w = fmaf(w, x[u].w, a.w);
-        }
-      }
-    }
-  }
-  accs[sl * NV + e] = a;
-  __syncthreads();
-  if (sl == 0) {
-#pragma unroll
-    for (int s2 = 1; s2 < SL; ++s2) {
-      const float4 b = accs[s2 * NV + e];
-      a.x += b.x;
-      a.y += b.y;
-      a.z += b.z;
-      a.w += b.w;
-    }
-    float W = 0.f;
-    for (int i = 0; i < S; ++i) W += ls[i * G + h];
-    const float inv = W > 0.f ? 1.f / W : 0.f;
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + (size_t)(row0 + h) * D + 4 * d4);
-    dst[0] = __floats2bfloat162_rn(a.x * inv, a.y * inv);
-    dst[1] = __floats2bfloat162_rn(a.z * inv, a.w * inv);
-    if (d4 == 0 && lse2_out) lse2_out[row0 + h] = W > 0.f ? mh[h] + log2f(W) : -INFINITY;
-  }
-}
-
 // Split plan. Fixed: num_splits splits per sequence (the host refuses a
 // count above max_splits).
 // Automatic: pages are cut into pieces of about total pages / target, so the
@@ -388,8 +284,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   constexpr int VCELLS = VTOK ? 1 : CELLS;
   using SmemT = Smem<HQ>;
 
-  extern __shared__ uint8_t smem_raw[];
-  SmemT& sm = *reinterpret_cast<SmemT*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-aligned (the 128-byte swizzle atom) by pointer arithmetic on the
+  // shared array itself, so the compiler keeps every access through `sm` in
+  // the shared window (32-bit addresses, shared loads) instead of generic
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  SmemT& sm = *reinterpret_cast<SmemT*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
 
   // Programmatic dependent launch. The kernel lets its successor launch at
   // once (the fused instance: once the CTA that writes the step's new token
@@ -1110,17 +1009,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (d4 == 0) lse_out[h] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
     }
   }
-  if (p.out == nullptr) return;
-  // The fold: every CTA's partial is visible before it takes its ticket;
-  // the last CTA of the (sequence, KV head) merges them.
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) sm.fold_last = take_ticket(p.tickets + (size_t)seq * p.kv_heads + kvh, S) ? 1 : 0;
-  __syncthreads();
-  if (sm.fold_last == 0) return;
-  __threadfence();
-  fold_parts<G>(p.o_parts, p.lse2_parts, rows, row0, S, p.out, p.lse2_final,
-                reinterpret_cast<float*>(&sm.grp[0].k[0][0]));
 }
 
 }  // namespace qkv
@@ -1232,20 +1120,16 @@ extern "C" int32_t qkv_paged_decode_auto_splits(int32_t kv_heads, int32_t block_
   return (int32_t)std::max(1, occ * sms / kv_heads);
 }
 
-// Workspace of the one-call decode attention: the fold's ticket counters in
-// a fixed first QKV_DECODE_FOLD_TICKET_BYTES (so a workspace reused with
-// other shapes, or the library's static array, keeps them where every call
-// leaves them at zero), then o_parts and lse2_parts, each from a 256-byte
-// boundary.
+// Workspace of the one-call decode attention: o_parts, then lse2_parts from
+// the next 256-byte boundary.
 struct DecodeWs {
-  size_t o, lse, tickets, total;
+  size_t o, lse, total;
 };
 DecodeWs decode_ws(int64_t n_seq, int64_t q_heads, int64_t head_dim, int64_t max_splits) {
   const size_t rows = (size_t)n_seq * q_heads;
   DecodeWs w;
-  w.tickets = 0;
-  w.o = QKV_DECODE_FOLD_TICKET_BYTES;
-  w.lse = w.o + ((rows * max_splits * head_dim * 4 + 255) & ~size_t(255));
+  w.o = 0;
+  w.lse = (rows * max_splits * head_dim * 4 + 255) & ~size_t(255);
   w.total = w.lse + ((rows * max_splits * 4 + 255) & ~size_t(255));
   return w;
 }
@@ -1273,9 +1157,7 @@ static int split_impl(float* o_parts, float* lse2_parts, int32_t max_splits, con
                       const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq, int32_t q_heads,
                       int32_t kv_heads, int32_t head_dim, int32_t block_size, int32_t max_pages_per_seq,
                       int64_t num_pages, float softmax_scale, int32_t num_splits, int32_t v_group,
-                      int32_t* device_status, qkv_stream_t stream, const StepArgs* step,
-                      uint16_t* fold_out = nullptr, float* fold_lse2 = nullptr,
-                      unsigned int* tickets = nullptr) {
+                      int32_t* device_status, qkv_stream_t stream, const StepArgs* step) {
   if (!o_parts || !lse2_parts || !q || !k_data || !k_scale || !v_data || !v_scale || !page_table || !seq_lens)
     return QKV_EINVAL;
   if (n_seq < 0 || q_heads < 1 || kv_heads < 1 || max_pages_per_seq < 1 || num_pages < 1 || max_splits < 1 ||
@@ -1325,9 +1207,6 @@ static int split_impl(float* o_parts, float* lse2_parts, int32_t max_splits, con
   p.target = std::max(1, occ * sms / kv_heads);
   const float sc = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
   p.score_scale = sc * 1.4426950408889634f;
-  p.out = reinterpret_cast<__nv_bfloat16*>(fold_out);
-  p.lse2_final = fold_lse2;
-  p.tickets = tickets;
   KParams<true> pf;  // the fused instances' parameters: Params + the step's inputs
   static_cast<Params&>(pf) = p;
   if (step) {
@@ -1384,9 +1263,8 @@ extern "C" int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int3
                                      stream);
 }
 
-// a4 + a5 (+ a2 + a3 with step): the split pass into the workspace; its
-// partials folded inside the launch when max_splits * G is at most
-// QKV_DECODE_FOLD_MAX_ROWS, else by a merge launch.
+// a4 + a5 (+ a2 + a3 with step): the split pass into the workspace, then
+// the merge of its partials.
 static int attn_impl(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t* k_data,
                      const uint16_t* k_scale, const uint8_t* v_data, const uint16_t* v_scale,
                      const int32_t* page_table, const int32_t* seq_lens, int32_t n_seq, int32_t q_heads,
@@ -1406,14 +1284,10 @@ static int attn_impl(uint16_t* out, float* lse2_out, const uint16_t* q, const ui
   char* ws = static_cast<char*>(workspace);
   float* o_parts = reinterpret_cast<float*>(ws + L.o);
   float* lse_parts = reinterpret_cast<float*>(ws + L.lse);
-  const bool fold = q_heads % kv_heads == 0 && (int64_t)max_splits * (q_heads / kv_heads) <= QKV_DECODE_FOLD_MAX_ROWS &&
-                    (int64_t)n_seq * kv_heads * 4 <= QKV_DECODE_FOLD_TICKET_BYTES;
   int rc = split_impl(o_parts, lse_parts, max_splits, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens,
                       n_seq, q_heads, kv_heads, head_dim, block_size, max_pages_per_seq, num_pages, softmax_scale,
-                      num_splits, v_group, device_status, stream, step, fold ? out : nullptr,
-                      fold ? lse2_out : nullptr,
-                      fold ? reinterpret_cast<unsigned int*>(ws + L.tickets) : nullptr);
-  if (rc != QKV_OK || fold) return rc;
+                      num_splits, v_group, device_status, stream, step);
+  if (rc != QKV_OK) return rc;
   return qkv_lse_merge(o_parts, lse_parts, max_splits, (int32_t)rows, head_dim, out, lse2_out, stream);
 }
 

@@ -110,10 +110,9 @@ extern "C" int qkv_paged_decode_attn_f4_static(uint16_t* out, float* lse2_out, c
   int dev = -1;
   void* scratch = static_scratch_address(dev);
   if (!scratch) return QKV_ECUDA;
-  // The array is zero when the library is loaded. The partials need no
-  // clearing (the split pass writes the lse2 of every slot it reads back, and
-  // the o row of every slot whose lse2 is finite); the fold's ticket
-  // counters must start at zero, and every call leaves them at zero.
+  // Nothing in the array has to start at zero: the split pass writes the
+  // lse2 of every slot the merge reads, and the o row of every slot whose
+  // lse2 is finite.
   const int rc = qkv_paged_decode_attn_f4(out, lse2_out, q, k_data, k_scale, v_data, v_scale, page_table, seq_lens,
                                           n_seq, q_heads, kv_heads, head_dim, block_size, max_pages_per_seq,
                                           num_pages, softmax_scale, num_splits, max_splits, scratch,

@@ -53,18 +53,9 @@ def test_workspace_bytes(qkv):
     n = qkv.qkv_paged_decode_workspace_bytes(3, 16, 256, 74)
     rows = 3 * 16 * 74
     a = lambda x: (x + 255) // 256 * 256
-    assert n == 4096 + a(rows * 256 * 4) + a(rows * 4)   # fold tickets, o_parts, lse2_parts
+    assert n == a(rows * 256 * 4) + a(rows * 4)   # o_parts, lse2_parts
     assert qkv.qkv_paged_decode_workspace_bytes(-1, 16, 256, 4) == 0
 
-
-def test_fold_limit_mirrors_header(qkv):
-    src = open(HEADER).read()
-    m = re.search(r"#define QKV_DECODE_FOLD_MAX_ROWS (\d+)", src)
-    assert m and int(m.group(1)) == qkv.DECODE_FOLD_MAX_ROWS
-    m = re.search(r"#define QKV_DECODE_FOLD_TICKET_BYTES (\d+)", src)
-    assert m and int(m.group(1)) == qkv.DECODE_FOLD_TICKET_BYTES
-    assert qkv.decode_folds(37, 1, 16, 4) and not qkv.decode_folds(148, 1, 16, 4)
-    assert not qkv.decode_folds(37, 257, 16, 4)
 
 
 FAKE = ctypes.c_void_p(4096)  # never dereferenced: validation fails first

@@ -290,6 +290,3 @@ def test_workspace_reuse_across_calls(qkv):
         assert int(st.item()) == 0
         ref_out, ref_lse = _oracle_attn(w, x, ref)
         _assert_close(to_host(out, np.uint16), to_host(lse), ref_out, ref_lse)
-        # the in-launch fold left its ticket counters at zero for the next call
-        assert qkv.decode_folds(16, w.n_seq, w.q_heads, w.kv_heads)
-        assert int(att.workspace[:qkv.DECODE_FOLD_TICKET_BYTES].count_nonzero()) == 0
