@@ -226,7 +226,7 @@ QKV_API size_t qkv_paged_decode_workspace_bytes(int32_t n_seq, int32_t q_heads, 
  *   lse2_parts float [max_splits][n_seq * q_heads]: log2 of the split's
  *             softmax normaliser, log2 sum_t 2^(score_t log2 e); -inf for an
  *             empty or unused split (its o_parts row is then unspecified).
- * Shapes compiled: head_dim 256, q_heads / kv_heads in {1, 2, 4, 8},
+ * Shapes compiled: head_dim 256 and 128, q_heads / kv_heads in {1, 2, 4, 8},
  * block_size in {16, 32, 64}; others return QKV_EUNSUPPORTED. Cache and q
  * pointers must be 16-byte aligned (EINVAL otherwise). */
 QKV_API int qkv_paged_decode_split_f4(float* o_parts, float* lse2_parts, int32_t max_splits,

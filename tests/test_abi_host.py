@@ -86,7 +86,8 @@ def test_invalid_arguments_rejected_before_launch(qkv):
     # split pass: unsupported head_dim / group / block, bad group divisibility, null
     args = lambda hq, hkv, d, blk, ms=4: (FAKE, FAKE, ms, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, hq, hkv, d,
                                           blk, 16, 64, ctypes.c_float(0.0), 0, NUL, NUL)
-    assert L.qkv_paged_decode_split_f4(*args(16, 4, 128, 64)) == 2
+    assert L.qkv_paged_decode_split_f4(*args(16, 4, 192, 64)) == 2     # head_dim: 256 and 128 are compiled
+    assert L.qkv_paged_decode_split_f4(*args(16, 4, 64, 64)) == 2
     assert L.qkv_paged_decode_split_f4(*args(12, 4, 256, 64)) == 2     # group of 3
     assert L.qkv_paged_decode_split_f4(*args(16, 4, 256, 128)) == 2    # block 128
     assert L.qkv_paged_decode_split_f4(*args(16, 3, 256, 64)) == 1     # 16 % 3

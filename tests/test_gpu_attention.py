@@ -258,8 +258,79 @@ def test_softmax_scale_argument_gpu(qkv):
     _assert_close(out, lse, ro, rl)
 
 
+# head_dim 128: 64-byte rows (64-byte TMA swizzle), two cell pairs in Q K^T,
+# one cell per warp in P V; every block size, G 1/2/4/8, ragged and empty
+# contexts, both V layouts
+D128_CASES = [
+    # seq_lens, block, q_heads, kv_heads, num_pages, num_splits
+    ((4096,), 16, 16, 4, 256, 4),
+    ((1, 2, 15, 16, 17), 16, 16, 4, 16, 3),
+    ((63, 64, 65, 127, 129), 64, 8, 2, 16, 2),
+    ((1000, 31, 4097, 0, 1), 32, 32, 4, 200, 0),
+    ((333,), 64, 8, 8, 8, 1),
+    ((5000, 3000, 10), 64, 16, 4, 140, 0),
+]
+
+
+@pytest.mark.parametrize("v_group", [32, 128])
+@pytest.mark.parametrize("case", D128_CASES, ids=[f"L{c[0]}-B{c[1]}-G{c[2] // c[3]}-S{c[5]}" for c in D128_CASES])
+def test_decode_attention_head_dim_128(qkv, case, v_group):
+    seq_lens, block, hq, hkv, pages, splits = case
+    w = workloads.small("d128", seq_lens=seq_lens, num_pages=pages, block_size=block, q_heads=hq, kv_heads=hkv,
+                        head_dim=128, page_alloc="interleaved" if len(seq_lens) > 1 else "contiguous",
+                        head_scale=True)
+    x, ref = oracle_layer(w, v_group=v_group)
+    cache = _dev_cache(qkv, w, x, v_group=v_group)
+    _check_cache_equal(cache, ref)
+    out, lse, st = _run_attn(qkv, w, x, cache, num_splits=splits)
+    assert st == 0
+    ref_out, ref_lse = _oracle_attn(w, x, ref)
+    _assert_close(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("v_group", [32, 128])
+def test_split_partials_head_dim_128(qkv, v_group):
+    """Per-split fp32 partials at head_dim 128 against the oracle's sub-range
+    attention (strict 2e-3, no bf16 allowance)."""
+    S = 5
+    w = workloads.small("parts128", seq_lens=(1900, 130), num_pages=140, block_size=16, head_dim=128, head_scale=True)
+    x, ref = oracle_layer(w, v_group=v_group)
+    cache = _dev_cache(qkv, w, x, v_group=v_group)
+    rows = w.n_seq * w.q_heads
+    o_parts = torch.empty((S, rows, 128), dtype=torch.float32, device="cuda")
+    l_parts = torch.empty((S, rows), dtype=torch.float32, device="cuda")
+    qkv.qkv_paged_decode_split_f4(o_parts, l_parts, to_dev(x["q"]), cache.k_data, cache.k_scale, cache.v_data,
+                                  cache.v_scale, to_dev(x["page_table"]), to_dev(x["seq_lens"]), w.kv_heads,
+                                  num_splits=S)
+    o_parts, l_parts = to_host(o_parts), to_host(l_parts)
+    for i in range(S):
+        tb, te = [], []
+        for L in w.seq_lens:
+            n = -(-L // w.block_size)
+            tb.append(i * n // S * w.block_size)
+            te.append(min((i + 1) * n // S * w.block_size, L))
+        ro, rl = oracle.paged_attention(x["q"], ref, x["page_table"], tb, te, w.q_heads, w.kv_heads, 128,
+                                        w.block_size)
+        ro, rl = ro.reshape(rows, 128), rl.reshape(rows)
+        fin = np.isfinite(rl)
+        assert np.array_equal(np.isfinite(l_parts[i]), fin)
+        assert np.max(np.abs(o_parts[i][fin] - ro[fin]), initial=0.0) <= ATOL_ATTN
+        assert np.max(np.abs(l_parts[i][fin] - rl[fin]), initial=0.0) <= 2e-4
+
+
+@pytest.mark.parametrize("v_group", [32, 128])
+def test_single_token_is_exact_value_head_dim_128(qkv, v_group):
+    w = workloads.small("one128", seq_lens=(1, 1), num_pages=2, block_size=64, head_dim=128)
+    x, ref = oracle_layer(w, v_group=v_group)
+    cache = _dev_cache(qkv, w, x, v_group=v_group)
+    out, lse, st = _run_attn(qkv, w, x, cache)
+    ro, rl = _oracle_attn(w, x, ref)
+    assert np.array_equal(out, oracle.f64_to_bf16(ro))
+
+
 def test_unsupported_shapes_raise(qkv):
-    w = workloads.small("bad", seq_lens=(10,), num_pages=2, block_size=64, head_dim=128)
+    """head_dim 256 and 128 are the compiled decode shapes; 192 is refused."""
+    w = workloads.small("bad", seq_lens=(10,), num_pages=2, block_size=64, head_dim=192)
     x, _ = oracle_layer(w)
     cache = _dev_cache(qkv, w, x)
     with pytest.raises(qkv.QkvError) as e:

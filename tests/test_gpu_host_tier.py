@@ -64,12 +64,17 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("v_group", [32, 256])
-@pytest.mark.parametrize("case", CASES, ids=[f"L{c[0]}-B{c[1]}-G{c[2] // c[3]}-W{c[6]}" for c in CASES])
+@pytest.mark.parametrize("v_group", [32, "head_dim"])
+@pytest.mark.parametrize("case", CASES + [CASES[1] + (128,)],
+                         ids=[f"L{c[0]}-B{c[1]}-G{c[2] // c[3]}-W{c[6]}" + ("-D128" if len(c) > 7 else "")
+                              for c in CASES + [CASES[1] + (128,)]])
 def test_tiered_decode_matches_oracle(qkv, case, v_group):
-    seq_lens, block, hq, hkv, pages, host_pages, window = case
+    seq_lens, block, hq, hkv, pages, host_pages, window = case[:7]
+    head_dim = case[7] if len(case) > 7 else 256
+    v_group = head_dim if v_group == "head_dim" else v_group
     w = workloads.small("tier", seq_lens=seq_lens, num_pages=pages, block_size=block, q_heads=hq, kv_heads=hkv,
-                        page_alloc="interleaved" if len(seq_lens) > 1 else "contiguous", head_scale=True)
+                        page_alloc="interleaved" if len(seq_lens) > 1 else "contiguous", head_scale=True,
+                        head_dim=head_dim)
     x, ref, dev, host = _pools(qkv, w, v_group)
     hpt, dpt, host_lens, dev_lens = _split_tables(x["page_table"], x["seq_lens"], host_pages, block)
     att = qkv.TieredDecodeAttention(hq, hkv, w.head_dim, block, hpt.shape[1], window, v_group=v_group)

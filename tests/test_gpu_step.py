@@ -100,10 +100,29 @@ def test_step_matches_two_calls(qkv, case, v_group):
     _same_cache(*caches)
 
 
-def test_step_matches_oracle(qkv):
+@pytest.mark.parametrize("v_group", [32, 128])
+@pytest.mark.parametrize("case", [((4096,), 16, 16, 4, 256, 4), ((63, 64, 65, 127, 129), 64, 8, 2, 16, 2),
+                                  ((1000, 31, 4097, 0, 1), 32, 32, 4, 200, 0)],
+                         ids=["L4096-B16-G4", "L5-B64-G4", "L5-B32-G8"])
+def test_step_matches_two_calls_head_dim_128(qkv, case, v_group):
+    seq_lens, block, hq, hkv, pages, splits = case
+    w = workloads.small("step128", seq_lens=seq_lens, num_pages=pages, block_size=block, q_heads=hq, kv_heads=hkv,
+                        head_dim=128, page_alloc="interleaved" if len(seq_lens) > 1 else "contiguous",
+                        head_scale=True, yarn_factor=4.0, first_position=300000)
+    x = workloads.host_layer(w)
+    outs, caches = _both(qkv, w, x, v_group, YARN4, num_splits=splits)
+    (oa, la, sa), (ob, lb, sb) = outs
+    assert sa == 0 and sb == 0
+    assert np.array_equal(oa, ob)
+    assert np.array_equal(la.view(np.uint32), lb.view(np.uint32))
+    _same_cache(*caches)
+
+
+@pytest.mark.parametrize("head_dim", [256, 128])
+def test_step_matches_oracle(qkv, head_dim):
     """rotary (oracle) -> F4 write (oracle) -> exact attention (oracle)."""
     w = workloads.small("step_o", seq_lens=(3000, 70, 1), num_pages=64, block_size=64, head_scale=True,
-                        page_alloc="interleaved", yarn_factor=4.0, first_position=400000)
+                        page_alloc="interleaved", yarn_factor=4.0, first_position=400000, head_dim=head_dim)
     x = workloads.host_layer(w)
     outs, caches = _both(qkv, w, x, 32, YARN4)
     ob, lb, sb = outs[1]
