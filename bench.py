@@ -108,9 +108,14 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+KERNEL_SOURCES = {"decode_split.cu": ("decode_split.cuh", "decode_split.cu", "common.cuh")}
+
+
 def kernel_source_hash(source: str = "decode_split.cu") -> str:
+    """Hash of the sources a profiled kernel is built from: a committed ncu
+    summary counts for the bench only while it matches."""
     h = hashlib.sha256()
-    for name in (source, "common.cuh"):
+    for name in KERNEL_SOURCES.get(source, (source, "common.cuh")):
         with open(os.path.join(ROOT, "quantized_paged_kv_yarn_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -230,8 +230,19 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Bounded wait that also gives up once another role of this CTA has
-// aborted. Waiting threads sleep in the barrier instead of spinning.
+// Give up the pair's work: this CTA's abort flag and the peer CTA's (a
+// store to its shared memory through the cluster window), so that the
+// roles of both CTAs stop waiting at once instead of at their own limits.
+__device__ __forceinline__ void abort_pair(int* abort) {
+  *reinterpret_cast<volatile int*>(abort) = 1;
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(abort)), "r"(cluster_rank() ^ 1u));
+  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(1u) : "memory");
+}
+
+// Bounded wait that also gives up once another role of this CTA, or of the
+// peer CTA, has aborted. Waiting threads sleep in the barrier instead of
+// spinning.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const unsigned long long t0 = globaltimer();
   for (;;) {
@@ -327,14 +338,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     bars.abort = 0;
     fence_barrier_init();
   }
+  // Tensor memory is taken only after the wait: the CTA holds none of the
+  // SM's tensor memory (nor its allocation permit) while the kernel ahead of
+  // it in the stream still runs.
+  pdl_wait();
+  pdl_release();
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&bars.tmem)),
                  "r"(TMEM_COLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
-  pdl_wait();
-  pdl_release();
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
@@ -388,7 +402,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       if (ok) ok = pv(n_st - 1);
       if (!ok) {
-        *abort = 1;
+        abort_pair(&bars.abort);
         flag(p.status, QKV_DEV_TIMEOUT);
       }
       // every MMA issued so far has completed once this commit lands (both CTAs)
@@ -559,7 +573,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (valid && part) p.lse_part[(size_t)blockIdx.z * p.n_q * p.q_heads + row] = lse;
       else if (valid && p.lse2) p.lse2[row] = lse;
     } else {
-      *abort = 1;
+      abort_pair(&bars.abort);
       flag(p.status, QKV_DEV_TIMEOUT);
     }
     tc_fence_before();
@@ -655,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
     }
     if (!ok) {
-      *abort = 1;
+      abort_pair(&bars.abort);
       flag(p.status, QKV_DEV_TIMEOUT);
     }
   }
