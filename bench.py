@@ -74,6 +74,8 @@ def parse_args():
     ap.add_argument("--chunk", type=int, default=2048, help="prefill chunk size (queries)")
     ap.add_argument("--window-pages", type=int, default=2048, help="host tier: device window (pages)")
     ap.add_argument("--device-pages", type=int, default=64, help="host tier: newest pages kept on the device")
+    ap.add_argument("--num-splits", type=int, default=-1,
+                    help="split count of the decode step (-1: the workload's own, 0: the automatic plan)")
     ap.add_argument("--layers", type=int, default=0,
                     help="run fewer layers than the workload has (a smaller case for profiler captures)")
     return ap.parse_args()
@@ -281,7 +283,8 @@ def run_reference(args, rank: int):
 
 
 def config_of(w, args):
-    return {"workload": w.name, "layers": w.n_layers, "seq_lens": list(w.seq_lens), "q_heads": w.q_heads,
+    return {"workload": w.name, "layers": w.n_layers, "seq_lens": list(w.seq_lens), "num_splits": w.num_splits,
+            "q_heads": w.q_heads,
             "kv_heads": w.kv_heads, "head_dim": w.head_dim, "rot_dim": w.rot_dim, "block_size": w.block_size,
             "yarn_factor": w.yarn_factor, "step_positions": w.step_positions, "parallelism": f"replicas{args.gpus}",
             "l2": "inputs larger than L2: each layer's cache exceeds 126 MB and the step walks all layers"}
@@ -437,6 +440,8 @@ def run_ours(args, rank, world, local_rank):
     w = workloads.BY_NAME[args.workload]
     if args.layers:
         w = dataclass_replace(w, n_layers=args.layers)
+    if args.num_splits >= 0:
+        w = dataclass_replace(w, num_splits=args.num_splits)
     b = Bench(w, dev, seed_offset=rank, two_call=args.two_call)
 
     def barrier():

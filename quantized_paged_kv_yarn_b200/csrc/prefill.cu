@@ -581,11 +581,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ dequantisation
     const bool is_k = warp < 12;
     const int d = is_k ? tid - 256 : tid - 384;  // 0..127
-    // K: token 32 rank + d / 4 of the stage, dims 64 (d % 4) .. + 63
-    // V: token d / 2 of the stage, dims 128 rank + 64 (d % 2) .. + 63
-    const int tk = is_k ? NTL * rank + (d >> 2) : (d >> 1);
-    const int trow = is_k ? (d >> 2) : (d >> 1);  // row in this CTA's tile
-    const int chunk = is_k ? (d & 3) : (d & 1);
+    // K: row d % 8 + 8 (d / 32) of this CTA's 32 tokens, dims 64 ((d / 8) % 4) .. + 63
+    // V: token d % 8 + 8 (d / 16) of the stage, dims 128 rank + 64 ((d / 8) % 2) .. + 63
+    // The eight lanes of a quarter-warp take eight consecutive rows: their
+    // 16-byte stores (a quarter-warp per shared-memory wavefront) land in
+    // eight different 16-byte columns of the swizzled tile, one wavefront
+    // each (with the chunk as the fastest index, four lanes of a quarter hit
+    // the same column: 16 wavefronts per K store, 8 per V store).
+    const int trow = is_k ? (d & 7) + 8 * (d >> 5) : (d & 7) + 8 * (d >> 4);  // row in this CTA's tile
+    const int tk = is_k ? NTL * rank + trow : trow;
+    const int chunk = is_k ? ((d >> 3) & 3) : ((d >> 3) & 1);
     const int byte_off = is_k ? 32 * chunk : 64 * rank + 32 * chunk;  // in the 128-byte packed row
     const int cell = byte_off / 16;                                    // first 32-dim cell
     const uint8_t* data = is_k ? p.k_data : p.v_data;
