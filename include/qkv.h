@@ -399,8 +399,8 @@ QKV_API int qkv_gather_kv_f4(uint16_t* k_out, uint16_t* v_out, int64_t n_out, co
  *   workspace  device buffer (256-byte aligned) of at least
  *              qkv_paged_prefill_workspace_bytes(n_q, q_heads, head_dim,
  *              num_splits) bytes, owned by the caller.
- * Compiled shapes: head_dim 256, q_heads / kv_heads in {1, 2, 4, 8}, a
- * power-of-two block_size (else QKV_EUNSUPPORTED). Runs on the tensor cores
+ * Compiled shapes: head_dim 256 and 128, q_heads / kv_heads in {1, 2, 4,
+ * 8}, a power-of-two block_size (else QKV_EUNSUPPORTED). Runs on the tensor cores
  * (tcgen05 on clusters of two CTAs, fp16 operands, fp32 accumulators in
  * tensor memory): K (as exact hi + lo halves) and V are dequantised to fp16
  * in shared memory, q scaled by a power of two per row; outputs match
@@ -560,7 +560,7 @@ QKV_API size_t qkv_paged_prefill_tiered_workspace_bytes(int32_t n_q, int32_t q_h
  * prefix_len + i.
  *   out, lse2_out, q, the device pool, page_table, n_q, prefix_len,
  *               softmax_scale, v_group: as in qkv_paged_prefill_attn_f4
- *               (head_dim 256, power-of-two block_size).
+ *               (head_dim 256 or 128, power-of-two block_size).
  *   host_*      the host pool (host_num_pages pages, same shape), pinned and
  *               mapped as for qkv_stage_pages_f4; host_page_table int32
  *               [host_len / block_size], device or mapped pinned memory.

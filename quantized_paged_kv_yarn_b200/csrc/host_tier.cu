@@ -50,8 +50,9 @@ constexpr int STAGE_UNROLL = 4;  // loads in flight per thread before its stores
 // attention kernels that follow it would otherwise sit on the same SMs while
 // its loads of host memory are outstanding. (With a prefill kernel running
 // beside a live staging grid -- staging on a second stream -- a bounded wait
-// of the prefill ran out once in three chunk-layers at full size; the
-// library therefore never overlaps the two.)
+// of the prefill ran out at full size, both before and after the prefill
+// took its tensor memory only after its dependency wait; the cause is not
+// known, so the library never overlaps the two.)
 __global__ void __launch_bounds__(STAGE_THREADS) stage_pages_f4_kernel(const StageParams p) {
   pdl_wait();
   if (blockIdx.x == 0) {

@@ -11,17 +11,18 @@
 //
 // This is a dense contraction (256 query rows share every dequantised
 // page), so it runs on tcgen05.mma with fp32 accumulators in TMEM, issued
-// for a pair of CTAs on two SMs (cta_group::2, M = 256):
+// for a pair of CTAs on two SMs (cta_group::2, M = 256). With head_dim D
+// (256 or 128):
 //
-//   S[256 x 64]  = Q'[256 x 256] . (K^'hi + K^'lo)[64 x 256]^T   (2 x 16 MMAs, K = 16)
-//   O[256 x 256] += P[256 x 64] . V^'[64 x 256]                  (4 MMAs, N = 256)
+//   S[256 x 64] = Q'[256 x D] . (K^'hi + K^'lo)[64 x D]^T   (2 x D/16 MMAs, K = 16)
+//   O[256 x D] += P[256 x 64] . V^'[64 x D]                 (4 MMAs, N = D)
 //
 // Rows are (query head of the GQA group, query): 256 = G x (256 / G); CTA
 // rank r of the pair owns rows 128 r .. 128 r + 127 (its lanes of Q', S, P
 // and O). The B operands are split by N: of each 64-token stage, rank r
-// dequantises the K of tokens 32 r .. 32 r + 31 (all 256 dims) and the V of
-// dims 128 r .. 128 r + 127 (all 64 tokens) into its own shared memory, so
-// each SM writes and the tensor core reads half of every tile, and the
+// dequantises the K of tokens 32 r .. 32 r + 31 (all D dims) and the V of
+// dims D/2 r .. D/2 r + D/2 - 1 (all 64 tokens) into its own shared memory,
+// so each SM writes and the tensor core reads half of every tile, and the
 // shared-memory pipe (the bound of a one-SM version) carries half the bytes.
 // One pair per (256 / G queries, KV head).
 //
@@ -32,8 +33,8 @@
 //                 its row of Q' into tensor memory, reads S, keeps the running
 //                 max and sum, writes P, rescales O when the max moves, and
 //                 writes the output
-//   warps 8..11   K dequantisation: one token's 64 dims of K per thread
-//   warps 12..15  V dequantisation: one token's 64 of this CTA's 128 dims
+//   warps 8..11   K dequantisation: D/4 dims of one token's K per thread
+//   warps 12..15  V dequantisation: D/4 of one token's D/2 dims of this CTA
 //                 Packed bytes are read two stages ahead, page ids one
 //                 load ahead of those.
 // Producers signal rank 0's barriers (a remote arrive from rank 1); the MMA
@@ -56,8 +57,8 @@
 // after the P . V reading it (issued earlier by the same thread, and the
 // tensor core keeps one thread's MMAs in order). Shared-memory tiles use the
 // 128-byte swizzle in the canonical UMMA layouts: the K^' tiles (K-major)
-// are [4 chunks of 64 dims][32 tokens][128 B]; the V^' tile, the MN-major
-// B operand of P . V, is [2 chunks of 64 dims][64 tokens][128 B]. Within
+// are [D/64 chunks of 64 dims][32 tokens][128 B]; the V^' tile, the
+// MN-major B operand of P . V, is [D/128 chunks of 64 dims][64 tokens][128 B]. Within
 // each 8-dim unit the dims are stored in the order 0,4,1,5,2,6,3,7 (the
 // order in which four nibble masks of a packed word yield them); Q' uses the
 // same order, and the output un-permutes O's columns.
@@ -70,7 +71,6 @@ namespace qkv {
 namespace prefill {
 
 constexpr int THREADS = 512;
-constexpr int D = 256;
 constexpr int M = 256;          // rows per CTA pair
 constexpr int ML = 128;         // rows per CTA
 constexpr int NT = 64;          // tokens per stage
@@ -78,20 +78,30 @@ constexpr int NTL = NT / 2;     // K tokens per CTA per stage
 constexpr int NS = 3;           // shared-memory slots of K^ and V^
 constexpr float TH = 8.f;       // lazy-rescale threshold (log2 units)
 
-// shared-memory map (offsets from a 1024-byte aligned base)
-constexpr int KT = 4 * NTL * 128;               // one K^ tile (hi or lo): [4][32][128 B] = 16 KB
-constexpr int VT = 2 * NT * 128;                // one V^ tile: [2][64][128 B] = 16 KB
-constexpr int K_OFF = 0;                        // NS slots x (hi, lo)
-constexpr int V_OFF = K_OFF + NS * 2 * KT;      // NS slots
-constexpr int BAR_OFF = V_OFF + NS * VT;
-constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;  // barriers, flags, alignment slack
-static_assert(SMEM_BYTES > 116 * 1024, "one CTA per SM: TMEM is allocated whole");
-
-// TMEM columns (each CTA, its 128 rows): O 0..255, S slot b at 256 + 64 b
-// (P of that stage, fp16, overwrites its first 32 columns once S is read),
-// Q' at 384..511
+// Sizes that follow from the head dim D.
+template <int D>
+struct Geo {
+  static_assert(D == 256 || D == 128, "head_dim 256 or 128");
+  // shared-memory map (offsets from a 1024-byte aligned base)
+  static constexpr int KT = (D / 64) * NTL * 128;   // one K^ tile (hi or lo): [D/64][32][128 B]
+  static constexpr int VT = (D / 128) * NT * 128;   // one V^ tile: [D/128][64][128 B]
+  static constexpr int K_OFF = 0;                   // NS slots x (hi, lo)
+  static constexpr int V_OFF = K_OFF + NS * 2 * KT;  // NS slots
+  static constexpr int BAR_OFF = V_OFF + NS * VT;
+  // barriers, flags and alignment slack; at least 117 KB, so that no two
+  // CTAs share an SM (the tensor memory is allocated whole)
+  static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024 > 117 * 1024 ? BAR_OFF + 256 + 1024 : 117 * 1024;
+  // TMEM columns (each CTA, its 128 rows): O 0..D-1, S slot b at D + 64 b
+  // (P of that stage, fp16, overwrites its first 32 columns once S is
+  // read), Q' (two fp16 per column) at D + 128 .. D + 128 + D/2 - 1
+  static constexpr uint32_t TS = D;
+  static constexpr uint32_t TQ = D + 128;
+  // dims one dequantising thread converts per stage, and its 16-byte units
+  static constexpr int DPT = D / 4;
+  static constexpr int UPT = DPT / 8;
+};
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TQ = 384;
+static_assert(Geo<256>::TQ + 128 <= TMEM_COLS && Geo<128>::TQ + 64 <= TMEM_COLS, "tensor memory map");
 
 struct Bars {
   // signalled by producers of both CTAs, waited on in rank 0
@@ -301,8 +311,12 @@ struct Raw {
   int32_t page;   // page id of the stage this set loads next (read one load ahead)
 };
 
+template <int D>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     paged_prefill_kernel(const Params p) {
+  using Gm = Geo<D>;
+  constexpr int KT = Gm::KT, VT = Gm::VT, K_OFF = Gm::K_OFF, V_OFF = Gm::V_OFF, BAR_OFF = Gm::BAR_OFF;
+  constexpr uint32_t TS = Gm::TS, TQ = Gm::TQ;
   // 1024-aligned by pointer arithmetic on the shared array (keeps accesses in
   // the shared window)
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -373,7 +387,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint64_t dv = dv0 + (uint64_t)((b * VT) >> 4);
 #pragma unroll
         for (int kk = 0; kk < NT / 16; ++kk)  // A = P in tensor memory (S slot sb)
-          umma2_ts(tmem, tmem + 256 + 64 * sb + 8 * kk, dv + (uint64_t)((2048 * kk) >> 4), ID_PV,
+          umma2_ts(tmem, tmem + TS + 64 * sb + 8 * kk, dv + (uint64_t)((2048 * kk) >> 4), ID_PV,
                    (i > 0 || kk > 0) ? 1u : 0u);
         umma2_commit_both(&bars.odone);
         umma2_commit_both(&bars.vfree[b]);
@@ -387,7 +401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // core runs one thread's MMAs in order
         tc_fence_after();
         const uint64_t dk = dk0 + (uint64_t)((b * 2 * KT) >> 4);
-        const uint32_t ts = tmem + 256 + 64 * sb;
+        const uint32_t ts = tmem + TS + 64 * sb;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // K^'hi, then K^'lo into the same accumulator
 #pragma unroll
@@ -445,7 +459,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const float up = __int_as_float((127 + e / 2) << 23) * __int_as_float((127 + (e - e / 2)) << 23);
       c_row = p.score_scale * 16.f / up;  // S = S' * 2^(4 - e)
 #pragma unroll 1
-      for (int g = 0; g < 4; ++g) {  // 8 units = 32 columns per store
+      for (int g = 0; g < D / 64; ++g) {  // 8 units = 32 columns per store
         uint32_t o[32];
 #pragma unroll
         for (int uu = 0; uu < 8; ++uu) {
@@ -476,8 +490,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (!__all_sync(FULL_MASK, ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[2][32];
-      tmem_ld32(tmem + lane_base + 256 + 64 * sb, sr[0]);
-      tmem_ld32(tmem + lane_base + 256 + 64 * sb + 32, sr[1]);
+      tmem_ld32(tmem + lane_base + TS + 64 * sb, sr[0]);
+      tmem_ld32(tmem + lane_base + TS + 64 * sb + 32, sr[1]);
       tmem_wait_ld();
       float s[64];
 #pragma unroll
@@ -513,7 +527,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         pw[i] = h2_as_u32(h);
       }
       // P into the first 32 columns of S slot sb (its S is in registers)
-      tmem_st32(tmem + lane_base + 256 + 64 * sb, pw);
+      tmem_st32(tmem + lane_base + TS + 64 * sb, pw);
       if (any_need && j >= 1) {  // rescale O once P . V of the previous stage is done
         ok = wait_bar(&bars.odone, (uint32_t)(j - 1) & 1u, abort);
         if (!__all_sync(FULL_MASK, ok)) { ok = false; break; }
@@ -579,20 +593,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_fence_before();
   } else if (warp >= 8) {
     // ------------------------------------------------------------ dequantisation
+    constexpr int DPT = Gm::DPT, UPT = Gm::UPT;
     const bool is_k = warp < 12;
     const int d = is_k ? tid - 256 : tid - 384;  // 0..127
-    // K: row d % 8 + 8 (d / 32) of this CTA's 32 tokens, dims 64 ((d / 8) % 4) .. + 63
-    // V: token d % 8 + 8 (d / 16) of the stage, dims 128 rank + 64 ((d / 8) % 2) .. + 63
+    // K: row d % 8 + 8 (d / 32) of this CTA's 32 tokens, dims DPT ((d / 8) % 4) .. + DPT - 1
+    // V: token d % 8 + 8 (d / 16) of the stage, dims D/2 rank + DPT ((d / 8) % 2) .. + DPT - 1
     // The eight lanes of a quarter-warp take eight consecutive rows: their
     // 16-byte stores (a quarter-warp per shared-memory wavefront) land in
     // eight different 16-byte columns of the swizzled tile, one wavefront
-    // each (with the chunk as the fastest index, four lanes of a quarter hit
-    // the same column: 16 wavefronts per K store, 8 per V store).
+    // each (with the dim slot as the fastest index, four lanes of a quarter
+    // hit the same column: 16 wavefronts per K store, 8 per V store).
     const int trow = is_k ? (d & 7) + 8 * (d >> 5) : (d & 7) + 8 * (d >> 4);  // row in this CTA's tile
     const int tk = is_k ? NTL * rank + trow : trow;
-    const int chunk = is_k ? ((d >> 3) & 3) : ((d >> 3) & 1);
-    const int byte_off = is_k ? 32 * chunk : 64 * rank + 32 * chunk;  // in the 128-byte packed row
-    const int cell = byte_off / 16;                                    // first 32-dim cell
+    const int slot = is_k ? ((d >> 3) & 3) : ((d >> 3) & 1);
+    const int tdim = DPT * slot;       // first dim in the tile (K: of D, V: of this CTA's D/2)
+    const int chunk = tdim / 64;       // 64-dim chunk of the tile
+    const int unit0 = (tdim % 64) / 8;  // first 16-byte unit in the chunk's row
+    const int byte_off = (is_k ? tdim : (D / 2) * rank + tdim) / 2;  // in the packed row
+    const int cell = byte_off / 16;                                   // first 32-dim cell
     const uint8_t* data = is_k ? p.k_data : p.v_data;
     const uint16_t* scales = is_k ? p.k_scale : p.v_scale;
     const bool per_tok = !is_k && p.v_tok;
@@ -618,16 +636,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const size_t row = ((size_t)page * p.kv_heads + kvh) * p.block + (t & (p.block - 1));
       const uint4* src = reinterpret_cast<const uint4*>(data + row * row_bytes + byte_off);
       x.a = ldg_early16(src);
-      x.b = ldg_early16(src + 1);
+      if constexpr (UPT == 8) x.b = ldg_early16(src + 1);
       if (per_tok) {
         const uint32_t h = ldg_early2(scales + row);
         x.sc = h | (h << 16);
+      } else if constexpr (UPT == 8) {
+        x.sc = ldg_early4(scales + row * (D / 32) + cell);  // two cells (cell is even)
       } else {
-        x.sc = ldg_early4(scales + row * 8 + cell);
+        const uint32_t h = ldg_early2(scales + row * (D / 32) + cell);
+        x.sc = h | (h << 16);
       }
       x.ok = 1;
     };
-    // one token's 64 dims into chunk `chunk` of a tile slot (K: hi and lo tiles)
+    // this thread's DPT dims of one token into its units of a tile slot (K: hi and lo tiles)
     auto put = [&](uint32_t chunk_base, const Raw& x, auto with_lo) {
       constexpr bool LO = decltype(with_lo)::value;
       // s' = scale * 2^-4 per cell (low half: first cell, high half: second)
@@ -635,16 +656,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const __half2 s_lo = __low2half2(s16), s_hi = __high2half2(s16);
       const uint32_t wd[8] = {x.a.x, x.a.y, x.a.z, x.a.w, x.b.x, x.b.y, x.b.z, x.b.w};
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < UPT; ++u) {
         uint32_t o[4] = {0u, 0u, 0u, 0u}, r[4] = {0u, 0u, 0u, 0u};
         if (x.ok == 1) dequant_word<LO>(wd[u], u < 4 ? s_lo : s_hi, o, r);
-        sts128(chunk_base + swz(trow, u), o[0], o[1], o[2], o[3]);
-        if constexpr (LO) sts128(chunk_base + KT + swz(trow, u), r[0], r[1], r[2], r[3]);
+        sts128(chunk_base + swz(trow, unit0 + u), o[0], o[1], o[2], o[3]);
+        if constexpr (LO) sts128(chunk_base + KT + swz(trow, unit0 + u), r[0], r[1], r[2], r[3]);
       }
     };
     auto process = [&](int j, const Raw& x) -> bool {
       const int b = j % NS, u = j / NS;
-      if (x.ok == 2 && chunk == 0 && kvh == 0 && (((st0 + j) * NT + tk) & (p.block - 1)) == 0)
+      if (x.ok == 2 && slot == 0 && kvh == 0 && (((st0 + j) * NT + tk) & (p.block - 1)) == 0)
         flag(p.status, QKV_DEV_BAD_PAGE);
       if (is_k) {
         if (u >= 1 && !wait_bar(&bars.kfree[b], (uint32_t)(u - 1) & 1u, abort)) return false;
@@ -754,7 +775,7 @@ int prefill_run(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t
   if (((uintptr_t)k_scale | (uintptr_t)v_scale | (uintptr_t)lse2_out | (uintptr_t)lse_part) & 3) return QKV_EINVAL;
   if (o_part && !lse_part) return QKV_EINVAL;
   const int G = q_heads / kv_heads;
-  if (head_dim != prefill::D || (G != 1 && G != 2 && G != 4 && G != 8)) return QKV_EUNSUPPORTED;
+  if ((head_dim != 256 && head_dim != 128) || (G != 1 && G != 2 && G != 4 && G != 8)) return QKV_EUNSUPPORTED;
   if (block_size & (block_size - 1)) return QKV_EUNSUPPORTED;  // pages of a power-of-two size
   if (kv_heads > 65535) return QKV_EUNSUPPORTED;
   if (n_q == 0) {
@@ -796,29 +817,30 @@ int prefill_run(uint16_t* out, float* lse2_out, const uint16_t* q, const uint8_t
   p.block_shift = 0;
   while ((1 << p.block_shift) < block_size) ++p.block_shift;
   p.v_tok = v_group != 32;
-  const float sc = softmax_scale > 0.f ? softmax_scale : 0.0625f;  // 1 / sqrt(256)
+  const float sc = softmax_scale > 0.f ? softmax_scale : 1.f / sqrtf((float)head_dim);
   p.score_scale = sc * 1.4426950408889634f;
   p.status = device_status;
   p.n_splits = S;
   p.o_part = o_part;
   p.lse_part = lse_part;
 
-  static bool attr_set[64];
+  const bool d128 = head_dim == 128;
+  const void* fn = d128 ? (const void*)prefill::paged_prefill_kernel<128> : (const void*)prefill::paged_prefill_kernel<256>;
+  const int smem = d128 ? prefill::Geo<128>::SMEM_BYTES : prefill::Geo<256>::SMEM_BYTES;
+  static bool attr_set[64][2];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QKV_ECUDA;
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(prefill::paged_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             prefill::SMEM_BYTES) != cudaSuccess) {
+  if (!attr_set[dev][d128]) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
       (void)cudaGetLastError();
       return QKV_ECUDA;
     }
-    attr_set[dev] = true;
+    attr_set[dev][d128] = true;
   }
   // one CTA pair (a cluster of two, compiled in) per (256 / G queries, KV head, part)
   const dim3 grid(2u * (unsigned)pairs_x, (unsigned)kv_heads, (unsigned)S);
   void* args[] = {&p};
-  if (launch_pdl((const void*)prefill::paged_prefill_kernel, grid, dim3(prefill::THREADS), prefill::SMEM_BYTES,
-                 stream, args) != cudaSuccess) {
+  if (launch_pdl(fn, grid, dim3(prefill::THREADS), smem, stream, args) != cudaSuccess) {
     (void)cudaGetLastError();
     return QKV_ECUDA;
   }
@@ -837,7 +859,8 @@ static int prefill_max_parts(int32_t n_q, int32_t q_heads, int32_t head_dim, siz
 
 extern "C" int32_t qkv_paged_prefill_auto_splits(int32_t n_q, int32_t prefix_len, int32_t q_heads,
                                                  int32_t kv_heads, int32_t head_dim, size_t workspace_bytes) {
-  if (n_q < 1 || prefix_len < 0 || q_heads < 1 || kv_heads < 1 || q_heads % kv_heads || head_dim != prefill::D)
+  if (n_q < 1 || prefix_len < 0 || q_heads < 1 || kv_heads < 1 || q_heads % kv_heads ||
+      (head_dim != 256 && head_dim != 128))
     return 0;
   const int G = q_heads / kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return 0;

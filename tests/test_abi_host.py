@@ -98,6 +98,12 @@ def test_invalid_arguments_rejected_before_launch(qkv):
     assert L.qkv_paged_decode_split_f4(*a) == 1
     a = list(args(16, 4, 256, 64)); a[4] = ctypes.c_void_p(4100)       # cache not 16-byte aligned
     assert L.qkv_paged_decode_split_f4(*a) == 1
+    # prefill: head_dim 256 and 128 are compiled (v_group = head_dim: one V scale per token)
+    pf = lambda d: (FAKE, NUL, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 0, 16, 4, d, 64, 16, 64,
+                    ctypes.c_float(0.0), d, 1, NUL, 0, NUL, NUL)
+    assert L.qkv_paged_prefill_attn_f4(*pf(192)) == 2
+    assert L.qkv_paged_prefill_attn_f4(*pf(64)) == 2
+    assert qkv.qkv_paged_prefill_auto_splits(64, 0, 16, 4, 192, 0) == 0
     # merge: bad head_dim, no parts, empty rows
     assert L.qkv_lse_merge(FAKE, FAKE, 4, 8, 30, FAKE, NUL, NUL) == 1
     assert L.qkv_lse_merge(FAKE, FAKE, 0, 8, 256, FAKE, NUL, NUL) == 1

@@ -186,23 +186,27 @@ PF_CASES = [
     (8, 130, 130, 64, 8, 8, 3, 2),        # the chunk is the whole device part, G = 1, windows 3, 3, 2
     (0, 1000, 257, 32, 32, 4, 4, 4),      # no host part, G = 8
     (20, 64, 1, 64, 16, 4, 64, 8),        # one query, the window larger than the host part
+    (30, 500, 200, 16, 16, 4, 12, 4, 128),  # head_dim 128
 ]
 
 
-@pytest.mark.parametrize("v_group", [32, 256])
-@pytest.mark.parametrize("case", PF_CASES, ids=[f"H{c[0]}-L{c[1]}-Q{c[2]}-B{c[3]}-W{c[6]}" for c in PF_CASES])
+@pytest.mark.parametrize("v_group", [32, "head_dim"])
+@pytest.mark.parametrize("case", PF_CASES, ids=[f"H{c[0]}-L{c[1]}-Q{c[2]}-B{c[3]}-W{c[6]}" +
+                                                ("-D128" if len(c) > 8 else "") for c in PF_CASES])
 def test_tiered_prefill_matches_oracle(qkv, case, v_group):
-    hp, dev_tokens, n_q, block, hq, hkv, window, ppl = case
+    hp, dev_tokens, n_q, block, hq, hkv, window, ppl = case[:8]
+    d = case[8] if len(case) > 8 else 256
+    v_group = d if v_group == "head_dim" else v_group
     ctx = hp * block + dev_tokens
     w = workloads.small("tier_pf", seq_lens=(ctx,), num_pages=-(-ctx // block) + 2, block_size=block, q_heads=hq,
-                        kv_heads=hkv, head_scale=True)
+                        kv_heads=hkv, head_scale=True, head_dim=d)
     x, ref, dev, host = _pools(qkv, w, v_group)
     row = x["page_table"][0]
     hrow, drow = np.ascontiguousarray(row[:max(hp, 1)]), np.ascontiguousarray(row[hp:])
     prefix = dev_tokens - n_q
     q = workloads.chunk_queries_host(w, 0, n_q)
-    att = qkv.TieredPrefillAttention(n_q, hq, hkv, 256, block, hp, window, v_group=v_group, parts_per_launch=ppl)
-    out = torch.full((n_q, hq, 256), 0x7FC1, dtype=torch.int16, device="cuda")
+    att = qkv.TieredPrefillAttention(n_q, hq, hkv, d, block, hp, window, v_group=v_group, parts_per_launch=ppl)
+    out = torch.full((n_q, hq, d), 0x7FC1, dtype=torch.int16, device="cuda")
     lse = torch.empty((n_q, hq), dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     att(out, to_dev(q), dev, to_dev(drow), prefix, host, torch.from_numpy(hrow).pin_memory(), hp * block,
@@ -210,7 +214,7 @@ def test_tiered_prefill_matches_oracle(qkv, case, v_group):
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     ro, rl = oracle.tiered_prefill_attention(q, ref, hrow, hp * block, ref, drow, np.arange(prefix, dev_tokens), hq,
-                                             hkv, 256, block)
+                                             hkv, d, block)
     err, bound = attn_within(to_host(out, np.uint16), ro)
     assert np.all(err <= bound), f"max err {err.max():.3e} (excess {np.max(err - bound):.3e})"
     assert np.max(np.abs(to_host(lse) - rl)) <= 2e-3

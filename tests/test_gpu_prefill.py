@@ -1,8 +1,8 @@
 """GPU parity of the chunked causal prefill attention over the paged F4
 cache (qkv_paged_prefill_attn_f4, tcgen05) with the oracle: every query of a
 chunk against exact attention over its causal prefix, for ragged chunk sizes,
-empty and long prefixes, every GQA ratio, three block sizes and both V scale
-layouts; bad page ids are flagged."""
+empty and long prefixes, every GQA ratio, three block sizes, both V scale
+layouts and head_dim 256 and 128; bad page ids are flagged."""
 import numpy as np
 import pytest
 import torch
@@ -20,11 +20,13 @@ def qkv():
     return q
 
 
-def _setup(qkv, L, n_q, block, hq, hkv, v_group=256, pages=None, seed=0, head_scale=True, outliers=0.0):
+def _setup(qkv, L, n_q, block, hq, hkv, v_group=256, pages=None, seed=0, head_scale=True, outliers=0.0,
+           head_dim=256):
     w = workloads.small("prefill", seq_lens=(L,), num_pages=pages or -(-L // block) + 3, block_size=block,
-                        q_heads=hq, kv_heads=hkv, head_scale=head_scale, seed=seed, k_outlier_frac=outliers)
+                        q_heads=hq, kv_heads=hkv, head_scale=head_scale, seed=seed, k_outlier_frac=outliers,
+                        head_dim=head_dim)
     x, ref = oracle_layer(w, v_group=v_group)
-    cache = qkv.PagedF4Cache.allocate(w.num_pages, hkv, block, 256, v_group=v_group)
+    cache = qkv.PagedF4Cache.allocate(w.num_pages, hkv, block, head_dim, v_group=v_group)
     cache.write(to_dev(x["k_cache"]), to_dev(x["v_cache"]), to_dev(x["cache_slots"]))
     cache.write(to_dev(x["k_new"]), to_dev(x["v_new"]), to_dev(x["step_slots"]))
     q = workloads.chunk_queries_host(w, 0, n_q)
@@ -33,11 +35,11 @@ def _setup(qkv, L, n_q, block, hq, hkv, v_group=256, pages=None, seed=0, head_sc
 
 def _run(qkv, w, x, cache, q, prefix, page_table=None, softmax_scale=0.0, num_splits=1, ws_splits=0):
     n_q = q.shape[0]
-    out = torch.full((n_q, w.q_heads, 256), 0x7FC1, dtype=torch.int16, device="cuda")
+    out = torch.full((n_q, w.q_heads, w.head_dim), 0x7FC1, dtype=torch.int16, device="cuda")
     lse = torch.empty((n_q, w.q_heads), dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     pt = x["page_table"][0] if page_table is None else page_table
-    nb = qkv.qkv_paged_prefill_workspace_bytes(n_q, w.q_heads, 256, ws_splits) if ws_splits > 1 else 0
+    nb = qkv.qkv_paged_prefill_workspace_bytes(n_q, w.q_heads, w.head_dim, ws_splits) if ws_splits > 1 else 0
     ws = torch.empty(nb, dtype=torch.uint8, device="cuda") if nb else None
     qkv.qkv_paged_prefill_attn_f4(out, to_dev(q), cache.k_data, cache.k_scale, cache.v_data, cache.v_scale,
                                   to_dev(np.ascontiguousarray(pt)), prefix, w.kv_heads, lse2_out=lse,
@@ -74,6 +76,45 @@ def test_prefill_matches_oracle(qkv, case, v_group):
     assert st == 0
     ro, rl = oracle.prefill_attention(q, ref, x["page_table"][0], np.arange(prefix, L), hq, hkv, 256, block)
     _check(out, lse, ro, rl)
+
+
+D128_CASES = [
+    (100, 100, 16, 16, 4),
+    (1600, 257, 32, 16, 4),
+    (300, 129, 64, 4, 4),
+    (400, 130, 16, 8, 4),
+    (333, 40, 64, 16, 2),
+    (65, 1, 64, 16, 4),
+]
+
+
+@pytest.mark.parametrize("v_group", [32, 128])
+@pytest.mark.parametrize("case", D128_CASES, ids=[f"L{c[0]}-n{c[1]}-B{c[2]}-G{c[3] // c[4]}" for c in D128_CASES])
+def test_prefill_d128_matches_oracle(qkv, case, v_group):
+    """head_dim 128: 64-byte packed rows, one 64-dim chunk of V per CTA of the pair."""
+    L, n_q, block, hq, hkv = case
+    w, x, ref, cache, q = _setup(qkv, L, n_q, block, hq, hkv, v_group, head_dim=128)
+    prefix = L - n_q
+    out, lse, st = _run(qkv, w, x, cache, q, prefix)
+    assert st == 0
+    ro, rl = oracle.prefill_attention(q, ref, x["page_table"][0], np.arange(prefix, L), hq, hkv, 128, block)
+    _check(out, lse, ro, rl)
+
+
+def test_prefill_d128_context_split_and_first_query(qkv):
+    """head_dim 128 with the context in three parts, and query 0 of a chunk
+    without prefix (token 0's value within one bf16 ulp)."""
+    L, n_q = 1600, 257
+    w, x, ref, cache, q = _setup(qkv, L, n_q, 32, 16, 4, 32, head_dim=128)
+    out, lse, st = _run(qkv, w, x, cache, q, L - n_q, num_splits=3, ws_splits=3)
+    assert st == 0
+    ro, rl = oracle.prefill_attention(q, ref, x["page_table"][0], np.arange(L - n_q, L), 16, 4, 128, 32)
+    _check(out, lse, ro, rl)
+    w, x, ref, cache, q = _setup(qkv, 70, 70, 16, 16, 4, head_dim=128, v_group=128)
+    out, _, st = _run(qkv, w, x, cache, q, 0)
+    ro, _ = oracle.prefill_attention(q[:1], ref, x["page_table"][0], np.arange(0, 1), 16, 4, 128, 16)
+    got = oracle.bf16_to_f64(out[0])
+    assert st == 0 and np.all(np.abs(got - ro[0]) <= bf16_ulp(ro[0]))
 
 
 @pytest.mark.parametrize("splits", [(2, 2), (3, 3), (0, 8)], ids=["S2", "S3", "auto"])
