@@ -319,7 +319,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   // these: the library's writers of the cache never do, and the fused
   // instance's own write is ordered before the copies of its stage below.
   if constexpr (!FUSE) pdl_release();
-  const int split = blockIdx.x, seq = blockIdx.y, kvh = blockIdx.z;
+  // Splits in reverse launch order: CTAs are placed in launch order as SMs
+  // free up, so the last one lands on the SM that frees last and starts
+  // late; that is then split 0 rather than the sequence's last split, which
+  // holds the new token's page (the decode step's write) and the plan's
+  // unused slots (which leave at once).
+  const int split = (int)(gridDim.x - 1 - blockIdx.x), seq = blockIdx.y, kvh = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = warp / GWARPS, gw = warp % GWARPS;  // group, warp within the group
   const int g = lane >> 2, t = lane & 3;
