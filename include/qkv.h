@@ -219,7 +219,11 @@ QKV_API size_t qkv_paged_decode_workspace_bytes(int32_t n_seq, int32_t q_heads, 
  *             to fit); 0: the plan balances pages over the device (splits of
  *             about sum(pages) / auto_splits pages each, at most max_splits
  *             per sequence). Split i of a sequence with n pages covers pages
- *             [i*n/S, (i+1)*n/S).
+ *             [b(i), b(i+1)): b(i) = i*n/S, except that with S >= 8 the
+ *             first m = ceil(S/7) splits are d pages shorter each (d: 400
+ *             tokens at head_dim 256, 800 at 128, at most a quarter split),
+ *             the others sharing those pages; the grid places the first
+ *             splits last, and the last CTAs placed start late.
  *   o_parts   float [max_splits][n_seq * q_heads][head_dim]: partial output
  *             of split i for row (s, h) at [i][s * q_heads + h], normalised
  *             by its own softmax sum.

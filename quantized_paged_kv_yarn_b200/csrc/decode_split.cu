@@ -165,7 +165,7 @@ static int split_impl(float* o_parts, float* lse2_parts, int32_t max_splits, con
   const uint64_t cache_rows = (uint64_t)num_pages * kv_heads * block_size;
   if (cache_rows > 0x7fffffffull) return QKV_EUNSUPPORTED;  // TMA row coordinate is int32
   if ((int64_t)max_pages_per_seq * block_size > 0x7fffffffLL) return QKV_EUNSUPPORTED;
-  if (max_splits > 65535 * 16 || n_seq > 65535 || kv_heads > 65535) return QKV_EUNSUPPORTED;
+  if (max_splits > 65535 || n_seq > 65535 || kv_heads > 65535) return QKV_EUNSUPPORTED;
   if (n_seq == 0) return QKV_OK;
 
   const int occ = prepare(fn, head_dim, block_size, G, vtok, step != nullptr);
@@ -217,7 +217,7 @@ static int split_impl(float* o_parts, float* lse2_parts, int32_t max_splits, con
 
   // Slots past the plan's split count still get lse2 = -inf: the grid
   // covers every slot the merge reads.
-  dim3 grid((unsigned)max_splits, (unsigned)n_seq, (unsigned)kv_heads);
+  dim3 grid((unsigned)kv_heads, (unsigned)max_splits, (unsigned)n_seq);
   void* args[] = {(void*)&tm_k, (void*)&tm_v, step ? (void*)&pf : (void*)&p};
   if (launch_pdl(fn, grid, dim3(THREADS), kernel_smem(head_dim, G), stream, args) != cudaSuccess) {
     (void)cudaGetLastError();

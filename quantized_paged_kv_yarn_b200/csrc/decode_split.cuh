@@ -247,19 +247,37 @@ __device__ __forceinline__ int muldiv(uint32_t a, uint32_t b, uint32_t c) {
   return (ab >> 32) == 0 ? (int)((uint32_t)ab / c) : (int)(ab / c);
 }
 
+// First page of split s (0 <= s <= S) of a sequence of n pages: S equal
+// parts, except that splits 0 .. m-1 take d pages fewer each (the others
+// share them). Those are the CTAs placed last (the grid runs splits in
+// reverse order), which start a prologue's time after the rest when they
+// get the SMs that the previous launch or its merge freed last. With
+// P = n / S: bound(s) = s (P - d) for s <= m, and s P + d m (s - m) / (S - m)
+// - d m for s >= m, rounded down (d <= P / 4 keeps it increasing).
+__device__ inline int split_bound(uint32_t s, uint32_t n, uint32_t S, uint32_t m, uint32_t d) {
+  if (m == 0 || d == 0) return muldiv(s, n, S);
+  const long long den = (long long)S * (S - m);
+  const long long num = s <= m ? ((long long)s * n - (long long)s * d * S) * (S - m)
+                               : (long long)n * (S - m) * s - (long long)m * d * S * (S - s);
+  return (int)(num / den);
+}
+
 // Split plan. Fixed: num_splits splits per sequence (the host refuses a
 // count above max_splits).
 // Automatic: pages are cut into pieces of about total pages / target, so the
 // grid holds at most `target` busy CTAs per KV head whatever the mix of
-// lengths. Split i of a sequence with n pages covers [i*n/S, (i+1)*n/S).
+// lengths. Split i covers pages [bound(i), bound(i + 1)) of its sequence:
+// with S >= 8 splits the first ceil(S / 7) of them (the ones placed last)
+// are `late_tok` tokens (at most a quarter split) shorter.
 __device__ inline long long splits_for(const Params& p, int block, uint32_t P) {
   long long total = 0;
   for (int s = 0; s < p.n_seq; ++s) total += cdiv(cdiv((uint32_t)seq_len_of(p, s, block, false), block), P);
   return total;
 }
 
-__device__ inline void plan(const Params& p, int seq, int split, int block, int& S, int& pg0, int& pg1, int& L) {
-  L = seq_len_of(p, seq, block, split == 0 && blockIdx.z == 0);
+__device__ inline void plan(const Params& p, int seq, int split, int block, int late_tok, int& S, int& pg0, int& pg1,
+                            int& L) {
+  L = seq_len_of(p, seq, block, split == 0 && blockIdx.x == 0);  // one report per sequence (KV head 0)
   const uint32_t n = cdiv((uint32_t)L, (uint32_t)block);
   if (p.num_splits > 0) {
     S = p.num_splits;
@@ -284,8 +302,10 @@ __device__ inline void plan(const Params& p, int seq, int split, int block, int&
     }
     S = (int)min((uint32_t)p.max_splits, max(1u, cdiv(n, P)));
   }
-  pg0 = muldiv((uint32_t)split, n, (uint32_t)S);
-  pg1 = muldiv((uint32_t)split + 1, n, (uint32_t)S);
+  const uint32_t m = S >= 8 ? ((uint32_t)S + 6) / 7 : 0;
+  const uint32_t d = min((uint32_t)late_tok / (uint32_t)block, n / (uint32_t)S / 4);
+  pg0 = split_bound((uint32_t)split, n, (uint32_t)S, m, d);
+  pg1 = split_bound((uint32_t)split + 1, n, (uint32_t)S, m, d);
 }
 
 template <int D, int BLOCK, int G, bool VTOK, bool FUSE>
@@ -319,12 +339,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   // these: the library's writers of the cache never do, and the fused
   // instance's own write is ordered before the copies of its stage below.
   if constexpr (!FUSE) pdl_release();
-  // Splits in reverse launch order: CTAs are placed in launch order as SMs
-  // free up, so the last one lands on the SM that frees last and starts
-  // late; that is then split 0 rather than the sequence's last split, which
-  // holds the new token's page (the decode step's write) and the plan's
-  // unused slots (which leave at once).
-  const int split = (int)(gridDim.x - 1 - blockIdx.x), seq = blockIdx.y, kvh = blockIdx.z;
+  // CTAs are placed in launch order as SMs free up, so the last ones land on
+  // the SMs that the previous launch (or its merge) frees last and start
+  // late. The grid runs the KV heads fastest and the splits in reverse
+  // order: the late ones are the first splits of every KV head, which the
+  // plan makes shorter, and not the sequence's last split, which holds the
+  // new token's page (the decode step's write), nor the plan's unused slots
+  // (which leave at once).
+  const int kvh = blockIdx.x, split = (int)(gridDim.y - 1 - blockIdx.y), seq = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = warp / GWARPS, gw = warp % GWARPS;  // group, warp within the group
   const int g = lane >> 2, t = lane & 3;
@@ -334,7 +356,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   GroupSmem<D>& gs = sm.grp[grp];
 
   int S, pg0, pg1, L;
-  plan(p, seq, split, BLOCK, S, pg0, pg1, L);
+  // ~3 us of a late start at an SM's ~38 GB/s: 400 tokens of 288 bytes (head_dim 256)
+  plan(p, seq, split, BLOCK, D == 256 ? 400 : 800, S, pg0, pg1, L);
   if (split >= S) {  // unused slot of the plan
     if constexpr (FUSE) pdl_release();
     pdl_wait();  // the workspace may still be read by the kernels ahead

@@ -43,6 +43,19 @@ def _run_attn(qkv, w, x, cache, num_splits=0, max_splits=0, softmax_scale=0.0):
     return to_host(out, np.uint16), to_host(lse), int(st.item())
 
 
+def _split_bound(i, n, S, block, head_dim):
+    """First page of split i of a sequence of n pages, as include/qkv.h states
+    the plan: i * n / S, except that with S >= 8 the first ceil(S / 7) splits
+    are d pages shorter (d = 400 tokens at head_dim 256, 800 at 128, at most a
+    quarter split), the other splits sharing those pages."""
+    m = (S + 6) // 7 if S >= 8 else 0
+    d = min((400 if head_dim == 256 else 800) // block, n // S // 4)
+    if m == 0 or d == 0:
+        return i * n // S
+    num = (i * n - i * d * S) * (S - m) if i <= m else n * (S - m) * i - m * d * S * (S - i)
+    return num // (S * (S - m))
+
+
 def _oracle_attn(w, x, ref, softmax_scale=None):
     return oracle.paged_attention(x["q"], ref, x["page_table"], np.zeros(w.n_seq, np.int32), x["seq_lens"],
                                   w.q_heads, w.kv_heads, w.head_dim, w.block_size, softmax_scale)
@@ -124,8 +137,8 @@ def test_split_partials_match_oracle_ranges(qkv, num_splits, v_group):
         tb, te = [], []
         for L in w.seq_lens:
             n = -(-L // w.block_size)
-            tb.append(i * n // num_splits * w.block_size)
-            te.append(min((i + 1) * n // num_splits * w.block_size, L))
+            tb.append(_split_bound(i, n, num_splits, w.block_size, 256) * w.block_size)
+            te.append(min(_split_bound(i + 1, n, num_splits, w.block_size, 256) * w.block_size, L))
         ro, rl = oracle.paged_attention(x["q"], ref, x["page_table"], tb, te, w.q_heads, w.kv_heads, 256,
                                         w.block_size)
         ro, rl = ro.reshape(rows, 256), rl.reshape(rows)
@@ -292,7 +305,7 @@ def test_decode_attention_head_dim_128(qkv, case, v_group):
 def test_split_partials_head_dim_128(qkv, v_group):
     """Per-split fp32 partials at head_dim 128 against the oracle's sub-range
     attention (strict 2e-3, no bf16 allowance)."""
-    S = 5
+    S = 9   # >= 8: the plan's shorter first splits
     w = workloads.small("parts128", seq_lens=(1900, 130), num_pages=140, block_size=16, head_dim=128, head_scale=True)
     x, ref = oracle_layer(w, v_group=v_group)
     cache = _dev_cache(qkv, w, x, v_group=v_group)
@@ -307,8 +320,8 @@ def test_split_partials_head_dim_128(qkv, v_group):
         tb, te = [], []
         for L in w.seq_lens:
             n = -(-L // w.block_size)
-            tb.append(i * n // S * w.block_size)
-            te.append(min((i + 1) * n // S * w.block_size, L))
+            tb.append(_split_bound(i, n, S, w.block_size, 128) * w.block_size)
+            te.append(min(_split_bound(i + 1, n, S, w.block_size, 128) * w.block_size, L))
         ro, rl = oracle.paged_attention(x["q"], ref, x["page_table"], tb, te, w.q_heads, w.kv_heads, 128,
                                         w.block_size)
         ro, rl = ro.reshape(rows, 128), rl.reshape(rows)
