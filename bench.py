@@ -329,12 +329,34 @@ class Bench:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.two_call = two_call
         self.launches_per_step = 1 + (3 if two_call else 2) * self.L
-        # host side of the end-to-end measurement (pinned)
-        self.h_q = [t.cpu().pin_memory() for t in self.q_raw]
-        self.h_kn = [t.cpu().pin_memory() for t in self.kn_raw]
-        self.h_vn = [t.cpu().pin_memory() for t in self.vn]
-        self.h_pos = self.positions.cpu().pin_memory()
-        self.h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.out]
+        # End-to-end measurement: the step's inputs (q, new k and v of every
+        # layer, the positions) live in one device buffer with a pinned host
+        # mirror, the outputs of all layers in another, so a step's transfers
+        # are one host-to-device and one device-to-host copy.
+        L = self.L
+        self.d_in, ins = self._pack(self.q_raw + self.kn_raw + self.vn + [self.positions])
+        self.q_raw, self.kn_raw, self.vn = ins[:L], ins[L:2 * L], ins[2 * L:3 * L]
+        self.positions = ins[3 * L]
+        self.d_out, self.out = self._pack(self.out)
+        self.h_in = torch.empty(self.d_in.shape, dtype=torch.uint8).pin_memory()
+        self.h_in.copy_(self.d_in)
+        self.h_out = torch.empty(self.d_out.shape, dtype=torch.uint8).pin_memory()
+
+    def _pack(self, tensors):
+        """One uint8 device buffer holding `tensors` at 256-byte aligned
+        offsets (their data copied in) and views of it in their shapes."""
+        torch = self.torch
+        offs, n = [], 0
+        for t in tensors:
+            offs.append(n)
+            n += (t.numel() * t.element_size() + 255) // 256 * 256
+        buf = torch.empty(n, dtype=torch.uint8, device=self.dev)
+        views = []
+        for t, o in zip(tensors, offs):
+            v = buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+            v.copy_(t)
+            views.append(v)
+        return buf, views
 
     def step(self):
         q, w = self.qkv, self.w
@@ -357,19 +379,13 @@ class Bench:
                      device_status=self.status)
 
     def e2e_step(self):
-        """Host buffers in, the step, the result back to the host."""
-        for l in range(self.L):
-            self.q_raw[l].copy_(self.h_q[l], non_blocking=True)
-            self.kn_raw[l].copy_(self.h_kn[l], non_blocking=True)
-            self.vn[l].copy_(self.h_vn[l], non_blocking=True)
-        self.positions.copy_(self.h_pos, non_blocking=True)
+        """Host buffers in (one copy), the step, the results back to the host (one copy)."""
+        self.d_in.copy_(self.h_in, non_blocking=True)
         self.step()
-        for l in range(self.L):
-            self.h_out[l].copy_(self.out[l], non_blocking=True)
+        self.h_out.copy_(self.d_out, non_blocking=True)
 
     def io_bytes(self):
-        nb = lambda ts: sum(t.numel() * t.element_size() for t in ts)
-        return nb(self.h_q) + nb(self.h_kn) + nb(self.h_vn) + nb([self.h_pos]), nb(self.h_out)
+        return self.h_in.numel(), self.h_out.numel()
 
     def capture(self, fn):
         torch = self.torch
