@@ -1037,7 +1037,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     __syncthreads();
     // Fold the groups: weights 2^(m_ref of the group - M) per head.
-    float* slab = reinterpret_cast<float*>(&sm.grp[0].k[0][0]);  // [group][head][dim], in idle rings
+    // [group][head][D + 4 dims], in group 0's idle rings: the 4-float pad
+    // puts the heads of one quarter-warp's stores in different banks
+    constexpr int SLAB_ROW = D + 4;
+    static_assert(GROUPS * 8 * SLAB_ROW * 4 <= (NSK + NSV) * STAGE_TOK * Geo<D>::ROW_BYTES, "slab fits the rings");
+    float* slab = reinterpret_cast<float*>(&sm.grp[0].k[0][0]);
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const int h = 2 * t + j;
@@ -1047,7 +1051,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int q = 0; q < GROUPS; ++q)
           if (sm.gl[q][h] > 0.f) M = fmaxf(M, sm.gm[q][h]);
         const float f = (sm.gl[grp][h] > 0.f) ? exp2f(sm.gm[grp][h] - M) : 0.f;
-        float* dst = slab + ((size_t)grp * G + h) * D + 4 * g;
+        float* dst = slab + ((size_t)grp * G + h) * SLAB_ROW + 4 * g;
 #pragma unroll
         for (int c = 0; c < CPW; ++c) {
           const float4 o = make_float4(f * acc[c][0][j], f * acc[c][0][j + 2], f * acc[c][1][j], f * acc[c][1][j + 2]);
@@ -1069,7 +1073,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int q = 0; q < GROUPS; ++q) {
         const float f = (sm.gl[q][h] > 0.f) ? exp2f(sm.gm[q][h] - M) : 0.f;
         Ls = fmaf(f, sm.gl[q][h], Ls);
-        const float4 x = *reinterpret_cast<const float4*>(slab + ((size_t)q * G + h) * D + 4 * d4);
+        const float4 x = *reinterpret_cast<const float4*>(slab + ((size_t)q * G + h) * SLAB_ROW + 4 * d4);
         o.x += x.x;
         o.y += x.y;
         o.z += x.z;
