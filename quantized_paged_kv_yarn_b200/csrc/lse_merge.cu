@@ -13,15 +13,17 @@
 
 namespace qkv {
 
-// One CTA per (row, 64-dim chunk); 16 warps split the parts (warp w takes
-// parts w, w + 16, ...). A warp loads the lse2 of up to 32 of its parts (one
+// One CTA per (row, 64-dim chunk); 8 warps split the parts (warp w takes
+// parts w, w + 8, ...). A warp loads the lse2 of up to 32 of its parts (one
 // per lane) together with the 64-dim rows (2 dims per lane) of the first 8 of
 // them, before their weights are known: the rows of parts without weight are
 // selected away, never multiplied, so whatever they hold is harmless. With
-// up to 8 parts per warp (128 per row) the fold costs one global-latency
+// up to 8 parts per warp (64 per row) the fold costs one global-latency
 // round. The warps' (max, weight sum, weighted sum) are combined in shared
-// memory.
-constexpr int MERGE_WARPS = 16;
+// memory. (Eight warps rather than sixteen: the merge's CTAs then hold fewer
+// of the SMs that the next split launch's CTAs wait for; 0.607 against
+// 0.612 ms per 16-layer decode step at 131,072 tokens, the same at 262,144.)
+constexpr int MERGE_WARPS = 8;
 constexpr int MERGE_THREADS = MERGE_WARPS * 32;
 constexpr int MERGE_DIMS = 64;
 constexpr int MERGE_BATCH = 8;  // part rows a lane has in flight at once

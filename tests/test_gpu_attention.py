@@ -149,8 +149,8 @@ def test_split_partials_match_oracle_ranges(qkv, num_splits, v_group):
 
 
 # part counts: the automatic plan's 37 on a B200, the 1M-token workload's 148
-# (>= 128 weighted parts per row), and 600, past the merge's first round of
-# 512 parts (16 warps x 32 lanes) into its second
+# (>= 128 weighted parts per row), and 600, past the merge's first rounds of
+# 256 parts (8 warps x 32 lanes) into its third
 @pytest.mark.parametrize("n", [37, 148, 600])
 def test_lse_merge_matches_oracle(qkv, n):
     rng = np.random.default_rng(21 + n)
