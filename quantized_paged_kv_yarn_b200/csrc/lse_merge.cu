@@ -117,6 +117,57 @@ __global__ void __launch_bounds__(MERGE_THREADS) lse_merge_kernel(const float* _
   }
 }
 
+// Few parts per row (the chunked prefill's context split, a short decode
+// plan): one warp per (row, 64-dim chunk), eight to a CTA, each lane holding
+// the lse2 of part `lane` and the rows of every part for its 2 dims, all
+// loaded at once; no shared memory and no block barrier. (The 2048-query
+// prefill chunk with its 4-part split: 10.77 against 11.05 ms with the
+// many-part kernel, whose idle warps then outnumber the busy ones.)
+constexpr int MERGE_SMALL_PARTS = 8;
+
+__global__ void __launch_bounds__(256) lse_merge_small_kernel(const float* __restrict__ o_parts,
+                                                              const float* __restrict__ lse2_parts, int n_parts,
+                                                              int rows, int head_dim, int chunks,
+                                                              __nv_bfloat16* __restrict__ out,
+                                                              float* __restrict__ lse2_out) {
+  pdl_release();
+  pdl_wait();
+  const int item = blockIdx.x * 8 + (threadIdx.x >> 5);  // (row, chunk)
+  const int lane = threadIdx.x & 31;
+  if (item >= rows * chunks) return;
+  const int row = item / chunks, chunk = item - row * chunks;
+  const int d = chunk * MERGE_DIMS + 2 * lane;
+  const bool dim_ok = d < head_dim;
+  float2 x[MERGE_SMALL_PARTS];
+#pragma unroll
+  for (int j = 0; j < MERGE_SMALL_PARTS; ++j) {
+    x[j] = make_float2(0.f, 0.f);
+    if (j < n_parts && dim_ok)
+      x[j] = *reinterpret_cast<const float2*>(o_parts + ((size_t)j * rows + row) * head_dim + d);
+  }
+  const float l = lane < n_parts ? lse2_parts[(size_t)lane * rows + row] : -INFINITY;
+  float M = l;
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, o));  // lanes 0-7 hold the parts
+  M = __shfl_sync(FULL_MASK, M, 0);
+  const float wt = (l == -INFINITY) ? 0.f : exp2f(l - M);
+  float W = 0.f;
+  float2 o = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < MERGE_SMALL_PARTS; ++j) {
+    const float w = __shfl_sync(FULL_MASK, wt, j);
+    W += w;
+    if (j < n_parts && w != 0.f) {  // unweighted rows are never multiplied
+      o.x = fmaf(w, x[j].x, o.x);
+      o.y = fmaf(w, x[j].y, o.y);
+    }
+  }
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+  if (dim_ok)
+    *reinterpret_cast<__nv_bfloat162*>(out + (size_t)row * head_dim + d) = __floats2bfloat162_rn(o.x * inv, o.y * inv);
+  if (lane == 0 && chunk == 0 && lse2_out) lse2_out[row] = W > 0.f ? M + log2f(W) : -INFINITY;
+}
+
 }  // namespace qkv
 
 using namespace qkv;
@@ -129,9 +180,21 @@ extern "C" int qkv_lse_merge(const float* o_parts, const float* lse2_parts, int3
       ((uintptr_t)lse2_out & 3))
     return QKV_EINVAL;
   if (rows == 0) return QKV_OK;
-  dim3 grid((unsigned)rows, (unsigned)((head_dim + MERGE_DIMS - 1) / MERGE_DIMS));
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
   int np = n_parts, nr = rows, hd = head_dim;
+  if (n_parts <= MERGE_SMALL_PARTS) {
+    int chunks = (head_dim + MERGE_DIMS - 1) / MERGE_DIMS;
+    const long long items = (long long)rows * chunks;
+    if (items > 0x7fffffffLL) return QKV_EUNSUPPORTED;
+    void* sargs[] = {&o_parts, &lse2_parts, &np, &nr, &hd, &chunks, &o, &lse2_out};
+    if (launch_pdl((const void*)lse_merge_small_kernel, dim3((unsigned)((items + 7) / 8)), dim3(256), 0, stream,
+                   sargs) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return QKV_ECUDA;
+    }
+    return QKV_OK;
+  }
+  dim3 grid((unsigned)rows, (unsigned)((head_dim + MERGE_DIMS - 1) / MERGE_DIMS));
   void* args[] = {&o_parts, &lse2_parts, &np, &nr, &hd, &o, &lse2_out};
   if (launch_pdl((const void*)lse_merge_kernel, grid, dim3(MERGE_THREADS), 0, stream, args) != cudaSuccess) {
     (void)cudaGetLastError();

@@ -148,10 +148,12 @@ def test_split_partials_match_oracle_ranges(qkv, num_splits, v_group):
         assert np.max(np.abs(l_parts[i][fin] - rl[fin]), initial=0.0) <= 2e-4
 
 
-# part counts: the automatic plan's 37 on a B200, the 1M-token workload's 148
-# (>= 128 weighted parts per row), and 600, past the merge's first rounds of
-# 256 parts (8 warps x 32 lanes) into its third
-@pytest.mark.parametrize("n", [37, 148, 600])
+# part counts: 1, 5 and 8 (the one-warp-per-row merge for up to 8 parts:
+# the prefill's context split, short decode plans), the automatic plan's 37
+# on a B200, the 1M-token workload's 148 (>= 128 weighted parts per row),
+# and 600, past the merge's first rounds of 256 parts (8 warps x 32 lanes)
+# into its third
+@pytest.mark.parametrize("n", [1, 5, 8, 37, 148, 600])
 def test_lse_merge_matches_oracle(qkv, n):
     rng = np.random.default_rng(21 + n)
     rows, d = 48, 256
