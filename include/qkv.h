@@ -265,7 +265,8 @@ QKV_API int qkv_paged_decode_split_f4_v(float* o_parts, float* lse2_parts, int32
  * hold anything, NaN included); a row without any weighted part gives
  * out = 0 and lse2 = -inf.
  * EINVAL: null pointer, n_parts < 1, rows < 0, head_dim not a multiple of 4
- * or > 1024. */
+ * or > 1024. EUNSUPPORTED: n_parts <= 8 and rows * ceil(head_dim / 64) above
+ * 2^31 - 1 (that case runs one warp per row and 64 dims). */
 QKV_API int qkv_lse_merge(const float* o_parts, const float* lse2_parts, int32_t n_parts, int32_t rows,
                   int32_t head_dim, uint16_t* out, float* lse2_out, qkv_stream_t stream);
 
