@@ -162,8 +162,8 @@ def test_lse_merge_matches_oracle(qkv, n):
     l[rng.random((n, rows)) < 0.2] = -np.inf
     l[:, 5] = -np.inf                     # a row without any weighted part
     if n > 512:
-        l[:512, 7] = -np.inf              # weighted parts only in the second round
-        l[600 - 3, 9] = 400.0             # the row's maximum in the second round
+        l[:512, 7] = -np.inf              # weighted parts only in the last round (past part 512)
+        l[600 - 3, 9] = 400.0             # the row's maximum in the last round
     o[np.isinf(l)] = np.nan               # unweighted parts are never read
     out = torch.empty((rows, d), dtype=torch.int16, device="cuda")
     lo = torch.empty(rows, dtype=torch.float32, device="cuda")
