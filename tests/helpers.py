@@ -75,3 +75,16 @@ def attn_within(gpu_bf16_bits, ref_f64, atol=ATOL_ATTN):
     err = np.abs(g - ref_f64)
     bound = atol + 0.5 * bf16_ulp(ref_f64)
     return err, bound
+
+
+def split_bound(i, n, S, block, head_dim):
+    """First page of split i of a sequence of n pages, as include/qkv.h states
+    the plan: i * n / S, except that with S >= 8 the first ceil(S / 7) splits
+    are d pages shorter (d = 400 tokens at head_dim 256, 800 at 128, at most a
+    quarter split), the other splits sharing those pages."""
+    m = (S + 6) // 7 if S >= 8 else 0
+    d = min((400 if head_dim == 256 else 800) // block, n // S // 4)
+    if m == 0 or d == 0:
+        return i * n // S
+    num = (i * n - i * d * S) * (S - m) if i <= m else n * (S - m) * i - m * d * S * (S - i)
+    return num // (S * (S - m))

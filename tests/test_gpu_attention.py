@@ -6,7 +6,7 @@ import torch
 
 import oracle
 import workloads
-from helpers import ATOL_ATTN, attn_within, oracle_layer, to_dev, to_host
+from helpers import ATOL_ATTN, attn_within, oracle_layer, split_bound, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -41,19 +41,6 @@ def _run_attn(qkv, w, x, cache, num_splits=0, max_splits=0, softmax_scale=0.0):
     att(out, to_dev(x["q"]), cache, to_dev(x["page_table"]), to_dev(x["seq_lens"]), lse2_out=lse,
         softmax_scale=softmax_scale, num_splits=num_splits, device_status=st)
     return to_host(out, np.uint16), to_host(lse), int(st.item())
-
-
-def _split_bound(i, n, S, block, head_dim):
-    """First page of split i of a sequence of n pages, as include/qkv.h states
-    the plan: i * n / S, except that with S >= 8 the first ceil(S / 7) splits
-    are d pages shorter (d = 400 tokens at head_dim 256, 800 at 128, at most a
-    quarter split), the other splits sharing those pages."""
-    m = (S + 6) // 7 if S >= 8 else 0
-    d = min((400 if head_dim == 256 else 800) // block, n // S // 4)
-    if m == 0 or d == 0:
-        return i * n // S
-    num = (i * n - i * d * S) * (S - m) if i <= m else n * (S - m) * i - m * d * S * (S - i)
-    return num // (S * (S - m))
 
 
 def _oracle_attn(w, x, ref, softmax_scale=None):
@@ -137,8 +124,8 @@ def test_split_partials_match_oracle_ranges(qkv, num_splits, v_group):
         tb, te = [], []
         for L in w.seq_lens:
             n = -(-L // w.block_size)
-            tb.append(_split_bound(i, n, num_splits, w.block_size, 256) * w.block_size)
-            te.append(min(_split_bound(i + 1, n, num_splits, w.block_size, 256) * w.block_size, L))
+            tb.append(split_bound(i, n, num_splits, w.block_size, 256) * w.block_size)
+            te.append(min(split_bound(i + 1, n, num_splits, w.block_size, 256) * w.block_size, L))
         ro, rl = oracle.paged_attention(x["q"], ref, x["page_table"], tb, te, w.q_heads, w.kv_heads, 256,
                                         w.block_size)
         ro, rl = ro.reshape(rows, 256), rl.reshape(rows)
@@ -322,8 +309,8 @@ def test_split_partials_head_dim_128(qkv, v_group):
         tb, te = [], []
         for L in w.seq_lens:
             n = -(-L // w.block_size)
-            tb.append(_split_bound(i, n, S, w.block_size, 128) * w.block_size)
-            te.append(min(_split_bound(i + 1, n, S, w.block_size, 128) * w.block_size, L))
+            tb.append(split_bound(i, n, S, w.block_size, 128) * w.block_size)
+            te.append(min(split_bound(i + 1, n, S, w.block_size, 128) * w.block_size, L))
         ro, rl = oracle.paged_attention(x["q"], ref, x["page_table"], tb, te, w.q_heads, w.kv_heads, 128,
                                         w.block_size)
         ro, rl = ro.reshape(rows, 128), rl.reshape(rows)

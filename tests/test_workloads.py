@@ -38,3 +38,30 @@ def test_binding_rejects_mismatched_slot_mapping():
              torch.zeros((8, 4, 64, 128), dtype=torch.uint8), torch.zeros((8, 4, 64, 8), dtype=torch.int16)]
     with pytest.raises(ValueError):
         _abi.qkv_kv_write_f4(k, k, torch.zeros(6, dtype=torch.int64), *cache)
+
+
+def test_split_plan_as_stated():
+    """The split boundaries the GPU tests expect (the plan include/qkv.h
+    states): they start at 0, end at n, never decrease, keep splits equal
+    below 8 splits, and from 8 on make the first ceil(S/7) splits shorter than
+    the rest by the stated amount (at most a quarter split)."""
+    from helpers import split_bound
+    for n in (1, 7, 57, 118, 2048, 4096, 16384):
+        for S in (1, 3, 7, 8, 9, 37, 100, 148):
+            for block in (16, 32, 64):
+                for hd in (256, 128):
+                    b = [split_bound(i, n, S, block, hd) for i in range(S + 1)]
+                    assert b[0] == 0 and b[-1] == n
+                    assert all(b[i] <= b[i + 1] for i in range(S))
+                    sizes = [b[i + 1] - b[i] for i in range(S)]
+                    if S < 8:
+                        assert max(sizes) - min(sizes) <= 1
+                    else:
+                        m = (S + 6) // 7
+                        d = min((400 if hd == 256 else 800) // block, n // S // 4)
+                        if d:
+                            assert max(sizes[:m]) < min(sizes[m:])
+                            assert sum(sizes[:m]) <= m * (n // S) - m * d + m
+    # the 262,144-token workload's plan: 6 of 37 splits ~6 pages shorter per KV head
+    sizes = [split_bound(i + 1, 4096, 37, 64, 256) - split_bound(i, 4096, 37, 64, 256) for i in range(37)]
+    assert sizes[:6] == [104, 105, 105, 104, 105, 105] and min(sizes[6:]) >= 111
