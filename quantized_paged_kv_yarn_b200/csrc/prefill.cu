@@ -14,8 +14,13 @@
 // for a pair of CTAs on two SMs (cta_group::2, M = 256). With head_dim D
 // (256 or 128):
 //
-//   S[256 x 64] = Q'[256 x D] . (K^'hi + K^'lo)[64 x D]^T   (2 x D/16 MMAs, K = 16)
+//   S[256 x 64] = Q'[256 x D] . (K^'hi + K^'lo)[64 x D]^T   (D/16 MMAs, K = 16, N = 128)
 //   O[256 x D] += P[256 x 64] . V^'[64 x D]                 (4 MMAs, N = D)
+//
+// The hi and lo tiles of K^' stand side by side as one B operand of 128
+// rows, so Q K^T takes D/16 MMAs of N = 128 instead of 2 D/16 of N = 64 (on
+// this part an N = 64 MMA takes 45 cycles, an N = 128 one 64); the softmax
+// adds the two products of each token.
 //
 // Rows are (query head of the GQA group, query): 256 = G x (256 / G); CTA
 // rank r of the pair owns rows 128 r .. 128 r + 127 (its lanes of Q', S, P
@@ -30,7 +35,7 @@
 //   warp 0        TMEM allocation (both CTAs); in rank 0, lane 0 issues every
 //                 MMA and commit of the pair
 //   warps 4..7    softmax: thread r owns row r of its CTA (TMEM lane r): puts
-//                 its row of Q' into tensor memory, reads S, keeps the running
+//                 its row of Q' into shared memory, reads S, keeps the running
 //                 max and sum, writes P, rescales O when the max moves, and
 //                 writes the output
 //   warps 8..11   K dequantisation: D/4 dims of one token's K per thread
@@ -47,21 +52,24 @@
 // scores see K exactly (one fp16 rounding of K alone moved scores by up to
 // ~1e-3, more than the attention tolerance allows at short contexts).
 // V^' = fp16((code - 8) s') is rounded once. Q' = fp16(q * 2^e) with a power
-// of two per row (exact for bf16 q in range). The scores and P . V
-// accumulate in fp32; p = 2^(s - m_ref) in fp16 with the reference max moved
+// of two per row (exact for bf16 q in range). The hi and lo products of a
+// score accumulate apart in fp32 and are added in fp32, P . V accumulates
+// in fp32; p = 2^(s - m_ref) in fp16 with the reference max moved
 // lazily (only when a score exceeds it by more than 8, so p <= 256).
 //
-// Q' and P live in tensor memory (the A operands; row r in lane r, two fp16
-// per column); P of a stage overwrites the first half of the S columns it
-// was computed from, which the next Q K^T into that slot may overwrite only
+// P lives in tensor memory (the A operand of P . V; row r in lane r, two
+// fp16 per column) and overwrites the first quarter of the S columns it was
+// computed from, which the next Q K^T into that slot may overwrite only
 // after the P . V reading it (issued earlier by the same thread, and the
 // tensor core keeps one thread's MMAs in order). Shared-memory tiles use the
 // 128-byte swizzle in the canonical UMMA layouts: the K^' tiles (K-major)
-// are [D/64 chunks of 64 dims][32 tokens][128 B]; the V^' tile, the
-// MN-major B operand of P . V, is [D/128 chunks of 64 dims][64 tokens][128 B]. Within
-// each 8-dim unit the dims are stored in the order 0,4,1,5,2,6,3,7 (the
-// order in which four nibble masks of a packed word yield them); Q' uses the
-// same order, and the output un-permutes O's columns.
+// are [D/64 chunks of 64 dims][32 tokens' hi, then their lo][128 B]; Q'
+// (K-major, the A operand of Q K^T) is [D/64 chunks][128 rows][128 B]; the
+// V^' tile, the MN-major B operand of P . V, is [D/128 chunks of 64
+// dims][64 tokens][128 B]. Within each 8-dim unit the dims are stored in
+// the order 0,4,1,5,2,6,3,7 (the order in which four nibble masks of a
+// packed word yield them); Q' uses the same order, and the output
+// un-permutes O's columns.
 #include <algorithm>
 #include <type_traits>
 
@@ -83,25 +91,27 @@ template <int D>
 struct Geo {
   static_assert(D == 256 || D == 128, "head_dim 256 or 128");
   // shared-memory map (offsets from a 1024-byte aligned base)
-  static constexpr int KT = (D / 64) * NTL * 128;   // one K^ tile (hi or lo): [D/64][32][128 B]
+  static constexpr int KT = (D / 64) * NTL * 128;   // the hi (or lo) rows of a K^ slot: D/64 x [32][128 B]
   static constexpr int VT = (D / 128) * NT * 128;   // one V^ tile: [D/128][64][128 B]
-  static constexpr int K_OFF = 0;                   // NS slots x (hi, lo)
+  static constexpr int K_OFF = 0;                   // NS slots of [D/64][hi 32 rows, lo 32 rows][128 B]
   static constexpr int V_OFF = K_OFF + NS * 2 * KT;  // NS slots
-  static constexpr int BAR_OFF = V_OFF + NS * VT;
+  static constexpr int Q_OFF = V_OFF + NS * VT;      // Q' of this CTA's rows: [D/64][128 rows][128 B]
+  static constexpr int BAR_OFF = Q_OFF + (D / 64) * ML * 128;
   // barriers, flags and alignment slack; at least 117 KB, so that no two
   // CTAs share an SM (the tensor memory is allocated whole)
   static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024 > 117 * 1024 ? BAR_OFF + 256 + 1024 : 117 * 1024;
-  // TMEM columns (each CTA, its 128 rows): O 0..D-1, S slot b at D + 64 b
-  // (P of that stage, fp16, overwrites its first 32 columns once S is
-  // read), Q' (two fp16 per column) at D + 128 .. D + 128 + D/2 - 1
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
+  // TMEM columns (each CTA, its 128 rows): O 0..D-1, S slot b at D + 128 b
+  // (columns 0..31 the hi products of rank 0's tokens, 32..63 their lo
+  // products, 64..127 the same for rank 1's; P of that stage, fp16,
+  // overwrites the first 32 columns once S is read)
   static constexpr uint32_t TS = D;
-  static constexpr uint32_t TQ = D + 128;
   // dims one dequantising thread converts per stage, and its 16-byte units
   static constexpr int DPT = D / 4;
   static constexpr int UPT = DPT / 8;
 };
 constexpr uint32_t TMEM_COLS = 512;
-static_assert(Geo<256>::TQ + 128 <= TMEM_COLS && Geo<128>::TQ + 64 <= TMEM_COLS, "tensor memory map");
+static_assert(Geo<256>::TS + 4 * NT <= TMEM_COLS && Geo<128>::TS + 4 * NT <= TMEM_COLS, "tensor memory map");
 
 struct Bars {
   // signalled by producers of both CTAs, waited on in rank 0
@@ -149,6 +159,15 @@ __device__ __forceinline__ void umma2_ts(uint32_t d_tmem, uint32_t a_tmem, uint6
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// Pair MMA with A and B from shared memory (A: each CTA its M / 2 rows; B:
+// each CTA N / 2 columns, at the same offsets in both CTAs).
+__device__ __forceinline__ void umma2_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
 }
 
 // Arrive, once the pair's MMAs issued so far are done, on the barrier at
@@ -315,8 +334,9 @@ template <int D>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     paged_prefill_kernel(const Params p) {
   using Gm = Geo<D>;
-  constexpr int KT = Gm::KT, VT = Gm::VT, K_OFF = Gm::K_OFF, V_OFF = Gm::V_OFF, BAR_OFF = Gm::BAR_OFF;
-  constexpr uint32_t TS = Gm::TS, TQ = Gm::TQ;
+  constexpr int KT = Gm::KT, VT = Gm::VT, K_OFF = Gm::K_OFF, V_OFF = Gm::V_OFF, Q_OFF = Gm::Q_OFF;
+  constexpr int BAR_OFF = Gm::BAR_OFF;
+  constexpr uint32_t TS = Gm::TS;
   // 1024-aligned by pointer arithmetic on the shared array (keeps accesses in
   // the shared window)
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -372,13 +392,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ MMA issue (rank 0)
     if (rank == 0 && lane == 0) {
-      constexpr uint32_t ID_QK = (1u << 4) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+      // Q K^T with N = 2 NT: K^'hi and K^'lo side by side as one B operand
+      constexpr uint32_t ID_QK = (1u << 4) | ((uint32_t)((2 * NT) >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
       constexpr uint32_t ID_PV = (1u << 4) | (1u << 16) | ((uint32_t)(D >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
       bool ok = wait_bar(&bars.qready, 0, abort);
       // descriptors of slot 0 at offset 0; each MMA adds its byte offset >> 4
       // to the start-address field (no carry: smem offsets stay below 2^18)
       const uint64_t dv0 = sdesc(s_base + V_OFF, NT * 128, 1024);
       const uint64_t dk0 = sdesc(s_base + K_OFF, 16, 1024);
+      const uint64_t dq0 = sdesc(s_base + Q_OFF, 16, 1024);
       auto pv = [&](int i) -> bool {
         const int b = i % NS, u = i / NS, sb = i & 1;
         if (!wait_bar(&bars.pready, (uint32_t)i & 1u, abort)) return false;
@@ -387,7 +409,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint64_t dv = dv0 + (uint64_t)((b * VT) >> 4);
 #pragma unroll
         for (int kk = 0; kk < NT / 16; ++kk)  // A = P in tensor memory (S slot sb)
-          umma2_ts(tmem, tmem + TS + 64 * sb + 8 * kk, dv + (uint64_t)((2048 * kk) >> 4), ID_PV,
+          umma2_ts(tmem, tmem + TS + 2 * NT * sb + 8 * kk, dv + (uint64_t)((2048 * kk) >> 4), ID_PV,
                    (i > 0 || kk > 0) ? 1u : 0u);
         umma2_commit_both(&bars.odone);
         umma2_commit_both(&bars.vfree[b]);
@@ -401,14 +423,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // core runs one thread's MMAs in order
         tc_fence_after();
         const uint64_t dk = dk0 + (uint64_t)((b * 2 * KT) >> 4);
-        const uint32_t ts = tmem + TS + 64 * sb;
+        const uint32_t ts = tmem + TS + 2 * NT * sb;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // K^'hi, then K^'lo into the same accumulator
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = h * KT + (kk >> 2) * (NTL * 128) + 32 * (kk & 3);
-            umma2_ts(ts, tmem + TQ + 8 * kk, dk + (uint64_t)(off >> 4), ID_QK, (h > 0 || kk > 0) ? 1u : 0u);
-          }
+        for (int kk = 0; kk < D / 16; ++kk) {  // 16 dims per MMA: 32 bytes into a 128-byte row
+          const uint32_t koff = (kk >> 2) * (2 * NTL * 128) + 32 * (kk & 3);
+          const uint32_t qoff = (kk >> 2) * (ML * 128) + 32 * (kk & 3);
+          umma2_ss(ts, dq0 + (uint64_t)(qoff >> 4), dk + (uint64_t)(koff >> 4), ID_QK, kk > 0 ? 1u : 0u);
         }
         umma2_commit_both(&bars.sfull[sb]);
         umma2_commit_both(&bars.kfree[b]);
@@ -436,7 +456,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int lim = min(p.prefix_len + qi, p.kv_limit - 1);  // last token this row attends
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
-    // Q' = fp16(q * 2^e) into tensor memory, dims permuted per 8-dim unit
+    // Q' = fp16(q * 2^e) into row r of this CTA's Q' tile, dims permuted per 8-dim unit
     float c_row;
     {
       const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)qi * p.q_heads + qhead) * D);
@@ -459,8 +479,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const float up = __int_as_float((127 + e / 2) << 23) * __int_as_float((127 + (e - e / 2)) << 23);
       c_row = p.score_scale * 16.f / up;  // S = S' * 2^(4 - e)
 #pragma unroll 1
-      for (int g = 0; g < D / 64; ++g) {  // 8 units = 32 columns per store
-        uint32_t o[32];
+      for (int g = 0; g < D / 64; ++g) {  // one 128-byte row of a 64-dim chunk
 #pragma unroll
         for (int uu = 0; uu < 8; ++uu) {
           uint4 w = make_uint4(0u, 0u, 0u, 0u);
@@ -472,13 +491,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             f[2 * i] = __uint_as_float(ws[i] << 16) * up;
             f[2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u) * up;
           }
+          uint32_t o[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) o[4 * uu + i] = h2_as_u32(__floats2half2_rn(f[i], f[i + 4]));
+          for (int i = 0; i < 4; ++i) o[i] = h2_as_u32(__floats2half2_rn(f[i], f[i + 4]));
+          sts128(s_base + Q_OFF + g * (ML * 128) + swz(r, uu), o[0], o[1], o[2], o[3]);
         }
-        tmem_st32(tmem + lane_base + TQ + 32 * g, o);
       }
-      tmem_wait_st();
-      tc_fence_before();
+      fence_async_smem();  // the tensor core reads the tile through the async proxy
       arrive_rank0(&bars.qready);
     }
 
@@ -489,13 +508,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       ok = wait_bar(&bars.sfull[sb], (uint32_t)(j >> 1) & 1u, abort);
       if (!__all_sync(FULL_MASK, ok)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(tmem + lane_base + TS + 64 * sb, sr[0]);
-      tmem_ld32(tmem + lane_base + TS + 64 * sb + 32, sr[1]);
-      tmem_wait_ld();
+      // score of token i = hi + lo products: columns 64 h + i % 32 and 64 h + 32 + i % 32 (h = i / 32)
+      const uint32_t ts = tmem + lane_base + TS + 2 * NT * sb;
       float s[64];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(sr[i >> 5][i & 31]);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sr[2][32];
+        tmem_ld32(ts + 64 * h, sr[0]);
+        tmem_ld32(ts + 64 * h + 32, sr[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[32 * h + i] = __uint_as_float(sr[0][i]) + __uint_as_float(sr[1][i]);
+      }
       const int base = (st0 + j) * NT;
       if (base + NT - 1 > lim) {
 #pragma unroll
@@ -527,7 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         pw[i] = h2_as_u32(h);
       }
       // P into the first 32 columns of S slot sb (its S is in registers)
-      tmem_st32(tmem + lane_base + TS + 64 * sb, pw);
+      tmem_st32(ts, pw);
       if (any_need && j >= 1) {  // rescale O once P . V of the previous stage is done
         ok = wait_bar(&bars.odone, (uint32_t)(j - 1) & 1u, abort);
         if (!__all_sync(FULL_MASK, ok)) { ok = false; break; }
@@ -547,9 +571,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       arrive_rank0(&bars.pready);
     }
 
-    // epilogue: O / l, columns un-permuted; bf16 out, or this part's fp32 partial
+    // epilogue: O / l, columns un-permuted; bf16 out, or this part's fp32 partial.
+    // O is complete once the drain commit lands (one phase, after every MMA of
+    // the pair). A parity wait on odone cannot say so: P . V of stage n_st - 2
+    // is issued after the last Q K^T, so odone may still be in phase n_st - 2,
+    // whose parity differs from that of n_st - 1, and the wait would return
+    // before the last two P . V products are in O.
     if (ok) {
-      ok = wait_bar(&bars.odone, (uint32_t)(n_st - 1) & 1u, abort);
+      ok = wait_bar(&bars.drain, 0u, abort) && !*abort;
       ok = __all_sync(FULL_MASK, ok);
     }
     if (ok) {
@@ -660,7 +689,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         uint32_t o[4] = {0u, 0u, 0u, 0u}, r[4] = {0u, 0u, 0u, 0u};
         if (x.ok == 1) dequant_word<LO>(wd[u], u < 4 ? s_lo : s_hi, o, r);
         sts128(chunk_base + swz(trow, unit0 + u), o[0], o[1], o[2], o[3]);
-        if constexpr (LO) sts128(chunk_base + KT + swz(trow, unit0 + u), r[0], r[1], r[2], r[3]);
+        if constexpr (LO) sts128(chunk_base + NTL * 128 + swz(trow, unit0 + u), r[0], r[1], r[2], r[3]);
       }
     };
     auto process = [&](int j, const Raw& x) -> bool {
@@ -669,7 +698,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         flag(p.status, QKV_DEV_BAD_PAGE);
       if (is_k) {
         if (u >= 1 && !wait_bar(&bars.kfree[b], (uint32_t)(u - 1) & 1u, abort)) return false;
-        put(s_base + K_OFF + b * (2 * KT) + chunk * (NTL * 128), x, std::true_type{});
+        put(s_base + K_OFF + b * (2 * KT) + chunk * (2 * NTL * 128), x, std::true_type{});
         fence_async_smem();
         arrive_rank0(&bars.kready[b]);
       } else {
