@@ -129,6 +129,22 @@ def test_prefill_context_split(qkv, splits):
     _check(out, lse, ro, rl)
 
 
+@pytest.mark.parametrize("case", [(700, 64, 64, 16, 4), (200, 64, 64, 16, 4)], ids=["L700-n64", "L200-n64"])
+def test_prefill_repeated_calls_hold_the_last_stages(qkv, case):
+    """One short-context chunk 16 times over: every output must hold the
+    P.V products of the last two stages. (The epilogue once took O as done
+    on a parity wait that the per-stage barrier could pass a phase early,
+    when the last P.V finished late: lse right, the output without those
+    stages, in about one call of a few hundred.)"""
+    L, n_q, block, hq, hkv = case
+    w, x, ref, cache, q = _setup(qkv, L, n_q, block, hq, hkv, 32)
+    ro, rl = oracle.prefill_attention(q, ref, x["page_table"][0], np.arange(L - n_q, L), hq, hkv, 256, block)
+    for _ in range(16):
+        out, lse, st = _run(qkv, w, x, cache, q, L - n_q)
+        assert st == 0
+        _check(out, lse, ro, rl)
+
+
 def test_prefill_outliers_and_scale(qkv):
     """1 % of K rows x20 (the 1M workload's outliers) and an explicit softmax scale."""
     w, x, ref, cache, q = _setup(qkv, 1200, 96, 64, 16, 4, outliers=0.01, seed=3)
