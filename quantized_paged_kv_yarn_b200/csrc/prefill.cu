@@ -114,8 +114,11 @@ constexpr uint32_t TMEM_COLS = 512;
 static_assert(Geo<256>::TS + 4 * NT <= TMEM_COLS && Geo<128>::TS + 4 * NT <= TMEM_COLS, "tensor memory map");
 
 struct Bars {
-  // signalled by producers of both CTAs, waited on in rank 0
-  uint64_t kready[NS], vready[NS], pready, qready;
+  // signalled by producers of both CTAs, waited on in rank 0. P of stage i
+  // signals pready[i % 2]: with one barrier, the softmax of one CTA (which
+  // needs only its own S) could finish stage i + 1 before its partner
+  // finished stage i, and its arrivals would complete stage i's phase.
+  uint64_t kready[NS], vready[NS], pready[2], qready;
   // signalled by the MMA commits of the pair, waited on in each CTA
   uint64_t kfree[NS], vfree[NS], sfull[2], odone, drain;
   uint32_t tmem;
@@ -365,7 +368,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&bars.vfree[b], 1);
     }
     for (int b = 0; b < 2; ++b) mbar_init(&bars.sfull[b], 1);
-    mbar_init(&bars.pready, 2 * 128);
+    for (int b = 0; b < 2; ++b) mbar_init(&bars.pready[b], 2 * 128);
     mbar_init(&bars.qready, 2 * 128);
     mbar_init(&bars.odone, 1);
     mbar_init(&bars.drain, 1);
@@ -403,7 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const uint64_t dq0 = sdesc(s_base + Q_OFF, 16, 1024);
       auto pv = [&](int i) -> bool {
         const int b = i % NS, u = i / NS, sb = i & 1;
-        if (!wait_bar(&bars.pready, (uint32_t)i & 1u, abort)) return false;
+        if (!wait_bar(&bars.pready[i & 1], (uint32_t)(i >> 1) & 1u, abort)) return false;
         if (!wait_bar(&bars.vready[b], (uint32_t)u & 1u, abort)) return false;
         tc_fence_after();
         const uint64_t dv = dv0 + (uint64_t)((b * VT) >> 4);
@@ -568,7 +571,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      arrive_rank0(&bars.pready);
+      arrive_rank0(&bars.pready[j & 1]);
     }
 
     // epilogue: O / l, columns un-permuted; bf16 out, or this part's fp32 partial.
