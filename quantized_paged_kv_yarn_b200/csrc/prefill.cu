@@ -118,6 +118,8 @@ struct Bars {
   // signals pready[i % 2]: with one barrier, the softmax of one CTA (which
   // needs only its own S) could finish stage i + 1 before its partner
   // finished stage i, and its arrivals would complete stage i's phase.
+  // (tests/test_prefill_protocol.py models these roles and barriers and
+  // checks every wait's phase over skewed schedules.)
   uint64_t kready[NS], vready[NS], pready[2], qready;
   // signalled by the MMA commits of the pair, waited on in each CTA
   uint64_t kfree[NS], vfree[NS], sfull[2], odone, drain;
