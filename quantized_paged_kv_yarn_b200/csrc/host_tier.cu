@@ -51,8 +51,13 @@ constexpr int STAGE_UNROLL = 4;  // loads in flight per thread before its stores
 // its loads of host memory are outstanding. (With a prefill kernel running
 // beside a live staging grid -- staging on a second stream -- a bounded wait
 // of the prefill ran out at full size, both before and after the prefill
-// took its tensor memory only after its dependency wait; the cause is not
-// known, so the library never overlaps the two.)
+// took its tensor memory only after its dependency wait. A race found later
+// fits it: the prefill's one P-ready barrier let a CTA running a stage ahead
+// of its partner complete the partner's phase, after which the partner
+// could wait for scores that never came; a staging CTA on one SM of a pair
+// is what slows one CTA of it. That barrier is now split by stage parity,
+// but the overlap has not been run since, so the library still never
+// overlaps the two.)
 __global__ void __launch_bounds__(STAGE_THREADS) stage_pages_f4_kernel(const StageParams p) {
   pdl_wait();
   if (blockIdx.x == 0) {
