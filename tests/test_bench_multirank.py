@@ -1,6 +1,6 @@
 """The bench's multi-rank plumbing on CPU: two gloo ranks, the max-over-ranks
 timing and the weak-scaling whole-job rate; the reference arm's non-zero
-ranks do no work."""
+ranks do no work, and its rank 0 prints the one JSON line the driver reads."""
 import os
 import socket
 
@@ -51,3 +51,24 @@ def test_reference_arm_other_ranks_do_nothing(capsys):
         workload, steps, warmup, gpus = "yarn262k", 2, 1, 2
     assert bench.run_reference(A(), rank=1) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_its_contract_line(capsys, monkeypatch):
+    """Rank 0 of the reference arm: one JSON line with the keys the driver
+    reads (the oracle's sample kept small here)."""
+    import json
+    monkeypatch.setattr(bench, "calibrate_sample", lambda w, seconds, n_threads=0: 4 * w.block_size)
+
+    class A:
+        workload, steps, warmup, gpus = "tiny_4k", 2, 1, 1
+    bench.run_reference(A(), rank=0)
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "GB/s"
+    assert d["higher_is_better"] is True and d["n_gpus"] == 1 and d["steps"] == 2 and d["warmup"] == 1
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and "64 of 4096" in d["cpu_baseline"]["sample"]
+    assert d["config"]["workload"] == "tiny_4k"
