@@ -23,10 +23,11 @@
 // adds the two products of each token.
 //
 // Rows are (query head of the GQA group, query): 256 = G x (256 / G); CTA
-// rank r of the pair owns rows 128 r .. 128 r + 127 (its lanes of Q', S, P
-// and O). The B operands are split by N: of each 64-token stage, rank r
-// dequantises the K of tokens 32 r .. 32 r + 31 (all D dims) and the V of
-// dims D/2 r .. D/2 r + D/2 - 1 (all 64 tokens) into its own shared memory,
+// rank r of the pair owns rows 128 r .. 128 r + 127 (its rows of the Q'
+// tile, its lanes of S, P and O). The B operands are split by N: of each
+// 64-token stage, rank r dequantises the K of tokens 32 r .. 32 r + 31 (all
+// D dims) and the V of dims D/2 r .. D/2 r + D/2 - 1 (all 64 tokens) into
+// its own shared memory,
 // so each SM writes and the tensor core reads half of every tile, and the
 // shared-memory pipe (the bound of a one-SM version) carries half the bytes.
 // One pair per (256 / G queries, KV head).
